@@ -1,0 +1,215 @@
+"""CPU oracle for the NVFP4 quantized linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may import
+this package. The product path (``nvfp4_block_scaled_14_b200``) never imports it and shares
+no code with it. The arithmetic lives in ``nvfp4_oracle.c`` (plain scalar C); this module only
+marshals numpy arrays into it.
+
+Sources of each step (see the header of nvfp4_oracle.c for the full list):
+  * "Qwen-Image NVFP4 on a 16 GB Ada GPU", "What NVFP4 is and how it differs from NF4" and
+    the figure "First NVFP4 block, as stored in the file" -- the format and decode equation.
+  * "Qwen-Rapid-AIO FP8 -> NVFP4", "1. Double Quantization" -- FP8 upcast, then NVFP4.
+  * "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details" -- dynamic per-tensor amax.
+  * "Qwen-Rapid-AIO FP8 -> NVFP4", "Recommended Model" -- p99.9 static input scales.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build_oracle
+
+_lib = None
+
+F32, BF16, E4M3 = 0, 1, 2
+
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = build_oracle.build()
+        L = ctypes.CDLL(path)
+        L.ora_e2m1_decode.argtypes = [ctypes.c_int]
+        L.ora_e2m1_decode.restype = ctypes.c_double
+        L.ora_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.ora_e4m3_decode.restype = ctypes.c_double
+        L.ora_e2m1_encode.argtypes = [ctypes.c_float]
+        L.ora_e2m1_encode.restype = ctypes.c_int
+        L.ora_e4m3_encode_nonneg.argtypes = [ctypes.c_float]
+        L.ora_e4m3_encode_nonneg.restype = ctypes.c_uint8
+        L.ora_swizzled_offset.argtypes = [_i64, _i64, _i64]
+        L.ora_swizzled_offset.restype = _i64
+        L.ora_swizzled_bytes.argtypes = [_i64, _i64]
+        L.ora_swizzled_bytes.restype = _i64
+        L.ora_quantize.argtypes = [_vp, ctypes.c_int, _f32p, _i64, _i64, _f32p, _u8p, _u8p,
+                                   _u8p, _f32p]
+        L.ora_quantize.restype = ctypes.c_int
+        L.ora_dequantize_f32.argtypes = [_u8p, _u8p, ctypes.c_float, _i64, _i64, _f32p]
+        L.ora_dequantize_bf16.argtypes = [_u8p, _u8p, ctypes.c_float, _i64, _i64,
+                                          ctypes.POINTER(ctypes.c_uint16)]
+        L.ora_gemm_f64.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
+                                   _i64, _i64, _i64, _f64p]
+        L.ora_gemm_f64_sampled.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p,
+                                           ctypes.c_float, _i64, _i64p, _i64p, _i64, _f64p]
+        L.ora_percentile_abs.argtypes = [ctypes.POINTER(_f32p), _i64p, ctypes.c_int,
+                                         ctypes.c_uint32, ctypes.c_uint32, _f32p, _f32p]
+        L.ora_percentile_abs.restype = ctypes.c_int
+        L.ora_e2m1_encode_array.argtypes = [_f32p, _i64, _u8p]
+        L.ora_e4m3_encode_array.argtypes = [_f32p, _i64, _u8p]
+        L.ora_amax.argtypes = [_f32p, _i64]
+        L.ora_amax.restype = ctypes.c_float
+        _lib = L
+    return _lib
+
+
+def _p(a, t):
+    return a.ctypes.data_as(t)
+
+
+# ---- scalar codecs ---------------------------------------------------------------------
+
+def e2m1_decode(code: int) -> float:
+    return lib().ora_e2m1_decode(int(code))
+
+
+def e4m3_decode(b: int) -> float:
+    return lib().ora_e4m3_decode(int(b))
+
+
+def e2m1_encode(y: float) -> int:
+    return lib().ora_e2m1_encode(float(np.float32(y)))
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().ora_e4m3_encode_nonneg(float(np.float32(v)))
+
+
+def e2m1_encode_array(y: np.ndarray) -> np.ndarray:
+    y = np.ascontiguousarray(y, np.float32).ravel()
+    out = np.zeros(y.size, np.uint8)
+    lib().ora_e2m1_encode_array(_p(y, _f32p), y.size, _p(out, _u8p))
+    return out
+
+
+def e4m3_encode_array(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32).ravel()
+    out = np.zeros(v.size, np.uint8)
+    lib().ora_e4m3_encode_array(_p(v, _f32p), v.size, _p(out, _u8p))
+    return out
+
+
+def swizzled_offset(row: int, block: int, nblocks: int) -> int:
+    return lib().ora_swizzled_offset(row, block, nblocks)
+
+
+def swizzled_bytes(rows: int, cols: int) -> int:
+    return lib().ora_swizzled_bytes(rows, cols)
+
+
+# ---- array ops -------------------------------------------------------------------------
+
+class Quantized:
+    """codes [rows, cols/2] u8, scales_lin [rows, cols/16] u8, scales_swz (flat u8), sg f32."""
+
+    def __init__(self, codes, scales_lin, scales_swz, sg, rows, cols):
+        self.codes, self.scales_lin, self.scales_swz = codes, scales_lin, scales_swz
+        self.sg, self.rows, self.cols = sg, rows, cols
+
+
+def _src_dtype(x):
+    if x.dtype == np.float32:
+        return F32
+    if x.dtype == np.uint16:  # bf16 bit patterns
+        return BF16
+    if x.dtype == np.uint8:  # E4M3 bit patterns
+        return E4M3
+    raise TypeError(f"unsupported source dtype {x.dtype}")
+
+
+def quantize(x: np.ndarray, amax=None, fp8_scale=None) -> Quantized:
+    """x: float32, or uint16 (bf16 bits), or uint8 (E4M3 bits, times fp8_scale or 1.0)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    lin = np.zeros((rows, cols // 16), np.uint8)
+    swz = np.zeros(max(swizzled_bytes(rows, cols), 1), np.uint8)
+    sg = np.zeros(1, np.float32)
+    am = None if amax is None else np.array([amax], np.float32)
+    s8 = None if fp8_scale is None else np.array([fp8_scale], np.float32)
+    rc = lib().ora_quantize(x.ctypes.data_as(_vp), _src_dtype(x),
+                            None if s8 is None else _p(s8, _f32p), rows, cols,
+                            None if am is None else _p(am, _f32p),
+                            _p(codes, _u8p), _p(lin, _u8p), _p(swz, _u8p), _p(sg, _f32p))
+    if rc != 0:
+        raise ValueError(f"oracle quantize failed ({rc}); cols must be a multiple of 16")
+    return Quantized(codes, lin, swz, float(sg[0]), rows, cols)
+
+
+def dequantize(q: Quantized, out_dtype="f32") -> np.ndarray:
+    codes = np.ascontiguousarray(q.codes)
+    lin = np.ascontiguousarray(q.scales_lin)
+    if out_dtype == "f32":
+        out = np.zeros((q.rows, q.cols), np.float32)
+        lib().ora_dequantize_f32(_p(codes, _u8p), _p(lin, _u8p), q.sg, q.rows, q.cols,
+                                 _p(out, _f32p))
+    else:
+        out = np.zeros((q.rows, q.cols), np.uint16)
+        lib().ora_dequantize_bf16(_p(codes, _u8p), _p(lin, _u8p), q.sg, q.rows, q.cols,
+                                  out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
+    return out
+
+
+def gemm(a: Quantized, w: Quantized) -> np.ndarray:
+    """Y = dequant(A) . dequant(W)^T in fp64, [M, N]."""
+    assert a.cols == w.cols
+    M, N, K = a.rows, w.rows, a.cols
+    out = np.zeros((M, N), np.float64)
+    lib().ora_gemm_f64(_p(a.codes, _u8p), _p(a.scales_lin, _u8p), a.sg,
+                       _p(w.codes, _u8p), _p(w.scales_lin, _u8p), w.sg, M, N, K, _p(out, _f64p))
+    return out
+
+
+def gemm_sampled(a: Quantized, w: Quantized, ms, ns) -> np.ndarray:
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    out = np.zeros(len(ms), np.float64)
+    lib().ora_gemm_f64_sampled(_p(a.codes, _u8p), _p(a.scales_lin, _u8p), a.sg,
+                               _p(w.codes, _u8p), _p(w.scales_lin, _u8p), w.sg, a.cols,
+                               _p(ms, _i64p), _p(ns, _i64p), len(ms), _p(out, _f64p))
+    return out
+
+
+def percentile_abs(arrays, num=999, den=1000):
+    """Nearest-rank percentile of |x| over the union of float32 arrays, and the max."""
+    arrs = [np.ascontiguousarray(a, np.float32).ravel() for a in arrays]
+    ptrs = (_f32p * len(arrs))(*[_p(a, _f32p) for a in arrs])
+    lens = np.array([a.size for a in arrs], np.int64)
+    pct = np.zeros(1, np.float32)
+    mx = np.zeros(1, np.float32)
+    rc = lib().ora_percentile_abs(ptrs, _p(lens, _i64p), len(arrs), num, den, _p(pct, _f32p),
+                                  _p(mx, _f32p))
+    if rc != 0:
+        raise ValueError("oracle percentile: empty input or bad ratio")
+    return float(pct[0]), float(mx[0])
+
+
+def source_to_f32(x: np.ndarray, fp8_scale=None) -> np.ndarray:
+    """The oracle's own upcast of a bf16 (uint16 bits) / E4M3 (uint8 bits) array to fp32."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x.copy()
+    f = np.zeros(x.shape, np.float32)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).reshape(x.shape)
+    L = lib()
+    lut = np.array([L.ora_e4m3_decode(b) for b in range(256)], np.float32)
+    f = lut[x]
+    s8 = np.float32(1.0 if fp8_scale is None else fp8_scale)
+    return (f * s8).astype(np.float32)

@@ -1,0 +1,167 @@
+/*
+ * nvfp4.h -- C ABI of the NVFP4 quantized linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The format (from "Qwen-Image NVFP4 on a 16 GB Ada GPU", section "What NVFP4 is and how it
+ * differs from NF4", and the figure "First NVFP4 block, as stored in the file"):
+ *   - each value is a 4-bit E2M1 code: sign, two exponent bits, one mantissa bit;
+ *     magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6};
+ *   - each block of 16 consecutive values of a row carries one FP8 E4M3 scale;
+ *   - each tensor carries one FP32 global scale;
+ *   - value = E2M1(code) x block scale x global scale;
+ *   - two codes per byte, the first (even-index) code in the low nibble.
+ *
+ * Conventions for every call:
+ *   - Matrices are row-major. A quantized matrix of [rows x cols] values has
+ *       codes      : rows x cols/2 bytes, row-major;
+ *       scales_lin : rows x cols/16 bytes (E4M3 bit patterns), row-major ("linear" layout);
+ *       scales_swz : nvfp4_scales_bytes(rows, cols, 1) bytes, the tensor-core operand layout:
+ *                    the [rows x cols/16] scale matrix cut into atoms of 128 rows x 4 blocks,
+ *                    512 bytes each; atoms of one 128-row band are stored one after another
+ *                    along the blocks, bands one after another; inside an atom, (r, b) sits at
+ *                    byte 16*(r%32) + 4*((r%128)/32) + b%4. Padding rows / blocks are zero;
+ *       global_scale: one fp32 in device memory.
+ *   - Blocks run along cols (the GEMM's K dimension). cols must be a multiple of 32.
+ *   - The caller owns every buffer; the library never allocates or frees memory. Every
+ *     pointer is a device pointer unless stated otherwise, 16-byte aligned.
+ *   - Every call is asynchronous on the given stream. Argument checks run on the host before
+ *     any launch and return an error without touching memory.
+ *   - Numbers of rows, cols, M, N, K are >= 0 and < 2^31. Empty inputs are allowed.
+ *   - Inputs must be finite; a NaN or Inf input gives unspecified codes.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1, /* NULL pointer, bad enum, bad ratio */
+    NVFP4_ERR_SHAPE = 2,       /* negative or too large size, cols not a multiple of 32 */
+    NVFP4_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+    NVFP4_ERR_WORKSPACE = 4,   /* workspace smaller than nvfp4_workspace_bytes() */
+    NVFP4_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed */
+    NVFP4_ERR_TIMEOUT = 6,     /* a device-side wait gave up (reported by nvfp4_sync_status) */
+    NVFP4_ERR_UNSUPPORTED = 7  /* the device is not sm_100 */
+} nvfp4_status;
+
+typedef enum { NVFP4_F32 = 0, NVFP4_BF16 = 1 } nvfp4_dtype;
+
+/* Operations whose workspace can be queried with nvfp4_workspace_bytes. */
+typedef enum {
+    NVFP4_OP_QUANTIZE = 0,   /* m = rows, k = cols (n ignored) */
+    NVFP4_OP_LINEAR = 1,     /* m = M, n = N, k = K */
+    NVFP4_OP_CALIB_BF16 = 2, /* m, n, k ignored */
+    NVFP4_OP_CALIB_F32 = 3   /* m, n, k ignored */
+} nvfp4_op;
+
+/* Human-readable name of a status. Never NULL. */
+const char *nvfp4_status_str(nvfp4_status st);
+
+/* Bytes of the packed codes of a rows x cols matrix: rows * cols / 2. */
+size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of its scales: linear rows * cols/16 (swizzled = 0), or the swizzled layout padded to
+ * whole 128 x 4 atoms (swizzled = 1). */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int swizzled);
+
+/* Device workspace the call needs (0 if none). Returns 0 for an unknown op. */
+size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k);
+
+/*
+ * Quantize a fp32 or bf16 matrix x [rows x cols] to NVFP4.
+ *
+ * Global scale: sg = amax / (6 * 448) where amax is either the dynamic per-tensor max |x|
+ * (static_amax == NULL; "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details":
+ * activations quantized at runtime from the per-tensor amax) or the calibrated value that
+ * static_amax points to (device fp32; "Qwen-Rapid-AIO FP8 -> NVFP4", "Recommended Model":
+ * p99.9 input scales). Values above a static amax saturate to +-6 x 448 x sg.
+ * Block scale: sb = E4M3(bmax / (6 * sg)), round to nearest even, saturating at 448.
+ * Code: E2M1(x * (1 / (sb * sg))), round to nearest even, saturating at 6, sign kept.
+ * All code-deciding arithmetic is IEEE fp32 round-to-nearest in that order; sg == 0 or
+ * sb == 0 gives all-zero codes for the block.
+ *
+ * Outputs: codes (required); scales_swz and / or scales_lin (at least one non-NULL; padding of
+ * scales_swz is written with zeros); global_scale (required, device fp32).
+ * ws: device workspace of nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols) bytes
+ * (may be NULL when static_amax is given).
+ */
+nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dt, int64_t rows, int64_t cols,
+                            const float *static_amax, uint8_t *codes, uint8_t *scales_swz,
+                            uint8_t *scales_lin, float *global_scale, void *ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/*
+ * Double quantization ("Qwen-Rapid-AIO FP8 -> NVFP4", "Why This Exists" and
+ * "1. Double Quantization"): x_e4m3 holds FP8 E4M3 bit patterns; each value is upcast to
+ * fp32 as e4m3 * (*fp8_scale) (one fp32 multiply; fp8_scale is a device fp32, or NULL for
+ * layers that ship without a weight_scale, read as 1.0) and then quantized exactly as
+ * nvfp4_quantize does. Same outputs, workspace and rules as nvfp4_quantize.
+ */
+nvfp4_status nvfp4_quantize_fp8_src(const uint8_t *x_e4m3, const float *fp8_scale, int64_t rows,
+                                    int64_t cols, const float *static_amax, uint8_t *codes,
+                                    uint8_t *scales_swz, uint8_t *scales_lin,
+                                    float *global_scale, void *ws, size_t ws_bytes,
+                                    cudaStream_t stream);
+
+/*
+ * Dequantize ("Qwen-Image NVFP4 on a 16 GB Ada GPU", worked example under "First NVFP4
+ * block, as stored in the file": weight = E2M1 x block scale x global scale).
+ * out[r, k] = (E2M1(code) * sb) * sg in fp32 (two round-to-nearest multiplies in that order);
+ * for NVFP4_BF16 output, that fp32 value rounded to nearest even. Reads linear scales.
+ * out: rows x cols of out_dt. No workspace.
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales_lin,
+                              const float *global_scale, int64_t rows, int64_t cols,
+                              nvfp4_dtype out_dt, void *out, cudaStream_t stream);
+
+/*
+ * Block-scaled W4A4 linear layer Y = dequant(A) . dequant(W)^T on the FP4 tensor cores
+ * ("Qwen-Image NVFP4 on a 16 GB Ada GPU", "What NVFP4 is...": on Blackwell the tensor cores
+ * multiply in FP4 with weights and activations both in 4 bits).
+ *   A: M x K (activations: a_codes, a_scales_swz, a_gs), W: N x K (weights, nn.Linear layout).
+ *   Y[m, n] = (sgA * sgW) * sum_b sA[m,b] * sW[n,b] * sum_{k in b} eA[m,k] * eW[n,k],
+ *   accumulated in fp32 by the tensor cores, scaled by sgA * sgW (fp32), then stored as out_dt
+ *   (bf16 rounded to nearest even). y: M x N of out_dt.
+ * K must be a multiple of 32. ws: nvfp4_workspace_bytes(NVFP4_OP_LINEAR, M, N, K) bytes.
+ */
+nvfp4_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales_swz, const float *a_gs,
+                          const uint8_t *w_codes, const uint8_t *w_scales_swz, const float *w_gs,
+                          int64_t M, int64_t N, int64_t K, nvfp4_dtype out_dt, void *y, void *ws,
+                          size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Static-scale calibration ("Qwen-Rapid-AIO FP8 -> NVFP4", "Recommended Model": p99.9
+ * percentile aggregation over calibration generations instead of max aggregation).
+ * Over the union of num_batches device arrays (batches is a HOST array of device pointers),
+ * each of elems_per_batch values of dt, computes exactly:
+ *   *out_pct = the nearest-rank pct_num/pct_den percentile of |x|: the rank-th smallest |x|
+ *              with rank = ceil(n * pct_num / pct_den) (1-based, at least 1), n = all values;
+ *   *out_max = max |x|.
+ * out_pct / out_max are device fp32; either may be used as the static_amax of nvfp4_quantize.
+ * Requires 0 < pct_num <= pct_den and n > 0.
+ * ws: nvfp4_workspace_bytes(NVFP4_OP_CALIB_BF16 or _F32, 0, 0, 0) bytes.
+ */
+nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_batches,
+                                         int64_t elems_per_batch, nvfp4_dtype dt,
+                                         uint32_t pct_num, uint32_t pct_den, float *out_pct,
+                                         float *out_max, void *ws, size_t ws_bytes,
+                                         cudaStream_t stream);
+
+/*
+ * Synchronize the stream, then report and clear the library's device-side status word
+ * (set by a kernel whose bounded wait gave up: NVFP4_ERR_TIMEOUT). Returns NVFP4_ERR_CUDA if
+ * the synchronization itself failed.
+ */
+nvfp4_status nvfp4_sync_status(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

@@ -1,0 +1,182 @@
+"""NVFP4 quantized linear layer for NVIDIA B200 (sm_100a).
+
+The compute runs in libnvfp4.so (hand-written CUDA for sm_100a behind the C ABI of
+include/nvfp4.h). This module marshals torch tensors into those calls: PyTorch supplies
+device memory and the current stream, nothing else.
+
+    q_w = quantize_fp8(w_e4m3, w_scale)       # double quantization of an FP8 checkpoint
+    q_x = quantize(x_bf16)                    # dynamic per-tensor amax
+    y = linear(q_x, q_w)                      # block-scaled W4A4 GEMM, bf16 out
+    pct, mx = calib_percentile_amax(batches)  # static p99.9 input scale
+    q_s = quantize(x_bf16, static_amax=pct)
+
+The C entry points are also available under their own names (``nvfp4_quantize`` ...).
+"""
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_OP_CALIB_BF16, NVFP4_OP_CALIB_F32,
+                   NVFP4_OP_LINEAR, NVFP4_OP_QUANTIZE, NVFP4Error, check, load)
+
+__all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "dequantize", "linear",
+           "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
+
+
+def __getattr__(name):
+    if name.startswith("nvfp4_"):
+        return getattr(_lib, name)
+    raise AttributeError(name)
+
+
+@dataclass
+class NVFP4Tensor:
+    """A quantized [rows x cols] matrix: codes [rows, cols/2] u8, scales in the tensor-core
+    layout (flat u8) and / or linear [rows, cols/16] u8, global scale (1-element fp32)."""
+    codes: torch.Tensor
+    scales_swz: torch.Tensor
+    scales_lin: torch.Tensor
+    global_scale: torch.Tensor
+    rows: int
+    cols: int
+
+
+def _stream(device):
+    return ctypes_ptr(torch.cuda.current_stream(device).cuda_stream)
+
+
+def ctypes_ptr(v):
+    return v if v else None
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+_ws_cache = {}
+
+
+def _workspace(device, nbytes):
+    if nbytes == 0:
+        return None
+    key = (device.index if device.index is not None else torch.cuda.current_device())
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def _alloc_outputs(rows, cols, device, swizzled, linear):
+    L = load()
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+    swz = (torch.empty(L.nvfp4_scales_bytes(rows, cols, 1), dtype=torch.uint8, device=device)
+           if swizzled else None)
+    lin = torch.empty((rows, cols // 16), dtype=torch.uint8, device=device) if linear else None
+    gs = torch.empty(1, dtype=torch.float32, device=device)
+    return codes, swz, lin, gs
+
+
+def quantize(x: torch.Tensor, static_amax: torch.Tensor = None, swizzled=True, linear=False,
+             out: NVFP4Tensor = None) -> NVFP4Tensor:
+    """NVFP4-quantize a 2-D fp32 / bf16 CUDA tensor (row-major, cols % 32 == 0)."""
+    if x.dtype not in (torch.float32, torch.bfloat16) or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("quantize expects a 2-D CUDA fp32 or bf16 tensor")
+    x = x.contiguous()
+    rows, cols = x.shape
+    if out is None:
+        codes, swz, lin, gs = _alloc_outputs(rows, cols, x.device, swizzled, linear)
+        out = NVFP4Tensor(codes, swz, lin, gs, rows, cols)
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols)
+    ws = _workspace(x.device, ws_bytes)
+    dt = NVFP4_F32 if x.dtype == torch.float32 else NVFP4_BF16
+    st = L.nvfp4_quantize(_ptr(x), dt, rows, cols, _ptr(static_amax), _ptr(out.codes),
+                          _ptr(out.scales_swz), _ptr(out.scales_lin), _ptr(out.global_scale),
+                          _ptr(ws), ws_bytes, _stream(x.device))
+    check(st, "nvfp4_quantize")
+    return out
+
+
+def quantize_fp8(x_e4m3: torch.Tensor, fp8_scale: torch.Tensor = None,
+                 static_amax: torch.Tensor = None, swizzled=True, linear=False,
+                 out: NVFP4Tensor = None) -> NVFP4Tensor:
+    """Double quantization: FP8 E4M3 (uint8 bits or float8_e4m3fn) x fp8_scale -> NVFP4."""
+    if x_e4m3.dtype == torch.float8_e4m3fn:
+        x_e4m3 = x_e4m3.view(torch.uint8)
+    if x_e4m3.dtype != torch.uint8 or x_e4m3.dim() != 2 or not x_e4m3.is_cuda:
+        raise TypeError("quantize_fp8 expects a 2-D CUDA uint8 / float8_e4m3fn tensor")
+    x_e4m3 = x_e4m3.contiguous()
+    rows, cols = x_e4m3.shape
+    if out is None:
+        codes, swz, lin, gs = _alloc_outputs(rows, cols, x_e4m3.device, swizzled, linear)
+        out = NVFP4Tensor(codes, swz, lin, gs, rows, cols)
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols)
+    ws = _workspace(x_e4m3.device, ws_bytes)
+    st = L.nvfp4_quantize_fp8_src(_ptr(x_e4m3), _ptr(fp8_scale), rows, cols, _ptr(static_amax),
+                                  _ptr(out.codes), _ptr(out.scales_swz), _ptr(out.scales_lin),
+                                  _ptr(out.global_scale), _ptr(ws), ws_bytes,
+                                  _stream(x_e4m3.device))
+    check(st, "nvfp4_quantize_fp8_src")
+    return out
+
+
+def dequantize(q: NVFP4Tensor, out_dtype=torch.float32) -> torch.Tensor:
+    if q.scales_lin is None:
+        raise ValueError("dequantize needs the linear scales (quantize(..., linear=True))")
+    out = torch.empty((q.rows, q.cols), dtype=out_dtype, device=q.codes.device)
+    dt = NVFP4_F32 if out_dtype == torch.float32 else NVFP4_BF16
+    st = load().nvfp4_dequantize(_ptr(q.codes), _ptr(q.scales_lin), _ptr(q.global_scale),
+                                 q.rows, q.cols, dt, _ptr(out), _stream(q.codes.device))
+    check(st, "nvfp4_dequantize")
+    return out
+
+
+def linear(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
+           out: torch.Tensor = None) -> torch.Tensor:
+    """Y = dequant(a) . dequant(w)^T, [a.rows x w.rows], fp32 accumulation."""
+    if a.cols != w.cols:
+        raise ValueError("K mismatch")
+    M, N, K = a.rows, w.rows, a.cols
+    dev = a.codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(NVFP4_OP_LINEAR, M, N, K)
+    ws = _workspace(dev, ws_bytes)
+    dt = NVFP4_F32 if out.dtype == torch.float32 else NVFP4_BF16
+    st = L.nvfp4_linear(_ptr(a.codes), _ptr(a.scales_swz), _ptr(a.global_scale), _ptr(w.codes),
+                        _ptr(w.scales_swz), _ptr(w.global_scale), M, N, K, dt, _ptr(out),
+                        _ptr(ws), ws_bytes, _stream(dev))
+    check(st, "nvfp4_linear")
+    return out
+
+
+def calib_percentile_amax(batches, num=999, den=1000):
+    """Exact nearest-rank num/den percentile of |x| over all batches, and max |x|.
+    Returns two 1-element fp32 CUDA tensors (usable as static_amax)."""
+    import ctypes
+    batches = [b.contiguous() for b in batches]
+    dtype = batches[0].dtype
+    n = batches[0].numel()
+    if any(b.dtype != dtype or b.numel() != n for b in batches):
+        raise ValueError("all batches must share dtype and size")
+    dev = batches[0].device
+    dt = NVFP4_BF16 if dtype == torch.bfloat16 else NVFP4_F32
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(NVFP4_OP_CALIB_BF16 if dt == NVFP4_BF16
+                                       else NVFP4_OP_CALIB_F32, 0, 0, 0)
+    ws = _workspace(dev, ws_bytes)
+    out = torch.empty(2, dtype=torch.float32, device=dev)
+    ptrs = (ctypes.c_void_p * len(batches))(*[b.data_ptr() for b in batches])
+    st = L.nvfp4_calib_percentile_amax(ptrs, len(batches), n, dt, num, den, out.data_ptr(),
+                                       out.data_ptr() + 4, _ptr(ws), ws_bytes, _stream(dev))
+    check(st, "nvfp4_calib_percentile_amax")
+    return out[0:1], out[1:2]
+
+
+def sync_status(device=None):
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    return load().nvfp4_sync_status(_stream(dev))

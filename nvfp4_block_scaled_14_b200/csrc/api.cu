@@ -1,0 +1,299 @@
+// api.cu -- the C ABI declared in include/nvfp4.h: argument checks (on the host, before any
+// launch), workspace sizing, dispatch to the kernels, status mapping.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "nvfp4_internal.cuh"
+
+namespace nvfp4 {
+
+// Library status word (one per device). Kernels whose bounded waits give up write
+// NVFP4_ERR_TIMEOUT here; nvfp4_sync_status reads and clears it.
+__device__ int g_device_status;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];
+int *g_status_ptr[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+int current_device()
+{
+    int d = 0;
+    cudaGetDevice(&d);
+    return d < 0 ? 0 : (d >= kMaxDevices ? kMaxDevices - 1 : d);
+}
+
+void init_device(int d)
+{
+    std::call_once(g_dev_once[d], [d]() {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d);
+        g_sms[d] = v > 0 ? v : 1;
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) == cudaSuccess)
+            g_status_ptr[d] = reinterpret_cast<int *>(p);
+    });
+}
+} // namespace
+
+int num_sms()
+{
+    const int d = current_device();
+    init_device(d);
+    return g_sms[d];
+}
+
+int *device_status_ptr()
+{
+    const int d = current_device();
+    init_device(d);
+    return g_status_ptr[d];
+}
+
+} // namespace nvfp4
+
+using namespace nvfp4;
+
+namespace {
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nvfp4_status map_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+nvfp4_status check_device()
+{
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, d) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return major == 10 ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED;
+}
+
+nvfp4_status check_matrix(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0 || rows >= kMaxDim || cols >= kMaxDim)
+        return NVFP4_ERR_SHAPE;
+    if (cols % 32 != 0)
+        return NVFP4_ERR_SHAPE;
+    return NVFP4_OK;
+}
+
+size_t quantize_ws_bytes() { return (size_t)kAmaxPartials * sizeof(float); }
+
+nvfp4_status quantize_common(const void *x, int src_type, const float *fp8_scale, int64_t rows,
+                             int64_t cols, const float *static_amax, uint8_t *codes,
+                             uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,
+                             void *ws, size_t ws_bytes, cudaStream_t s)
+{
+    nvfp4_status st = check_matrix(rows, cols);
+    if (st != NVFP4_OK)
+        return st;
+    const bool empty = rows == 0 || cols == 0;
+    if (!global_scale)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!empty && (!x || !codes || (!scales_swz && !scales_lin)))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales_swz) || !aligned16(scales_lin) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u) || !aligned16(ws))
+        return NVFP4_ERR_ALIGNMENT;
+    if (!static_amax && (!ws || ws_bytes < quantize_ws_bytes()))
+        return NVFP4_ERR_WORKSPACE;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    return map_cuda(launch_quantize(x, src_type, fp8_scale, rows, cols, static_amax, codes,
+                                    scales_swz, scales_lin, global_scale,
+                                    reinterpret_cast<float *>(ws), s));
+}
+
+} // namespace
+
+extern "C" {
+
+const char *nvfp4_status_str(nvfp4_status st)
+{
+    switch (st) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_SHAPE: return "invalid shape (sizes >= 0, < 2^31, cols a multiple of 32)";
+    case NVFP4_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case NVFP4_ERR_WORKSPACE: return "workspace too small";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
+    case NVFP4_ERR_UNSUPPORTED: return "device is not sm_100";
+    }
+    return "unknown status";
+}
+
+size_t nvfp4_codes_bytes(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0)
+        return 0;
+    return (size_t)(rows * (cols / 2));
+}
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int swizzled)
+{
+    if (rows < 0 || cols < 0)
+        return 0;
+    const int64_t nb = cols / 16;
+    if (!swizzled)
+        return (size_t)(rows * nb);
+    return (size_t)(((rows + 127) / 128) * 128 * ((nb + 3) / 4) * 4);
+}
+
+size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
+{
+    switch (op) {
+    case NVFP4_OP_QUANTIZE: return quantize_ws_bytes();
+    case NVFP4_OP_LINEAR:
+        if (m <= 0 || n <= 0 || k <= 0)
+            return 0;
+        return plan_linear(m, n, k).ws_bytes;
+    case NVFP4_OP_CALIB_BF16: return calib_workspace_bytes(1);
+    case NVFP4_OP_CALIB_F32: return calib_workspace_bytes(0);
+    }
+    return 0;
+}
+
+nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dt, int64_t rows, int64_t cols,
+                            const float *static_amax, uint8_t *codes, uint8_t *scales_swz,
+                            uint8_t *scales_lin, float *global_scale, void *ws, size_t ws_bytes,
+                            cudaStream_t stream)
+{
+    if (dt != NVFP4_F32 && dt != NVFP4_BF16)
+        return NVFP4_ERR_INVALID_ARG;
+    return quantize_common(x, dt == NVFP4_F32 ? kSrcF32 : kSrcBF16, nullptr, rows, cols,
+                           static_amax, codes, scales_swz, scales_lin, global_scale, ws,
+                           ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_quantize_fp8_src(const uint8_t *x_e4m3, const float *fp8_scale, int64_t rows,
+                                    int64_t cols, const float *static_amax, uint8_t *codes,
+                                    uint8_t *scales_swz, uint8_t *scales_lin,
+                                    float *global_scale, void *ws, size_t ws_bytes,
+                                    cudaStream_t stream)
+{
+    if (reinterpret_cast<uintptr_t>(fp8_scale) & 3u)
+        return NVFP4_ERR_ALIGNMENT;
+    return quantize_common(x_e4m3, kSrcE4M3, fp8_scale, rows, cols, static_amax, codes,
+                           scales_swz, scales_lin, global_scale, ws, ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales_lin,
+                              const float *global_scale, int64_t rows, int64_t cols,
+                              nvfp4_dtype out_dt, void *out, cudaStream_t stream)
+{
+    nvfp4_status st = check_matrix(rows, cols);
+    if (st != NVFP4_OK)
+        return st;
+    if (out_dt != NVFP4_F32 && out_dt != NVFP4_BF16)
+        return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0)
+        return NVFP4_OK;
+    if (!codes || !scales_lin || !global_scale || !out)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(out) || (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+        return NVFP4_ERR_ALIGNMENT;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    return map_cuda(launch_dequantize(codes, scales_lin, global_scale, rows, cols,
+                                      out_dt == NVFP4_BF16, out, stream));
+}
+
+nvfp4_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales_swz, const float *a_gs,
+                          const uint8_t *w_codes, const uint8_t *w_scales_swz, const float *w_gs,
+                          int64_t M, int64_t N, int64_t K, nvfp4_dtype out_dt, void *y, void *ws,
+                          size_t ws_bytes, cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || K % 32 != 0)
+        return NVFP4_ERR_SHAPE;
+    if (out_dt != NVFP4_F32 && out_dt != NVFP4_BF16)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (!y)
+        return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    const size_t esz = out_dt == NVFP4_BF16 ? 2 : 4;
+    if (K == 0)
+        return map_cuda(cudaMemsetAsync(y, 0, (size_t)M * N * esz, stream));
+    if (!a_codes || !a_scales_swz || !a_gs || !w_codes || !w_scales_swz || !w_gs)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_scales_swz) || !aligned16(w_codes) ||
+        !aligned16(w_scales_swz) || !aligned16(y) || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(a_gs) & 3u) || (reinterpret_cast<uintptr_t>(w_gs) & 3u))
+        return NVFP4_ERR_ALIGNMENT;
+    const LinearPlan pl = plan_linear(M, N, K);
+    if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes))
+        return NVFP4_ERR_WORKSPACE;
+    st = NVFP4_OK;
+    cudaError_t e = launch_linear(pl, a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs,
+                                  M, N, K, out_dt == NVFP4_BF16, y, ws, stream, &st);
+    if (st != NVFP4_OK)
+        return st;
+    return map_cuda(e);
+}
+
+nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_batches,
+                                         int64_t elems_per_batch, nvfp4_dtype dt,
+                                         uint32_t pct_num, uint32_t pct_den, float *out_pct,
+                                         float *out_max, void *ws, size_t ws_bytes,
+                                         cudaStream_t stream)
+{
+    if (dt != NVFP4_F32 && dt != NVFP4_BF16)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!batches || num_batches <= 0 || !out_pct || !out_max)
+        return NVFP4_ERR_INVALID_ARG;
+    if (pct_den == 0 || pct_num == 0 || pct_num > pct_den)
+        return NVFP4_ERR_INVALID_ARG;
+    if (elems_per_batch <= 0 || elems_per_batch >= kMaxDim)
+        return NVFP4_ERR_SHAPE;
+    for (int i = 0; i < num_batches; ++i) {
+        if (!batches[i])
+            return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(batches[i]))
+            return NVFP4_ERR_ALIGNMENT;
+    }
+    if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(out_pct) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out_max) & 3u))
+        return NVFP4_ERR_ALIGNMENT;
+    const int bf16 = dt == NVFP4_BF16;
+    if (!ws || ws_bytes < calib_workspace_bytes(bf16))
+        return NVFP4_ERR_WORKSPACE;
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    const unsigned __int128 n = (unsigned __int128)num_batches * (uint64_t)elems_per_batch;
+    unsigned __int128 rank = (n * pct_num + pct_den - 1) / pct_den;
+    if (rank < 1)
+        rank = 1;
+    return map_cuda(launch_calib(batches, num_batches, elems_per_batch, bf16, (uint64_t)rank,
+                                 out_pct, out_max, ws, stream));
+}
+
+nvfp4_status nvfp4_sync_status(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    int *p = device_status_ptr();
+    if (!p)
+        return NVFP4_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    }
+    return (nvfp4_status)v;
+}
+
+} // extern "C"

@@ -1,0 +1,69 @@
+// nvfp4_internal.cuh -- declarations shared by the library's translation units.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "nvfp4.h"
+
+namespace nvfp4 {
+
+// Source element types of the quantizer.
+enum SrcType : int { kSrcF32 = 0, kSrcBF16 = 1, kSrcE4M3 = 2 };
+
+// Byte offset of the scale of (row, block) in the tensor-core scale layout: atoms of
+// 128 rows x 4 blocks (512 B), atoms of a 128-row band consecutive along the blocks.
+__host__ __device__ __forceinline__ int64_t swz_offset(int64_t row, int64_t blk,
+                                                       int64_t atoms_per_band)
+{
+    return ((row >> 7) * atoms_per_band + (blk >> 2)) * 512 + ((row & 31) << 4) +
+           (((row >> 5) & 3) << 2) + (blk & 3);
+}
+
+// Device-side status word of the current device (bounded waits that give up write
+// NVFP4_ERR_TIMEOUT here). Resolved once per device.
+int *device_status_ptr();
+
+int num_sms();
+
+// ---- quantize.cu --------------------------------------------------------------------
+// Number of partial maxima the amax pass writes (the workspace holds that many floats).
+constexpr int kAmaxPartials = 1184; // 8 per SM on a 148-SM part
+
+cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale, int64_t rows,
+                            int64_t cols, const float *static_amax, uint8_t *codes,
+                            uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,
+                            float *ws_partials, cudaStream_t s);
+
+// ---- dequantize.cu ------------------------------------------------------------------
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales_lin,
+                              const float *global_scale, int64_t rows, int64_t cols,
+                              int out_bf16, void *out, cudaStream_t s);
+
+// ---- calib.cu -----------------------------------------------------------------------
+size_t calib_workspace_bytes(int is_bf16);
+cudaError_t launch_calib(const void *const *batches, int num_batches, int64_t elems_per_batch,
+                         int is_bf16, uint64_t rank, float *out_pct, float *out_max, void *ws,
+                         cudaStream_t s);
+
+// ---- gemm_sm100.cu ------------------------------------------------------------------
+struct LinearPlan {
+    bool swap_ab;       // operand "A" of the MMA is W (rows N), "B" is the activations
+    int bn;             // MMA N (tile width on the B side)
+    int64_t rows_a;     // rows of the MMA A operand
+    int64_t rows_b;     // rows of the MMA B operand
+    int64_t tiles_a;    // ceil(rows_a / 128)
+    int64_t tiles_b;    // ceil(rows_b / bn)
+    int kt;             // k-tiles of 256 elements
+    int splits;         // split-K factor (1 = no split)
+    int kt_per_split;
+    size_t ws_bytes;    // workspace for split-K partials
+};
+LinearPlan plan_linear(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_linear(const LinearPlan &p, const uint8_t *a_codes, const uint8_t *a_sf,
+                          const float *a_gs, const uint8_t *w_codes, const uint8_t *w_sf,
+                          const float *w_gs, int64_t M, int64_t N, int64_t K, int out_bf16,
+                          void *y, void *ws, cudaStream_t s, nvfp4_status *st);
+
+} // namespace nvfp4

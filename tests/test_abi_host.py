@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and loads, exports every
+function include/nvfp4.h declares, sizes the buffers correctly, and rejects bad arguments on
+the host before touching the device."""
+import ctypes
+
+import pytest
+
+from nvfp4_block_scaled_14_b200 import _lib as L
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return L.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = L.declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L._SIGNATURES)
+
+
+def test_status_strings(lib):
+    for st in range(8):
+        assert lib.nvfp4_status_str(st)
+    assert lib.nvfp4_status_str(99) == b"unknown status"
+
+
+def test_buffer_sizes(lib):
+    assert lib.nvfp4_codes_bytes(4096, 3072) == 4096 * 1536
+    assert lib.nvfp4_scales_bytes(4096, 3072, 0) == 4096 * 192
+    assert lib.nvfp4_scales_bytes(4096, 3072, 1) == 4096 * 192
+    # padding to 128-row x 4-block atoms
+    assert lib.nvfp4_scales_bytes(1, 32, 1) == 512
+    assert lib.nvfp4_scales_bytes(129, 96, 1) == 2 * 128 * 8
+    # 4.5 bits per weight (codes + linear scales)
+    assert (lib.nvfp4_codes_bytes(64, 256) + lib.nvfp4_scales_bytes(64, 256, 0)) * 8 == \
+        64 * 256 * 4.5
+    assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_QUANTIZE, 10, 0, 64) >= 4
+    assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_CALIB_BF16, 0, 0, 0) > 0
+    assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_CALIB_F32, 0, 0, 0) > \
+        lib.nvfp4_workspace_bytes(L.NVFP4_OP_CALIB_BF16, 0, 0, 0)
+    assert lib.nvfp4_workspace_bytes(99, 1, 1, 1) == 0
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails its host-side check first
+
+
+def test_quantize_argument_checks(lib):
+    q = lib.nvfp4_quantize
+    ws = lib.nvfp4_workspace_bytes(L.NVFP4_OP_QUANTIZE, 8, 0, 64)
+    # cols not a multiple of 32, negative rows
+    assert q(FAKE, 1, 8, 48, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == L.NVFP4_ERR_SHAPE
+    assert q(FAKE, 1, -1, 64, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == L.NVFP4_ERR_SHAPE
+    assert q(FAKE, 1, 8, 1 << 31, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == \
+        L.NVFP4_ERR_SHAPE
+    # bad dtype, missing outputs
+    assert q(FAKE, 7, 8, 64, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    assert q(FAKE, 1, 8, 64, None, FAKE, None, None, FAKE, FAKE, ws, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    assert q(FAKE, 1, 8, 64, None, FAKE, FAKE, None, None, FAKE, ws, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    assert q(None, 1, 8, 64, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    # misaligned input / codes
+    assert q(FAKE + 8, 1, 8, 64, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == \
+        L.NVFP4_ERR_ALIGNMENT
+    assert q(FAKE, 1, 8, 64, None, FAKE + 4, FAKE, None, FAKE, FAKE, ws, None) == \
+        L.NVFP4_ERR_ALIGNMENT
+    # dynamic amax needs the workspace
+    assert q(FAKE, 1, 8, 64, None, FAKE, FAKE, None, FAKE, None, 0, None) == \
+        L.NVFP4_ERR_WORKSPACE
+    assert q(FAKE, 1, 8, 64, None, FAKE, FAKE, None, FAKE, FAKE, ws - 4, None) == \
+        L.NVFP4_ERR_WORKSPACE
+
+
+def test_fp8_and_dequant_checks(lib):
+    f = lib.nvfp4_quantize_fp8_src
+    assert f(FAKE, FAKE + 2, 8, 64, None, FAKE, FAKE, None, FAKE, FAKE, 1 << 20, None) == \
+        L.NVFP4_ERR_ALIGNMENT
+    assert f(FAKE, None, 8, 40, None, FAKE, FAKE, None, FAKE, FAKE, 1 << 20, None) == \
+        L.NVFP4_ERR_SHAPE
+    d = lib.nvfp4_dequantize
+    assert d(FAKE, FAKE, FAKE, 8, 48, 0, FAKE, None) == L.NVFP4_ERR_SHAPE
+    assert d(FAKE, FAKE, FAKE, 8, 64, 5, FAKE, None) == L.NVFP4_ERR_INVALID_ARG
+    assert d(None, FAKE, FAKE, 8, 64, 0, FAKE, None) == L.NVFP4_ERR_INVALID_ARG
+    assert d(FAKE, FAKE, FAKE, 8, 64, 0, FAKE + 8, None) == L.NVFP4_ERR_ALIGNMENT
+    # empty input is a no-op
+    assert d(None, None, None, 0, 64, 0, None, None) == L.NVFP4_OK
+
+
+def test_linear_and_calib_checks(lib):
+    li = lib.nvfp4_linear
+    args = [FAKE] * 6
+    assert li(*args, 64, 64, 48, 1, FAKE, None, 0, None) == L.NVFP4_ERR_SHAPE
+    assert li(*args, -1, 64, 64, 1, FAKE, None, 0, None) == L.NVFP4_ERR_SHAPE
+    assert li(*args, 64, 64, 64, 3, FAKE, None, 0, None) == L.NVFP4_ERR_INVALID_ARG
+    assert li(*args, 0, 64, 64, 1, None, None, 0, None) == L.NVFP4_OK  # empty output
+    assert li(*args, 64, 64, 64, 1, None, None, 0, None) == L.NVFP4_ERR_INVALID_ARG
+    c = lib.nvfp4_calib_percentile_amax
+    one = (ctypes.c_void_p * 1)(FAKE)
+    assert c(one, 1, 1024, 1, 1001, 1000, FAKE, FAKE, FAKE, 1 << 20, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    assert c(one, 1, 1024, 1, 0, 1000, FAKE, FAKE, FAKE, 1 << 20, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    assert c(one, 0, 1024, 1, 999, 1000, FAKE, FAKE, FAKE, 1 << 20, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    assert c(one, 1, 0, 1, 999, 1000, FAKE, FAKE, FAKE, 1 << 20, None) == L.NVFP4_ERR_SHAPE
+    mis = (ctypes.c_void_p * 1)(FAKE + 2)
+    assert c(mis, 1, 1024, 1, 999, 1000, FAKE, FAKE, FAKE, 1 << 20, None) == \
+        L.NVFP4_ERR_ALIGNMENT
+    assert c(one, 1, 1024, 1, 999, 1000, FAKE, FAKE, FAKE, 16, None) == L.NVFP4_ERR_WORKSPACE
+
+
+def test_product_path_never_imports_oracle():
+    import os
+    import re
+    pkg = os.path.dirname(L.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
+                assert "nvfp4_oracle" not in text, f

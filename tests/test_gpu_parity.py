@@ -1,0 +1,259 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded
+inputs. Codes, E4M3 scales (both layouts), global scales and percentiles are compared bit for
+bit; GEMM outputs within 1e-3 * max|Y_ref| (plus one bf16 unit for bf16 outputs)."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_14_b200 as nv
+import oracle as O
+from gpu_helpers import (assert_quant_equal, dev_tensor, gemm_tolerance, gpu_quantize, host,
+                         scalar_dev, to_numpy_f64)
+from nvfp4_block_scaled_14_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    nv.load()
+
+
+# ---------------------------------------------------------------------------------------
+# quantize
+# ---------------------------------------------------------------------------------------
+
+def test_quantize_tiny_workload():
+    t = W.tiny()
+    for x in (t.W, t.X):
+        assert_quant_equal(gpu_quantize(x), O.quantize(x))
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (7, 96), (127, 160), (129, 64), (300, 1056),
+                                       (64, 32), (256, 4096)])
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+def test_quantize_ragged_shapes(rows, cols, kind):
+    x = W.normal((rows, cols), 1.0, 20, rows * 7 + cols)
+    x[rows // 2, cols // 3] = 17.0  # an outlier channel value
+    if kind == "bf16":
+        x = W.to_bf16_bits(x)
+    assert_quant_equal(gpu_quantize(x), O.quantize(x))
+
+
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+def test_quantize_static_amax_saturates(kind):
+    x = W.normal((200, 288), 1.0, 21, 1)
+    if kind == "bf16":
+        x = W.to_bf16_bits(x)
+    for amax in (0.5, 2.0, 3.3, 1e3):
+        assert_quant_equal(gpu_quantize(x, amax=amax), O.quantize(x, amax=amax))
+
+
+def test_quantize_fp8_source_double_quant():
+    w8, s8 = W.to_fp8_tensorwise(W.normal((320, 384), 0.02, 22, 1))
+    assert_quant_equal(gpu_quantize(w8, fp8_scale=s8), O.quantize(w8, fp8_scale=s8))
+    # a layer without weight_scale: scale read as 1.0
+    assert_quant_equal(gpu_quantize(w8), O.quantize(w8))
+    # static amax on the upcast values
+    assert_quant_equal(gpu_quantize(w8, amax=0.03, fp8_scale=s8),
+                       O.quantize(w8, amax=0.03, fp8_scale=s8))
+
+
+def test_quantize_degenerate_inputs():
+    z = np.zeros((130, 64), np.float32)
+    q = gpu_quantize(z)
+    codes, swz, lin, sg = host(q)
+    assert sg == 0.0 and not codes.any() and not swz.any() and not lin.any()
+    # empty tensor: global scale 0
+    e = nv.quantize(torch.zeros((0, 64), device="cuda"), linear=True)
+    torch.cuda.synchronize()
+    assert float(e.global_scale.cpu()[0]) == 0.0
+    # zero blocks inside a nonzero tensor, subnormal block scales
+    x = np.zeros((3, 64), np.float32)
+    x[0, 0] = 2688.0
+    x[1, 16:32] = 6 * 2.0 ** -9
+    x[2, 5] = -1e-3
+    assert_quant_equal(gpu_quantize(x), O.quantize(x))
+
+
+def _probe_values(grid, n_random, lo, hi, seed):
+    g = np.float32(grid)
+    mids = (g[:-1] + g[1:]) / 2
+    base = np.concatenate([g, mids]).astype(np.float32)
+    pts = [base]
+    cur_up, cur_dn = base.copy(), base.copy()
+    for _ in range(4):  # four ulps either side of every grid point and midpoint
+        cur_up = np.nextafter(cur_up, np.float32(np.inf))
+        cur_dn = np.nextafter(cur_dn, np.float32(0))
+        pts += [cur_up, cur_dn]
+    r = np.random.Generator(np.random.PCG64(seed))
+    pts.append(r.uniform(lo, hi, n_random).astype(np.float32))
+    v = np.concatenate(pts)
+    return v[(v >= lo) & (v <= hi)]
+
+
+def test_e2m1_rounding_of_the_hardware_matches_oracle():
+    # static amax 2688 -> sg = 1; each block holds one 6.0, so its scale is 1.0 and every
+    # other value is encoded as itself: the codes show the E2M1 rounding directly.
+    vals = _probe_values([0, 0.5, 1, 1.5, 2, 3, 4, 6], 20000, 0.0, 6.0, 30)
+    tiny = np.float32([1e-30, 1e-10, 2.0 ** -126, 2.0 ** -149, 0.0])
+    vals = np.concatenate([vals, -vals, tiny, -tiny]).astype(np.float32)
+    per = 15
+    nblk = -(-vals.size // per)
+    buf = np.zeros(nblk * per, np.float32)
+    buf[:vals.size] = vals
+    blocks = np.concatenate([np.full((nblk, 1), 6.0, np.float32), buf.reshape(nblk, per)], 1)
+    rows = -(-nblk // 2)
+    x = np.zeros((rows * 2, 16), np.float32)
+    x[:nblk] = blocks
+    x = x.reshape(rows, 32)
+    assert_quant_equal(gpu_quantize(x, amax=2688.0), O.quantize(x, amax=2688.0))
+
+
+def test_e4m3_rounding_of_the_hardware_matches_oracle():
+    # static amax 448 -> sg * 6 == 1.0 in fp32, so each block's scale is E4M3(block max).
+    e4m3 = np.array([O.e4m3_decode(c) for c in range(127)], np.float32)
+    vals = _probe_values(e4m3, 20000, 2.0 ** -12, 448.0, 31)
+    vals = np.concatenate([vals, np.float32([500.0, 1e4])])
+    rows = -(-vals.size // 2)
+    x = np.zeros((rows, 32), np.float32)
+    flat = np.zeros(rows * 2, np.float32)
+    flat[:vals.size] = vals
+    x[:, 0] = flat[0::2]
+    x[:, 16] = flat[1::2]
+    x[:, 1] = flat[0::2] * np.float32(0.37)
+    ref = O.quantize(x, amax=448.0)
+    sg = np.float32(448.0) / np.float32(2688.0)
+    assert np.float32(sg) * np.float32(6.0) == np.float32(1.0)
+    assert_quant_equal(gpu_quantize(x, amax=448.0), ref)
+
+
+# ---------------------------------------------------------------------------------------
+# dequantize
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols", [(64, 256), (33, 96), (1, 32)])
+def test_dequantize_bit_exact(rows, cols):
+    x = W.normal((rows, cols), 0.02, 23, rows)
+    ref = O.quantize(x)
+    q = gpu_quantize(x)
+    f = nv.dequantize(q, torch.float32).cpu().numpy()
+    b = nv.dequantize(q, torch.bfloat16).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(f.view(np.uint32), O.dequantize(ref, "f32").view(np.uint32))
+    assert np.array_equal(b, O.dequantize(ref, "bf16"))
+
+
+# ---------------------------------------------------------------------------------------
+# GEMM
+# ---------------------------------------------------------------------------------------
+
+def _run_linear(xa, xw, out_dtype, amax_a=None):
+    qa, qw = gpu_quantize(xa, amax=amax_a), gpu_quantize(xw)
+    y = nv.linear(qa, qw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    ra, rw = O.quantize(xa, amax=amax_a), O.quantize(xw)
+    assert_quant_equal(qa, ra)
+    assert_quant_equal(qw, rw)
+    return to_numpy_f64(y), ra, rw
+
+
+def test_linear_tiny_workload_fp32_out():
+    t = W.tiny()
+    y, ra, rw = _run_linear(t.X, t.W, torch.float32)
+    ref = O.gemm(ra, rw)
+    assert np.all(np.abs(y - ref) <= gemm_tolerance(ref, False))
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (300, 520, 1056),   # >128 rows: BN=256 tiles, ragged M, N and K, split-K
+    (129, 256, 256),
+    (256, 264, 512),
+    (1, 384, 512), (5, 384, 512), (8, 384, 512), (16, 200, 320), (17, 256, 256),
+    (33, 384, 512), (100, 384, 512), (128, 384, 512),   # small M: swap-AB
+    (64, 1024, 2048),   # swap-AB, many k-tiles per split
+])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_linear_matches_oracle(M, N, K, out):
+    xa = W.to_bf16_bits(W.normal((M, K), 1.0, 24, M))
+    xw = W.to_bf16_bits(W.normal((N, K), 0.02, 25, N))
+    odt = torch.bfloat16 if out == "bf16" else torch.float32
+    y, ra, rw = _run_linear(xa, xw, odt)
+    ref = O.gemm(ra, rw)
+    err = np.abs(y - ref)
+    tol = gemm_tolerance(ref, out == "bf16")
+    assert np.all(err <= tol), f"max err {err.max()} vs tol {np.max(tol)}"
+
+
+def test_linear_exact_with_unit_scales():
+    # all block scales 1.0 and both global scales 1: 2 * each value is an integer in
+    # [-12, 12], the sums are exact in fp32, so the fp32 output must equal the exact product.
+    g = np.random.Generator(np.random.PCG64(26))
+    for M, N, K in [(64, 256, 512), (200, 300, 1024), (8, 512, 2048)]:
+        ac = g.integers(0, 256, (M, K // 2), dtype=np.uint8)
+        wc = g.integers(0, 256, (N, K // 2), dtype=np.uint8)
+
+        def swz_ones(rows):
+            s = np.zeros(O.swizzled_bytes(rows, K), np.uint8)
+            for r in range(rows):
+                for b in range(K // 16):
+                    s[O.swizzled_offset(r, b, K // 16)] = 0x38
+            return s
+
+        ta = nv.NVFP4Tensor(torch.from_numpy(ac).cuda(), torch.from_numpy(swz_ones(M)).cuda(),
+                            None, scalar_dev(1.0), M, K)
+        tw = nv.NVFP4Tensor(torch.from_numpy(wc).cuda(), torch.from_numpy(swz_ones(N)).cuda(),
+                            None, scalar_dev(1.0), N, K)
+        y = nv.linear(ta, tw, out_dtype=torch.float32)
+        ra = O.Quantized(ac, np.full((M, K // 16), 0x38, np.uint8), None, 1.0, M, K)
+        rw = O.Quantized(wc, np.full((N, K // 16), 0x38, np.uint8), None, 1.0, N, K)
+        assert np.array_equal(to_numpy_f64(y), O.gemm(ra, rw)), (M, N, K)
+
+
+def test_linear_large_tile_path_sampled():
+    # enough 128x256 tiles that no K split is used
+    M, N, K = 1280, 2048, 512
+    xa = W.to_bf16_bits(W.normal((M, K), 1.0, 27, 1))
+    xw = W.to_bf16_bits(W.normal((N, K), 0.02, 27, 2))
+    y, ra, rw = _run_linear(xa, xw, torch.bfloat16)
+    r = np.random.Generator(np.random.PCG64(28))
+    ms = np.concatenate([r.integers(0, M, 3000), [0, M - 1, 127, 128, 255, 256]])
+    ns = np.concatenate([r.integers(0, N, 3000), [N - 1, 0, 255, 256, 511, 512]])
+    ref = O.gemm_sampled(ra, rw, ms, ns)
+    full_max = np.abs(y).max()
+    tol = 1e-3 * full_max + np.abs(ref) * 2.0 ** -8
+    assert np.all(np.abs(y[ms, ns] - ref) <= tol)
+
+
+# ---------------------------------------------------------------------------------------
+# calibration percentile
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+def test_calib_percentile_matches_oracle(kind):
+    batches = []
+    for b in range(5):
+        x = W.normal((64, 96 + 32), 1.0, 29, b)
+        x.reshape(-1)[::97] *= np.float32(7.0)
+        batches.append(W.to_bf16_bits(x) if kind == "bf16" else x)
+    f32 = [W.bf16_bits_to_f32(b) if kind == "bf16" else b for b in batches]
+    dev = [dev_tensor(b) for b in batches]
+    for num, den in [(999, 1000), (1, 2), (1, 1), (1, 1000000)]:
+        p, m = nv.calib_percentile_amax(dev, num, den)
+        torch.cuda.synchronize()
+        rp, rm = O.percentile_abs(f32, num, den)
+        assert float(p.cpu()[0]) == rp and float(m.cpu()[0]) == rm, (num, den)
+
+
+def test_calib_ragged_element_count():
+    x = W.normal((1, 1000 + 3), 2.0, 29, 9).ravel()[:1003].copy()
+    xs = [x[:1001].copy(), x[1:1002].copy()]
+    dev = [torch.from_numpy(a).cuda() for a in xs]
+    p, m = nv.calib_percentile_amax(dev)
+    torch.cuda.synchronize()
+    assert (float(p.cpu()[0]), float(m.cpu()[0])) == O.percentile_abs(xs)
+
+
+def test_sync_status_clean():
+    assert nv.sync_status() == 0

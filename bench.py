@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 quantized linear layer on B200.
+
+One step = the whole hot path on the double-quant diffusion attention projection
+(W 3072x3072 stored as FP8 E4M3 with a per-tensor scale, X 4096x3072 bf16 with 0.1 %
+outlier channels): NVFP4-quantize W from FP8 (double quantization), quantize X with its
+dynamic per-tensor amax, and run the block-scaled W4A4 GEMM to a bf16 Y.
+
+The headline `value` is the linear layer's throughput in TFLOP/s (2*M*N*K per step over the
+whole step, quantization included), summed over ranks. Each rank runs its own independent
+batch (weak scaling, no collective on the data path). Inputs rotate over enough buffer sets
+that every step reads them cold from HBM (more than 3x the L2 size in flight). Steps are
+replayed from CUDA graphs; per-kernel durations come from CUDA events captured inside those
+graphs, on the launching stream.
+
+The other rows of the hot path (MLP-pair GEMMs, small-M decode GEMV, p99.9 calibration,
+dequantize) are measured after the timed region and reported under "rows".
+
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, N, K = 4096, 3072, 3072
+FLOPS = 2.0 * M * N * K
+METRIC = "NVFP4 GEMM TFLOPS & quantize GB/s at 1 B200 (fraction of FP4/HBM peak)"
+WORKLOAD = "attn_proj_fp8w_m4096_n3072_k3072"
+FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        self.gpu = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self, t_lo, t_hi):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        self.out.flush()
+        rows = []
+        for line in open(self.out.name):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(f[1]), float(f[2]), f[3], f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        inside = [r for r in rows if t_lo - 1.0 <= r[0] <= t_hi + 1.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[4])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+
+class Step:
+    """Preallocated buffers of one step over several input sets."""
+
+    def __init__(self, nv, wl, n_sets, dev):
+        self.nv = nv
+        w8 = torch.from_numpy(wl.W_e4m3).to(dev)
+        xb = torch.from_numpy(wl.X_bf16.view(np.int16)).to(dev).view(torch.bfloat16)
+        s8 = torch.tensor([wl.w_scale], dtype=torch.float32, device=dev)
+        self.W = [w8.clone() for _ in range(n_sets)]
+        self.X = [xb.clone() for _ in range(n_sets)]
+        self.s8 = s8
+        self.qw = nv.quantize_fp8(self.W[0], s8)
+        self.qx = nv.quantize(self.X[0])
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def run(self, i, ev=None):
+        nv = self.nv
+        if ev is not None:
+            ev[0].record()
+        nv.quantize_fp8(self.W[i], self.s8, out=self.qw)
+        if ev is not None:
+            ev[1].record()
+        nv.quantize(self.X[i], out=self.qx)
+        if ev is not None:
+            ev[2].record()
+        nv.linear(self.qx, self.qw, out=self.Y)
+        if ev is not None:
+            ev[3].record()
+
+
+def launches_per_step(nv):
+    L = nv.load()
+    ws = L.nvfp4_workspace_bytes(nv.NVFP4_OP_LINEAR, M, N, K)
+    return 2 + 2 + (2 if ws > 0 else 1)
+
+
+def time_graph_replays(graphs, n_total, stream):
+    """Replay graphs round-robin for n_total steps; return elapsed ms (device events)."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(n_total):
+        graphs[i % len(graphs)].replay()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def op_timer(fns, reps_per_fn=3):
+    """Average device time of one call of each closure in fns (rotating buffer sets),
+    captured in one CUDA graph with external events around every call."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for f in fns:
+            f()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in fns]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for (a, b), f in zip(evs, fns):
+            a.record()
+            f()
+            b.record()
+    times = []
+    for _ in range(reps_per_fn):
+        g.replay()
+        torch.cuda.synchronize()
+        times += [a.elapsed_time(b) for a, b in evs]
+    del g
+    return statistics.mean(times), statistics.median(times)
+
+
+def extras(nv, W, dev, hbm, fp4_peak):
+    """The other hot-path rows: MLP-pair GEMMs, small-M decode, calibration, dequantize."""
+    rows = {}
+    L2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def sets_for(nbytes):
+        return max(2, math.ceil(3 * L2 / max(nbytes, 1)))
+
+    # --- MLP pair (4096x3072 -> 12288 -> 3072), weights pre-quantized
+    mp = W.mlp_pair()
+    t = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    W1, W2, X1, X2 = t(mp.W1), t(mp.W2), t(mp.X1), t(mp.X2)
+    q1, q2 = nv.quantize(W1), nv.quantize(W2)
+    n_x2 = sets_for(X2.numel() * 2)
+    X2s = [X2.clone() for _ in range(n_x2)]
+    qx2 = nv.quantize(X2)
+    qx1 = nv.quantize(X1)
+    Y1 = torch.empty((4096, 12288), dtype=torch.bfloat16, device=dev)
+    Y2 = torch.empty((4096, 3072), dtype=torch.bfloat16, device=dev)
+    avg, med = op_timer([lambda x=x: nv.quantize(x, out=qx2) for x in X2s])
+    elems = X2.numel()
+    gbs = (elems * 2 + elems / 2 + elems / 16 + 4) / (avg * 1e-3) / 1e9
+    rows["quantize_x2_bf16_4096x12288"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    for name, a, w, y, kk, nn in [("gemm1_m4096_n12288_k3072", qx1, q1, Y1, 3072, 12288),
+                                  ("gemm2_m4096_n3072_k12288", qx2, q2, Y2, 12288, 3072)]:
+        avg, med = op_timer([lambda a=a, w=w, y=y: nv.linear(a, w, out=y)] * 6)
+        tf = 2.0 * 4096 * nn * kk / (avg * 1e-3) / 1e12
+        rows[name] = {"us": avg * 1e3, "TFLOP/s": tf, "frac_fp4": tf / fp4_peak}
+    del X2s, W1, W2, X1, X2, Y1, Y2, q1, q2, qx1, qx2
+    torch.cuda.empty_cache()
+
+    # --- small-M decode: W 12288x4096 packed, M in {1, 8, 32, 128}
+    dc = W.decode()
+    Wd = t(dc.W)
+    wbytes = 12288 * 4096 // 2 + 12288 * 4096 // 16
+    n_w = sets_for(wbytes)
+    qws = [nv.quantize(Wd) for _ in range(n_w)]
+    small = {}
+    for m, xa in dc.X.items():
+        qa = nv.quantize(t(xa))
+        y = torch.empty((m, 12288), dtype=torch.bfloat16, device=dev)
+        avg, med = op_timer([lambda q=q: nv.linear(qa, q, out=y) for q in qws])
+        gbs = wbytes / (avg * 1e-3) / 1e9
+        small[f"M{m}"] = {"us": avg * 1e3, "GB/s_weights": gbs, "frac_hbm": gbs / hbm,
+                          "TFLOP/s": 2.0 * m * 12288 * 4096 / (avg * 1e-3) / 1e12}
+    rows["small_m_n12288_k4096"] = small
+    del qws, Wd
+    torch.cuda.empty_cache()
+
+    # --- p99.9 calibration over 53 batches of 4096x3072 bf16 (8 distinct seeded batches,
+    #     each read several times; 8 x 25 MB exceeds L2, so every read comes from HBM)
+    distinct = [t(W.calib_batch(b)) for b in range(8)]
+    batches = [distinct[b % 8] for b in range(53)]
+    avg, med = op_timer([lambda: nv.calib_percentile_amax(batches)], reps_per_fn=5)
+    nbytes = 53 * 4096 * 3072 * 2
+    gbs = nbytes / (avg * 1e-3) / 1e9
+    rows["calib_p999_53x4096x3072_bf16"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    del distinct, batches
+
+    # --- dequantize 12288x3072 to bf16
+    wq = nv.quantize(t(W.mlp_pair(M=8).W1), linear=True)
+    avg, med = op_timer([lambda: nv.dequantize(wq, torch.bfloat16)] * 4)
+    elems = 12288 * 3072
+    gbs = (elems / 2 + elems / 16 + elems * 2) / (avg * 1e-3) / 1e9
+    rows["dequantize_12288x3072_bf16"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    return rows
+
+
+def cpu_baseline(seconds=10.0):
+    """The oracle, as it stands, on a bounded sample of the step: quantize W rows 0..511
+    (FP8 source, with the full-tensor amax), X rows 0..63 (full-tensor amax), and the
+    64 x 512 outputs of Y in fp64. Repeated for about `seconds`; TFLOP/s of the GEMM part
+    over the whole sample time."""
+    import oracle as O
+    from nvfp4_block_scaled_14_b200 import workloads as W
+    wl = W.attn_proj()
+    ms, ns = 64, 512
+    x_all = wl.X_bf16
+    w8 = wl.W_e4m3
+    reps, t0 = 0, time.time()
+    while True:
+        w_f32 = O.source_to_f32(w8, wl.w_scale)
+        amax_w = float(np.abs(w_f32).max())
+        amax_x = float(np.abs(W.bf16_bits_to_f32(x_all)).max())
+        qw = O.quantize(w8[:ns], amax=amax_w, fp8_scale=wl.w_scale)
+        qx = O.quantize(x_all[:ms], amax=amax_x)
+        O.gemm(qx, qw)
+        reps += 1
+        if time.time() - t0 >= seconds:
+            break
+    dt = (time.time() - t0) / reps
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": 2.0 * ms * ns * K / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"quantize W[0:{ns}] (fp8 source) and X[0:{ms}] with full-tensor amax, "
+                      f"Y[0:{ms},0:{ns}] in fp64; {reps} repetitions, {dt:.3f} s each"}
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    import nvfp4_block_scaled_14_b200 as nv
+    from nvfp4_block_scaled_14_b200 import workloads as W
+    nv.load()
+    hbm, bf16, peak_kind = peaks()
+    fp4_peak = bf16 * FP4_PER_BF16
+
+    wl = W.attn_proj(x_tensor=2 + 100 * rank)
+    L2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    set_bytes = wl.W_e4m3.nbytes + wl.X_bf16.nbytes
+    n_sets = max(3, math.ceil(3 * L2 / set_bytes))
+    st = Step(nv, wl, n_sets, dev)
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        st.run(i % n_sets)
+    torch.cuda.synchronize()
+
+    # one graph per input set, with external events between the three ops
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+           for _ in range(n_sets)]
+    graphs = []
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        st.run(0)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    for i in range(n_sets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            st.run(i, evs[i])
+        graphs.append(g)
+    for i in range(max(args.warmup, n_sets)):
+        graphs[i % n_sets].replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_lo = time.time()
+    ms = time_graph_replays(graphs, args.steps, stream)
+    t_hi = time.time()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop(t_lo, t_hi)
+
+    # per-op device durations from the events of the last replay of every graph
+    qw_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    qx_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    gemm_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # e2e: host inputs in pinned memory, copies inside the timed region
+    e2e_steps = max(3, min(args.steps, 50))
+    w_host = torch.from_numpy(wl.W_e4m3).pin_memory()
+    x_host = torch.from_numpy(wl.X_bf16.view(np.int16)).pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    for _ in range(2):
+        st.W[0].copy_(w_host, non_blocking=True)
+        st.X[0].view(torch.int16).copy_(x_host, non_blocking=True)
+        st.run(0)
+        y_host.copy_(st.Y.view(torch.int16), non_blocking=True)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(e2e_steps):
+        st.W[0].copy_(w_host, non_blocking=True)
+        st.X[0].view(torch.int16).copy_(x_host, non_blocking=True)
+        st.run(0)
+        y_host.copy_(st.Y.view(torch.int16), non_blocking=True)
+    b.record()
+    b.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+
+    rows = None
+    if not args.no_extras and rank == 0:
+        del graphs
+        rows = extras(nv, W, dev, hbm, fp4_peak)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms_step = ms_max / args.steps
+    value = world * FLOPS / (ms_step * 1e-3) / 1e12
+    gemm_tf = FLOPS / (gemm_ms * 1e-3) / 1e12
+    qx_bytes = M * K * (2 + 0.5 + 1 / 16) + 4
+    qw_bytes = N * K * (1 + 0.5 + 1 / 16) + 4
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if os.path.exists(tp):
+        traffic = json.load(open(tp)).get("nvfp4_gemm_kernel", {}).get(WORKLOAD)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4-e2m1",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K,
+                   "weights": "fp8 e4m3 tensorwise -> nvfp4 each step", "activations":
+                   "bf16, dynamic per-tensor amax", "out": "bf16",
+                   "l2": f"inputs rotate over {n_sets} buffer sets "
+                         f"({n_sets * set_bytes / 1e6:.0f} MB > 3x L2)",
+                   "parallelism": f"{world} independent ranks"},
+        "gemm_tflops": gemm_tf,
+        "quantize_gbs": {"x_bf16": qx_bytes / (qx_ms * 1e-3) / 1e9,
+                         "w_fp8": qw_bytes / (qw_ms * 1e-3) / 1e9},
+        "op_us": {"quantize_w_fp8": qw_ms * 1e3, "quantize_x_bf16": qx_ms * 1e3,
+                  "gemm": gemm_ms * 1e3},
+        "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel<256>",
+                     "achieved": gemm_tf, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tf / fp4_peak, "traffic": traffic,
+                     "peak_note": f"{peak_kind} bf16 burst {bf16} TFLOP/s x {FP4_PER_BF16} "
+                                  "(nominal FP4/BF16 ratio)"},
+        "e2e": {"value": FLOPS / (e2e_ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(wl.W_e4m3.nbytes + wl.X_bf16.nbytes),
+                "d2h_bytes_per_step": int(M * N * 2)},
+        "gpu_launches": launches_per_step(nv) * args.steps,
+        "clocks": clk,
+    }
+    if rows is not None:
+        line["rows"] = rows
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+def run_reference(args):
+    """The CPU oracle as it stands on a bounded sample of the same workload per step."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle as O
+    from nvfp4_block_scaled_14_b200 import workloads as W
+    wl = W.attn_proj()
+    ms, ns = 16, 256
+    amax_x = float(np.abs(W.bf16_bits_to_f32(wl.X_bf16)).max())
+
+    def step():
+        amax_w = float(np.abs(O.source_to_f32(wl.W_e4m3, wl.w_scale)).max())
+        qw = O.quantize(wl.W_e4m3[:ns], amax=amax_w, fp8_scale=wl.w_scale)
+        qx = O.quantize(wl.X_bf16[:ms], amax=amax_x)
+        O.gemm(qx, qw)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.time()
+    for _ in range(args.steps):
+        step()
+    dt = (time.time() - t0) / args.steps
+    value = 2.0 * ms * ns * K / dt / 1e12
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = (f"per step: quantize W[0:{ns}] (fp8 source, full-tensor amax) and X[0:{ms}], "
+              f"Y[0:{ms},0:{ns}] in fp64 over K={K}")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

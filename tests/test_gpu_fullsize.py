@@ -1,0 +1,112 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration bench.py times:
+codes / scales / global scales bit-exact against the oracle over the whole tensors, GEMM
+outputs on sampled positions (the oracle computes them one by one), calibration by the
+nearest-rank property that holds at any size."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_14_b200 as nv
+import oracle as O
+from gpu_helpers import assert_quant_equal, dev_tensor, gpu_quantize, to_numpy_f64
+from nvfp4_block_scaled_14_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    nv.load()
+
+
+def _sampled_check(y, ra, rw, n_samples, seed, bf16=True, extra=()):
+    Mr, Nr = y.shape
+    g = np.random.Generator(np.random.PCG64(seed))
+    ms = np.concatenate([g.integers(0, Mr, n_samples), [0, Mr - 1] + [e[0] for e in extra]])
+    ns = np.concatenate([g.integers(0, Nr, n_samples), [Nr - 1, 0] + [e[1] for e in extra]])
+    ref = O.gemm_sampled(ra, rw, ms, ns)
+    # tolerance from the oracle's own values (max over the samples <= max over all of Y)
+    tol = 1e-3 * np.abs(ref).max() + (np.abs(ref) * 2.0 ** -8 if bf16 else 0.0)
+    err = np.abs(y[ms, ns] - ref)
+    assert np.all(err <= tol), f"max err {err.max()} (tol {np.max(tol)})"
+
+
+def test_attn_proj_double_quant_full():
+    wl = W.attn_proj()
+    qw = gpu_quantize(wl.W_e4m3, fp8_scale=wl.w_scale)
+    qx = gpu_quantize(wl.X_bf16)
+    rw = O.quantize(wl.W_e4m3, fp8_scale=wl.w_scale)
+    rx = O.quantize(wl.X_bf16)
+    assert_quant_equal(qw, rw)
+    assert_quant_equal(qx, rx)
+    y = to_numpy_f64(nv.linear(qx, qw))
+    _sampled_check(y, rx, rw, 2000, 40, extra=[(4095, 3071), (128, 256), (127, 255)])
+
+
+def test_mlp_pair_full():
+    mp = W.mlp_pair()
+    q1, r1 = gpu_quantize(mp.W1), O.quantize(mp.W1)
+    assert_quant_equal(q1, r1)
+    qa1, ra1 = gpu_quantize(mp.X1), O.quantize(mp.X1)
+    assert_quant_equal(qa1, ra1)
+    y1 = to_numpy_f64(nv.linear(qa1, q1))
+    _sampled_check(y1, ra1, r1, 1500, 41)
+    del q1, qa1, y1
+    q2, r2 = gpu_quantize(mp.W2), O.quantize(mp.W2)
+    assert_quant_equal(q2, r2)
+    qa2, ra2 = gpu_quantize(mp.X2), O.quantize(mp.X2)
+    assert_quant_equal(qa2, ra2)
+    y2 = to_numpy_f64(nv.linear(qa2, q2))
+    _sampled_check(y2, ra2, r2, 1000, 42)
+
+
+def test_decode_small_m_full():
+    dc = W.decode()
+    qw, rw = gpu_quantize(dc.W), O.quantize(dc.W)
+    assert_quant_equal(qw, rw)
+    for m, x in dc.X.items():
+        qa, ra = gpu_quantize(x), O.quantize(x)
+        assert_quant_equal(qa, ra)
+        y = to_numpy_f64(nv.linear(qa, qw))
+        if m <= 8:
+            ref = O.gemm(ra, rw)
+            tol = 1e-3 * np.abs(ref).max() + np.abs(ref) * 2.0 ** -8
+            assert np.all(np.abs(y - ref) <= tol), m
+        else:
+            _sampled_check(y, ra, rw, 1500, 43 + m)
+
+
+def test_calibration_full_53_batches():
+    nb = 53
+    dev_batches, counts_lt, counts_le = [], 0, 0
+    host = []
+    for b in range(nb):
+        xb = W.calib_batch(b)
+        dev_batches.append(dev_tensor(xb))
+        host.append(xb)
+    p, mx = nv.calib_percentile_amax(dev_batches)
+    torch.cuda.synchronize()
+    p, mx = float(p.cpu()[0]), float(mx.cpu()[0])
+    n = nb * 4096 * 3072
+    rank = -(-n * 999 // 1000)
+    # nearest-rank property: #{|x| < p} < rank <= #{|x| <= p}; max is the largest |x|
+    true_max = 0.0
+    for xb in host:
+        a = np.abs(W.bf16_bits_to_f32(xb))
+        counts_lt += int(np.count_nonzero(a < p))
+        counts_le += int(np.count_nonzero(a <= p))
+        true_max = max(true_max, float(a.max()))
+    assert counts_lt < rank <= counts_le
+    assert mx == true_max
+    # quantize an evaluation batch with the p99.9 static scale and with the max, run the GEMM
+    ev = W.calib_batch(53)
+    wt = W.calib_weight()
+    qw, rw = gpu_quantize(wt), O.quantize(wt)
+    assert_quant_equal(qw, rw)
+    for amax in (p, mx):
+        qa, ra = gpu_quantize(ev, amax=amax), O.quantize(ev, amax=amax)
+        assert_quant_equal(qa, ra)
+        y = to_numpy_f64(nv.linear(qa, qw))
+        _sampled_check(y, ra, rw, 1000, 44)

@@ -5,18 +5,24 @@
 // Ada GPU", "What NVFP4 is and how it differs from NF4": on Blackwell the tensor cores
 // multiply in FP4 with weights and activations both in 4 bits).
 //
-// Kernel structure (one CTA per SM, persistent over work units):
+// Kernel structure (one CTA per SM, persistent over work units, 10 warps):
 //   warp 0      TMA producer: per 256-wide k-tile loads the A tile (128 rows x 128 B of packed
 //               codes), the B tile (BN rows x 128 B), both 128B-swizzled, and the scale-factor
 //               atoms of both (512-byte atoms of the tensor-core scale layout) into a
 //               STAGES-deep shared-memory ring; completion is tracked by mbarrier tx counts.
-//   warp 1      MMA issuer (one thread): copies the k-tile's scale atoms shared -> TMEM with
-//               tcgen05.cp (32x128b, replicated to the four lane quarters), then issues four
+//   warps 6..9  scale-factor feeders: move each k-tile's scale atoms shared -> registers ->
+//               TMEM with tcgen05.st (every lane quarter receives the full atom, the layout
+//               the block-scaled MMA reads), into one of kSfSlots TMEM slots. Doing this on
+//               the SIMT side keeps it off the tensor pipe, where a tcgen05.cp per atom would
+//               serialize with the MMAs.
+//   warp 1      MMA issuer (one thread): per k-tile four
 //               tcgen05.mma.kind::mxf4nvf4.block_scale.scale_vec::4X (M128 x BN x K64) into a
-//               fp32 accumulator in TMEM, and frees the ring slot with tcgen05.commit.
+//               fp32 accumulator in TMEM; tcgen05.commit frees the smem stage and the SF slot.
 //               Also allocates / frees TMEM.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp owns one 32-lane quarter),
-//               times alpha = sgA * sgW, cast, store (or raw fp32 partials for split-K).
+//               times alpha = sgA * sgW, cast to bf16 and held in registers; the accumulator
+//               is released to the MMA warp before the global stores, so the stores overlap
+//               the next tile's mainloop. (fp32 outputs / split-K partials store chunk-wise.)
 // Small M (<= 128) runs swap-AB: the weights take the MMA's M side (128 rows of W per tile)
 // and the activation rows the N side (8..128), so the tensor cores stream the weight matrix
 // at full width; with few tiles the K range is split over CTAs and a second kernel adds the
@@ -25,6 +31,7 @@
 // status word, lets the CTA drain its in-flight copies / MMAs, frees TMEM and returns.
 // No TMA multicast is used.
 #include <cuda.h>
+#include <cstring>
 #include <mutex>
 
 #include "nvfp4_internal.cuh"
@@ -34,11 +41,14 @@ namespace nvfp4 {
 namespace {
 
 constexpr int BM = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kWaitLimit = 1u << 20;
+#ifndef NVFP4_STAGES_256
+#define NVFP4_STAGES_256 3
+#endif
 
 template <int BN> struct Cfg {
-    static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 7);
+    static constexpr int kStages = BN == 256 ? NVFP4_STAGES_256 : (BN == 128 ? 6 : 7);
     static constexpr int kSfbBands = BN > 128 ? 2 : 1;
     static constexpr int kABytes = BM * 128;
     static constexpr int kBBytes = BN * 128;
@@ -48,14 +58,20 @@ template <int BN> struct Cfg {
     static constexpr int kOffB = kStages * kABytes;
     static constexpr int kOffSfa = kOffB + kStages * kBBytes;
     static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
-    static constexpr int kOffBar = kOffSfb + kStages * kSfbBytes;
-    static constexpr int kSmemBytes = 1024 + kOffBar + 256;
-    // TMEM columns: accumulator, then double-buffered scale factors.
+    // bf16 output staging for the TMA-store epilogue (BN = 256): four 128-row x 128-byte
+    // boxes, 128B-swizzled
+    static constexpr int kStagingBytes = BN == 256 ? BM * BN * 2 : 0;
+    static constexpr int kOffStaging = kOffSfb + kStages * kSfbBytes;
+    static constexpr int kOffBar = kOffStaging + kStagingBytes;
+    static constexpr int kSmemBytes = kOffBar + 512;
+    // TMEM columns: accumulator, then kSfSlots scale-factor slots; a slot holds one k-tile:
+    // SFA in 16 columns (4 k-blocks x 4), SFB in 4 * kSfbColsPerKb columns.
     static constexpr int kAccCols = BN < 32 ? 32 : BN;
-    static constexpr int kSfaCol = kAccCols;
-    static constexpr int kSfbCol = kSfaCol + 2 * 16;
+    static constexpr int kSfSlots = 4;
     static constexpr int kSfbColsPerKb = 4 * kSfbBands;
-    static constexpr int kUsedCols = kSfbCol + 2 * 4 * kSfbColsPerKb;
+    static constexpr int kSlotCols = 16 + 4 * kSfbColsPerKb;
+    static constexpr int kSfCol = kAccCols;
+    static constexpr int kUsedCols = kSfCol + kSfSlots * kSlotCols;
     static constexpr int kTmemCols = kUsedCols <= 32    ? 32
                                      : kUsedCols <= 64  ? 64
                                      : kUsedCols <= 128 ? 128
@@ -80,6 +96,7 @@ struct GemmParams {
     int out_bf16, swap;
     float *partial;            // split-K partials [splits][tiles_a*128][tiles_b*BN]
     int *status;
+    int tma_store; // 1: bf16 output through the shared-memory staging + TMA store
 };
 
 __device__ __forceinline__ void set_timeout(int *status)
@@ -87,6 +104,13 @@ __device__ __forceinline__ void set_timeout(int *status)
     atomicExch(status, (int)NVFP4_ERR_TIMEOUT);
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Chunk-wise store of 32 (or fewer) accumulator columns: fp32 outputs and split-K partials.
 template <int BN>
 __device__ __forceinline__ void store_chunk(const GemmParams &p, int64_t arow, int64_t bcol0,
                                             int split, const uint32_t *v, int n, float alpha)
@@ -94,16 +118,12 @@ __device__ __forceinline__ void store_chunk(const GemmParams &p, int64_t arow, i
     if (arow >= p.rows_a)
         return;
     if (p.splits > 1) {
-        float *dst = p.partial + ((int64_t)split * p.tiles_a * BM + arow) * (p.tiles_b * BN) + bcol0;
-        if (n % 4 == 0) {
-            for (int j = 0; j < n; j += 4)
-                *reinterpret_cast<float4 *>(dst + j) =
-                    make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-        } else {
-            for (int j = 0; j < n; ++j)
-                dst[j] = __uint_as_float(v[j]);
-        }
+        float *dst =
+            p.partial + ((int64_t)split * p.tiles_a * BM + arow) * (p.tiles_b * BN) + bcol0;
+        for (int j = 0; j < n; j += 4)
+            *reinterpret_cast<float4 *>(dst + j) =
+                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                            __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
         return;
     }
     if (p.swap) {
@@ -120,26 +140,12 @@ __device__ __forceinline__ void store_chunk(const GemmParams &p, int64_t arow, i
         }
         return;
     }
-    // A row = output row m, B rows = output columns
     const int64_t base = arow * p.ldy + bcol0;
     const bool full = bcol0 + n <= p.rows_b;
     if (p.out_bf16) {
         __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.y) + base;
-        if (full && (p.ldy % 8 == 0) && (n % 8 == 0)) {
-            for (int j = 0; j < n; j += 8) {
-                uint32_t w[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[j + 2 * t]) * alpha,
-                                                             __uint_as_float(v[j + 2 * t + 1]) * alpha);
-                    w[t] = *reinterpret_cast<uint32_t *>(&h);
-                }
-                *reinterpret_cast<uint4 *>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-        } else {
-            for (int j = 0; j < n && bcol0 + j < p.rows_b; ++j)
-                dst[j] = __float2bfloat16_rn(__uint_as_float(v[j]) * alpha);
-        }
+        for (int j = 0; j < n && bcol0 + j < p.rows_b; ++j)
+            dst[j] = __float2bfloat16_rn(__uint_as_float(v[j]) * alpha);
     } else {
         float *dst = reinterpret_cast<float *>(p.y) + base;
         if (full && (p.ldy % 4 == 0) && (n % 4 == 0)) {
@@ -155,20 +161,104 @@ __device__ __forceinline__ void store_chunk(const GemmParams &p, int64_t arow, i
     }
 }
 
+// Read NC (<= 32) accumulator columns starting at `col` of this warp's lanes into v.
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t *v)
+{
+    if constexpr (NC == 32) {
+        tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
+    } else if constexpr (NC == 16) {
+        tmem_ld_32x32b_x16(taddr, v);
+    } else {
+        tmem_ld_32x32b_x8(taddr, v);
+    }
+}
+
+// Whole accumulator row of this thread -> bf16 pairs in registers (alpha applied).
+template <int BN>
+__device__ __forceinline__ void acc_row_to_bf16(uint32_t trow, float alpha, uint32_t *pk)
+{
+    constexpr int NC = BN < 16 ? BN : 16;
+#pragma unroll
+    for (int c0 = 0; c0 < BN; c0 += NC) {
+        uint32_t v[NC];
+        tmem_ld_cols<NC>(trow + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < NC; j += 2)
+            pk[(c0 + j) / 2] =
+                pack_bf16x2(__uint_as_float(v[j]) * alpha, __uint_as_float(v[j + 1]) * alpha);
+    }
+}
+
+__device__ __forceinline__ __nv_bfloat16 bf16_half(uint32_t w, int hi)
+{
+    __nv_bfloat16_raw r;
+    r.x = (unsigned short)(hi ? (w >> 16) : (w & 0xFFFFu));
+    return __nv_bfloat16(r);
+}
+
+// Y[arow, bcol0 .. bcol0+BN) from a register-held row (A rows are output rows).
+template <int BN>
+__device__ __forceinline__ void store_row_bf16(const GemmParams &p, int64_t arow, int64_t bcol0,
+                                               const uint32_t *pk)
+{
+    if (arow >= p.rows_a)
+        return;
+    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.y) + arow * p.ldy + bcol0;
+    if (bcol0 + BN <= p.rows_b && (p.ldy % 8) == 0) {
+#pragma unroll
+        for (int j = 0; j < BN; j += 8)
+            *reinterpret_cast<uint4 *>(dst + j) =
+                make_uint4(pk[j / 2], pk[j / 2 + 1], pk[j / 2 + 2], pk[j / 2 + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < BN; j += 2) {
+            if (bcol0 + j < p.rows_b)
+                dst[j] = bf16_half(pk[j / 2], 0);
+            if (bcol0 + j + 1 < p.rows_b)
+                dst[j + 1] = bf16_half(pk[j / 2], 1);
+        }
+    }
+}
+
+// Swap-AB: A rows are output columns, B rows (accumulator columns) are output rows; each
+// store instruction of the warp covers 32 consecutive output columns.
+template <int BN>
+__device__ __forceinline__ void store_row_bf16_swap(const GemmParams &p, int64_t arow,
+                                                    int64_t bcol0, const uint32_t *pk)
+{
+    if (arow >= p.rows_a)
+        return;
+    __nv_bfloat16 *y = reinterpret_cast<__nv_bfloat16 *>(p.y);
+#pragma unroll
+    for (int j = 0; j < BN; ++j) {
+        const int64_t m = bcol0 + j;
+        if (m < p.rows_b)
+            y[m * p.ldy + arow] = bf16_half(pk[j / 2], j & 1);
+    }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmSFA,
-                      const __grid_constant__ CUtensorMap tmSFB, const GemmParams p)
+                      const __grid_constant__ CUtensorMap tmSFB,
+                      const __grid_constant__ CUtensorMap tmY, const GemmParams p)
 {
     using C = Cfg<BN>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((smem_u32(smem) & 1023u) != 0) { // the swizzled operand tiles need 1024-B alignment
+        if (threadIdx.x == 0)
+            atomicExch(p.status, (int)NVFP4_ERR_CUDA);
+        return;
+    }
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *empty_bar = full_bar + C::kStages;
-    uint64_t *acc_full = empty_bar + C::kStages;
+    uint64_t *sf_full = empty_bar + C::kStages;
+    uint64_t *sf_empty = sf_full + C::kSfSlots;
+    uint64_t *acc_full = sf_empty + C::kSfSlots;
     uint64_t *acc_empty = acc_full + 1;
     uint64_t *drain_bar = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 3);
@@ -180,6 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
+        }
+        for (int s = 0; s < C::kSfSlots; ++s) {
+            mbar_init(&sf_full[s], 4);
+            mbar_init(&sf_empty[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 4);
@@ -250,10 +344,89 @@ __global__ void __launch_bounds__(kThreads, 1)
                     set_timeout(p.status);
             }
         }
+    } else if (warp >= 6) {
+        // ------------------------------- scale-factor feeders -----------------------
+        const int q = warp & 3; // the TMEM lane quarter this warp may write
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, sphase = 0;
+        bool ok = true;
+        for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+            const int split = (int)(u / tiles_ab);
+            const int k0 = split * p.kt_per_split;
+            const int k1 = min(p.kt_total, k0 + p.kt_per_split);
+            for (int kt = k0; kt < k1; ++kt) {
+                if (!mbar_wait(&full_bar[stage], phase, kWaitLimit) ||
+                    !mbar_wait(&sf_empty[slot], sphase ^ 1, kWaitLimit)) {
+                    if (lane == 0)
+                        set_timeout(p.status);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t ssfa = smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes);
+                const uint32_t ssfb = smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes);
+                const uint32_t tslot =
+                    tmem + ((uint32_t)(q * 32) << 16) + C::kSfCol + slot * C::kSlotCols;
+                // SFA: atom kb -> columns 4*kb .. 4*kb+3 (row r of the atom in lane r)
+                uint32_t ra[16];
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    const uint4 w = lds128(ssfa + kb * 512 + lane * 16);
+                    ra[4 * kb] = w.x;
+                    ra[4 * kb + 1] = w.y;
+                    ra[4 * kb + 2] = w.z;
+                    ra[4 * kb + 3] = w.w;
+                }
+                tmem_st_32x32b_x16(tslot, ra);
+                // SFB: atom (band h, kb) -> columns 16 + kb*kSfbColsPerKb + 4*h
+#pragma unroll
+                for (int h = 0; h < C::kSfbBands; ++h) {
+                    uint32_t rb[16];
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        const uint4 w = lds128(ssfb + (h * 4 + kb) * 512 + lane * 16);
+                        rb[4 * kb] = w.x;
+                        rb[4 * kb + 1] = w.y;
+                        rb[4 * kb + 2] = w.z;
+                        rb[4 * kb + 3] = w.w;
+                    }
+                    if constexpr (C::kSfbBands == 1) {
+                        tmem_st_32x32b_x16(tslot + 16, rb);
+                    } else {
+                        // interleave bands: kb-major, band-minor
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb) {
+                            uint32_t t4[16];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                t4[i] = rb[4 * kb + i];
+                            asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], "
+                                         "{%1, %2, %3, %4};" ::"r"(tslot + 16 +
+                                                                     kb * C::kSfbColsPerKb + 4 * h),
+                                         "r"(t4[0]), "r"(t4[1]), "r"(t4[2]), "r"(t4[3])
+                                         : "memory");
+                        }
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sf_full[slot]);
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+                if (++slot == C::kSfSlots) {
+                    slot = 0;
+                    sphase ^= 1;
+                }
+            }
+        }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
-        int stage = 0;
-        uint32_t phase = 0, acc_phase = 0, sfbuf = 0;
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, sphase = 0, acc_phase = 0;
         bool ok = true;
         for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
             const int split = (int)(u / tiles_ab);
@@ -266,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             for (int kt = k0; kt < k1; ++kt) {
-                if (!mbar_wait(&full_bar[stage], phase, kWaitLimit)) {
+                if (!mbar_wait(&full_bar[stage], phase, kWaitLimit) ||
+                    !mbar_wait(&sf_full[slot], sphase, kWaitLimit)) {
                     if (lane == 0)
                         set_timeout(p.status);
                     ok = false;
@@ -274,20 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t ssfa = smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes);
-                    const uint32_t ssfb = smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes);
-                    const uint32_t tsfa = tmem + C::kSfaCol + sfbuf * 16;
-                    const uint32_t tsfb = tmem + C::kSfbCol + sfbuf * (4 * C::kSfbColsPerKb);
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        tc_cp_sf_atom(tsfa + kb * 4,
-                                      smem_desc(ssfa + kb * 512, 0, 128, kLayoutSwizzleNone));
-#pragma unroll
-                        for (int h = 0; h < C::kSfbBands; ++h)
-                            tc_cp_sf_atom(tsfb + kb * C::kSfbColsPerKb + h * 4,
-                                          smem_desc(ssfb + (h * 4 + kb) * 512, 0, 128,
-                                                    kLayoutSwizzleNone));
-                    }
+                    const uint32_t tsfa = tmem + C::kSfCol + slot * C::kSlotCols;
+                    const uint32_t tsfb = tsfa + 16;
                     const uint64_t adesc = smem_desc(smem_u32(smem + stage * C::kABytes), 16,
                                                      1024, kLayoutSwizzle128B);
                     const uint64_t bdesc =
@@ -301,12 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     (kt > k0 || kb > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty_bar[stage]);
+                    tc_commit(&sf_empty[slot]);
                 }
                 __syncwarp();
-                sfbuf ^= 1;
                 if (++stage == C::kStages) {
                     stage = 0;
                     phase ^= 1;
+                }
+                if (++slot == C::kSfSlots) {
+                    slot = 0;
+                    sphase ^= 1;
                 }
             }
             if (!ok)
@@ -316,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             acc_phase ^= 1;
         }
-        // Drain: every MMA / copy issued by this thread completes before TMEM is freed.
+        // Drain: every MMA issued by this thread completes before TMEM is freed.
         if (lane == 0) {
             tc_commit(drain_bar);
             if (!mbar_wait(drain_bar, 0, kWaitLimit))
@@ -324,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------- epilogue -----------------------------------
+        // ------------------------------- epilogue (warps 2..5) ----------------------
         const int q = warp & 3; // TMEM lane quarter this warp may access
         const float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
         uint32_t acc_phase = 0;
@@ -340,33 +506,79 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int64_t arow = ta * BM + q * 32 + lane;
             const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-            if constexpr (BN >= 32) {
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(trow + c0, v);
-                    tmem_ld_wait();
-                    store_chunk<BN>(p, arow, tb * BN + c0, split, v, 32, alpha);
+            if constexpr (BN == 256) {
+                if (p.tma_store) {
+                    // previous tile's bulk stores must have read the staging buffer
+                    if (threadIdx.x == 64)
+                        bulk_wait_group_read0();
+                    named_bar_sync(1, 128);
+                    const uint32_t stg = smem_u32(smem + C::kOffStaging);
+                    const int r = q * 32 + lane; // row inside the tile
+#pragma unroll 2
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(trow + c0, v);
+                        tmem_ld_wait();
+                        uint32_t w[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            w[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * alpha,
+                                               __uint_as_float(v[2 * j + 1]) * alpha);
+                        // box c0/64, 16-byte chunk (c0 % 64) / 8 (+1), swizzled by row % 8
+                        const uint32_t box = stg + (c0 >> 6) * (BM * 128) + r * 128;
+                        const int ch = (c0 & 63) >> 3;
+                        sts128(box + (((ch) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                        sts128(box + (((ch + 1) ^ (r & 7)) << 4), w[4], w[5], w[6], w[7]);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(acc_empty); // accumulator free: next tile's MMAs may start
+                    fence_proxy_async_smem();
+                    named_bar_sync(1, 128);
+                    if (threadIdx.x == 64) {
+#pragma unroll
+                        for (int b = 0; b < BN / 64; ++b)
+                            tma_store_2d(&tmY, smem + C::kOffStaging + b * (BM * 128),
+                                         (int)(tb * BN + b * 64), (int)(ta * BM));
+                        bulk_commit_group();
+                    }
+                    acc_phase ^= 1;
+                    continue;
                 }
-            } else if constexpr (BN == 16) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(trow, v);
-                tmem_ld_wait();
-                store_chunk<BN>(p, arow, tb * BN, split, v, 16, alpha);
-            } else {
-                uint32_t v[8];
-                tmem_ld_32x32b_x8(trow, v);
-                tmem_ld_wait();
-                store_chunk<BN>(p, arow, tb * BN, split, v, 8, alpha);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(acc_empty);
+            if (p.splits == 1 && p.out_bf16 && BN <= 128) {
+                // bf16 row in registers, accumulator released before the stores
+                uint32_t pk[BN / 2 > 0 ? BN / 2 : 1];
+                acc_row_to_bf16<BN>(trow, alpha, pk);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(acc_empty);
+                if (p.swap)
+                    store_row_bf16_swap<BN>(p, arow, tb * BN, pk);
+                else
+                    store_row_bf16<BN>(p, arow, tb * BN, pk);
+            } else {
+                constexpr int NC = BN < 32 ? BN : 32;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += NC) {
+                    uint32_t v[NC];
+                    tmem_ld_cols<NC>(trow + c0, v);
+                    tmem_ld_wait();
+                    store_chunk<BN>(p, arow, tb * BN + c0, split, v, NC, alpha);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(acc_empty);
+            }
             acc_phase ^= 1;
         }
     }
 
+    if (threadIdx.x == 64)
+        bulk_wait_group0(); // bulk stores complete before the CTA's shared memory goes away
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -457,13 +669,32 @@ bool make_sf_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, int 
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output Y [rows x cols], box 64 columns x 128 rows, 128B swizzle (TMA store).
+bool make_out_map(CUtensorMap *m, void *base, int64_t rows, int64_t cols)
+{
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+    cuuint32_t box[2] = {64u, 128u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN>
 cudaError_t launch_bn(const LinearPlan &pl, const uint8_t *a_codes, const uint8_t *a_sf,
                       const uint8_t *b_codes, const uint8_t *b_sf, int64_t K, GemmParams gp,
                       cudaStream_t s, nvfp4_status *st)
 {
     using C = Cfg<BN>;
-    CUtensorMap tmA, tmB, tmSFA, tmSFB;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
+    memset(&tmY, 0, sizeof(tmY));
+    gp.tma_store = 0;
+    if (BN == 256 && gp.splits == 1 && gp.out_bf16 && !gp.swap && gp.ldy % 8 == 0 &&
+        (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0 && encode_fn() &&
+        make_out_map(&tmY, gp.y, gp.rows_a, gp.rows_b))
+        gp.tma_store = 1;
     if (!encode_fn() || !make_codes_map(&tmA, a_codes, pl.rows_a, K, BM) ||
         !make_codes_map(&tmB, b_codes, pl.rows_b, K, BN) ||
         !make_sf_map(&tmSFA, a_sf, pl.rows_a, K, 1) ||
@@ -486,7 +717,7 @@ cudaError_t launch_bn(const LinearPlan &pl, const uint8_t *a_codes, const uint8_
     if (grid < 1)
         grid = 1;
     nvfp4_gemm_kernel<BN><<<(unsigned)grid, kThreads, C::kSmemBytes, s>>>(tmA, tmB, tmSFA,
-                                                                          tmSFB, gp);
+                                                                          tmSFB, tmY, gp);
     return cudaGetLastError();
 }
 

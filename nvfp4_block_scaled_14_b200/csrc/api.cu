@@ -81,10 +81,12 @@ nvfp4_status check_matrix(int64_t rows, int64_t cols)
         return NVFP4_ERR_SHAPE;
     if (cols % 32 != 0)
         return NVFP4_ERR_SHAPE;
+    if ((rows / 128 + 1) * (cols / 64 + 1) >= ((int64_t)1 << 31)) // tile indices fit in int32
+        return NVFP4_ERR_SHAPE;
     return NVFP4_OK;
 }
 
-size_t quantize_ws_bytes() { return (size_t)kAmaxPartials * sizeof(float); }
+size_t quantize_ws_bytes() { return quantize_workspace_bytes(); }
 
 nvfp4_status quantize_common(const void *x, int src_type, const float *fp8_scale, int64_t rows,
                              int64_t cols, const float *static_amax, uint8_t *codes,
@@ -107,8 +109,7 @@ nvfp4_status quantize_common(const void *x, int src_type, const float *fp8_scale
     if ((st = check_device()) != NVFP4_OK)
         return st;
     return map_cuda(launch_quantize(x, src_type, fp8_scale, rows, cols, static_amax, codes,
-                                    scales_swz, scales_lin, global_scale,
-                                    reinterpret_cast<float *>(ws), s));
+                                    scales_swz, scales_lin, global_scale, ws, s));
 }
 
 } // namespace

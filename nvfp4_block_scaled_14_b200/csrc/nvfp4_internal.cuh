@@ -28,13 +28,14 @@ int *device_status_ptr();
 int num_sms();
 
 // ---- quantize.cu --------------------------------------------------------------------
-// Number of partial maxima the amax pass writes (the workspace holds that many floats).
-constexpr int kAmaxPartials = 1184; // 8 per SM on a 148-SM part
+// Per-CTA maxima the quantizer's workspace holds (one amax CTA per SM).
+constexpr int kAmaxPartials = 1024;
+size_t quantize_workspace_bytes();
 
 cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale, int64_t rows,
                             int64_t cols, const float *static_amax, uint8_t *codes,
                             uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,
-                            float *ws_partials, cudaStream_t s);
+                            void *ws, cudaStream_t s);
 
 // ---- dequantize.cu ------------------------------------------------------------------
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales_lin,

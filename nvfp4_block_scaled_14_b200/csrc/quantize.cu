@@ -7,15 +7,19 @@
 // "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details". FP8 source (double
 // quantization): "Qwen-Rapid-AIO FP8 -> NVFP4", "1. Double Quantization".
 //
-// Two kernels, both HBM-bound:
-//   amax_kernel   -- grid-stride max |x| with 128-bit loads; one partial per CTA (no atomics,
-//                    no zeroing, order-free and therefore exact).
-//   encode_kernel -- one CTA per 128-row x 64-column tile (exactly one 512-byte atom of the
-//                    tensor-core scale layout); each thread encodes two 16-value blocks:
-//                    block amax, E4M3 scale, reciprocal, E2M1 codes by the hardware cvt,
-//                    8-byte code stores (four lanes write 32 contiguous bytes of a row) and
-//                    byte stores of the swizzled and / or linear scales. Padding entries of
-//                    the swizzled atom are written as zero by the same CTA.
+// Two kernels per call, both HBM-bound, chained by programmatic dependent launch:
+//   amax_kernel   (dynamic amax only) -- one CTA per SM streams a contiguous byte range of
+//                 the tensor through a 4 x 32 KB shared-memory ring of 1-D bulk copies and
+//                 reduces max |x| with SIMD integer max on the magnitude bits (exact,
+//                 order-free); one partial per CTA, no atomics, nothing to zero.
+//   encode_kernel -- one CTA per SM owns a contiguous range of rows; each warp takes a
+//                 32-block run of one row (512 values, fully coalesced), one 16-value block per
+//                 lane. It loads its first items before griddepcontrol.wait, so the loads
+//                 overlap the amax kernel's tail (the tensor is then mostly in L2), reduces the
+//                 partial maxima to the global scale, and fills a 128-entry table of
+//                 1 / (E4M3(c) * sg). Per block: block amax, E4M3 scale, E2M1 codes by the
+//                 hardware cvt, an 8-byte code store (a warp writes 256 contiguous bytes) and
+//                 byte stores of the swizzled and / or linear scales; atom padding is zeroed.
 // Code-deciding arithmetic is IEEE fp32 round-to-nearest in a fixed order (__fdiv_rn,
 // __fmul_rn, __frcp_rn): sg = amax / 2688, sb = E4M3(bmax / (sg * 6)),
 // code = E2M1(x * (1 / (sb * sg))).
@@ -25,50 +29,51 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kAmaxThreads = 512;
-constexpr int kEncThreads = 256;
+constexpr int kThreads = 1024;      // encode: 32 warps, one 16-value block per lane per item
+constexpr int kAmaxThreads = 1024;  // amax: one CTA per SM streaming its byte range
+constexpr int kChunk = 32 * 1024;   // amax ring: 4 x 32 KB bulk copies in flight per SM
+constexpr int kRing = 4;
+constexpr uint32_t kSpinLimit = 1u << 24;
 
 template <int SRC> struct Src;
 
+// |x| orders like the magnitude bits of x for finite values, so maxima are taken on the bit
+// patterns with SIMD integer max: exact, order-free.
 template <> struct Src<kSrcF32> {
     static constexpr int kBytes = 4;
-    __device__ static float vec_absmax(uint4 v)
+    __device__ static uint32_t vec_magmax(uint4 v) // fp32 magnitude bits
     {
-        float a = fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y)));
-        float b = fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)));
-        return fmaxf(a, b);
+        return max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu),
+                   max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu));
     }
+    __device__ static float mag_to_f32(uint32_t m) { return __uint_as_float(m); }
 };
 
 template <> struct Src<kSrcBF16> {
     static constexpr int kBytes = 2;
-    __device__ static float vec_absmax(uint4 v)
+    __device__ static uint32_t vec_magmax(uint4 v) // two 16-bit lanes of magnitude bits
     {
-        // |x| of a bf16 is monotone in its low 15 bits: take the max of the magnitude bits.
-        uint32_t m = 0;
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            m = max(m, w[i] & 0x7FFFu);
-            m = max(m, (w[i] >> 16) & 0x7FFFu);
-        }
-        return __uint_as_float(m << 16);
+        const uint32_t k = 0x7FFF7FFFu;
+        return __vmaxu2(__vmaxu2(v.x & k, v.y & k), __vmaxu2(v.z & k, v.w & k));
+    }
+    __device__ static float mag_to_f32(uint32_t m)
+    {
+        return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
     }
 };
 
 template <> struct Src<kSrcE4M3> {
     static constexpr int kBytes = 1;
-    __device__ static float vec_absmax(uint4 v)
+    __device__ static uint32_t vec_magmax(uint4 v) // four 8-bit lanes of magnitude bits
     {
-        // |e4m3| is monotone in its low 7 bits (finite inputs).
-        uint32_t m = 0;
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-                m = max(m, (w[i] >> (8 * b)) & 0x7Fu);
-        return e4m3_to_f32(m);
+        const uint32_t k = 0x7F7F7F7Fu;
+        return __vmaxu4(__vmaxu4(v.x & k, v.y & k), __vmaxu4(v.z & k, v.w & k));
+    }
+    __device__ static float mag_to_f32(uint32_t m) // |e4m3| (before the fp8 scale)
+    {
+        const uint32_t b = max(max(m & 0xFFu, (m >> 8) & 0xFFu),
+                               max((m >> 16) & 0xFFu, m >> 24));
+        return e4m3_to_f32(b);
     }
 };
 
@@ -81,57 +86,35 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4 *p)
     return v;
 }
 
-template <int SRC>
-__global__ void __launch_bounds__(kAmaxThreads)
-    amax_kernel(const uint4 *__restrict__ x, int64_t nvec, float *__restrict__ partials)
-{
-    float m = 0.0f;
-    const int64_t stride = (int64_t)gridDim.x * kAmaxThreads;
-    int64_t i = (int64_t)blockIdx.x * kAmaxThreads + threadIdx.x;
-    for (; i + 3 * stride < nvec; i += 4 * stride) {
-        uint4 v0 = ldg_stream(x + i), v1 = ldg_stream(x + i + stride);
-        uint4 v2 = ldg_stream(x + i + 2 * stride), v3 = ldg_stream(x + i + 3 * stride);
-        m = fmaxf(m, fmaxf(fmaxf(Src<SRC>::vec_absmax(v0), Src<SRC>::vec_absmax(v1)),
-                           fmaxf(Src<SRC>::vec_absmax(v2), Src<SRC>::vec_absmax(v3))));
-    }
-    for (; i < nvec; i += stride)
-        m = fmaxf(m, Src<SRC>::vec_absmax(ldg_stream(x + i)));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __shared__ float red[kAmaxThreads / 32];
-    if ((threadIdx.x & 31) == 0)
-        red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        m = threadIdx.x < kAmaxThreads / 32 ? red[threadIdx.x] : 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        if (threadIdx.x == 0)
-            partials[blockIdx.x] = m;
-    }
-}
+// Raw 16-byte vectors of one 16-value block: 4 (fp32), 2 (bf16) or 1 (fp8).
+template <int SRC> constexpr int kVecs = SRC == kSrcF32 ? 4 : (SRC == kSrcBF16 ? 2 : 1);
 
-// Load one 16-value block as fp32 (fp8: upcast by one fp32 multiply with s8).
 template <int SRC>
-__device__ __forceinline__ void load_block(const uint8_t *p, float s8, float (&v)[16])
+__device__ __forceinline__ void load_raw(const uint8_t *p, uint4 (&r)[4])
 {
     const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < kVecs<SRC>; ++i)
+        r[i] = ldg_stream(q + i);
+}
+
+// Raw block -> 16 fp32 values (bf16 widening is exact; fp8 is upcast by one fp32 multiply
+// with s8).
+template <int SRC>
+__device__ __forceinline__ void to_f32(const uint4 (&r)[4], float s8, float (&v)[16])
+{
     if constexpr (SRC == kSrcF32) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            uint4 w = ldg_stream(q + i);
-            v[4 * i + 0] = __uint_as_float(w.x);
-            v[4 * i + 1] = __uint_as_float(w.y);
-            v[4 * i + 2] = __uint_as_float(w.z);
-            v[4 * i + 3] = __uint_as_float(w.w);
+            v[4 * i + 0] = __uint_as_float(r[i].x);
+            v[4 * i + 1] = __uint_as_float(r[i].y);
+            v[4 * i + 2] = __uint_as_float(r[i].z);
+            v[4 * i + 3] = __uint_as_float(r[i].w);
         }
     } else if constexpr (SRC == kSrcBF16) {
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-            uint4 w = ldg_stream(q + i);
-            uint32_t u[4] = {w.x, w.y, w.z, w.w};
+            const uint32_t u[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 v[8 * i + 2 * j + 0] = __uint_as_float(u[j] << 16);
@@ -139,165 +122,389 @@ __device__ __forceinline__ void load_block(const uint8_t *p, float s8, float (&v
             }
         }
     } else {
-        uint4 w = ldg_stream(q);
-        uint32_t u[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t u[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float2 a = e4m3x2_to_f32x2(u[j] & 0xFFFFu);
-            float2 b = e4m3x2_to_f32x2(u[j] >> 16);
-            v[4 * j + 0] = __fmul_rn(a.x, s8);
-            v[4 * j + 1] = __fmul_rn(a.y, s8);
-            v[4 * j + 2] = __fmul_rn(b.x, s8);
-            v[4 * j + 3] = __fmul_rn(b.y, s8);
+            const float2 ss = make_float2(s8, s8);
+            const float2 a = __fmul2_rn(e4m3x2_to_f32x2(u[j] & 0xFFFFu), ss);
+            const float2 b = __fmul2_rn(e4m3x2_to_f32x2(u[j] >> 16), ss);
+            v[4 * j + 0] = a.x;
+            v[4 * j + 1] = a.y;
+            v[4 * j + 2] = b.x;
+            v[4 * j + 3] = b.y;
         }
     }
 }
 
-// Encode one block: returns the E4M3 scale byte and writes the 8 code bytes.
-__device__ __forceinline__ uint32_t encode_block(const float (&v)[16], float sg, float t,
+// Block maximum |x| (fp32) from the raw vectors (fp8: times s8, which commutes with the max
+// because rounding is monotone).
+template <int SRC>
+__device__ __forceinline__ float block_absmax(const uint4 (&r)[4], float s8)
+{
+    if constexpr (SRC == kSrcF32) {
+        return __uint_as_float(max(max(Src<SRC>::vec_magmax(r[0]), Src<SRC>::vec_magmax(r[1])),
+                                   max(Src<SRC>::vec_magmax(r[2]), Src<SRC>::vec_magmax(r[3]))));
+    } else if constexpr (SRC == kSrcBF16) {
+        return Src<SRC>::mag_to_f32(
+            __vmaxu2(Src<SRC>::vec_magmax(r[0]), Src<SRC>::vec_magmax(r[1])));
+    } else {
+        return __fmul_rn(Src<SRC>::mag_to_f32(Src<SRC>::vec_magmax(r[0])), s8);
+    }
+}
+
+// E4M3 code of RN(bmax / t), exactly as cvt_e4m3(__fdiv_rn(bmax, t)) gives it, usually without
+// the division. rt = RN(1/t). q0 = RN(bmax * rt) is within 3 fp32 ulps of RN(bmax / t) (two
+// roundings of relative size 2^-24 each, plus the rounding of the quotient itself). For
+// q0 >= 2^-6 (normal E4M3 range) the E4M3 rounding decision depends on the 20 fp32 mantissa
+// bits below the 3 kept ones and flips only at 0x80000 (the midpoint between two E4M3
+// values; saturation at 448 leaves no further boundary above). If q0 sits more than 4 ulps
+// from that midpoint, q0 and RN(bmax / t) round to the same E4M3 code; otherwise, below
+// 2^-6, and when q0 is not finite (1/t overflowed), the correctly rounded division decides.
+__device__ __forceinline__ uint32_t e4m3_of_quotient(float bmax, float t, float rt)
+{
+    if (bmax == 0.0f)
+        return 0u;
+    const float q0 = __fmul_rn(bmax, rt);
+    const int d = (int)(__float_as_uint(q0) & 0xFFFFFu) - 0x80000;
+    if (q0 >= 0.015625f && q0 <= 3.0e38f && (d > 4 || d < -4))
+        return cvt_e4m3(q0);
+    return cvt_e4m3(__fdiv_rn(bmax, t));
+}
+
+// Encode one block: returns the E4M3 scale byte and writes the 8 code bytes. rcp_tab[c] holds
+// 1 / (E4M3(c) * sg), computed with the same two round-to-nearest operations per code.
+template <int SRC>
+__device__ __forceinline__ uint32_t encode_block(const uint4 (&r)[4], float s8, float sg,
+                                                 float t, float rt, const float *rcp_tab,
                                                  uint2 &packed)
 {
-    float bmax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-        bmax = fmaxf(bmax, fabsf(v[j]));
+    const float bmax = block_absmax<SRC>(r, s8);
     uint32_t sb = 0;
     if (sg > 0.0f)
-        sb = cvt_e4m3(__fdiv_rn(bmax, t));
-    const float fsb = e4m3_to_f32(sb);
+        sb = e4m3_of_quotient(bmax, t, rt);
     packed = make_uint2(0u, 0u);
-    if (fsb != 0.0f) {
-        const float rcp = __frcp_rn(__fmul_rn(fsb, sg));
+    if (sb != 0u) {
+        float v[16];
+        to_f32<SRC>(r, s8, v);
+        const float rcp = rcp_tab[sb];
+        const float2 rr = make_float2(rcp, rcp);
         float y[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            y[j] = __fmul_rn(v[j], rcp);
+        for (int j = 0; j < 16; j += 2) {
+            const float2 p = __fmul2_rn(make_float2(v[j], v[j + 1]), rr);
+            y[j] = p.x;
+            y[j + 1] = p.y;
+        }
         packed.x = cvt_e2m1x8(y);
         packed.y = cvt_e2m1x8(y + 8);
     }
     return sb;
 }
 
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Fold a magnitude-bit accumulator (per source type) into another.
+template <int SRC> __device__ __forceinline__ uint32_t mag_fold(uint32_t a, uint32_t b)
+{
+    if constexpr (SRC == kSrcF32)
+        return max(a, b);
+    else if constexpr (SRC == kSrcBF16)
+        return __vmaxu2(a, b);
+    else
+        return __vmaxu4(a, b);
+}
+
+template <int SRC> __device__ __forceinline__ uint32_t raw_magmax(const uint4 (&r)[4])
+{
+    uint32_t m = Src<SRC>::vec_magmax(r[0]);
+#pragma unroll
+    for (int i = 1; i < kVecs<SRC>; ++i)
+        m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(r[i]));
+    return m;
+}
+
+struct QuantArgs {
+    const uint8_t *x;
+    const float *fp8_scale;
+    int rows, cols;
+    const float *static_amax;
+    uint8_t *codes, *sf_swz, *sf_lin;
+    float *global_scale;
+    const float *partials; // one max |x| per amax CTA (dynamic amax)
+    int npartials;
+    uint32_t chunks_magic; // ceil(2^32 / chunks) for chunks >= 2: item / chunks by umulhi
+};
+
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// K1: max |x| over a contiguous byte range per CTA, streamed through a shared-memory ring
+// with 1-D bulk copies; one partial per CTA.
 template <int SRC>
-__global__ void __launch_bounds__(kEncThreads)
-    encode_kernel(const uint8_t *__restrict__ x, const float *__restrict__ fp8_scale,
-                  int64_t rows, int64_t cols, const float *__restrict__ static_amax,
-                  const float *__restrict__ partials, int npartials, uint8_t *__restrict__ codes,
-                  uint8_t *__restrict__ sf_swz, uint8_t *__restrict__ sf_lin,
-                  float *__restrict__ global_scale)
+__global__ void __launch_bounds__(kAmaxThreads, 1)
+    amax_kernel(const uint8_t *__restrict__ x, int64_t nbytes, float *__restrict__ partials,
+                int *status)
+{
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ uint64_t bars[kRing];
+    __shared__ float s_red[kAmaxThreads / 32];
+    const int64_t nvec = nbytes >> 4;
+    const int64_t per = ((nvec + gridDim.x - 1) / gridDim.x) << 4;
+    const int64_t b0 = min(nbytes, per * (int64_t)blockIdx.x);
+    const int64_t b1 = min(nbytes, b0 + per);
+    const int nchunks = (int)((b1 - b0 + kChunk - 1) / kChunk);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kRing; ++i)
+            mbar_init(&bars[i], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    auto issue = [&](int c) {
+        const int64_t off = b0 + (int64_t)c * kChunk;
+        const uint32_t n = (uint32_t)min((int64_t)kChunk, b1 - off);
+        mbar_arrive_expect_tx(&bars[c % kRing], n);
+        bulk_load_1d(ring + (c % kRing) * kChunk, x + off, n, &bars[c % kRing]);
+    };
+    if (threadIdx.x == 0)
+        for (int c = 0; c < min(nchunks, kRing); ++c)
+            issue(c);
+    pdl_launch_dependents(); // the encode kernel may start its own loads meanwhile
+    uint32_t m = 0;
+    for (int c = 0; c < nchunks; ++c) {
+        const int slot = c % kRing;
+        if (!mbar_wait(&bars[slot], (uint32_t)(c / kRing) & 1u, kSpinLimit))
+            atomicExch(status, (int)NVFP4_ERR_TIMEOUT);
+        const int nv = (int)(min((int64_t)kChunk, b1 - (b0 + (int64_t)c * kChunk)) >> 4);
+        const uint32_t base = smem_u32(ring + slot * kChunk);
+        for (int i = threadIdx.x; i < nv; i += kAmaxThreads)
+            m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(lds128(base + 16 * i)));
+        __syncthreads(); // every thread is done with this slot
+        if (threadIdx.x == 0 && c + kRing < nchunks)
+            issue(c + kRing);
+    }
+    float f = Src<SRC>::mag_to_f32(m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
+    if ((threadIdx.x & 31) == 0)
+        s_red[threadIdx.x >> 5] = f;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        f = threadIdx.x < kAmaxThreads / 32 ? s_red[threadIdx.x] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
+        if (threadIdx.x == 0)
+            partials[blockIdx.x] = f;
+    }
+}
+
+// K2: encode. Each CTA owns a contiguous range of rows; each warp takes a 32-block run of
+// one row (one 16-value block per lane). The first items are loaded before waiting on the
+// amax kernel (programmatic dependent launch), so the loads overlap its tail.
+template <int SRC>
+__global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
 {
     __shared__ float s_sg;
-    const float s8 = (SRC == kSrcE4M3 && fp8_scale) ? *fp8_scale : 1.0f;
+    __shared__ float s_rcp[128];
+    constexpr int kBlkBytes = 16 * Src<SRC>::kBytes;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = a.cols >> 4;        // blocks per row
+    const int chunks = (nb + 31) >> 5; // 32-block runs per row (one per warp item)
+    const int apb = (nb + 3) >> 2;     // scale atoms per 128-row band
+    const int64_t row_bytes = (int64_t)a.cols * Src<SRC>::kBytes;
+    const int r0 = (int)((int64_t)a.rows * blockIdx.x / gridDim.x);
+    const int r1 = (int)((int64_t)a.rows * (blockIdx.x + 1) / gridDim.x);
+    const int items = (r1 - r0) * chunks;
+    const uint8_t *xbase = a.x + (int64_t)r0 * row_bytes;
+
+    // item -> (row offset, block). The quotient by multiply-high is exact or one too large
+    // (item < 2^31, chunks < 2^27); one correction.
+    auto item_rb = [&](int it, int &ro, int &blk) {
+        if (chunks == 1) {
+            ro = it;
+            blk = lane;
+            return;
+        }
+        ro = (int)__umulhi((uint32_t)it, a.chunks_magic);
+        if (ro * chunks > it)
+            --ro;
+        blk = (it - ro * chunks) * 32 + lane;
+    };
+    auto load_item = [&](int it, uint4 (&r)[4], int &ro, int &blk) {
+        item_rb(it, ro, blk);
+        if (it < items && blk < nb)
+            load_raw<SRC>(xbase + (int64_t)ro * row_bytes + blk * kBlkBytes, r);
+    };
+
+    // first two items of this warp: loaded before the dependency wait
+    int it = warp;
+    uint4 r[2][4];
+    int ro[2], blk[2];
+    load_item(it, r[0], ro[0], blk[0]);
+    load_item(it + 32, r[1], ro[1], blk[1]);
+
+    const float s8 = (SRC == kSrcE4M3 && a.fp8_scale) ? *a.fp8_scale : 1.0f;
+    if (!a.static_amax)
+        pdl_wait(); // the amax kernel's partial maxima are complete and visible
     if (threadIdx.x < 32) {
-        float a = 0.0f;
-        if (static_amax) {
-            a = *static_amax;
+        float g = 0.0f;
+        if (a.static_amax) {
+            g = *a.static_amax;
         } else {
-            for (int i = threadIdx.x; i < npartials; i += 32)
-                a = fmaxf(a, partials[i]);
+            for (int i = threadIdx.x; i < a.npartials; i += 32)
+                g = fmaxf(g, __ldcg(a.partials + i));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
-                a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
             if (SRC == kSrcE4M3)
-                a = __fmul_rn(a, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
+                g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
         }
         if (threadIdx.x == 0) {
-            const float sg = __fdiv_rn(a, 2688.0f); // 6 * 448
+            const float sg = __fdiv_rn(g, 2688.0f); // 6 * 448
             s_sg = sg;
             if (blockIdx.x == 0)
-                *global_scale = sg;
+                *a.global_scale = sg;
         }
     }
     __syncthreads();
     const float sg = s_sg;
     const float t = __fmul_rn(sg, 6.0f);
+    const float rt = __frcp_rn(t);
+    if (threadIdx.x < 128)
+        s_rcp[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
+    __syncthreads();
 
-    const int64_t nb = cols >> 4;
-    const int64_t apb = (nb + 3) >> 2; // atoms per 128-row band
-    const int64_t ntiles = ((rows + 127) >> 7) * apb;
-    const int64_t row_bytes = cols * Src<SRC>::kBytes;
-
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t band = tile / apb, atom = tile - band * apb;
-        float v[2][16];
-        int64_t row[2], blk[2];
-        bool valid[2];
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const int local = threadIdx.x + it * kEncThreads; // 0..511
-            row[it] = band * 128 + (local >> 2);
-            blk[it] = atom * 4 + (local & 3);
-            valid[it] = row[it] < rows && blk[it] < nb;
-            if (valid[it])
-                load_block<SRC>(x + row[it] * row_bytes + blk[it] * 16 * Src<SRC>::kBytes, s8,
-                                v[it]);
+    // valid block: codes + scales; atom padding block (nb <= blk < 4 * apb): zero scale
+    auto encode_store = [&](int rowo, int b, const uint4 (&rr)[4]) {
+        const int row = r0 + rowo;
+        uint32_t sb = 0;
+        if (b < nb) {
+            uint2 packed;
+            sb = encode_block<SRC>(rr, s8, sg, t, rt, s_rcp, packed);
+            *reinterpret_cast<uint2 *>(a.codes + (int64_t)row * (a.cols >> 1) + b * 8) = packed;
+            if (a.sf_lin)
+                a.sf_lin[(int64_t)row * nb + b] = (uint8_t)sb;
         }
+        if (a.sf_swz && b < 4 * apb)
+            a.sf_swz[((int64_t)(row >> 7) * apb + (b >> 2)) * 512 + ((row & 31) << 4) +
+                     (((row >> 5) & 3) << 2) + (b & 3)] = (uint8_t)sb;
+    };
+    while (it < items) {
+        // two items in flight: encode the loaded pair, then load the next pair
+        uint4 n[2][4];
+        int nro[2], nblk[2];
+        load_item(it + 64, n[0], nro[0], nblk[0]);
+        load_item(it + 96, n[1], nro[1], nblk[1]);
+        encode_store(ro[0], blk[0], r[0]);
+        if (it + 32 < items)
+            encode_store(ro[1], blk[1], r[1]);
 #pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            uint32_t sb = 0;
-            if (valid[it]) {
-                uint2 packed;
-                sb = encode_block(v[it], sg, t, packed);
-                *reinterpret_cast<uint2 *>(codes + row[it] * (cols >> 1) + blk[it] * 8) = packed;
-                if (sf_lin)
-                    sf_lin[row[it] * nb + blk[it]] = (uint8_t)sb;
-            }
-            if (sf_swz) {
-                const int local = threadIdx.x + it * kEncThreads;
-                const int r = local >> 2;
-                sf_swz[tile * 512 + ((r & 31) << 4) + ((r >> 5) << 2) + (local & 3)] =
-                    (uint8_t)sb;
-            }
+        for (int u = 0; u < 2; ++u) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                r[u][v] = n[u][v];
+            ro[u] = nro[u];
+            blk[u] = nblk[u];
         }
+        it += 64;
+    }
+    // zero the scale padding rows of the last 128-row band
+    if (a.sf_swz) {
+        const int rows_pad = ((a.rows + 127) >> 7) << 7;
+        for (int row = a.rows + blockIdx.x; row < rows_pad; row += gridDim.x)
+            for (int b = threadIdx.x; b < 4 * apb; b += kThreads)
+                a.sf_swz[((int64_t)(row >> 7) * apb + (b >> 2)) * 512 + ((row & 31) << 4) +
+                         (((row >> 5) & 3) << 2) + (b & 3)] = 0;
     }
 }
 
 template <int SRC>
 cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, int64_t cols,
                          const float *static_amax, uint8_t *codes, uint8_t *sf_swz,
-                         uint8_t *sf_lin, float *global_scale, float *partials, cudaStream_t s)
+                         uint8_t *sf_lin, float *global_scale, void *ws, cudaStream_t s)
 {
-    int npartials = 0;
+    const int sms = num_sms();
+    QuantArgs qa{};
+    qa.x = reinterpret_cast<const uint8_t *>(x);
+    qa.fp8_scale = fp8_scale;
+    qa.rows = (int)rows;
+    qa.cols = (int)cols;
+    qa.static_amax = static_amax;
+    qa.codes = codes;
+    qa.sf_swz = sf_swz;
+    qa.sf_lin = sf_lin;
+    qa.global_scale = global_scale;
+    qa.partials = reinterpret_cast<const float *>(ws);
+    const uint64_t chunks = (uint64_t)((cols / 16 + 31) / 32);
+    qa.chunks_magic = chunks > 1 ? (uint32_t)((((uint64_t)1 << 32) + chunks - 1) / chunks) : 0u;
+    cudaError_t e;
     if (!static_amax) {
-        const int64_t nvec = rows * cols * Src<SRC>::kBytes / 16;
-        int64_t g = (nvec + kAmaxThreads * 4 - 1) / (kAmaxThreads * 4);
-        g = g < 1 ? 1 : (g > kAmaxPartials ? kAmaxPartials : g);
-        npartials = (int)g;
-        amax_kernel<SRC><<<(unsigned)g, kAmaxThreads, 0, s>>>(
-            reinterpret_cast<const uint4 *>(x), nvec, partials);
-        cudaError_t e = cudaGetLastError();
+        const int64_t nbytes = rows * cols * Src<SRC>::kBytes;
+        int g = sms < kAmaxPartials ? sms : kAmaxPartials;
+        const int64_t need = (nbytes + kChunk - 1) / kChunk;
+        if (need < g)
+            g = need < 1 ? 1 : (int)need;
+        qa.npartials = g;
+        const size_t smem = (size_t)kRing * kChunk;
+        e = cudaFuncSetAttribute(amax_kernel<SRC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
         if (e != cudaSuccess)
             return e;
+        amax_kernel<SRC><<<g, kAmaxThreads, smem, s>>>(reinterpret_cast<const uint8_t *>(x),
+                                                       nbytes, reinterpret_cast<float *>(ws),
+                                                       device_status_ptr());
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
     }
-    const int64_t nb = cols >> 4;
-    const int64_t ntiles = ((rows + 127) >> 7) * ((nb + 3) >> 2);
-    int64_t g = ntiles < 1 ? 1 : ntiles;
-    const int64_t cap = (int64_t)num_sms() * 8;
-    if (g > cap)
-        g = cap;
-    encode_kernel<SRC><<<(unsigned)g, kEncThreads, 0, s>>>(
-        reinterpret_cast<const uint8_t *>(x), fp8_scale, rows, cols, static_amax, partials,
-        npartials, codes, sf_swz, sf_lin, global_scale);
-    return cudaGetLastError();
+    int grid = sms;
+    if (rows < grid)
+        grid = rows < 1 ? 1 : (int)rows;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = static_amax ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, encode_kernel<SRC>, qa);
 }
 
 } // namespace
 
+size_t quantize_workspace_bytes() { return (size_t)kAmaxPartials * sizeof(float); }
+
 cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale, int64_t rows,
                             int64_t cols, const float *static_amax, uint8_t *codes,
                             uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,
-                            float *ws_partials, cudaStream_t s)
+                            void *ws, cudaStream_t s)
 {
     switch (src_type) {
     case kSrcF32:
         return launch_typed<kSrcF32>(x, fp8_scale, rows, cols, static_amax, codes, scales_swz,
-                                     scales_lin, global_scale, ws_partials, s);
+                                     scales_lin, global_scale, ws, s);
     case kSrcBF16:
         return launch_typed<kSrcBF16>(x, fp8_scale, rows, cols, static_amax, codes, scales_swz,
-                                      scales_lin, global_scale, ws_partials, s);
+                                      scales_lin, global_scale, ws, s);
     default:
         return launch_typed<kSrcE4M3>(x, fp8_scale, rows, cols, static_amax, codes, scales_swz,
-                                      scales_lin, global_scale, ws_partials, s);
+                                      scales_lin, global_scale, ws, s);
     }
 }
 

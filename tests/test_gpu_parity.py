@@ -130,6 +130,38 @@ def test_e4m3_rounding_of_the_hardware_matches_oracle():
     assert_quant_equal(gpu_quantize(x, amax=448.0), ref)
 
 
+@pytest.mark.parametrize("amax", [333.3, 1.0, 0.0123, 7.77e3])
+def test_e4m3_scale_near_rounding_midpoints(amax):
+    # block maxima placed within a few ulps of (E4M3 midpoint) * (6 * sg) for a global scale
+    # whose reciprocal is inexact: the scale's rounding decision sits right at a boundary.
+    sg = np.float32(amax) / np.float32(2688.0)
+    t = np.float64(np.float32(sg * np.float32(6.0)))
+    e4 = np.array([O.e4m3_decode(c) for c in range(127)], np.float64)
+    mids = np.concatenate([(e4[:-1] + e4[1:]) / 2, e4])
+    base = (mids * t).astype(np.float32)
+    pts = [base]
+    up, dn = base.copy(), base.copy()
+    for _ in range(6):
+        up = np.nextafter(up, np.float32(np.inf))
+        dn = np.nextafter(dn, np.float32(0))
+        pts += [up, dn]
+    r = np.random.Generator(np.random.PCG64(32))
+    pts.append((r.uniform(0, 450, 5000) * t).astype(np.float32))
+    v = np.concatenate(pts)
+    v = v[(v > 0) & (v <= np.float32(amax))]
+    rows = -(-v.size // 2)
+    flat = np.zeros(rows * 2, np.float32)
+    flat[:v.size] = v
+    x = np.zeros((rows, 32), np.float32)
+    x[:, 0] = flat[0::2]
+    x[:, 16] = flat[1::2]
+    x[:, 5] = flat[0::2] * np.float32(0.5)
+    x[0, 1] = np.float32(amax)  # the tensor amax itself
+    assert_quant_equal(gpu_quantize(x, amax=amax), O.quantize(x, amax=amax))
+    # the same values through the dynamic-amax path
+    assert_quant_equal(gpu_quantize(x), O.quantize(x))
+
+
 # ---------------------------------------------------------------------------------------
 # dequantize
 # ---------------------------------------------------------------------------------------

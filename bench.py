@@ -10,8 +10,10 @@ The headline `value` is the linear layer's throughput in TFLOP/s (2*M*N*K per st
 whole step, quantization included), summed over ranks. Each rank runs its own independent
 batch (weak scaling, no collective on the data path). Inputs rotate over enough buffer sets
 that every step reads them cold from HBM (more than 3x the L2 size in flight). Steps are
-replayed from CUDA graphs; per-kernel durations come from CUDA events captured inside those
-graphs, on the launching stream.
+replayed from CUDA graphs (one graph per rotation of the input sets). Per-op durations come
+from CUDA events around graph loops of each op alone over the same rotating inputs, on the
+launching stream (event nodes inside the step graph would break the kernels' programmatic
+dependent launch and add ~15 us per step).
 
 The other rows of the hot path (MLP-pair GEMMs, small-M decode GEMV, p99.9 calibration,
 dequantize) are measured after the timed region and reported under "rows".
@@ -135,19 +137,11 @@ class Step:
         self.qx = nv.quantize(self.X[0])
         self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
 
-    def run(self, i, ev=None):
+    def run(self, i):
         nv = self.nv
-        if ev is not None:
-            ev[0].record()
         nv.quantize_fp8(self.W[i], self.s8, out=self.qw)
-        if ev is not None:
-            ev[1].record()
         nv.quantize(self.X[i], out=self.qx)
-        if ev is not None:
-            ev[2].record()
         nv.linear(self.qx, self.qw, out=self.Y)
-        if ev is not None:
-            ev[3].record()
 
 
 def launches_per_step(nv):
@@ -156,43 +150,44 @@ def launches_per_step(nv):
     return 2 + 2 + (2 if ws > 0 else 1)
 
 
-def time_graph_replays(graphs, n_total, stream):
-    """Replay graphs round-robin for n_total steps; return elapsed ms (device events)."""
+def capture(fns):
+    """One CUDA graph that runs every closure in fns in order (warmed up on a side stream)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for f in fns:
+            f()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in fns:
+            f()
+    return g
+
+
+def replay_ms(graphs, stream):
+    """Replay graphs in order; device time between events on the launching stream."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for i in range(n_total):
-        graphs[i % len(graphs)].replay()
+    for g in graphs:
+        g.replay()
     end.record(stream)
     end.synchronize()
     return start.elapsed_time(end)
 
 
-def op_timer(fns, reps_per_fn=3):
-    """Average device time of one call of each closure in fns (rotating buffer sets),
-    captured in one CUDA graph with external events around every call."""
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        for f in fns:
-            f()
-    torch.cuda.current_stream().wait_stream(s)
+def op_timer(fns, reps=3):
+    """Average device time of one call, over graphs that run every closure in fns (each on
+    its own buffer set, so inputs come from HBM), replayed `reps` times."""
+    g = capture(fns)
+    g.replay()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True, external=True),
-            torch.cuda.Event(enable_timing=True, external=True)) for _ in fns]
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for (a, b), f in zip(evs, fns):
-            a.record()
-            f()
-            b.record()
-    times = []
-    for _ in range(reps_per_fn):
-        g.replay()
-        torch.cuda.synchronize()
-        times += [a.elapsed_time(b) for a, b in evs]
+    ms = replay_ms([g] * reps, torch.cuda.current_stream())
     del g
-    return statistics.mean(times), statistics.median(times)
+    us = ms * 1e3 / (reps * len(fns))
+    return us / 1e3, us / 1e3
 
 
 def extras(nv, W, dev, hbm, fp4_peak):
@@ -218,11 +213,19 @@ def extras(nv, W, dev, hbm, fp4_peak):
     elems = X2.numel()
     gbs = (elems * 2 + elems / 2 + elems / 16 + 4) / (avg * 1e-3) / 1e9
     rows["quantize_x2_bf16_4096x12288"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    def clone_q(q):
+        return nv.NVFP4Tensor(q.codes.clone(), q.scales_swz.clone(), None,
+                              q.global_scale.clone(), q.rows, q.cols)
+
     for name, a, w, y, kk, nn in [("gemm1_m4096_n12288_k3072", qx1, q1, Y1, 3072, 12288),
                                   ("gemm2_m4096_n3072_k12288", qx2, q2, Y2, 12288, 3072)]:
-        avg, med = op_timer([lambda a=a, w=w, y=y: nv.linear(a, w, out=y)] * 6)
+        # rotate over copies of the quantized operands so each call reads them from HBM
+        nset = sets_for(a.codes.numel() + w.codes.numel())
+        sets = [(clone_q(a), clone_q(w)) for _ in range(nset)]
+        avg, med = op_timer([lambda p=p, y=y: nv.linear(p[0], p[1], out=y) for p in sets])
         tf = 2.0 * 4096 * nn * kk / (avg * 1e-3) / 1e12
         rows[name] = {"us": avg * 1e3, "TFLOP/s": tf, "frac_fp4": tf / fp4_peak}
+        del sets
     del X2s, W1, W2, X1, X2, Y1, Y2, q1, q2, qx1, qx2
     torch.cuda.empty_cache()
 
@@ -248,15 +251,17 @@ def extras(nv, W, dev, hbm, fp4_peak):
     #     each read several times; 8 x 25 MB exceeds L2, so every read comes from HBM)
     distinct = [t(W.calib_batch(b)) for b in range(8)]
     batches = [distinct[b % 8] for b in range(53)]
-    avg, med = op_timer([lambda: nv.calib_percentile_amax(batches)], reps_per_fn=5)
+    avg, med = op_timer([lambda: nv.calib_percentile_amax(batches)], reps=5)
     nbytes = 53 * 4096 * 3072 * 2
     gbs = nbytes / (avg * 1e-3) / 1e9
     rows["calib_p999_53x4096x3072_bf16"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
     del distinct, batches
 
     # --- dequantize 12288x3072 to bf16
-    wq = nv.quantize(t(W.mlp_pair(M=8).W1), linear=True)
-    avg, med = op_timer([lambda: nv.dequantize(wq, torch.bfloat16)] * 4)
+    w1 = nv.quantize(t(W.mlp_pair(M=8).W1), linear=True)
+    wqs = [nv.NVFP4Tensor(w1.codes.clone(), None, w1.scales_lin.clone(), w1.global_scale,
+                          w1.rows, w1.cols) for _ in range(3)]
+    avg, med = op_timer([lambda q=q: nv.dequantize(q, torch.bfloat16) for q in wqs])
     elems = 12288 * 3072
     gbs = (elems / 2 + elems / 16 + elems * 2) / (avg * 1e-3) / 1e9
     rows["dequantize_12288x3072_bf16"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
@@ -322,23 +327,14 @@ def run_ours(args):
         st.run(i % n_sets)
     torch.cuda.synchronize()
 
-    # one graph per input set, with external events between the three ops
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-           for _ in range(n_sets)]
-    graphs = []
-    side = torch.cuda.Stream()
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        st.run(0)
-    stream.wait_stream(side)
-    torch.cuda.synchronize()
-    for i in range(n_sets):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            st.run(i, evs[i])
-        graphs.append(g)
-    for i in range(max(args.warmup, n_sets)):
-        graphs[i % n_sets].replay()
+    # one graph per rotation of the input sets (n_sets steps, no nodes between the ops),
+    # plus one for the remaining steps, so exactly args.steps steps are replayed
+    full = capture([lambda i=i: st.run(i) for i in range(n_sets)])
+    rem = args.steps % n_sets
+    part = capture([lambda i=i: st.run(i) for i in range(rem)]) if rem else None
+    plan = [full] * (args.steps // n_sets) + ([part] if part is not None else [])
+    for _ in range(max(1, args.warmup // n_sets)):
+        full.replay()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
@@ -348,17 +344,22 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     t_lo = time.time()
-    ms = time_graph_replays(graphs, args.steps, stream)
+    ms = replay_ms(plan, stream)
     t_hi = time.time()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     clk = clocks.stop(t_lo, t_hi)
+    del plan, full, part
 
-    # per-op device durations from the events of the last replay of every graph
-    qw_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    qx_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    gemm_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    # per-op device durations: each op alone, over the rotating input sets
+    qw_ms, _ = op_timer([lambda i=i: nv.quantize_fp8(st.W[i], st.s8, out=st.qw)
+                         for i in range(n_sets)])
+    qx_ms, _ = op_timer([lambda i=i: nv.quantize(st.X[i], out=st.qx) for i in range(n_sets)])
+    qws = [nv.quantize_fp8(st.W[i], st.s8) for i in range(n_sets)]
+    qxs = [nv.quantize(st.X[i]) for i in range(n_sets)]
+    gemm_ms, _ = op_timer([lambda i=i: nv.linear(qxs[i], qws[i], out=st.Y) for i in range(n_sets)])
+    del qws, qxs
 
     t = torch.tensor([ms], dtype=torch.float64, device=dev)
     if dist is not None:
@@ -395,7 +396,6 @@ def run_ours(args):
 
     rows = None
     if not args.no_extras and rank == 0:
-        del graphs
         rows = extras(nv, W, dev, hbm, fp4_peak)
 
     if dist is not None:

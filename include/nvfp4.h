@@ -136,6 +136,30 @@ nvfp4_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales_swz, c
                           size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * nvfp4_linear without a caller-supplied workspace. No counterpart in the paper: it exists for
+ * callers that cannot call cudaMalloc or lend a device buffer, e.g. code that runs inside an
+ * engine or plugin host that owns all device memory, latency-critical loops where an
+ * allocation (which may synchronize the device) is not allowed, or callers with no buffer to
+ * spare. Same arguments, result and checks as nvfp4_linear minus ws / ws_bytes.
+ * Scratch: the split-K partial sums go to a 4 MiB array that the library keeps in device
+ * memory (every GPU that loads the library holds it until the process exits). Shapes whose
+ * partial sums need more than 4 MiB (nvfp4_workspace_bytes(NVFP4_OP_LINEAR, M, N, K) >
+ * 4 MiB) are rejected with NVFP4_ERR_WORKSPACE before any launch; shapes that need no partial
+ * sums (workspace 0) never touch the array. The call allocates nothing.
+ * The array is shared by every call on the device and keeps the last call's contents; each
+ * call writes every partial it later reads, so nothing needs clearing. Calls whose GPU work
+ * overlaps (other streams, or concurrent host threads) race on the array: serialize them.
+ * The first call on each device that needs the scratch resolves its address
+ * (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ * capture.
+ */
+nvfp4_status nvfp4_linear_noalloc(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                                  const float *a_gs, const uint8_t *w_codes,
+                                  const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
+                                  int64_t N, int64_t K, nvfp4_dtype out_dt, void *y,
+                                  cudaStream_t stream);
+
+/*
  * Static-scale calibration ("Qwen-Rapid-AIO FP8 -> NVFP4", "Recommended Model": p99.9
  * percentile aggregation over calibration generations instead of max aggregation).
  * Over the union of num_batches device arrays (batches is a HOST array of device pointers),

@@ -47,6 +47,8 @@ _SIGNATURES = {
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _int, _vp, _vp], _int),
     "nvfp4_linear": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _sz, _vp],
                      _int),
+    "nvfp4_linear_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp],
+                             _int),
     "nvfp4_calib_percentile_amax": ([ctypes.POINTER(_vp), _int, _i64, _int, _u32, _u32, _vp,
                                      _vp, _vp, _sz, _vp], _int),
     "nvfp4_sync_status": ([_vp], _int),

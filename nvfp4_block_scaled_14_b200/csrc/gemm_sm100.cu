@@ -806,4 +806,64 @@ cudaError_t launch_linear(const LinearPlan &pl, const uint8_t *a_codes, const ui
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------------
+// Allocation-free entry point
+// ---------------------------------------------------------------------------------------
+
+namespace {
+
+// Split-K partial sums of nvfp4_linear_noalloc live here instead of in a caller-supplied
+// workspace. Every GPU that loads the library holds this array until the process exits.
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20; // 4 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+void *g_noalloc_ptr[kNoAllocMaxDevices];
+cudaError_t g_noalloc_err[kNoAllocMaxDevices];
+
+// Device address of the scratch array on the current device. In host code the array's name
+// only stands for the symbol; the address kernels may use comes from cudaGetSymbolAddress,
+// resolved once per device with that device current.
+cudaError_t noalloc_scratch(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return cudaErrorInvalidDevice;
+    std::call_once(g_noalloc_once[dev], [dev]() {
+        void *p = nullptr;
+        g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        g_noalloc_ptr[dev] = p;
+    });
+    if (g_noalloc_err[dev] != cudaSuccess)
+        return g_noalloc_err[dev];
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+} // namespace
+
 } // namespace nvfp4
+
+extern "C" nvfp4_status nvfp4_linear_noalloc(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                                             const float *a_gs, const uint8_t *w_codes,
+                                             const uint8_t *w_scales_swz, const float *w_gs,
+                                             int64_t M, int64_t N, int64_t K,
+                                             nvfp4_dtype out_dt, void *y, cudaStream_t stream)
+{
+    using namespace nvfp4;
+    size_t need = 0;
+    if (M > 0 && N > 0 && K > 0 && K % 32 == 0 && M < ((int64_t)1 << 31) &&
+        N < ((int64_t)1 << 31) && K < ((int64_t)1 << 31))
+        need = plan_linear(M, N, K).ws_bytes;
+    if (need > kNoAllocScratchBytes)
+        return NVFP4_ERR_WORKSPACE; // this shape's split-K partials exceed the 4 MiB scratch
+    void *scratch = nullptr;
+    if (need > 0 && noalloc_scratch(&scratch) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return nvfp4_linear(a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs, M, N, K,
+                        out_dt, y, scratch, scratch ? kNoAllocScratchBytes : 0, stream);
+}

@@ -46,6 +46,10 @@ constexpr uint32_t kWaitLimit = 1u << 20;
 #ifndef NVFP4_STAGES_256
 #define NVFP4_STAGES_256 3
 #endif
+#ifndef NVFP4_PAIR_KERNEL
+#define NVFP4_PAIR_KERNEL 1
+#endif
+constexpr bool kUsePairKernel = NVFP4_PAIR_KERNEL != 0;
 
 template <int BN> struct Cfg {
     static constexpr int kStages = BN == 256 ? NVFP4_STAGES_256 : (BN == 128 ? 6 : 7);
@@ -171,6 +175,31 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t *v)
         tmem_ld_32x32b_x16(taddr, v);
     } else {
         tmem_ld_32x32b_x8(taddr, v);
+    }
+}
+
+// This thread's accumulator row (256 fp32 columns of its TMEM lane) x alpha -> bf16 into the
+// shared staging tile: four 128-row x 128-byte boxes, 16-byte chunks swizzled by row % 8 (the
+// TMA store's 128B swizzle). Four TMEM loads are in flight per wait.
+__device__ __forceinline__ void stage_tile_bf16(uint32_t trow, uint32_t stg, int r, float alpha)
+{
+#pragma unroll 1
+    for (int c0 = 0; c0 < 256; c0 += 64) {
+        uint32_t v[64];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            tmem_ld_32x32b_x16(trow + c0 + 16 * i, v + 16 * i);
+        tmem_ld_wait();
+        const uint32_t box = stg + (c0 >> 6) * (128 * 128) + r * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                w[j] = pack_bf16x2(__uint_as_float(v[8 * ch + 2 * j]) * alpha,
+                                   __uint_as_float(v[8 * ch + 2 * j + 1]) * alpha);
+            sts128(box + ((ch ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+        }
     }
 }
 
@@ -512,24 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (threadIdx.x == 64)
                         bulk_wait_group_read0();
                     named_bar_sync(1, 128);
-                    const uint32_t stg = smem_u32(smem + C::kOffStaging);
-                    const int r = q * 32 + lane; // row inside the tile
-#pragma unroll 2
-                    for (int c0 = 0; c0 < BN; c0 += 16) {
-                        uint32_t v[16];
-                        tmem_ld_32x32b_x16(trow + c0, v);
-                        tmem_ld_wait();
-                        uint32_t w[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            w[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * alpha,
-                                               __uint_as_float(v[2 * j + 1]) * alpha);
-                        // box c0/64, 16-byte chunk (c0 % 64) / 8 (+1), swizzled by row % 8
-                        const uint32_t box = stg + (c0 >> 6) * (BM * 128) + r * 128;
-                        const int ch = (c0 & 63) >> 3;
-                        sts128(box + (((ch) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
-                        sts128(box + (((ch + 1) ^ (r & 7)) << 4), w[4], w[5], w[6], w[7]);
-                    }
+                    stage_tile_bf16(trow, smem_u32(smem + C::kOffStaging), q * 32 + lane, alpha);
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
@@ -584,6 +596,308 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// 2-SM variant: a CTA pair (cluster of 2) computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M256 N256 K64). Each CTA loads its 128 rows of A and its 128
+// rows of B, so the shared-memory traffic per SM per k-tile drops from ~108 KB (1-SM 128x256
+// tile: TMA writes + MMA reads) to ~76 KB. The leader CTA (rank 0) issues the MMAs and
+// commits to barriers of both CTAs; the other CTA's TMA loads of A / B and its feeder and
+// epilogue warps arrive on the leader's barriers. Scale factors: each CTA's TMEM holds SFA
+// of its own 128 rows and SFB of all 256 columns (its feeders write both). Only the bf16,
+// un-split case uses it (TMA-store epilogue).
+// ---------------------------------------------------------------------------------------
+
+struct Pair {
+    static constexpr int kStages = 4;
+    static constexpr int kABytes = 128 * 128;     // this CTA's 128 rows of A
+    static constexpr int kBBytes = 128 * 128;     // this CTA's 128 rows of B
+    static constexpr int kSfaBytes = 4 * 512;     // SFA atoms of this CTA's rows
+    static constexpr int kSfbBytes = 2 * 4 * 512; // SFB atoms of all 256 columns
+    static constexpr int kOffB = kStages * kABytes;
+    static constexpr int kOffSfa = kOffB + kStages * kBBytes;
+    static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
+    static constexpr int kOffStaging = kOffSfb + kStages * kSfbBytes;
+    static constexpr int kStagingBytes = 128 * 256 * 2;
+    static constexpr int kOffBar = kOffStaging + kStagingBytes;
+    static constexpr int kSmemBytes = kOffBar + 512;
+    static constexpr uint32_t kTxAB = 2 * (kABytes + kBBytes); // both CTAs, on the leader
+    static constexpr uint32_t kTxSf = kSfaBytes + kSfbBytes;   // own CTA
+    static constexpr int kSfSlots = 4;
+    static constexpr int kSlotCols = 16 + 32; // SFA 4 x 4, SFB 4 x 8
+    static constexpr int kSfCol = 256;
+    static constexpr int kTmemCols = 512;
+    static constexpr uint32_t kIdesc =
+        (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kSfCol + kSfSlots * kSlotCols <= kTmemCols, "TMEM budget");
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmSFA,
+                           const __grid_constant__ CUtensorMap tmSFB,
+                           const __grid_constant__ CUtensorMap tmY, const GemmParams p)
+{
+    using C = Pair;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((smem_u32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0)
+            atomicExch(p.status, (int)NVFP4_ERR_CUDA);
+        return; // uniform across the cluster: both CTAs see the same layout
+    }
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kOffBar); // leader only
+    uint64_t *sfdata = full_bar + C::kStages;                            // own SF TMA
+    uint64_t *empty_bar = sfdata + C::kStages;                           // both
+    uint64_t *sf_full = empty_bar + C::kStages;                          // leader only
+    uint64_t *sf_empty = sf_full + C::kSfSlots;                          // both
+    uint64_t *acc_full = sf_empty + C::kSfSlots;                         // both
+    uint64_t *acc_empty = acc_full + 1;                                  // leader only
+    uint64_t *drain_bar = acc_full + 2;                                  // leader only
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 3);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&sfdata[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int s = 0; s < C::kSfSlots; ++s) {
+            mbar_init(&sf_full[s], 8); // four feeder warps in each CTA
+            mbar_init(&sf_empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 8); // four epilogue warps in each CTA
+        mbar_init(drain_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync(); // barriers of both CTAs initialised before any remote arrival
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int64_t tiles_ab = p.tiles_a * p.tiles_b; // tiles_a counts 256-row pairs
+    const int64_t cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+    if (warp == 0) {
+        // ------------------------------- TMA producer (both CTAs) ---------------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmSFA);
+            tma_prefetch_desc(&tmSFB);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int64_t u = cluster_id; u < tiles_ab && ok; u += nclusters) {
+                const int64_t ta = u % p.tiles_a, tb = u / p.tiles_a;
+                const int arow = (int)(ta * 256 + rank * 128);
+                const int brow = (int)(tb * 256 + rank * 128);
+                for (int kt = 0; kt < p.kt_total; ++kt) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimit)) {
+                        set_timeout(p.status);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t leader_full = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                    if (leader)
+                        mbar_arrive_expect_tx(&full_bar[stage], C::kTxAB);
+                    mbar_arrive_expect_tx(&sfdata[stage], C::kTxSf);
+                    tma_load_2d_pair(smem + stage * C::kABytes, &tmA, leader_full, kt * 128, arow);
+                    tma_load_2d_pair(smem + C::kOffB + stage * C::kBBytes, &tmB, leader_full,
+                                     kt * 128, brow);
+                    tma_load_3d(smem + C::kOffSfa + stage * C::kSfaBytes, &tmSFA, &sfdata[stage], 0,
+                                kt * 4, arow >> 7);
+                    tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmSFB, &sfdata[stage], 0,
+                                kt * 4, (int)(tb * 2));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        }
+    } else if (warp >= 6) {
+        // ------------------------------- scale-factor feeders (both CTAs) -------------
+        const int q = warp & 3;
+        const uint32_t leader_sf_full0 = mapa_shared(smem_u32(&sf_full[0]), 0);
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, sphase = 0;
+        bool ok = true;
+        for (int64_t u = cluster_id; u < tiles_ab && ok; u += nclusters) {
+            for (int kt = 0; kt < p.kt_total; ++kt) {
+                if (!mbar_wait(&sfdata[stage], phase, kWaitLimit) ||
+                    !mbar_wait(&sf_empty[slot], sphase ^ 1, kWaitLimit)) {
+                    if (lane == 0)
+                        set_timeout(p.status);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t ssfa = smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes);
+                const uint32_t ssfb = smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes);
+                const uint32_t tslot =
+                    tmem + ((uint32_t)(q * 32) << 16) + C::kSfCol + slot * C::kSlotCols;
+                uint32_t ra[16];
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    const uint4 w = lds128(ssfa + kb * 512 + lane * 16);
+                    ra[4 * kb] = w.x;
+                    ra[4 * kb + 1] = w.y;
+                    ra[4 * kb + 2] = w.z;
+                    ra[4 * kb + 3] = w.w;
+                }
+                tmem_st_32x32b_x16(tslot, ra);
+                // SFB: atom (band h, kb) -> columns 16 + 8*kb + 4*h
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    uint32_t rb[16];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 w = lds128(ssfb + (h * 4 + kb) * 512 + lane * 16);
+                        rb[4 * h] = w.x;
+                        rb[4 * h + 1] = w.y;
+                        rb[4 * h + 2] = w.z;
+                        rb[4 * h + 3] = w.w;
+                    }
+                    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], "
+                                 "{%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(tslot + 16 + 8 * kb),
+                                 "r"(rb[0]), "r"(rb[1]), "r"(rb[2]), "r"(rb[3]), "r"(rb[4]),
+                                 "r"(rb[5]), "r"(rb[6]), "r"(rb[7])
+                                 : "memory");
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_remote(leader_sf_full0 + 8 * slot);
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+                if (++slot == C::kSfSlots) {
+                    slot = 0;
+                    sphase ^= 1;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer (leader) ---------------------------
+        if (leader) {
+            int stage = 0, slot = 0;
+            uint32_t phase = 0, sphase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int64_t u = cluster_id; u < tiles_ab && ok; u += nclusters) {
+                if (!mbar_wait(acc_empty, acc_phase ^ 1, kWaitLimit)) {
+                    if (lane == 0)
+                        set_timeout(p.status);
+                    break;
+                }
+                tc_fence_after();
+                for (int kt = 0; kt < p.kt_total; ++kt) {
+                    if (!mbar_wait(&full_bar[stage], phase, kWaitLimit) ||
+                        !mbar_wait(&sf_full[slot], sphase, kWaitLimit)) {
+                        if (lane == 0)
+                            set_timeout(p.status);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t tsfa = tmem + C::kSfCol + slot * C::kSlotCols;
+                        const uint32_t tsfb = tsfa + 16;
+                        const uint64_t adesc = smem_desc(smem_u32(smem + stage * C::kABytes), 16,
+                                                         1024, kLayoutSwizzle128B);
+                        const uint64_t bdesc =
+                            smem_desc(smem_u32(smem + C::kOffB + stage * C::kBBytes), 16, 1024,
+                                      kLayoutSwizzle128B);
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb)
+                            tc_mma_nvf4_pair(tmem, adesc + (uint64_t)(2 * kb),
+                                             bdesc + (uint64_t)(2 * kb), C::kIdesc, tsfa + kb * 4,
+                                             tsfb + kb * 8, (kt > 0 || kb > 0) ? 1u : 0u);
+                        tc_commit_pair_mc(&empty_bar[stage], 0x3);
+                        tc_commit_pair_mc(&sf_empty[slot], 0x3);
+                    }
+                    __syncwarp();
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                    if (++slot == C::kSfSlots) {
+                        slot = 0;
+                        sphase ^= 1;
+                    }
+                }
+                if (!ok)
+                    break;
+                if (lane == 0)
+                    tc_commit_pair_mc(acc_full, 0x3);
+                __syncwarp();
+                acc_phase ^= 1;
+            }
+            if (lane == 0) {
+                tc_commit_pair(drain_bar);
+                if (!mbar_wait(drain_bar, 0, kWaitLimit))
+                    set_timeout(p.status);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ------------------------------- epilogue (both CTAs, warps 2..5) -------------
+        const int q = warp & 3;
+        const float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
+        const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
+        uint32_t acc_phase = 0;
+        for (int64_t u = cluster_id; u < tiles_ab; u += nclusters) {
+            const int64_t ta = u % p.tiles_a, tb = u / p.tiles_a;
+            if (!mbar_wait(acc_full, acc_phase, kWaitLimit)) {
+                if (lane == 0)
+                    set_timeout(p.status);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+            if (threadIdx.x == 64)
+                bulk_wait_group_read0();
+            named_bar_sync(1, 128);
+            stage_tile_bf16(trow, smem_u32(smem + C::kOffStaging), q * 32 + lane, alpha);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_remote(leader_acc_empty); // this CTA's accumulator is drained
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (threadIdx.x == 64) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    tma_store_2d(&tmY, smem + C::kOffStaging + b * (128 * 128),
+                                 (int)(tb * 256 + b * 64), (int)(ta * 256 + rank * 128));
+                bulk_commit_group();
+            }
+            acc_phase ^= 1;
+        }
+    }
+
+    if (threadIdx.x == 64)
+        bulk_wait_group0();
+    tc_fence_before();
+    cluster_sync(); // no CTA leaves while its pair may still signal its barriers
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, C::kTmemCols);
     }
 }
 
@@ -721,6 +1035,41 @@ cudaError_t launch_bn(const LinearPlan &pl, const uint8_t *a_codes, const uint8_
     return cudaGetLastError();
 }
 
+cudaError_t launch_pair(const LinearPlan &pl, const uint8_t *a_codes, const uint8_t *a_sf,
+                        const uint8_t *w_codes, const uint8_t *w_sf, int64_t M, int64_t N,
+                        int64_t K, GemmParams gp, cudaStream_t s, nvfp4_status *st)
+{
+    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
+    if (!encode_fn() || !make_codes_map(&tmA, a_codes, M, K, 128) ||
+        !make_codes_map(&tmB, w_codes, N, K, 128) || !make_sf_map(&tmSFA, a_sf, M, K, 1) ||
+        !make_sf_map(&tmSFB, w_sf, N, K, 2) || !make_out_map(&tmY, gp.y, M, N)) {
+        *st = NVFP4_ERR_CUDA;
+        return cudaErrorInvalidValue;
+    }
+    static std::once_flag flags[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaError_t attr_err = cudaSuccess;
+    std::call_once(flags[dev & 63], [&]() {
+        attr_err = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        Pair::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return attr_err;
+    gp.tiles_a = (M + 255) / 256;
+    gp.tiles_b = (N + 255) / 256;
+    gp.units = gp.tiles_a * gp.tiles_b;
+    int64_t clusters = num_sms() / 2;
+    if (clusters > gp.units)
+        clusters = gp.units;
+    if (clusters < 1)
+        clusters = 1;
+    nvfp4_gemm_pair_kernel<<<(unsigned)(2 * clusters), kThreads, Pair::kSmemBytes, s>>>(
+        tmA, tmB, tmSFA, tmSFB, tmY, gp);
+    return cudaGetLastError();
+}
+
 } // namespace
 
 LinearPlan plan_linear(int64_t M, int64_t N, int64_t K)
@@ -785,6 +1134,9 @@ cudaError_t launch_linear(const LinearPlan &pl, const uint8_t *a_codes, const ui
     const uint8_t *cb = pl.swap_ab ? a_codes : w_codes;
     const uint8_t *sb = pl.swap_ab ? a_sf : w_sf;
     cudaError_t e;
+    if (!pl.swap_ab && pl.splits == 1 && out_bf16 && N % 8 == 0 &&
+        (reinterpret_cast<uintptr_t>(y) & 15u) == 0 && kUsePairKernel)
+        return launch_pair(pl, a_codes, a_sf, w_codes, w_sf, M, N, K, gp, s, st);
     switch (pl.bn) {
     case 8: e = launch_bn<8>(pl, ca, sa, cb, sb, K, gp, s, st); break;
     case 16: e = launch_bn<16>(pl, ca, sa, cb, sb, K, gp, s, st); break;

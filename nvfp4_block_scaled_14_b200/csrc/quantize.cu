@@ -13,13 +13,13 @@
 //                 reduces max |x| with SIMD integer max on the magnitude bits (exact,
 //                 order-free); one partial per CTA, no atomics, nothing to zero.
 //   encode_kernel -- one CTA per SM owns a contiguous range of rows; each warp takes a
-//                 32-block run of one row (512 values, fully coalesced), one 16-value block per
+//                 64-block run of one row (1024 values, fully coalesced), two 16-value blocks per
 //                 lane. It loads its first items before griddepcontrol.wait, so the loads
 //                 overlap the amax kernel's tail (the tensor is then mostly in L2), reduces the
 //                 partial maxima to the global scale, and fills a 128-entry table of
 //                 1 / (E4M3(c) * sg). Per block: block amax, E4M3 scale, E2M1 codes by the
-//                 hardware cvt, an 8-byte code store (a warp writes 256 contiguous bytes) and
-//                 byte stores of the swizzled and / or linear scales; atom padding is zeroed.
+//                 hardware cvt, a 16-byte code store (a warp writes 512 contiguous bytes) and
+//                 16-bit stores of the swizzled and / or linear scales; atom padding is zeroed.
 // Code-deciding arithmetic is IEEE fp32 round-to-nearest in a fixed order (__fdiv_rn,
 // __fmul_rn, __frcp_rn): sg = amax / 2688, sb = E4M3(bmax / (sg * 6)),
 // code = E2M1(x * (1 / (sb * sg))).
@@ -237,7 +237,7 @@ struct QuantArgs {
     float *global_scale;
     const float *partials; // one max |x| per amax CTA (dynamic amax)
     int npartials;
-    uint32_t chunks_magic; // ceil(2^32 / chunks) for chunks >= 2: item / chunks by umulhi
+    uint32_t chunks_magic; // ceil(2^32 / runs) for runs >= 2: item / runs by umulhi
 };
 
 __device__ __forceinline__ void pdl_launch_dependents()
@@ -311,51 +311,60 @@ __global__ void __launch_bounds__(kAmaxThreads, 1)
     }
 }
 
-// K2: encode. Each CTA owns a contiguous range of rows; each warp takes a 32-block run of
-// one row (one 16-value block per lane). The first items are loaded before waiting on the
-// amax kernel (programmatic dependent launch), so the loads overlap its tail.
+// K2: encode. Each CTA owns a contiguous range of rows; each warp takes a 64-block run of one
+// row and each lane two adjacent 16-value blocks, so address arithmetic and loop control are
+// shared by two blocks, the codes leave as one 16-byte store and the two scale bytes as one
+// 16-bit store. The first item is loaded before waiting on the amax kernel (programmatic
+// dependent launch), so the loads overlap its tail; later items are double-buffered.
 template <int SRC>
 __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
 {
     __shared__ float s_sg;
     __shared__ float s_rcp[128];
     constexpr int kBlkBytes = 16 * Src<SRC>::kBytes;
+    constexpr int V = kVecs<SRC>; // 16-byte vectors per block
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nb = a.cols >> 4;        // blocks per row
-    const int chunks = (nb + 31) >> 5; // 32-block runs per row (one per warp item)
-    const int apb = (nb + 3) >> 2;     // scale atoms per 128-row band
+    const int nb = a.cols >> 4;       // blocks per row
+    const int runs = (nb + 63) >> 6;  // 64-block runs per row (one per warp item)
+    const int apb = (nb + 3) >> 2;    // scale atoms per 128-row band
     const int64_t row_bytes = (int64_t)a.cols * Src<SRC>::kBytes;
     const int r0 = (int)((int64_t)a.rows * blockIdx.x / gridDim.x);
     const int r1 = (int)((int64_t)a.rows * (blockIdx.x + 1) / gridDim.x);
-    const int items = (r1 - r0) * chunks;
+    const int items = (r1 - r0) * runs;
     const uint8_t *xbase = a.x + (int64_t)r0 * row_bytes;
 
-    // item -> (row offset, block). The quotient by multiply-high is exact or one too large
-    // (item < 2^31, chunks < 2^27); one correction.
-    auto item_rb = [&](int it, int &ro, int &blk) {
-        if (chunks == 1) {
+    // item -> (row offset, first block of this lane). The quotient by multiply-high is exact
+    // or one too large (item < 2^31, runs < 2^26); one correction.
+    auto item_rb = [&](int it, int &ro, int &b0) {
+        if (runs == 1) {
             ro = it;
-            blk = lane;
+            b0 = 2 * lane;
             return;
         }
         ro = (int)__umulhi((uint32_t)it, a.chunks_magic);
-        if (ro * chunks > it)
+        if (ro * runs > it)
             --ro;
-        blk = (it - ro * chunks) * 32 + lane;
+        b0 = (it - ro * runs) * 64 + 2 * lane;
     };
-    auto load_item = [&](int it, uint4 (&r)[4], int &ro, int &blk) {
-        item_rb(it, ro, blk);
-        if (it < items && blk < nb)
-            load_raw<SRC>(xbase + (int64_t)ro * row_bytes + blk * kBlkBytes, r);
+    // the lane's two blocks are contiguous in memory: 2 * V vectors
+    auto load_item = [&](int it, uint4 (&r)[8], int &ro, int &b0) {
+        item_rb(it, ro, b0);
+        if (it < items && b0 < nb) {
+            const uint4 *q =
+                reinterpret_cast<const uint4 *>(xbase + (int64_t)ro * row_bytes + b0 * kBlkBytes);
+            const int nv = b0 + 1 < nb ? 2 * V : V;
+#pragma unroll
+            for (int v = 0; v < 2 * V; ++v)
+                if (v < nv)
+                    r[v] = ldg_stream(q + v);
+        }
     };
 
-    // first two items of this warp: loaded before the dependency wait
     int it = warp;
-    uint4 r[2][4];
-    int ro[2], blk[2];
-    load_item(it, r[0], ro[0], blk[0]);
-    load_item(it + 32, r[1], ro[1], blk[1]);
+    uint4 ra[8], rb[8];
+    int roa, b0a, rob, b0b;
+    load_item(it, ra, roa, b0a);
 
     const float s8 = (SRC == kSrcE4M3 && a.fp8_scale) ? *a.fp8_scale : 1.0f;
     if (!a.static_amax)
@@ -388,39 +397,57 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
         s_rcp[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
     __syncthreads();
 
-    // valid block: codes + scales; atom padding block (nb <= blk < 4 * apb): zero scale
-    auto encode_store = [&](int rowo, int b, const uint4 (&rr)[4]) {
-        const int row = r0 + rowo;
-        uint32_t sb = 0;
-        if (b < nb) {
-            uint2 packed;
-            sb = encode_block<SRC>(rr, s8, sg, t, rt, s_rcp, packed);
-            *reinterpret_cast<uint2 *>(a.codes + (int64_t)row * (a.cols >> 1) + b * 8) = packed;
-            if (a.sf_lin)
-                a.sf_lin[(int64_t)row * nb + b] = (uint8_t)sb;
+    // blocks b0, b0 + 1 of row r0 + ro: codes, scales; atom padding blocks get zero scales
+    auto encode_store = [&](int ro, int b0, const uint4 (&r)[8]) {
+        const int row = r0 + ro;
+        uint32_t sb0 = 0, sb1 = 0;
+        uint2 p0 = make_uint2(0u, 0u), p1 = make_uint2(0u, 0u);
+        if (b0 < nb) {
+            uint4 x0[4], x1[4];
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                x0[v] = r[v];
+                x1[v] = r[V + v];
+            }
+            sb0 = encode_block<SRC>(x0, s8, sg, t, rt, s_rcp, p0);
+            uint8_t *c = a.codes + (int64_t)row * (a.cols >> 1) + b0 * 8;
+            if (b0 + 1 < nb) {
+                sb1 = encode_block<SRC>(x1, s8, sg, t, rt, s_rcp, p1);
+                *reinterpret_cast<uint4 *>(c) = make_uint4(p0.x, p0.y, p1.x, p1.y);
+            } else {
+                *reinterpret_cast<uint2 *>(c) = p0;
+            }
+            if (a.sf_lin) {
+                uint8_t *l = a.sf_lin + (int64_t)row * nb + b0;
+                if (b0 + 1 < nb)
+                    *reinterpret_cast<uint16_t *>(l) = (uint16_t)(sb0 | (sb1 << 8));
+                else
+                    *l = (uint8_t)sb0;
+            }
         }
-        if (a.sf_swz && b < 4 * apb)
-            a.sf_swz[((int64_t)(row >> 7) * apb + (b >> 2)) * 512 + ((row & 31) << 4) +
-                     (((row >> 5) & 3) << 2) + (b & 3)] = (uint8_t)sb;
+        if (a.sf_swz && b0 < 4 * apb) // b0 even: both bytes in one atom, adjacent
+            *reinterpret_cast<uint16_t *>(
+                a.sf_swz + ((int64_t)(row >> 7) * apb + (b0 >> 2)) * 512 + ((row & 31) << 4) +
+                (((row >> 5) & 3) << 2) + (b0 & 3)) = (uint16_t)(sb0 | (sb1 << 8));
     };
-    while (it < items) {
-        // two items in flight: encode the loaded pair, then load the next pair
-        uint4 n[2][4];
-        int nro[2], nblk[2];
-        load_item(it + 64, n[0], nro[0], nblk[0]);
-        load_item(it + 96, n[1], nro[1], nblk[1]);
-        encode_store(ro[0], blk[0], r[0]);
-        if (it + 32 < items)
-            encode_store(ro[1], blk[1], r[1]);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-                r[u][v] = n[u][v];
-            ro[u] = nro[u];
-            blk[u] = nblk[u];
+    if constexpr (SRC == kSrcF32) {
+        // fp32 blocks are 64 bytes: one item in flight keeps the registers in budget
+        while (it < items) {
+            encode_store(roa, b0a, ra);
+            it += 32;
+            load_item(it, ra, roa, b0a);
         }
-        it += 64;
+    } else {
+        while (it < items) {
+            load_item(it + 32, rb, rob, b0b);
+            encode_store(roa, b0a, ra);
+            it += 32;
+            if (it >= items)
+                break;
+            load_item(it + 32, ra, roa, b0a);
+            encode_store(rob, b0b, rb);
+            it += 32;
+        }
     }
     // zero the scale padding rows of the last 128-row band
     if (a.sf_swz) {
@@ -449,8 +476,8 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
     qa.sf_lin = sf_lin;
     qa.global_scale = global_scale;
     qa.partials = reinterpret_cast<const float *>(ws);
-    const uint64_t chunks = (uint64_t)((cols / 16 + 31) / 32);
-    qa.chunks_magic = chunks > 1 ? (uint32_t)((((uint64_t)1 << 32) + chunks - 1) / chunks) : 0u;
+    const uint64_t runs = (uint64_t)((cols / 16 + 63) / 64);
+    qa.chunks_magic = runs > 1 ? (uint32_t)((((uint64_t)1 << 32) + runs - 1) / runs) : 0u;
     cudaError_t e;
     if (!static_amax) {
         const int64_t nbytes = rows * cols * Src<SRC>::kBytes;

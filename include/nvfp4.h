@@ -135,6 +135,30 @@ nvfp4_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales_swz, c
                           int64_t M, int64_t N, int64_t K, nvfp4_dtype out_dt, void *y, void *ws,
                           size_t ws_bytes, cudaStream_t stream);
 
+/* Flags of nvfp4_linear_ex (bitwise or). */
+typedef enum {
+    NVFP4_LINEAR_DEFAULT = 0,
+    /* The weight operand (w_codes, w_scales_swz, w_gs) is resident: nothing that may still be
+     * running on the stream when this call's kernel starts writes it (model weights loaded or
+     * quantized ahead of time and only read since). The small-M (M <= 128) kernel then starts
+     * reading W while the previous kernel of the stream is still finishing (programmatic
+     * dependent launch), so consecutive decode-size layers stream weights back to back; the
+     * activations, the global scales' product and y still wait for that kernel. Ignored for
+     * M > 128. Results are identical with and without the flag. */
+    NVFP4_LINEAR_RESIDENT_WEIGHTS = 1
+} nvfp4_linear_flags;
+
+/*
+ * nvfp4_linear with flags (nvfp4_linear_flags). No counterpart in the paper: the flag is a
+ * scheduling hint about the caller's stream, the result is the one nvfp4_linear defines.
+ * An unknown flag bit gives NVFP4_ERR_INVALID_ARG.
+ */
+nvfp4_status nvfp4_linear_ex(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                             const float *a_gs, const uint8_t *w_codes,
+                             const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
+                             int64_t N, int64_t K, nvfp4_dtype out_dt, void *y, void *ws,
+                             size_t ws_bytes, uint32_t flags, cudaStream_t stream);
+
 /*
  * nvfp4_linear without a caller-supplied workspace. No counterpart in the paper: it exists for
  * callers that cannot call cudaMalloc or lend a device buffer, e.g. code that runs inside an

@@ -17,8 +17,9 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_OP_CALIB_BF16, NVFP4_OP_CALIB_F32,
-                   NVFP4_OP_LINEAR, NVFP4_OP_QUANTIZE, NVFP4Error, check, load)
+from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_LINEAR_DEFAULT, NVFP4_LINEAR_RESIDENT_WEIGHTS,
+                   NVFP4_OP_CALIB_BF16, NVFP4_OP_CALIB_F32, NVFP4_OP_LINEAR, NVFP4_OP_QUANTIZE,
+                   NVFP4Error, check, load)
 
 __all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "dequantize", "linear",
            "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
@@ -135,8 +136,11 @@ def dequantize(q: NVFP4Tensor, out_dtype=torch.float32) -> torch.Tensor:
 
 
 def linear(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
-           out: torch.Tensor = None) -> torch.Tensor:
-    """Y = dequant(a) . dequant(w)^T, [a.rows x w.rows], fp32 accumulation."""
+           out: torch.Tensor = None, resident_weights: bool = False) -> torch.Tensor:
+    """Y = dequant(a) . dequant(w)^T, [a.rows x w.rows], fp32 accumulation.
+
+    resident_weights: w is not written by work still running on the stream (weights quantized
+    ahead of time); lets small-M calls start reading w before the previous kernel finishes."""
     if a.cols != w.cols:
         raise ValueError("K mismatch")
     M, N, K = a.rows, w.rows, a.cols
@@ -147,10 +151,11 @@ def linear(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
     ws_bytes = L.nvfp4_workspace_bytes(NVFP4_OP_LINEAR, M, N, K)
     ws = _workspace(dev, ws_bytes)
     dt = NVFP4_F32 if out.dtype == torch.float32 else NVFP4_BF16
-    st = L.nvfp4_linear(_ptr(a.codes), _ptr(a.scales_swz), _ptr(a.global_scale), _ptr(w.codes),
-                        _ptr(w.scales_swz), _ptr(w.global_scale), M, N, K, dt, _ptr(out),
-                        _ptr(ws), ws_bytes, _stream(dev))
-    check(st, "nvfp4_linear")
+    flags = NVFP4_LINEAR_RESIDENT_WEIGHTS if resident_weights else NVFP4_LINEAR_DEFAULT
+    st = L.nvfp4_linear_ex(_ptr(a.codes), _ptr(a.scales_swz), _ptr(a.global_scale),
+                           _ptr(w.codes), _ptr(w.scales_swz), _ptr(w.global_scale), M, N, K, dt,
+                           _ptr(out), _ptr(ws), ws_bytes, flags, _stream(dev))
+    check(st, "nvfp4_linear_ex")
     return out
 
 

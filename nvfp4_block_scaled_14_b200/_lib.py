@@ -23,6 +23,9 @@ NVFP4_ERR_UNSUPPORTED = 7
 NVFP4_F32 = 0
 NVFP4_BF16 = 1
 
+NVFP4_LINEAR_DEFAULT = 0
+NVFP4_LINEAR_RESIDENT_WEIGHTS = 1
+
 NVFP4_OP_QUANTIZE = 0
 NVFP4_OP_LINEAR = 1
 NVFP4_OP_CALIB_BF16 = 2
@@ -47,6 +50,8 @@ _SIGNATURES = {
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _int, _vp, _vp], _int),
     "nvfp4_linear": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _sz, _vp],
                      _int),
+    "nvfp4_linear_ex": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _sz, _u32,
+                         _vp], _int),
     "nvfp4_linear_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp],
                              _int),
     "nvfp4_calib_percentile_amax": ([ctypes.POINTER(_vp), _int, _i64, _int, _u32, _u32, _vp,

@@ -212,6 +212,18 @@ nvfp4_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales_swz, c
                           int64_t M, int64_t N, int64_t K, nvfp4_dtype out_dt, void *y, void *ws,
                           size_t ws_bytes, cudaStream_t stream)
 {
+    return nvfp4_linear_ex(a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs, M, N, K,
+                           out_dt, y, ws, ws_bytes, 0u, stream);
+}
+
+nvfp4_status nvfp4_linear_ex(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                             const float *a_gs, const uint8_t *w_codes,
+                             const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
+                             int64_t N, int64_t K, nvfp4_dtype out_dt, void *y, void *ws,
+                             size_t ws_bytes, uint32_t flags, cudaStream_t stream)
+{
+    if (flags & ~(uint32_t)NVFP4_LINEAR_RESIDENT_WEIGHTS)
+        return NVFP4_ERR_INVALID_ARG;
     if (M < 0 || N < 0 || K < 0 || M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || K % 32 != 0)
         return NVFP4_ERR_SHAPE;
     if (out_dt != NVFP4_F32 && out_dt != NVFP4_BF16)
@@ -232,12 +244,12 @@ nvfp4_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales_swz, c
         !aligned16(w_scales_swz) || !aligned16(y) || !aligned16(ws) ||
         (reinterpret_cast<uintptr_t>(a_gs) & 3u) || (reinterpret_cast<uintptr_t>(w_gs) & 3u))
         return NVFP4_ERR_ALIGNMENT;
-    const LinearPlan pl = plan_linear(M, N, K);
+    const LinearPlan pl = plan_linear(M, N, K, flags);
     if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes))
         return NVFP4_ERR_WORKSPACE;
     st = NVFP4_OK;
     cudaError_t e = launch_linear(pl, a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs,
-                                  M, N, K, out_dt == NVFP4_BF16, y, ws, stream, &st);
+                                  M, N, K, out_dt == NVFP4_BF16, y, ws, flags, stream, &st);
     if (st != NVFP4_OK)
         return st;
     return map_cuda(e);

@@ -23,10 +23,12 @@
 //               times alpha = sgA * sgW, cast to bf16 and held in registers; the accumulator
 //               is released to the MMA warp before the global stores, so the stores overlap
 //               the next tile's mainloop. (fp32 outputs / split-K partials store chunk-wise.)
-// Small M (<= 128) runs swap-AB: the weights take the MMA's M side (128 rows of W per tile)
-// and the activation rows the N side (8..128), so the tensor cores stream the weight matrix
-// at full width; with few tiles the K range is split over CTAs and a second kernel adds the
-// fp32 partials in split order (deterministic).
+// Large M with few tiles splits K over CTAs of this kernel and a second kernel adds the fp32
+// partials in split order (deterministic).
+// Small M (<= 128) runs swap-AB in its own kernel (nvfp4_gemm_smallm_kernel): the weights take
+// the MMA's M side (128 rows of W per tile) and the activation rows the N side (8..128), so
+// the tensor cores stream the weight matrix at full width; K is split over a thread-block
+// cluster and the partials are summed through distributed shared memory.
 // Every wait is bounded; a wait that gives up records NVFP4_ERR_TIMEOUT in the library's
 // status word, lets the CTA drain its in-flight copies / MMAs, frees TMEM and returns.
 // No TMA multicast is used.
@@ -51,8 +53,9 @@ constexpr uint32_t kWaitLimit = 1u << 20;
 #endif
 constexpr bool kUsePairKernel = NVFP4_PAIR_KERNEL != 0;
 
-template <int BN> struct Cfg {
-    static constexpr int kStages = BN == 256 ? NVFP4_STAGES_256 : (BN == 128 ? 6 : 7);
+// Shared-memory / TMEM layout of the 1-SM kernels for a B tile of BN rows and STAGES stages.
+template <int BN, int STAGES = (BN == 256 ? NVFP4_STAGES_256 : (BN == 128 ? 6 : 7))> struct Cfg {
+    static constexpr int kStages = STAGES;
     static constexpr int kSfbBands = BN > 128 ? 2 : 1;
     static constexpr int kABytes = BM * 128;
     static constexpr int kBBytes = BN * 128;
@@ -933,6 +936,395 @@ __global__ void splitk_reduce_kernel(const float *__restrict__ partial, int spli
 }
 
 // ---------------------------------------------------------------------------------------
+// Small M (<= 128, swap-AB): one 128-row tile of W per thread-block cluster, its K range
+// split over the cluster's csplit CTAs. Each CTA streams its share of k-tiles through the
+// same warp-specialized pipeline as the persistent kernel (TMA producer, scale-factor
+// feeders, MMA issuer, epilogue), sized so that two CTAs fit on an SM. CTAs 1.. stage their
+// fp32 partial accumulators in their own (drained) shared memory; the leader (rank 0) adds
+// them to its own in rank order through distributed shared memory, scales and stores. So
+// every SM streams weights, with no workspace and no second kernel, and the sum order is
+// fixed. The kernel takes part in programmatic dependent launch: its set-up overlaps the
+// previous kernel of the stream, its global reads and writes wait for that kernel.
+// ---------------------------------------------------------------------------------------
+
+template <int BN> struct SmallCfg {
+    // stages that keep one CTA at <= 113 KB of shared memory (two per SM)
+    static constexpr int kStages = BN <= 16 ? 5 : BN <= 64 ? 4 : 3;
+    using L = Cfg<BN, kStages>;
+    static_assert(L::kSmemBytes <= 115712, "two CTAs per SM");
+    static_assert(L::kTmemCols <= 256, "two CTAs per SM");
+    // partial accumulators of a non-leader CTA, [BN][128] fp32, over the drained stages
+    static_assert(BN * 128 * 4 + BN * 128 * 2 <= L::kOffSfa,
+                  "partials and bf16 output staging fit in the operand stages");
+};
+
+struct SmallParams {
+    int64_t rows_a, rows_b; // weight rows (N), activation rows (M)
+    int kt_total;           // 256-wide k-tiles
+    int csplit;             // CTAs per cluster = K splits
+    const float *a_gs, *w_gs;
+    void *y;
+    int64_t ldy; // = N
+    int out_bf16;
+    int tma_store;  // 1: each CTA stages its slice of the output tile, one TMA store writes it
+    int resident_w; // 1: W is not written by earlier work still running on the stream, so
+                    // its first stages load before the programmatic-launch wait
+    int *status;
+};
+
+// Output rows [rank*BN/CS, (rank+1)*BN/CS) of the tile, summed over the CS partials of the
+// cluster in rank order (the same order on every CTA), scaled, cast and stored. Thread t owns
+// output column n = 128*ta + t. Remote loads are issued in batches of up to 32 so that one
+// distributed-shared-memory round trip serves a batch. bf16 results are staged after the
+// partials, fp32 results overwrite this CTA's own slice rows (each thread rewrites exactly the
+// elements it read; peers never read this CTA's slice), then one TMA store writes the
+// [BN/CS x 128] box (clipped at M and N). With CS > 1 the caller waits on the cluster barrier
+// this function arrives on once its remote reads are done, before the CTA may exit.
+template <int BN, int CS>
+__device__ __forceinline__ void reduce_slice(const SmallParams &p, uint8_t *smem, uint32_t rank,
+                                             int t, int64_t ta, float alpha,
+                                             const CUtensorMap *tmY)
+{
+    constexpr int SR = BN / CS;                         // output rows of this CTA
+    constexpr int RB = (32 / CS) < SR ? (32 / CS) : SR; // rows per batch
+    static_assert(BN % CS == 0 && SR % RB == 0, "slice shape");
+    const int m0 = (int)rank * SR;
+    const uint32_t col = smem_u32(smem) + (uint32_t)t * 4u;
+    uint32_t src[CS];
+#pragma unroll
+    for (int j = 0; j < CS; ++j)
+        src[j] = CS == 1 ? col : mapa_shared(col, (uint32_t)j);
+    float *part = reinterpret_cast<float *>(smem);
+    __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(smem + BN * BM * 4);
+    const int64_t n = ta * BM + t;
+#pragma unroll 1
+    for (int mb = 0; mb < SR; mb += RB) {
+        float v[RB][CS];
+#pragma unroll
+        for (int rr = 0; rr < RB; ++rr) {
+            const uint32_t off = (uint32_t)(m0 + mb + rr) * (BM * 4);
+#pragma unroll
+            for (int j = 0; j < CS; ++j) {
+                if constexpr (CS == 1)
+                    v[rr][j] = part[(m0 + mb + rr) * BM + t];
+                else
+                    v[rr][j] = ld_shared_cluster_f32(src[j] + off);
+            }
+        }
+#pragma unroll
+        for (int rr = 0; rr < RB; ++rr) {
+            float acc = v[rr][0];
+#pragma unroll
+            for (int j = 1; j < CS; ++j)
+                acc += v[rr][j];
+            const float r = acc * alpha;
+            const int m = m0 + mb + rr;
+            if (p.tma_store) {
+                if (p.out_bf16)
+                    ob[(mb + rr) * BM + t] = __float2bfloat16_rn(r);
+                else
+                    part[m * BM + t] = r;
+            } else if (m < p.rows_b && n < p.rows_a) {
+                if (p.out_bf16)
+                    reinterpret_cast<__nv_bfloat16 *>(p.y)[m * p.ldy + n] = __float2bfloat16_rn(r);
+                else
+                    reinterpret_cast<float *>(p.y)[m * p.ldy + n] = r;
+            }
+        }
+    }
+    if constexpr (CS > 1) {
+        __syncwarp();
+        cluster_arrive(); // done reading the other CTAs' partials (waited on before exit)
+    }
+    if (p.tma_store) {
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (t == 0 && m0 < p.rows_b) {
+            const void *src_tile = p.out_bf16 ? static_cast<const void *>(ob)
+                                              : static_cast<const void *>(part + m0 * BM);
+            tma_store_2d(tmY, src_tile, (int)(ta * BM), m0);
+            bulk_commit_group();
+            bulk_wait_group_read0(); // shared memory is read before the CTA may exit
+        }
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 2)
+    nvfp4_gemm_smallm_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmSFA,
+                             const __grid_constant__ CUtensorMap tmSFB,
+                             const __grid_constant__ CUtensorMap tmY, const SmallParams p)
+{
+    using C = typename SmallCfg<BN>::L;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((smem_u32(smem) & 1023u) != 0) { // same for every CTA: the whole grid returns here
+        if (threadIdx.x == 0)
+            atomicExch(p.status, (int)NVFP4_ERR_CUDA);
+        return;
+    }
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint64_t *empty_bar = full_bar + C::kStages;
+    uint64_t *sf_full = empty_bar + C::kStages;
+    uint64_t *sf_empty = sf_full + C::kSfSlots;
+    uint64_t *acc_full = sf_empty + C::kSfSlots;
+    uint64_t *drain_bar = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int cs = p.csplit;
+    const uint32_t rank = cs > 1 ? cluster_ctarank() : 0u;
+    const int64_t ta = blockIdx.x / cs;
+    const int k0 = (int)((int64_t)rank * p.kt_total / cs);
+    const int k1 = (int)((int64_t)(rank + 1) * p.kt_total / cs);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int s = 0; s < C::kSfSlots; ++s) {
+            mbar_init(&sf_full[s], 4);
+            mbar_init(&sf_empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    if (cs > 1)
+        cluster_sync(); // barriers initialised cluster-wide before any remote arrival
+    else
+        __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // Every CTA holds its TMEM by now, so a dependent grid's CTAs never take columns this
+    // grid still has to allocate.
+    pdl_launch_dependents();
+    float alpha = 0.0f; // sgA * sgW, read by the epilogue warps
+
+    if (warp == 0) {
+        // ------------------------------- TMA producer -------------------------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmSFA);
+            tma_prefetch_desc(&tmSFB);
+            // Resident weights: the first stages' W tiles and scales are requested while the
+            // previous kernel may still run (the stages start out free); the activations
+            // always wait for it.
+            const int pre = p.resident_w ? min(k1 - k0, C::kStages) : 0;
+            for (int i = 0; i < pre; ++i) {
+                mbar_arrive_expect_tx(&full_bar[i], C::kTx);
+                tma_load_2d(smem + i * C::kABytes, &tmA, &full_bar[i], (k0 + i) * 128,
+                            (int)(ta * BM));
+                tma_load_3d(smem + C::kOffSfa + i * C::kSfaBytes, &tmSFA, &full_bar[i], 0,
+                            (k0 + i) * 4, (int)ta);
+            }
+            pdl_wait(); // operands may come from the previous kernel
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int kt = k0; kt < k1; ++kt) {
+                uint8_t *sa = smem + stage * C::kABytes;
+                uint8_t *sb = smem + C::kOffB + stage * C::kBBytes;
+                uint8_t *ssfa = smem + C::kOffSfa + stage * C::kSfaBytes;
+                uint8_t *ssfb = smem + C::kOffSfb + stage * C::kSfbBytes;
+                if (kt - k0 >= pre) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimit)) {
+                        set_timeout(p.status);
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full_bar[stage], C::kTx);
+                    tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, (int)(ta * BM));
+                    tma_load_3d(ssfa, &tmSFA, &full_bar[stage], 0, kt * 4, (int)ta);
+                }
+                tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, 0);
+                tma_load_3d(ssfb, &tmSFB, &full_bar[stage], 0, kt * 4, 0);
+                ++issued;
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            // every copy issued has landed before the CTA may exit
+            int s = stage;
+            uint32_t ph = phase;
+            const int last = issued < C::kStages ? issued : C::kStages;
+            for (int i = 0; i < last; ++i) {
+                if (--s < 0) {
+                    s = C::kStages - 1;
+                    ph ^= 1;
+                }
+                if (!mbar_wait(&full_bar[s], ph, kWaitLimit))
+                    set_timeout(p.status);
+            }
+        }
+    } else if (warp >= 6) {
+        // ------------------------------- scale-factor feeders -----------------------
+        const int q = warp & 3;
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, sphase = 0;
+        for (int kt = k0; kt < k1; ++kt) {
+            if (!mbar_wait(&full_bar[stage], phase, kWaitLimit) ||
+                !mbar_wait(&sf_empty[slot], sphase ^ 1, kWaitLimit)) {
+                if (lane == 0)
+                    set_timeout(p.status);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t ssfa = smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes);
+            const uint32_t ssfb = smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes);
+            const uint32_t tslot =
+                tmem + ((uint32_t)(q * 32) << 16) + C::kSfCol + slot * C::kSlotCols;
+            uint32_t ra[16], rb[16];
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                const uint4 wa = lds128(ssfa + kb * 512 + lane * 16);
+                const uint4 wb = lds128(ssfb + kb * 512 + lane * 16);
+                ra[4 * kb] = wa.x;
+                ra[4 * kb + 1] = wa.y;
+                ra[4 * kb + 2] = wa.z;
+                ra[4 * kb + 3] = wa.w;
+                rb[4 * kb] = wb.x;
+                rb[4 * kb + 1] = wb.y;
+                rb[4 * kb + 2] = wb.z;
+                rb[4 * kb + 3] = wb.w;
+            }
+            tmem_st_32x32b_x16(tslot, ra);
+            tmem_st_32x32b_x16(tslot + 16, rb);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sf_full[slot]);
+            if (++stage == C::kStages) {
+                stage = 0;
+                phase ^= 1;
+            }
+            if (++slot == C::kSfSlots) {
+                slot = 0;
+                sphase ^= 1;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer ---------------------------------
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, sphase = 0;
+        bool ok = true;
+        for (int kt = k0; kt < k1; ++kt) {
+            if (!mbar_wait(&full_bar[stage], phase, kWaitLimit) ||
+                !mbar_wait(&sf_full[slot], sphase, kWaitLimit)) {
+                if (lane == 0)
+                    set_timeout(p.status);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t tsfa = tmem + C::kSfCol + slot * C::kSlotCols;
+                const uint64_t adesc = smem_desc(smem_u32(smem + stage * C::kABytes), 16, 1024,
+                                                 kLayoutSwizzle128B);
+                const uint64_t bdesc = smem_desc(smem_u32(smem + C::kOffB + stage * C::kBBytes),
+                                                 16, 1024, kLayoutSwizzle128B);
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb)
+                    tc_mma_nvf4(tmem, adesc + (uint64_t)(2 * kb), bdesc + (uint64_t)(2 * kb),
+                                C::kIdesc, tsfa + kb * 4, tsfa + 16 + kb * 4,
+                                (kt > k0 || kb > 0) ? 1u : 0u);
+                tc_commit(&empty_bar[stage]);
+                tc_commit(&sf_empty[slot]);
+            }
+            __syncwarp();
+            if (++stage == C::kStages) {
+                stage = 0;
+                phase ^= 1;
+            }
+            if (++slot == C::kSfSlots) {
+                slot = 0;
+                sphase ^= 1;
+            }
+        }
+        if (lane == 0) {
+            if (ok)
+                tc_commit(acc_full);
+            tc_commit(drain_bar); // every MMA issued completes before TMEM is freed
+            if (!mbar_wait(drain_bar, 0, kWaitLimit))
+                set_timeout(p.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------- epilogue (warps 2..5) ----------------------
+        // partial accumulator -> own shared memory, [BN][128] fp32 (row m of the output
+        // tile = accumulator column, 128 output columns n = TMEM lanes), over the drained
+        // operand stages
+        const int q = warp & 3;
+        const int t = q * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        constexpr int NC = BN < 32 ? BN : 32;
+        pdl_wait(); // global scales and y belong to the stream's earlier work
+        alpha = __fmul_rn(*p.a_gs, *p.w_gs);
+        const bool ok = mbar_wait(acc_full, 0, kWaitLimit);
+        if (!ok && lane == 0)
+            set_timeout(p.status);
+        tc_fence_after();
+        float *part = reinterpret_cast<float *>(smem);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += NC) {
+            uint32_t v[NC];
+            tmem_ld_cols<NC>(trow + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < NC; ++j)
+                part[(c0 + j) * BM + t] = (ok && k1 > k0) ? __uint_as_float(v[j]) : 0.0f;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    if (cs > 1)
+        cluster_sync(); // every CTA of the cluster has staged its partial
+    else
+        __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols); // the accumulator has been read
+    }
+    if (warp >= 2 && warp <= 5) {
+        const int t = (warp & 3) * 32 + lane;
+        switch (cs) {
+        case 1: reduce_slice<BN, 1>(p, smem, 0, t, ta, alpha, &tmY); break;
+        case 2: reduce_slice<BN, 2>(p, smem, rank, t, ta, alpha, &tmY); break;
+        case 4: reduce_slice<BN, 4>(p, smem, rank, t, ta, alpha, &tmY); break;
+        default: reduce_slice<BN, 8>(p, smem, rank, t, ta, alpha, &tmY); break;
+        }
+    } else if (cs > 1) {
+        __syncwarp();
+        cluster_arrive();
+    }
+    __syncwarp();
+    if (cs > 1)
+        cluster_wait(); // no CTA leaves while another may still read its partial
+}
+
+// Same threads and shared memory as nvfp4_gemm_smallm_kernel<BN> but no tensor memory. The
+// occupancy calculator counts a CTA that allocates tensor memory as filling its SM, while two
+// small-M CTAs (2 x 256 of the 512 columns) do run side by side; this kernel, never launched,
+// gives the calculator's count of resident clusters for that shape.
+template <int BN> __global__ void __launch_bounds__(kThreads, 2) smallm_occupancy_proxy(int *p)
+{
+    extern __shared__ uint8_t proxy_smem[];
+    if (p)
+        p[threadIdx.x] = proxy_smem[threadIdx.x];
+}
+
+// ---------------------------------------------------------------------------------------
 // Host side: tensor maps and launch
 // ---------------------------------------------------------------------------------------
 
@@ -993,6 +1385,22 @@ bool make_out_map(CUtensorMap *m, void *base, int64_t rows, int64_t cols)
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output Y [M x N] (bf16 or fp32) of the small-M kernel, box 128 columns x box_rows rows, no
+// swizzle: one CTA's staged slice of the output tile.
+bool make_out_map_swap(CUtensorMap *m, void *base, int64_t rows, int64_t cols, int bf16,
+                       int box_rows)
+{
+    const cuuint64_t esz = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * esz};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return encode_fn()(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                       2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1070,9 +1478,126 @@ cudaError_t launch_pair(const LinearPlan &pl, const uint8_t *a_codes, const uint
     return cudaGetLastError();
 }
 
+template <int BN> cudaError_t smallm_set_smem_attr()
+{
+    static std::once_flag flags[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaError_t e = cudaSuccess;
+    std::call_once(flags[dev & 63], [&]() {
+        e = cudaFuncSetAttribute(nvfp4_gemm_smallm_kernel<BN>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SmallCfg<BN>::L::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(smallm_occupancy_proxy<BN>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SmallCfg<BN>::L::kSmemBytes);
+    });
+    return e;
+}
+
+// Clusters of cs CTAs of the small-M kernel that can be resident at once on this device.
+template <int BN> int smallm_max_clusters(int cs)
+{
+    if (smallm_set_smem_attr<BN>() != cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(cs * 1024), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = SmallCfg<BN>::L::kSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, smallm_occupancy_proxy<BN>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+constexpr int kMaxCsplit = 8; // portable cluster size
+
+// Resident clusters per cluster size 1..8 for each small-M tile width, per device.
+struct SmallOccupancy {
+    int clusters[5][kMaxCsplit + 1];
+};
+
+const SmallOccupancy &small_occupancy()
+{
+    static std::once_flag flags[64];
+    static SmallOccupancy occ[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    dev &= 63;
+    std::call_once(flags[dev], [&]() {
+        for (int cs = 1; cs <= kMaxCsplit; ++cs) {
+            occ[dev].clusters[0][cs] = smallm_max_clusters<8>(cs);
+            occ[dev].clusters[1][cs] = smallm_max_clusters<16>(cs);
+            occ[dev].clusters[2][cs] = smallm_max_clusters<32>(cs);
+            occ[dev].clusters[3][cs] = smallm_max_clusters<64>(cs);
+            occ[dev].clusters[4][cs] = smallm_max_clusters<128>(cs);
+        }
+    });
+    return occ[dev];
+}
+
+int bn_index(int bn) { return bn <= 8 ? 0 : bn <= 16 ? 1 : bn <= 32 ? 2 : bn <= 64 ? 3 : 4; }
+
+template <int BN>
+cudaError_t launch_smallm(const LinearPlan &pl, const uint8_t *w_codes, const uint8_t *w_sf,
+                          const uint8_t *a_codes, const uint8_t *a_sf, int64_t K,
+                          const SmallParams &sp, cudaStream_t s, nvfp4_status *st)
+{
+    using C = typename SmallCfg<BN>::L;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
+    memset(&tmY, 0, sizeof(tmY));
+    SmallParams spl = sp;
+    spl.tma_store = 0;
+    const int64_t esz = sp.out_bf16 ? 2 : 4;
+    if ((sp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(sp.y) & 15u) == 0 &&
+        encode_fn() && make_out_map_swap(&tmY, sp.y, pl.rows_b, sp.ldy, sp.out_bf16, BN / pl.csplit))
+        spl.tma_store = 1;
+    if (!encode_fn() || !make_codes_map(&tmA, w_codes, pl.rows_a, K, BM) ||
+        !make_codes_map(&tmB, a_codes, pl.rows_b, K, BN) ||
+        !make_sf_map(&tmSFA, w_sf, pl.rows_a, K, 1) ||
+        !make_sf_map(&tmSFB, a_sf, pl.rows_b, K, 1)) {
+        *st = NVFP4_ERR_CUDA;
+        return cudaErrorInvalidValue;
+    }
+    cudaError_t e = smallm_set_smem_attr<BN>();
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(pl.tiles_a * pl.csplit), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    int na = 0;
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (pl.csplit > 1) {
+        at[na].id = cudaLaunchAttributeClusterDimension;
+        at[na].val.clusterDim.x = (unsigned)pl.csplit;
+        at[na].val.clusterDim.y = 1;
+        at[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = at;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_smallm_kernel<BN>, tmA, tmB, tmSFA, tmSFB, tmY,
+                              spl);
+}
+
 } // namespace
 
-LinearPlan plan_linear(int64_t M, int64_t N, int64_t K)
+LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, unsigned flags)
 {
     LinearPlan p{};
     p.kt = (int)((K + 255) / 256);
@@ -1091,7 +1616,31 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K)
     p.tiles_b = (p.rows_b + p.bn - 1) / p.bn;
     p.splits = 1;
     p.kt_per_split = p.kt;
+    p.csplit = 0;
     const int64_t tiles = p.tiles_a * p.tiles_b;
+    if (p.swap_ab) {
+        // One wave of clusters: the largest K split (8, 4 or 2, at most the k-tiles; a power
+        // of two so that it divides the tile width) whose clusters of one tile each are all
+        // resident at once; shapes with more tiles than one wave of single CTAs go to the
+        // persistent kernel.
+        // The grid stays within 4/3 of the SM count: a few SMs run two CTAs, the rest keep a
+        // slot free for the next kernel's CTAs (they start streaming resident weights there).
+        // Measured on 8 x {6144, 12288, 18944} x 4096: more CTAs only lengthen the tail.
+        (void)flags;
+        const SmallOccupancy &occ = small_occupancy();
+        const int bi = bn_index(p.bn);
+        const int64_t max_ctas = (int64_t)num_sms() * 4 / 3;
+        for (int cs = kMaxCsplit; cs >= 1; cs /= 2) {
+            if (cs <= p.kt && tiles <= occ.clusters[bi][cs] && (cs == 1 || tiles * cs <= max_ctas)) {
+                p.csplit = cs;
+                break;
+            }
+        }
+        if (p.csplit > 0) {
+            p.ws_bytes = 0;
+            return p;
+        }
+    }
     const int sms = num_sms();
     if (tiles > 0 && p.kt > 1 && tiles * 2 <= sms) {
         int64_t sp = sms / tiles;
@@ -1109,7 +1658,7 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K)
 cudaError_t launch_linear(const LinearPlan &pl, const uint8_t *a_codes, const uint8_t *a_sf,
                           const float *a_gs, const uint8_t *w_codes, const uint8_t *w_sf,
                           const float *w_gs, int64_t M, int64_t N, int64_t K, int out_bf16,
-                          void *y, void *ws, cudaStream_t s, nvfp4_status *st)
+                          void *y, void *ws, unsigned flags, cudaStream_t s, nvfp4_status *st)
 {
     GemmParams gp{};
     gp.rows_a = pl.rows_a;
@@ -1134,6 +1683,27 @@ cudaError_t launch_linear(const LinearPlan &pl, const uint8_t *a_codes, const ui
     const uint8_t *cb = pl.swap_ab ? a_codes : w_codes;
     const uint8_t *sb = pl.swap_ab ? a_sf : w_sf;
     cudaError_t e;
+    if (pl.csplit > 0) {
+        SmallParams sp{};
+        sp.rows_a = pl.rows_a;
+        sp.rows_b = pl.rows_b;
+        sp.kt_total = pl.kt;
+        sp.csplit = pl.csplit;
+        sp.a_gs = a_gs;
+        sp.w_gs = w_gs;
+        sp.y = y;
+        sp.ldy = N;
+        sp.out_bf16 = out_bf16;
+        sp.resident_w = (flags & NVFP4_LINEAR_RESIDENT_WEIGHTS) ? 1 : 0;
+        sp.status = device_status_ptr();
+        switch (pl.bn) {
+        case 8: return launch_smallm<8>(pl, ca, sa, cb, sb, K, sp, s, st);
+        case 16: return launch_smallm<16>(pl, ca, sa, cb, sb, K, sp, s, st);
+        case 32: return launch_smallm<32>(pl, ca, sa, cb, sb, K, sp, s, st);
+        case 64: return launch_smallm<64>(pl, ca, sa, cb, sb, K, sp, s, st);
+        default: return launch_smallm<128>(pl, ca, sa, cb, sb, K, sp, s, st);
+        }
+    }
     if (!pl.swap_ab && pl.splits == 1 && out_bf16 && N % 8 == 0 &&
         (reinterpret_cast<uintptr_t>(y) & 15u) == 0 && kUsePairKernel)
         return launch_pair(pl, a_codes, a_sf, w_codes, w_sf, M, N, K, gp, s, st);

@@ -59,12 +59,15 @@ struct LinearPlan {
     int kt;             // k-tiles of 256 elements
     int splits;         // split-K factor (1 = no split)
     int kt_per_split;
+    int csplit;         // small M: K split over a thread-block cluster of csplit CTAs (0 = the
+                        // persistent kernel runs the shape)
     size_t ws_bytes;    // workspace for split-K partials
 };
-LinearPlan plan_linear(int64_t M, int64_t N, int64_t K);
+// flags: nvfp4_linear_flags (they change the small-M launch shape, never the workspace)
+LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, unsigned flags = 0);
 cudaError_t launch_linear(const LinearPlan &p, const uint8_t *a_codes, const uint8_t *a_sf,
                           const float *a_gs, const uint8_t *w_codes, const uint8_t *w_sf,
                           const float *w_gs, int64_t M, int64_t N, int64_t K, int out_bf16,
-                          void *y, void *ws, cudaStream_t s, nvfp4_status *st);
+                          void *y, void *ws, unsigned flags, cudaStream_t s, nvfp4_status *st);
 
 } // namespace nvfp4

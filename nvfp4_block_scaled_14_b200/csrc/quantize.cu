@@ -240,16 +240,6 @@ struct QuantArgs {
     uint32_t chunks_magic; // ceil(2^32 / runs) for runs >= 2: item / runs by umulhi
 };
 
-__device__ __forceinline__ void pdl_launch_dependents()
-{
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-__device__ __forceinline__ void pdl_wait()
-{
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
 // K1: max |x| over a contiguous byte range per CTA, streamed through a shared-memory ring
 // with 1-D bulk copies; one partial per CTA.
 template <int SRC>

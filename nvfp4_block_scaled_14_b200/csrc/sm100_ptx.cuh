@@ -414,6 +414,17 @@ __device__ __forceinline__ void cluster_sync()
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Split cluster barrier: arrive (releasing this thread's prior accesses) now, wait later.
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // TMA 2-D load into this CTA's shared memory whose completion is counted on the mbarrier
 // at `bar_cluster` (the leader CTA's barrier of the pair). No multicast.
 __device__ __forceinline__ void tma_load_2d_pair(void *dst, const void *desc, uint32_t bar_cluster,
@@ -474,6 +485,32 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar)
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
                  : "memory");
+}
+
+// 32-bit load from the shared memory of a CTA of the cluster (address from mapa_shared).
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------------------------------
+// Programmatic dependent launch
+// ---------------------------------------------------------------------------------------
+
+// Lets the next kernel of the stream (launched with programmatic stream serialization) start
+// its CTAs once every CTA of this grid has executed this or exited.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the grids this one depends on have completed and their writes are visible
+// (returns at once for a kernel launched without the attribute).
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t elect_one()

@@ -205,6 +205,9 @@ def test_linear_tiny_workload_fp32_out():
     (1, 384, 512), (5, 384, 512), (8, 384, 512), (16, 200, 320), (17, 256, 256),
     (33, 384, 512), (100, 384, 512), (128, 384, 512),   # small M: swap-AB
     (64, 1024, 2048),   # swap-AB, many k-tiles per split
+    # small M: K split over a thread-block cluster, partials summed through distributed
+    # shared memory (uneven k-ranges, odd cluster sizes, the widest B tile)
+    (8, 1536, 3072), (3, 640, 1792), (128, 2560, 1024), (64, 12288, 512), (1, 128, 4096),
 ])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_linear_matches_oracle(M, N, K, out):
@@ -216,6 +219,42 @@ def test_linear_matches_oracle(M, N, K, out):
     err = np.abs(y - ref)
     tol = gemm_tolerance(ref, out == "bf16")
     assert np.all(err <= tol), f"max err {err.max()} vs tol {np.max(tol)}"
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 1536, 3072), (1, 12288, 1024), (64, 640, 768),
+                                   (128, 256, 2048)])
+def test_linear_resident_weights_back_to_back(M, N, K):
+    # the resident-weights flag lets each small-M call start reading W while the previous
+    # call still runs; a chain of calls with different W (and the activations quantized just
+    # before the first) must give every call's own result
+    xa = W.to_bf16_bits(W.normal((M, K), 1.0, 30, M))
+    a_dev = dev_tensor(xa)
+    ws = [W.to_bf16_bits(W.normal((N, K), 0.02, 31, N + i)) for i in range(3)]
+    qws = [gpu_quantize(x) for x in ws]
+    torch.cuda.synchronize()
+    qa = nv.quantize(a_dev)  # the chain starts right behind the activation quantizer
+    ys = [nv.linear(qa, qw, resident_weights=True) for qw in qws for _ in range(2)]
+    torch.cuda.synchronize()
+    ra = O.quantize(xa)
+    for i, x in enumerate(ws):
+        ref = O.gemm(ra, O.quantize(x))
+        tol = gemm_tolerance(ref, True)
+        for y in ys[2 * i:2 * i + 2]:
+            assert np.all(np.abs(to_numpy_f64(y) - ref) <= tol), i
+    assert nv.sync_status() == 0
+
+
+def test_linear_rejects_unknown_flag():
+    from nvfp4_block_scaled_14_b200 import _lib as L
+    qa = gpu_quantize(W.to_bf16_bits(W.normal((4, 64), 1.0, 32, 0)))
+    y = torch.zeros((4, 4), dtype=torch.bfloat16, device="cuda")
+    st = L.load().nvfp4_linear_ex(qa.codes.data_ptr(), qa.scales_swz.data_ptr(),
+                                  qa.global_scale.data_ptr(), qa.codes.data_ptr(),
+                                  qa.scales_swz.data_ptr(), qa.global_scale.data_ptr(), 4, 4,
+                                  64, L.NVFP4_BF16, y.data_ptr(), None, 0, 2, None)
+    assert st == L.NVFP4_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert not y.float().abs().sum().item()
 
 
 def test_linear_exact_with_unit_scales():

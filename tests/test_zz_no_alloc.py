@@ -47,8 +47,8 @@ def _call_noalloc(qa, qw, M, N, K, y):
         M, N, K, L.NVFP4_BF16, y.data_ptr(), stream or None)
 
 
-@pytest.mark.parametrize("M,N,K", [(8, 1024, 4096), (1, 384, 2048), (64, 512, 1024),
-                                   (8, 12288, 4096)])
+@pytest.mark.parametrize("M,N,K", [(256, 256, 2048), (8, 1024, 4096), (1, 384, 2048),
+                                   (64, 512, 1024), (8, 12288, 4096)])
 def test_noalloc_matches_linear_on_two_calls(M, N, K):
     lib = L.load()
     need = lib.nvfp4_workspace_bytes(L.NVFP4_OP_LINEAR, M, N, K)
@@ -68,7 +68,7 @@ def test_noalloc_matches_linear_on_two_calls(M, N, K):
 def test_noalloc_uses_the_scratch_for_split_k():
     # the first shape above splits K across CTAs, so its partial sums really go to the array
     lib = L.load()
-    assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_LINEAR, 8, 1024, 4096) > 0
+    assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_LINEAR, 256, 256, 2048) > 0
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch():

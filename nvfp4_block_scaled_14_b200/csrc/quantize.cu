@@ -7,14 +7,16 @@
 // "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details". FP8 source (double
 // quantization): "Qwen-Rapid-AIO FP8 -> NVFP4", "1. Double Quantization".
 //
-// Two kernels per call, both HBM-bound, chained by programmatic dependent launch:
+// Tensors of 16 MB up to what the CTAs' shared memory holds (148 x 192 KB) take one fused
+// single-pass kernel (fused_quantize_kernel, below). Every other size takes two kernels, both
+// HBM-bound, chained by programmatic dependent launch:
 //   amax_kernel   (dynamic amax only) -- one CTA per SM streams a contiguous byte range of
 //                 the tensor through a 4 x 32 KB shared-memory ring of 1-D bulk copies and
 //                 reduces max |x| with SIMD integer max on the magnitude bits (exact,
 //                 order-free); one partial per CTA, no atomics, nothing to zero.
 //   encode_kernel -- one CTA per SM owns a contiguous range of rows; each warp takes a
-//                 64-block run of one row (1024 values, fully coalesced), two 16-value blocks per
-//                 lane. It loads its first items before griddepcontrol.wait, so the loads
+//                 64-block run of one row (1024 values, fully coalesced), two 16-value blocks
+//                 per lane. It loads its first items before griddepcontrol.wait, so the loads
 //                 overlap the amax kernel's tail (the tensor is then mostly in L2), reduces the
 //                 partial maxima to the global scale, and fills a 128-entry table of
 //                 1 / (E4M3(c) * sg). Per block: block amax, E4M3 scale, E2M1 codes by the
@@ -23,16 +25,29 @@
 // Code-deciding arithmetic is IEEE fp32 round-to-nearest in a fixed order (__fdiv_rn,
 // __fmul_rn, __frcp_rn): sg = amax / 2688, sb = E4M3(bmax / (sg * 6)),
 // code = E2M1(x * (1 / (sb * sg))).
+#include <cooperative_groups.h>
+#include <mutex>
+
 #include "nvfp4_internal.cuh"
 #include "sm100_ptx.cuh"
 
 namespace nvfp4 {
 namespace {
 
-constexpr int kThreads = 1024;      // encode: 32 warps, one 16-value block per lane per item
 constexpr int kAmaxThreads = 1024;  // amax: one CTA per SM streaming its byte range
 constexpr int kChunk = 32 * 1024;   // amax ring: 4 x 32 KB bulk copies in flight per SM
 constexpr int kRing = 4;
+constexpr int kFusedThreads = 1024;    // fused quantizer: one CTA per SM
+constexpr int kFusedChunk = 32 * 1024;  // fused quantizer: bulk-copy size
+constexpr int kFusedMaxChunks = 6;
+constexpr int kFusedCap = kFusedChunk * kFusedMaxChunks; // tensor bytes per CTA (192 KB)
+constexpr int kEncThreads = 1024;      // encode: 32 warps, two 16-value blocks per lane per item
+// The fused kernel runs tensors from kFusedMinBytes up to its shared-memory capacity. Below,
+// its grid-wide barrier and one-CTA-per-SM launch cost more than the second kernel and the
+// second read (from L2) save: measured on B200, bf16 / fp32 / fp8 from 0.1 to 25 MB, the
+// fused kernel is ahead from about 12-16 MB (fp32 12.6 MB: 10.4 vs 11.5 us; bf16 25 MB:
+// 14.1 vs 14.9 us) and behind below (bf16 6.3 MB: 8.6 vs 7.3 us).
+constexpr int64_t kFusedMinBytes = (int64_t)16 << 20;
 constexpr uint32_t kSpinLimit = 1u << 24;
 
 template <int SRC> struct Src;
@@ -77,81 +92,6 @@ template <> struct Src<kSrcE4M3> {
     }
 };
 
-__device__ __forceinline__ uint4 ldg_stream(const uint4 *p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-// Raw 16-byte vectors of one 16-value block: 4 (fp32), 2 (bf16) or 1 (fp8).
-template <int SRC> constexpr int kVecs = SRC == kSrcF32 ? 4 : (SRC == kSrcBF16 ? 2 : 1);
-
-template <int SRC>
-__device__ __forceinline__ void load_raw(const uint8_t *p, uint4 (&r)[4])
-{
-    const uint4 *q = reinterpret_cast<const uint4 *>(p);
-#pragma unroll
-    for (int i = 0; i < kVecs<SRC>; ++i)
-        r[i] = ldg_stream(q + i);
-}
-
-// Raw block -> 16 fp32 values (bf16 widening is exact; fp8 is upcast by one fp32 multiply
-// with s8).
-template <int SRC>
-__device__ __forceinline__ void to_f32(const uint4 (&r)[4], float s8, float (&v)[16])
-{
-    if constexpr (SRC == kSrcF32) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[4 * i + 0] = __uint_as_float(r[i].x);
-            v[4 * i + 1] = __uint_as_float(r[i].y);
-            v[4 * i + 2] = __uint_as_float(r[i].z);
-            v[4 * i + 3] = __uint_as_float(r[i].w);
-        }
-    } else if constexpr (SRC == kSrcBF16) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const uint32_t u[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[8 * i + 2 * j + 0] = __uint_as_float(u[j] << 16);
-                v[8 * i + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
-            }
-        }
-    } else {
-        const uint32_t u[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 ss = make_float2(s8, s8);
-            const float2 a = __fmul2_rn(e4m3x2_to_f32x2(u[j] & 0xFFFFu), ss);
-            const float2 b = __fmul2_rn(e4m3x2_to_f32x2(u[j] >> 16), ss);
-            v[4 * j + 0] = a.x;
-            v[4 * j + 1] = a.y;
-            v[4 * j + 2] = b.x;
-            v[4 * j + 3] = b.y;
-        }
-    }
-}
-
-// Block maximum |x| (fp32) from the raw vectors (fp8: times s8, which commutes with the max
-// because rounding is monotone).
-template <int SRC>
-__device__ __forceinline__ float block_absmax(const uint4 (&r)[4], float s8)
-{
-    if constexpr (SRC == kSrcF32) {
-        return __uint_as_float(max(max(Src<SRC>::vec_magmax(r[0]), Src<SRC>::vec_magmax(r[1])),
-                                   max(Src<SRC>::vec_magmax(r[2]), Src<SRC>::vec_magmax(r[3]))));
-    } else if constexpr (SRC == kSrcBF16) {
-        return Src<SRC>::mag_to_f32(
-            __vmaxu2(Src<SRC>::vec_magmax(r[0]), Src<SRC>::vec_magmax(r[1])));
-    } else {
-        return __fmul_rn(Src<SRC>::mag_to_f32(Src<SRC>::vec_magmax(r[0])), s8);
-    }
-}
-
 // E4M3 code of RN(bmax / t), exactly as cvt_e4m3(__fdiv_rn(bmax, t)) gives it, usually without
 // the division. rt = RN(1/t). q0 = RN(bmax * rt) is within 3 fp32 ulps of RN(bmax / t) (two
 // roundings of relative size 2^-24 each, plus the rounding of the quotient itself). For
@@ -171,43 +111,6 @@ __device__ __forceinline__ uint32_t e4m3_of_quotient(float bmax, float t, float 
     return cvt_e4m3(__fdiv_rn(bmax, t));
 }
 
-// Encode one block: returns the E4M3 scale byte and writes the 8 code bytes. rcp_tab[c] holds
-// 1 / (E4M3(c) * sg), computed with the same two round-to-nearest operations per code.
-template <int SRC>
-__device__ __forceinline__ uint32_t encode_block(const uint4 (&r)[4], float s8, float sg,
-                                                 float t, float rt, const float *rcp_tab,
-                                                 uint2 &packed)
-{
-    const float bmax = block_absmax<SRC>(r, s8);
-    uint32_t sb = 0;
-    if (sg > 0.0f)
-        sb = e4m3_of_quotient(bmax, t, rt);
-    packed = make_uint2(0u, 0u);
-    if (sb != 0u) {
-        float v[16];
-        to_f32<SRC>(r, s8, v);
-        const float rcp = rcp_tab[sb];
-        const float2 rr = make_float2(rcp, rcp);
-        float y[16];
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-            const float2 p = __fmul2_rn(make_float2(v[j], v[j + 1]), rr);
-            y[j] = p.x;
-            y[j + 1] = p.y;
-        }
-        packed.x = cvt_e2m1x8(y);
-        packed.y = cvt_e2m1x8(y + 8);
-    }
-    return sb;
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 // Fold a magnitude-bit accumulator (per source type) into another.
 template <int SRC> __device__ __forceinline__ uint32_t mag_fold(uint32_t a, uint32_t b)
 {
@@ -219,25 +122,21 @@ template <int SRC> __device__ __forceinline__ uint32_t mag_fold(uint32_t a, uint
         return __vmaxu4(a, b);
 }
 
-template <int SRC> __device__ __forceinline__ uint32_t raw_magmax(const uint4 (&r)[4])
-{
-    uint32_t m = Src<SRC>::vec_magmax(r[0]);
-#pragma unroll
-    for (int i = 1; i < kVecs<SRC>; ++i)
-        m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(r[i]));
-    return m;
-}
-
 struct QuantArgs {
     const uint8_t *x;
+    int64_t nbytes; // rows * cols * element size
     const float *fp8_scale;
     int rows, cols;
     const float *static_amax;
     uint8_t *codes, *sf_swz, *sf_lin;
     float *global_scale;
     const float *partials; // one max |x| per amax CTA (dynamic amax)
+    float *partials_out;   // the fused kernel's per-CTA maxima (same workspace)
     int npartials;
-    uint32_t chunks_magic; // ceil(2^32 / runs) for runs >= 2: item / runs by umulhi
+    uint32_t nb_magic;     // ceil(2^32 / blocks per row): block / nb by multiply-high
+    uint32_t runs_magic;   // ceil(2^32 / runs) for runs >= 2: item / runs by multiply-high
+    int blocks_fit32;      // rows * blocks per row < 2^32 (the multiply-high path applies)
+    int *status;
 };
 
 // K1: max |x| over a contiguous byte range per CTA, streamed through a shared-memory ring
@@ -301,18 +200,324 @@ __global__ void __launch_bounds__(kAmaxThreads, 1)
     }
 }
 
-// K2: encode. Each CTA owns a contiguous range of rows; each warp takes a 64-block run of one
-// row and each lane two adjacent 16-value blocks, so address arithmetic and loop control are
-// shared by two blocks, the codes leave as one 16-byte store and the two scale bytes as one
-// 16-bit store. The first item is loaded before waiting on the amax kernel (programmatic
-// dependent launch), so the loads overlap its tail; later items are double-buffered.
+// Geometry of the fused kernel's warp items: a lane owns kBpl whole blocks (2 for bf16 / fp8,
+// 1 for fp32) of a 32 * kBpl-block item.
+template <int SRC> struct Enc {
+    static constexpr int kEsz = Src<SRC>::kBytes;
+    static constexpr int kBlk = 16 * kEsz;                    // bytes per block
+    static constexpr int kVecs = kBlk / 16;                   // 16-byte vectors per block
+    static constexpr int kBpl = SRC == kSrcF32 ? 1 : 2;       // blocks per lane
+    static constexpr int kItemBlocks = 32 * kBpl;
+    static constexpr int kItem = kItemBlocks * kBlk;          // bytes per warp item
+};
+
+// One block of raw vectors -> 16 fp32 values (bf16 widening exact; fp8 times s8).
 template <int SRC>
-__global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
+__device__ __forceinline__ void block_to_f32(const uint4 *r, float s8, float (&v)[16])
+{
+    if constexpr (SRC == kSrcF32) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[4 * i] = __uint_as_float(r[i].x);
+            v[4 * i + 1] = __uint_as_float(r[i].y);
+            v[4 * i + 2] = __uint_as_float(r[i].z);
+            v[4 * i + 3] = __uint_as_float(r[i].w);
+        }
+    } else if constexpr (SRC == kSrcBF16) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t u[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v[8 * i + 2 * j] = __uint_as_float(u[j] << 16);
+                v[8 * i + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+            }
+        }
+    } else {
+        const uint32_t u[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
+        const float2 ss = make_float2(s8, s8);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 a = __fmul2_rn(e4m3x2_to_f32x2(u[j] & 0xFFFFu), ss);
+            const float2 b = __fmul2_rn(e4m3x2_to_f32x2(u[j] >> 16), ss);
+            v[4 * j] = a.x;
+            v[4 * j + 1] = a.y;
+            v[4 * j + 2] = b.x;
+            v[4 * j + 3] = b.y;
+        }
+    }
+}
+
+// E4M3 scale byte of a block from its nv raw vectors.
+template <int SRC>
+__device__ __forceinline__ uint32_t block_scale(const uint4 *r, int nv, float s8, float sg,
+                                                float t, float rt)
+{
+    uint32_t m = Src<SRC>::vec_magmax(r[0]);
+    for (int i = 1; i < nv; ++i)
+        m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(r[i]));
+    float bmax = Src<SRC>::mag_to_f32(m);
+    if constexpr (SRC == kSrcE4M3)
+        bmax = __fmul_rn(bmax, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
+    return sg > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
+}
+
+// E2M1 codes of one 16-byte vector times rcp, low nibble first: 2 (fp32), 4 (bf16) or 8
+// (fp8) bytes; all zero when the block's scale is zero.
+template <int SRC>
+__device__ __forceinline__ uint2 vec_codes(uint4 u, float s8, uint32_t sb, const float *rcp_tab)
+{
+    if (sb == 0u)
+        return make_uint2(0u, 0u);
+    constexpr int NV = 16 / Src<SRC>::kBytes;
+    float v[16];
+    const uint4 r[4] = {u, u, u, u};
+    if constexpr (SRC == kSrcF32) {
+        v[0] = __uint_as_float(u.x);
+        v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z);
+        v[3] = __uint_as_float(u.w);
+    } else if constexpr (SRC == kSrcBF16) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    } else {
+        block_to_f32<SRC>(r, s8, v);
+    }
+    const float rcp = rcp_tab[sb];
+    const float2 rr = make_float2(rcp, rcp);
+    float y[16];
+#pragma unroll
+    for (int j = 0; j < NV; j += 2) {
+        const float2 q = __fmul2_rn(make_float2(v[j], v[j + 1]), rr);
+        y[j] = q.x;
+        y[j + 1] = q.y;
+    }
+    if constexpr (NV == 4) {
+        y[4] = y[5] = y[6] = y[7] = 0.0f;
+        return make_uint2(cvt_e2m1x8(y) & 0xFFFFu, 0u);
+    } else if constexpr (NV == 8) {
+        return make_uint2(cvt_e2m1x8(y), 0u);
+    } else {
+        return make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8));
+    }
+}
+
+// Maxima |x| (fp8: of |e|, before the fp8 scale) of a lane's kBpl blocks, in natural block
+// order, from its vectors read in rotated order: r[v] holds the lane's vector v ^ k (k = 0:
+// natural order; the rotation keeps each block's vectors together).
+template <int SRC>
+__device__ __forceinline__ void lane_block_max(const uint4 *r, uint32_t k, float &m0, float &m1)
+{
+    using S = Src<SRC>;
+    if constexpr (SRC == kSrcBF16) {
+        const float ma = S::mag_to_f32(mag_fold<SRC>(S::vec_magmax(r[0]), S::vec_magmax(r[1])));
+        const float mb = S::mag_to_f32(mag_fold<SRC>(S::vec_magmax(r[2]), S::vec_magmax(r[3])));
+        const bool sw = (k & 2u) != 0;
+        m0 = sw ? mb : ma;
+        m1 = sw ? ma : mb;
+    } else if constexpr (SRC == kSrcF32) {
+        m0 = S::mag_to_f32(mag_fold<SRC>(mag_fold<SRC>(S::vec_magmax(r[0]), S::vec_magmax(r[1])),
+                                         mag_fold<SRC>(S::vec_magmax(r[2]), S::vec_magmax(r[3]))));
+        m1 = 0.0f;
+    } else {
+        const float ma = S::mag_to_f32(S::vec_magmax(r[0]));
+        const float mb = S::mag_to_f32(S::vec_magmax(r[1]));
+        const bool sw = (k & 1u) != 0;
+        m0 = sw ? mb : ma;
+        m1 = sw ? ma : mb;
+    }
+}
+
+// E4M3 scale byte of a block from its maximum (fp8: times s8 first).
+template <int SRC>
+__device__ __forceinline__ uint32_t scale_of(float m, float s8, float sg, float t, float rt)
+{
+    const float bmax = SRC == kSrcE4M3 ? __fmul_rn(m, s8) : m;
+    return sg > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
+}
+
+// Natural-order code bytes (8 per block, as 32-bit words) of a lane's blocks with natural
+// scale bytes sb0, sb1, from its vectors read in rotated order (r[v] = vector v ^ k).
+template <int SRC>
+__device__ __forceinline__ void lane_codes(const uint4 *r, uint32_t k, uint32_t sb0,
+                                           uint32_t sb1, float s8, const float *rcp_tab,
+                                           uint32_t (&cw)[2 * Enc<SRC>::kBpl])
+{
+    if constexpr (SRC == kSrcBF16) {
+        const bool sw = (k & 2u) != 0;
+        const uint32_t sa = sw ? sb1 : sb0, sbb = sw ? sb0 : sb1; // scales of r[0..1], r[2..3]
+        uint32_t c[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            c[v] = vec_codes<SRC>(r[v], s8, v < 2 ? sa : sbb, rcp_tab).x;
+        const uint32_t a0 = (k & 1u) ? c[1] : c[0], a1 = (k & 1u) ? c[0] : c[1];
+        const uint32_t a2 = (k & 1u) ? c[3] : c[2], a3 = (k & 1u) ? c[2] : c[3];
+        cw[0] = sw ? a2 : a0;
+        cw[1] = sw ? a3 : a1;
+        cw[2] = sw ? a0 : a2;
+        cw[3] = sw ? a1 : a3;
+    } else if constexpr (SRC == kSrcF32) {
+        uint32_t h[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            h[v] = vec_codes<SRC>(r[v], s8, sb0, rcp_tab).x;
+        uint32_t o[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const uint32_t lo = (k & 1u) ? h[n ^ 1] : h[n];
+            const uint32_t hi = (k & 1u) ? h[n ^ 3] : h[n ^ 2];
+            o[n] = (k & 2u) ? hi : lo;
+        }
+        cw[0] = o[0] | (o[1] << 16);
+        cw[1] = o[2] | (o[3] << 16);
+    } else {
+        const bool sw = (k & 1u) != 0;
+        const uint2 ca = vec_codes<SRC>(r[0], s8, sw ? sb1 : sb0, rcp_tab);
+        const uint2 cb = vec_codes<SRC>(r[1], s8, sw ? sb0 : sb1, rcp_tab);
+        cw[0] = sw ? cb.x : ca.x;
+        cw[1] = sw ? cb.y : ca.y;
+        cw[2] = sw ? ca.x : cb.x;
+        cw[3] = sw ? ca.y : cb.y;
+    }
+}
+
+// Scales and codes of a lane's blocks (vectors in rotated order, see lane_block_max).
+template <int SRC>
+__device__ __forceinline__ void lane_encode(const uint4 *r, uint32_t k, float s8, float sg,
+                                            float t, float rt, const float *rcp_tab,
+                                            uint32_t (&cw)[2 * Enc<SRC>::kBpl], uint32_t &sb0,
+                                            uint32_t &sb1)
+{
+    float m0, m1;
+    lane_block_max<SRC>(r, k, m0, m1);
+    sb0 = scale_of<SRC>(m0, s8, sg, t, rt);
+    sb1 = Enc<SRC>::kBpl == 2 ? scale_of<SRC>(m1, s8, sg, t, rt) : 0u;
+    lane_codes<SRC>(r, k, sb0, sb1, s8, rcp_tab, cw);
+}
+
+// Store a lane's codes (blocks f0 .. f0 + kBpl - 1) and scales in the linear and / or
+// swizzled layout; the lane holding a row's last blocks also zeroes the atom's padding.
+template <int SRC>
+__device__ __forceinline__ void store_lane(const QuantArgs &a, int64_t f0, uint32_t nb, int apb,
+                                           const uint32_t (&cw)[2 * Enc<SRC>::kBpl],
+                                           uint32_t sb0, uint32_t sb1)
+{
+    uint8_t *cp = a.codes + f0 * 8;
+    if constexpr (Enc<SRC>::kBpl == 2)
+        *reinterpret_cast<uint4 *>(cp) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    else
+        *reinterpret_cast<uint2 *>(cp) = make_uint2(cw[0], cw[1]);
+    uint32_t row, b;
+    if (a.blocks_fit32) {
+        row = __umulhi((uint32_t)f0, a.nb_magic);
+        if (row * nb > (uint32_t)f0)
+            --row;
+        b = (uint32_t)f0 - row * nb;
+    } else {
+        row = (uint32_t)(f0 / nb);
+        b = (uint32_t)(f0 - (int64_t)row * nb);
+    }
+    const int64_t swz = ((int64_t)(row >> 7) * apb + (b >> 2)) * 512 + ((row & 31) << 4) +
+                        (((row >> 5) & 3) << 2) + (b & 3);
+    if constexpr (Enc<SRC>::kBpl == 2) {
+        // b is even: both scale bytes are adjacent in either layout
+        const uint16_t s2 = (uint16_t)(sb0 | (sb1 << 8));
+        if (a.sf_lin)
+            *reinterpret_cast<uint16_t *>(a.sf_lin + f0) = s2;
+        if (a.sf_swz) {
+            if (b + 2 == nb && (b & 3) == 0) // last pair of the row: zero the atom's pad
+                *reinterpret_cast<uint32_t *>(a.sf_swz + swz) = s2;
+            else
+                *reinterpret_cast<uint16_t *>(a.sf_swz + swz) = s2;
+        }
+    } else {
+        if (a.sf_lin)
+            a.sf_lin[f0] = (uint8_t)sb0;
+        if (a.sf_swz) {
+            a.sf_swz[swz] = (uint8_t)sb0;
+            if (b + 1 == nb && (b & 3) == 1) { // last block of the row: zero the pad
+                a.sf_swz[swz + 1] = 0;
+                a.sf_swz[swz + 2] = 0;
+            }
+        }
+    }
+}
+
+// Zero the swizzled padding rows of the last 128-row band. In an atom, the 16-byte line
+// i holds rows i, i + 32, i + 64, i + 96 of the band (4 bytes each), so one warp covers an
+// atom with one store per lane: 16 bytes when all four rows are padding, else only the
+// padding rows' words (the real rows' words belong to the encoding lanes). The pad blocks of
+// real rows are written with their row's last scales.
+__device__ __forceinline__ void zero_pad_rows(const QuantArgs &a, int apb)
+{
+    if (!a.sf_swz || (a.rows & 127) == 0)
+        return;
+    const int band = a.rows >> 7;     // the partly filled band
+    const int real = a.rows & 127;    // its real rows
+    const int i = threadIdx.x & 31;   // line of the atom
+    const int warps = blockDim.x >> 5;
+    for (int atom = blockIdx.x * warps + (threadIdx.x >> 5); atom < apb;
+         atom += gridDim.x * warps) {
+        uint8_t *line = a.sf_swz + ((int64_t)band * apb + atom) * 512 + i * 16;
+        if (i >= real) {
+            *reinterpret_cast<uint4 *>(line) = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+#pragma unroll
+            for (int q = 1; q < 4; ++q)
+                if (i + 32 * q >= real)
+                    *reinterpret_cast<uint32_t *>(line + 4 * q) = 0u;
+        }
+    }
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// One block from its kVecs raw vectors: the E4M3 scale byte, and the 8 code bytes.
+template <int SRC>
+__device__ __forceinline__ uint32_t encode_one(const uint4 *r, float s8, float sg, float t,
+                                               float rt, const float *rcp_tab, uint2 &packed)
+{
+    constexpr int V = Enc<SRC>::kVecs;
+    const uint32_t sb = block_scale<SRC>(r, V, s8, sg, t, rt);
+    if constexpr (V == 4) { // fp32: 2 code bytes per vector
+        uint32_t c[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            c[v] = vec_codes<SRC>(r[v], s8, sb, rcp_tab).x;
+        packed = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+    } else if constexpr (V == 2) { // bf16: 4 per vector
+        packed = make_uint2(vec_codes<SRC>(r[0], s8, sb, rcp_tab).x,
+                            vec_codes<SRC>(r[1], s8, sb, rcp_tab).x);
+    } else { // fp8: 8 per vector
+        packed = vec_codes<SRC>(r[0], s8, sb, rcp_tab);
+    }
+    return sb;
+}
+
+// K2: encode (tensors above the fused kernel's size). One CTA per SM owns a contiguous range
+// of rows; each warp takes a 64-block run of one row and each lane two adjacent 16-value
+// blocks, so address arithmetic and loop control are shared by two blocks, the codes leave as
+// one 16-byte store and the two scale bytes as one 16-bit store. The first item is loaded
+// before waiting on the amax kernel (programmatic dependent launch), so the loads overlap its
+// tail; later items are double-buffered.
+template <int SRC>
+__global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs a)
 {
     __shared__ float s_sg;
     __shared__ float s_rcp[128];
     constexpr int kBlkBytes = 16 * Src<SRC>::kBytes;
-    constexpr int V = kVecs<SRC>; // 16-byte vectors per block
+    constexpr int V = Enc<SRC>::kVecs; // 16-byte vectors per block
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nb = a.cols >> 4;       // blocks per row
@@ -332,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
             b0 = 2 * lane;
             return;
         }
-        ro = (int)__umulhi((uint32_t)it, a.chunks_magic);
+        ro = (int)__umulhi((uint32_t)it, a.runs_magic);
         if (ro * runs > it)
             --ro;
         b0 = (it - ro * runs) * 64 + 2 * lane;
@@ -364,8 +569,18 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
         if (a.static_amax) {
             g = *a.static_amax;
         } else {
-            for (int i = threadIdx.x; i < a.npartials; i += 32)
-                g = fmaxf(g, __ldcg(a.partials + i));
+            // up to 8 loads in flight per lane: one L2 round trip per 256 partials
+            for (int i0 = 0; i0 < a.npartials; i0 += 32 * 8) {
+                float pv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + threadIdx.x + 32 * u;
+                    pv[u] = i < a.npartials ? __ldcg(a.partials + i) : 0.0f;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    g = fmaxf(g, pv[u]);
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
@@ -393,16 +608,10 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
         uint32_t sb0 = 0, sb1 = 0;
         uint2 p0 = make_uint2(0u, 0u), p1 = make_uint2(0u, 0u);
         if (b0 < nb) {
-            uint4 x0[4], x1[4];
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                x0[v] = r[v];
-                x1[v] = r[V + v];
-            }
-            sb0 = encode_block<SRC>(x0, s8, sg, t, rt, s_rcp, p0);
+            sb0 = encode_one<SRC>(r, s8, sg, t, rt, s_rcp, p0);
             uint8_t *c = a.codes + (int64_t)row * (a.cols >> 1) + b0 * 8;
             if (b0 + 1 < nb) {
-                sb1 = encode_block<SRC>(x1, s8, sg, t, rt, s_rcp, p1);
+                sb1 = encode_one<SRC>(r + V, s8, sg, t, rt, s_rcp, p1);
                 *reinterpret_cast<uint4 *>(c) = make_uint4(p0.x, p0.y, p1.x, p1.y);
             } else {
                 *reinterpret_cast<uint2 *>(c) = p0;
@@ -439,14 +648,165 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const QuantArgs a)
             it += 32;
         }
     }
-    // zero the scale padding rows of the last 128-row band
-    if (a.sf_swz) {
-        const int rows_pad = ((a.rows + 127) >> 7) << 7;
-        for (int row = a.rows + blockIdx.x; row < rows_pad; row += gridDim.x)
-            for (int b = threadIdx.x; b < 4 * apb; b += kThreads)
-                a.sf_swz[((int64_t)(row >> 7) * apb + (b >> 2)) * 512 + ((row & 31) << 4) +
-                         (((row >> 5) & 3) << 2) + (b & 3)] = 0;
+    zero_pad_rows(a, apb);
+}
+
+// Fused single-pass quantizer for tensors that fit in the CTAs' shared memory (one CTA per
+// SM, up to kFusedCap bytes each): each CTA bulk-loads its contiguous share of warp items in
+// 32 KB copies. Dynamic amax: it folds max |x| over its share as the copies land, publishes
+// one partial, meets the other CTAs at a grid-wide barrier (cooperative launch: all CTAs are
+// co-resident), reduces the partials to the global scale and encodes from shared memory, so
+// the tensor is read from HBM once and no second kernel is launched. Static amax: no
+// barrier, each item is encoded as soon as its copy lands. Lanes read their 64 (32) bytes
+// in an order rotated by lane so that a warp's shared-memory reads are conflict-free.
+template <int SRC>
+__global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const QuantArgs a)
+{
+    using E = Enc<SRC>;
+    extern __shared__ __align__(128) uint8_t buf[];
+    __shared__ uint64_t bars[kFusedMaxChunks];
+    __shared__ float s_red[kFusedThreads / 32];
+    __shared__ float s_sg;
+    __shared__ float s_rcp[128];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nblocks = (int64_t)a.rows * (a.cols >> 4);
+    const int64_t nitems = (nblocks + E::kItemBlocks - 1) / E::kItemBlocks;
+    const int64_t c0 = nitems * blockIdx.x / gridDim.x;
+    const int64_t c1 = nitems * (blockIdx.x + 1) / gridDim.x;
+    const int64_t byte0 = c0 * E::kItem;
+    const int64_t nbytes = max((int64_t)0, min(a.nbytes, c1 * E::kItem) - byte0);
+    const int nch = (int)((nbytes + kFusedChunk - 1) / kFusedChunk);
+    __shared__ float s_scalars[2];
+    if (threadIdx.x == 0) {
+        // the scalar inputs go out ahead of the bulk copies, not behind them in the queue
+        s_scalars[0] = (SRC == kSrcE4M3 && a.fp8_scale) ? *a.fp8_scale : 1.0f;
+        s_scalars[1] = a.static_amax ? *a.static_amax : 0.0f;
+        for (int i = 0; i < nch; ++i)
+            mbar_init(&bars[i], 1);
+        fence_barrier_init();
+        for (int i = 0; i < nch; ++i) {
+            const int64_t off = (int64_t)i * kFusedChunk;
+            const uint32_t n = (uint32_t)min((int64_t)kFusedChunk, nbytes - off);
+            mbar_arrive_expect_tx(&bars[i], n);
+            bulk_load_1d(buf + off, a.x + byte0 + off, n, &bars[i]);
+        }
     }
+    __syncthreads();
+    const float s8 = s_scalars[0];
+    // rotation: bf16 / fp32 lanes read 64 bytes (4 vectors), fp8 lanes 32 bytes (2 vectors)
+    const uint32_t k = SRC == kSrcE4M3 ? (uint32_t)(lane >> 2) & 1u : (uint32_t)(lane >> 1) & 3u;
+    constexpr int NVL = E::kBpl * E::kVecs;
+    constexpr int kWarps = kFusedThreads / 32;
+    constexpr int MIW = kFusedCap / E::kItem / kWarps; // items per warp at most
+    const int items = (int)(c1 - c0);
+    auto load_lane = [&](int j, uint4 (&r)[NVL]) -> bool {
+        const int64_t f0 = (c0 + j) * E::kItemBlocks + lane * E::kBpl;
+        const bool valid = f0 < nblocks;
+        const uint32_t src = smem_u32(buf + j * E::kItem) + lane * (E::kBpl * E::kBlk);
+#pragma unroll
+        for (int v = 0; v < NVL; ++v)
+            r[v] = valid ? lds128(src + 16 * (v ^ k)) : make_uint4(0u, 0u, 0u, 0u);
+        return valid;
+    };
+    auto wait_item = [&](int j) {
+        if (!mbar_wait(&bars[(j * E::kItem) / kFusedChunk], 0, kSpinLimit) && lane == 0)
+            atomicExch(a.status, (int)NVFP4_ERR_TIMEOUT);
+    };
+    float bm0[MIW], bm1[MIW]; // block maxima of this lane's blocks, item by item
+    if (!a.static_amax) {
+        // block maxima as the copies land; the CTA maximum is their maximum
+        float lm = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < MIW; ++jj) {
+            const int j = warp + kWarps * jj;
+            bm0[jj] = bm1[jj] = 0.0f;
+            if (j < items) {
+                wait_item(j);
+                uint4 r[NVL];
+                load_lane(j, r);
+                lane_block_max<SRC>(r, k, bm0[jj], bm1[jj]);
+                lm = fmaxf(lm, fmaxf(bm0[jj], bm1[jj]));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            lm = fmaxf(lm, __shfl_xor_sync(0xFFFFFFFFu, lm, o));
+        if (lane == 0)
+            s_red[warp] = lm;
+        __syncthreads();
+        float g = 0.0f;
+        if (threadIdx.x < 32) {
+            g = s_red[threadIdx.x];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+            if (threadIdx.x == 0 && gridDim.x > 1)
+                a.partials_out[blockIdx.x] = g;
+        }
+        if (gridDim.x > 1) { // a single CTA already holds the tensor's maximum
+            cooperative_groups::this_grid().sync(); // every CTA's partial is visible
+            if (threadIdx.x < 32) {
+                // all loads in flight at once (gridDim <= 160): one L2 round trip
+                float pv[5];
+#pragma unroll
+                for (int u = 0; u < 5; ++u) {
+                    const int i = threadIdx.x + 32 * u;
+                    pv[u] = i < (int)gridDim.x ? __ldcg(a.partials_out + i) : 0.0f;
+                }
+                g = fmaxf(fmaxf(fmaxf(pv[0], pv[1]), fmaxf(pv[2], pv[3])), pv[4]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+            }
+        }
+        if (threadIdx.x < 32) {
+            if (SRC == kSrcE4M3)
+                g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
+            if (threadIdx.x == 0) {
+                const float sg = __fdiv_rn(g, 2688.0f); // 6 * 448
+                s_sg = sg;
+                if (blockIdx.x == 0)
+                    *a.global_scale = sg;
+            }
+        }
+    } else if (threadIdx.x == 0) {
+        const float sg = __fdiv_rn(s_scalars[1], 2688.0f);
+        s_sg = sg;
+        if (blockIdx.x == 0)
+            *a.global_scale = sg;
+    }
+    __syncthreads();
+    const float sg = s_sg;
+    const float t = __fmul_rn(sg, 6.0f);
+    const float rt = __frcp_rn(t);
+    if (threadIdx.x < 128)
+        s_rcp[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
+    __syncthreads();
+
+    const uint32_t nb = (uint32_t)(a.cols >> 4);
+    const int apb = (int)((nb + 3) >> 2);
+#pragma unroll
+    for (int jj = 0; jj < MIW; ++jj) {
+        const int j = warp + kWarps * jj;
+        if (j >= items)
+            break;
+        uint4 r[NVL];
+        if (a.static_amax) { // the copy may still be in flight; maxima not taken yet
+            wait_item(j);
+            load_lane(j, r);
+            lane_block_max<SRC>(r, k, bm0[jj], bm1[jj]);
+        } else {
+            load_lane(j, r);
+        }
+        const int64_t f0 = (c0 + j) * E::kItemBlocks + lane * E::kBpl;
+        const uint32_t sb0 = scale_of<SRC>(bm0[jj], s8, sg, t, rt);
+        const uint32_t sb1 = E::kBpl == 2 ? scale_of<SRC>(bm1[jj], s8, sg, t, rt) : 0u;
+        uint32_t cw[2 * E::kBpl];
+        lane_codes<SRC>(r, k, sb0, sb1, s8, s_rcp, cw);
+        if (f0 < nblocks)
+            store_lane<SRC>(a, f0, nb, apb, cw, sb0, sb1);
+    }
+    zero_pad_rows(a, apb);
 }
 
 template <int SRC>
@@ -466,8 +826,48 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
     qa.sf_lin = sf_lin;
     qa.global_scale = global_scale;
     qa.partials = reinterpret_cast<const float *>(ws);
-    const uint64_t runs = (uint64_t)((cols / 16 + 63) / 64);
-    qa.chunks_magic = runs > 1 ? (uint32_t)((((uint64_t)1 << 32) + runs - 1) / runs) : 0u;
+    qa.nbytes = rows * cols * Src<SRC>::kBytes;
+    const uint64_t nb = (uint64_t)(cols / 16);
+    qa.nb_magic = nb > 1 ? (uint32_t)((((uint64_t)1 << 32) + nb - 1) / nb) : 0u;
+    qa.blocks_fit32 = (uint64_t)rows * nb < ((uint64_t)1 << 32) ? 1 : 0;
+    const uint64_t runs = (nb + 63) / 64;
+    qa.runs_magic = runs > 1 ? (uint32_t)((((uint64_t)1 << 32) + runs - 1) / runs) : 0u;
+    qa.status = device_status_ptr();
+    qa.partials_out = reinterpret_cast<float *>(ws);
+    // fused single pass when every CTA's share fits in its shared memory
+    {
+        using E = Enc<SRC>;
+        const int64_t nitems = (rows * (cols / 16) + E::kItemBlocks - 1) / E::kItemBlocks;
+        int64_t g = (nitems + kFusedThreads / 32 - 1) / (kFusedThreads / 32);
+        if (g > sms)
+            g = sms;
+        if (g < 1)
+            g = 1;
+        if ((nitems + g - 1) / g * E::kItem <= kFusedCap && g <= 160 &&
+            qa.nbytes >= kFusedMinBytes) {
+            static std::once_flag fattr[64];
+            int dev = 0;
+            cudaGetDevice(&dev);
+            cudaError_t fe = cudaSuccess;
+            std::call_once(fattr[dev & 63], [&]() {
+                fe = cudaFuncSetAttribute(fused_quantize_kernel<SRC>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedCap);
+            });
+            if (fe != cudaSuccess)
+                return fe;
+            cudaLaunchConfig_t fc{};
+            fc.gridDim = dim3((unsigned)g);
+            fc.blockDim = dim3(kFusedThreads);
+            fc.dynamicSmemBytes = kFusedCap;
+            fc.stream = s;
+            cudaLaunchAttribute fa[1];
+            fa[0].id = cudaLaunchAttributeCooperative;
+            fa[0].val.cooperative = static_amax ? 0 : 1;
+            fc.attrs = fa;
+            fc.numAttrs = 1;
+            return cudaLaunchKernelEx(&fc, fused_quantize_kernel<SRC>, qa);
+        }
+    }
     cudaError_t e;
     if (!static_amax) {
         const int64_t nbytes = rows * cols * Src<SRC>::kBytes;
@@ -492,7 +892,7 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
         grid = rows < 1 ? 1 : (int)rows;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kEncThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

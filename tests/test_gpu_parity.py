@@ -51,6 +51,28 @@ def test_quantize_static_amax_saturates(kind):
         assert_quant_equal(gpu_quantize(x, amax=amax), O.quantize(x, amax=amax))
 
 
+# Tensors of 16 MB and more take the single-pass kernel (shared-memory resident, grid-wide
+# barrier); these shapes also have rows that end inside a 128-row band, and (4064 columns)
+# a block count per row that is not a multiple of 4, so the swizzled padding is exercised.
+@pytest.mark.parametrize("kind,rows,cols", [("f32", 1100, 4064), ("bf16", 2100, 4064),
+                                            ("e4m3", 4100, 4096)])
+@pytest.mark.parametrize("static", [False, True])
+def test_quantize_single_pass_sizes(kind, rows, cols, static):
+    x = W.normal((rows, cols), 1.0, 23, rows + cols)
+    x[rows - 1, cols - 1] = 19.0
+    amax = 7.5 if static else None
+    if kind == "e4m3":
+        w8, s8 = W.to_fp8_tensorwise(x)
+        assert w8.nbytes >= 16 << 20
+        assert_quant_equal(gpu_quantize(w8, amax=amax, fp8_scale=s8),
+                           O.quantize(w8, amax=amax, fp8_scale=s8))
+        return
+    if kind == "bf16":
+        x = W.to_bf16_bits(x)
+    assert x.nbytes >= 16 << 20
+    assert_quant_equal(gpu_quantize(x, amax=amax), O.quantize(x, amax=amax))
+
+
 def test_quantize_fp8_source_double_quant():
     w8, s8 = W.to_fp8_tensorwise(W.normal((320, 384), 0.02, 22, 1))
     assert_quant_equal(gpu_quantize(w8, fp8_scale=s8), O.quantize(w8, fp8_scale=s8))
@@ -208,6 +230,8 @@ def test_linear_tiny_workload_fp32_out():
     # small M: K split over a thread-block cluster, partials summed through distributed
     # shared memory (uneven k-ranges, odd cluster sizes, the widest B tile)
     (8, 1536, 3072), (3, 640, 1792), (128, 2560, 1024), (64, 12288, 512), (1, 128, 4096),
+    # output rows whose byte stride is not a multiple of 16: no TMA store, direct stores
+    (8, 1004, 512), (3, 100, 256), (130, 1004, 256),
 ])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_linear_matches_oracle(M, N, K, out):

@@ -109,6 +109,36 @@ nvfp4_status nvfp4_quantize_fp8_src(const uint8_t *x_e4m3, const float *fp8_scal
                                     float *global_scale, void *ws, size_t ws_bytes,
                                     cudaStream_t stream);
 
+/* Source element type of a batched quantize job. */
+typedef enum { NVFP4_SRC_F32 = 0, NVFP4_SRC_BF16 = 1, NVFP4_SRC_E4M3 = 2 } nvfp4_src;
+
+/* One tensor of nvfp4_quantize_batch: the arguments of nvfp4_quantize (F32 / BF16 source) or
+ * nvfp4_quantize_fp8_src (E4M3 source; fp8_scale ignored for the other types). */
+typedef struct {
+    const void *x;
+    int src; /* nvfp4_src */
+    const float *fp8_scale;
+    int64_t rows, cols;
+    const float *static_amax;
+    uint8_t *codes, *scales_swz, *scales_lin;
+    float *global_scale;
+} nvfp4_quant_job;
+
+#define NVFP4_MAX_QUANT_JOBS 8
+
+/*
+ * Several quantizations in one pass: job i gets exactly the outputs that nvfp4_quantize /
+ * nvfp4_quantize_fp8_src give for its arguments (its own amax and global scale). No
+ * counterpart in the paper: the per-tensor method above, batched so that the tensors share one
+ * amax launch and one encode launch (CTAs split in proportion to the bytes) and their memory
+ * traffic overlaps, e.g. a weight re-quantized from FP8 and the activations of the same layer.
+ * jobs: HOST array of njobs (1 .. NVFP4_MAX_QUANT_JOBS) descriptors, each checked as its own
+ * call would be (first failure returned, nothing launched). ws: one workspace of
+ * nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, ...) bytes serves the whole batch.
+ */
+nvfp4_status nvfp4_quantize_batch(const nvfp4_quant_job *jobs, int njobs, void *ws,
+                                  size_t ws_bytes, cudaStream_t stream);
+
 /*
  * Dequantize ("Qwen-Image NVFP4 on a 16 GB Ada GPU", worked example under "First NVFP4
  * block, as stored in the file": weight = E2M1 x block scale x global scale).

@@ -21,7 +21,7 @@ from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_LINEAR_DEFAULT, NVFP4_LINEAR_RES
                    NVFP4_OP_CALIB_BF16, NVFP4_OP_CALIB_F32, NVFP4_OP_LINEAR, NVFP4_OP_QUANTIZE,
                    NVFP4Error, check, load)
 
-__all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "dequantize", "linear",
+__all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "quantize_batch", "dequantize", "linear",
            "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
 
 
@@ -122,6 +122,56 @@ def quantize_fp8(x_e4m3: torch.Tensor, fp8_scale: torch.Tensor = None,
                                   _stream(x_e4m3.device))
     check(st, "nvfp4_quantize_fp8_src")
     return out
+
+
+def quantize_batch(jobs) -> list:
+    """Quantize several tensors in one pass (one amax launch and one encode launch for all);
+    every tensor gets exactly what quantize / quantize_fp8 give it. jobs: a list of dicts with
+    keys x (fp32 / bf16 tensor, or uint8 / float8_e4m3fn E4M3 bits), and optionally
+    fp8_scale, static_amax, swizzled, linear, out. Returns the NVFP4Tensors."""
+    import ctypes
+    if not 1 <= len(jobs) <= _lib.NVFP4_MAX_QUANT_JOBS:
+        raise ValueError("quantize_batch takes 1 to 8 tensors")
+    descs = (_lib.QuantJob * len(jobs))()
+    outs, keep = [], []
+    dev = None
+    for i, jb in enumerate(jobs):
+        x = jb["x"]
+        if x.dtype == torch.float8_e4m3fn:
+            x = x.view(torch.uint8)
+        if x.dim() != 2 or not x.is_cuda:
+            raise TypeError("quantize_batch expects 2-D CUDA tensors")
+        if x.dtype == torch.float32:
+            src = _lib.NVFP4_SRC_F32
+        elif x.dtype == torch.bfloat16:
+            src = _lib.NVFP4_SRC_BF16
+        elif x.dtype == torch.uint8:
+            src = _lib.NVFP4_SRC_E4M3
+        else:
+            raise TypeError("quantize_batch: fp32, bf16 or E4M3 tensors")
+        x = x.contiguous()
+        keep.append(x)
+        dev = x.device
+        rows, cols = x.shape
+        out = jb.get("out")
+        if out is None:
+            codes, swz, lin, gs = _alloc_outputs(rows, cols, x.device, jb.get("swizzled", True),
+                                                 jb.get("linear", False))
+            out = NVFP4Tensor(codes, swz, lin, gs, rows, cols)
+        outs.append(out)
+        d = descs[i]
+        d.x, d.src = _ptr(x), src
+        d.fp8_scale = _ptr(jb.get("fp8_scale"))
+        d.rows, d.cols = rows, cols
+        d.static_amax = _ptr(jb.get("static_amax"))
+        d.codes, d.scales_swz = _ptr(out.codes), _ptr(out.scales_swz)
+        d.scales_lin, d.global_scale = _ptr(out.scales_lin), _ptr(out.global_scale)
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, 0, 0, 0)
+    ws = _workspace(dev, ws_bytes)
+    st = L.nvfp4_quantize_batch(descs, len(jobs), _ptr(ws), ws_bytes, _stream(dev))
+    check(st, "nvfp4_quantize_batch")
+    return outs
 
 
 def dequantize(q: NVFP4Tensor, out_dtype=torch.float32) -> torch.Tensor:

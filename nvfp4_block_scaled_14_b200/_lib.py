@@ -39,6 +39,21 @@ _sz = ctypes.c_size_t
 _int = ctypes.c_int
 _u32 = ctypes.c_uint32
 
+NVFP4_SRC_F32 = 0
+NVFP4_SRC_BF16 = 1
+NVFP4_SRC_E4M3 = 2
+NVFP4_MAX_QUANT_JOBS = 8
+
+
+class QuantJob(ctypes.Structure):
+    """nvfp4_quant_job: one tensor of nvfp4_quantize_batch."""
+    _fields_ = [("x", ctypes.c_void_p), ("src", ctypes.c_int), ("fp8_scale", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("static_amax", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("scales_swz", ctypes.c_void_p), ("scales_lin", ctypes.c_void_p),
+                ("global_scale", ctypes.c_void_p)]
+
+
 _SIGNATURES = {
     "nvfp4_status_str": ([_int], ctypes.c_char_p),
     "nvfp4_codes_bytes": ([_i64, _i64], _sz),
@@ -47,6 +62,7 @@ _SIGNATURES = {
     "nvfp4_quantize": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "nvfp4_quantize_fp8_src": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
                                _int),
+    "nvfp4_quantize_batch": ([ctypes.POINTER(QuantJob), _int, _vp, _sz, _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _int, _vp, _vp], _int),
     "nvfp4_linear": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _sz, _vp],
                      _int),

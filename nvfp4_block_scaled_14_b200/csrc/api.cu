@@ -88,6 +88,28 @@ nvfp4_status check_matrix(int64_t rows, int64_t cols)
 
 size_t quantize_ws_bytes() { return quantize_workspace_bytes(); }
 
+// Host-side checks of one quantize call (shared by nvfp4_quantize, _fp8_src and _batch).
+nvfp4_status check_quantize(const void *x, int64_t rows, int64_t cols, const float *static_amax,
+                            const uint8_t *codes, const uint8_t *scales_swz,
+                            const uint8_t *scales_lin, const float *global_scale, const void *ws,
+                            size_t ws_bytes)
+{
+    nvfp4_status st = check_matrix(rows, cols);
+    if (st != NVFP4_OK)
+        return st;
+    const bool empty = rows == 0 || cols == 0;
+    if (!global_scale)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!empty && (!x || !codes || (!scales_swz && !scales_lin)))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales_swz) || !aligned16(scales_lin) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u) || !aligned16(ws))
+        return NVFP4_ERR_ALIGNMENT;
+    if (!static_amax && (!ws || ws_bytes < quantize_ws_bytes()))
+        return NVFP4_ERR_WORKSPACE;
+    return NVFP4_OK;
+}
+
 nvfp4_status quantize_common(const void *x, int src_type, const float *fp8_scale, int64_t rows,
                              int64_t cols, const float *static_amax, uint8_t *codes,
                              uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,
@@ -129,6 +151,32 @@ const char *nvfp4_status_str(nvfp4_status st)
     case NVFP4_ERR_UNSUPPORTED: return "device is not sm_100";
     }
     return "unknown status";
+}
+
+nvfp4_status nvfp4_quantize_batch(const nvfp4_quant_job *jobs, int njobs, void *ws,
+                                  size_t ws_bytes, cudaStream_t stream)
+{
+    if (!jobs || njobs < 1 || njobs > NVFP4_MAX_QUANT_JOBS)
+        return NVFP4_ERR_INVALID_ARG;
+    QuantJob jb[NVFP4_MAX_QUANT_JOBS];
+    for (int j = 0; j < njobs; ++j) {
+        const nvfp4_quant_job &q = jobs[j];
+        if (q.src != NVFP4_SRC_F32 && q.src != NVFP4_SRC_BF16 && q.src != NVFP4_SRC_E4M3)
+            return NVFP4_ERR_INVALID_ARG;
+        const nvfp4_status st =
+            check_quantize(q.x, q.rows, q.cols, q.static_amax, q.codes, q.scales_swz,
+                           q.scales_lin, q.global_scale, ws, ws_bytes);
+        if (st != NVFP4_OK)
+            return st;
+        jb[j] = QuantJob{q.x,          q.src,   q.src == NVFP4_SRC_E4M3 ? q.fp8_scale : nullptr,
+                         q.rows,       q.cols,  q.static_amax,
+                         q.codes,      q.scales_swz,
+                         q.scales_lin, q.global_scale};
+    }
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    return map_cuda(launch_quantize_batch(jb, njobs, ws, stream));
 }
 
 size_t nvfp4_codes_bytes(int64_t rows, int64_t cols)

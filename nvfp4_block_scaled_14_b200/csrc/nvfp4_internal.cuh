@@ -32,6 +32,18 @@ int num_sms();
 constexpr int kAmaxPartials = 1024;
 size_t quantize_workspace_bytes();
 
+// One tensor of a batched quantize (the fields of nvfp4_quant_job).
+struct QuantJob {
+    const void *x;
+    int src; // SrcType
+    const float *fp8_scale;
+    int64_t rows, cols;
+    const float *static_amax;
+    uint8_t *codes, *scales_swz, *scales_lin;
+    float *global_scale;
+};
+cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t s);
+
 cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale, int64_t rows,
                             int64_t cols, const float *static_amax, uint8_t *codes,
                             uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,

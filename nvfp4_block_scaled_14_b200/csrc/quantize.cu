@@ -41,7 +41,10 @@ constexpr int kFusedThreads = 1024;    // fused quantizer: one CTA per SM
 constexpr int kFusedChunk = 32 * 1024;  // fused quantizer: bulk-copy size
 constexpr int kFusedMaxChunks = 6;
 constexpr int kFusedCap = kFusedChunk * kFusedMaxChunks; // tensor bytes per CTA (192 KB)
-constexpr int kEncThreads = 1024;      // encode: 32 warps, two 16-value blocks per lane per item
+constexpr int kMaxQuantJobs = NVFP4_MAX_QUANT_JOBS; // tensors per batched quantize
+// encode: 24 warps, two 16-value blocks per lane per item (up to 80 registers a thread; at
+// 1024 threads the 64-register cap spills; measured 768 >= 1024 and 512 on 0.1-100 MB)
+constexpr int kEncThreads = 768;
 // The fused kernel runs tensors from kFusedMinBytes up to its shared-memory capacity. Below,
 // its grid-wide barrier and one-CTA-per-SM launch cost more than the second kernel and the
 // second read (from L2) save: measured on B200, bf16 / fp32 / fp8 from 0.1 to 25 MB, the
@@ -140,18 +143,19 @@ struct QuantArgs {
 };
 
 // K1: max |x| over a contiguous byte range per CTA, streamed through a shared-memory ring
-// with 1-D bulk copies; one partial per CTA.
+// with 1-D bulk copies; one partial per CTA. `bid` / `nblk`: this CTA's index among the CTAs
+// that share the tensor, and their number (the whole grid for one tensor, a slice of it in a
+// batch).
 template <int SRC>
-__global__ void __launch_bounds__(kAmaxThreads, 1)
-    amax_kernel(const uint8_t *__restrict__ x, int64_t nbytes, float *__restrict__ partials,
-                int *status)
+__device__ __forceinline__ void amax_body(const uint8_t *__restrict__ x, int64_t nbytes,
+                                          float *__restrict__ partials, int *status, int bid,
+                                          int nblk, uint8_t *ring)
 {
-    extern __shared__ __align__(128) uint8_t ring[];
     __shared__ uint64_t bars[kRing];
     __shared__ float s_red[kAmaxThreads / 32];
     const int64_t nvec = nbytes >> 4;
-    const int64_t per = ((nvec + gridDim.x - 1) / gridDim.x) << 4;
-    const int64_t b0 = min(nbytes, per * (int64_t)blockIdx.x);
+    const int64_t per = ((nvec + nblk - 1) / nblk) << 4;
+    const int64_t b0 = min(nbytes, per * (int64_t)bid);
     const int64_t b1 = min(nbytes, b0 + per);
     const int nchunks = (int)((b1 - b0 + kChunk - 1) / kChunk);
     if (threadIdx.x == 0) {
@@ -196,8 +200,17 @@ __global__ void __launch_bounds__(kAmaxThreads, 1)
         for (int o = 16; o > 0; o >>= 1)
             f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
         if (threadIdx.x == 0)
-            partials[blockIdx.x] = f;
+            partials[bid] = f;
     }
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(kAmaxThreads, 1)
+    amax_kernel(const uint8_t *__restrict__ x, int64_t nbytes, float *__restrict__ partials,
+                int *status)
+{
+    extern __shared__ __align__(128) uint8_t ring[];
+    amax_body<SRC>(x, nbytes, partials, status, blockIdx.x, gridDim.x, ring);
 }
 
 // Geometry of the fused kernel's warp items: a lane owns kBpl whole blocks (2 for bf16 / fp8,
@@ -452,7 +465,7 @@ __device__ __forceinline__ void store_lane(const QuantArgs &a, int64_t f0, uint3
 // atom with one store per lane: 16 bytes when all four rows are padding, else only the
 // padding rows' words (the real rows' words belong to the encoding lanes). The pad blocks of
 // real rows are written with their row's last scales.
-__device__ __forceinline__ void zero_pad_rows(const QuantArgs &a, int apb)
+__device__ __forceinline__ void zero_pad_rows(const QuantArgs &a, int apb, int bid, int nblk)
 {
     if (!a.sf_swz || (a.rows & 127) == 0)
         return;
@@ -460,8 +473,7 @@ __device__ __forceinline__ void zero_pad_rows(const QuantArgs &a, int apb)
     const int real = a.rows & 127;    // its real rows
     const int i = threadIdx.x & 31;   // line of the atom
     const int warps = blockDim.x >> 5;
-    for (int atom = blockIdx.x * warps + (threadIdx.x >> 5); atom < apb;
-         atom += gridDim.x * warps) {
+    for (int atom = bid * warps + (threadIdx.x >> 5); atom < apb; atom += nblk * warps) {
         uint8_t *line = a.sf_swz + ((int64_t)band * apb + atom) * 512 + i * 16;
         if (i >= real) {
             *reinterpret_cast<uint4 *>(line) = make_uint4(0u, 0u, 0u, 0u);
@@ -483,24 +495,42 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4 *p)
     return v;
 }
 
-// One block from its kVecs raw vectors: the E4M3 scale byte, and the 8 code bytes.
+// E2M1 codes of 16 fp32 values (already multiplied by the block's 1 / (sb * sg)), low
+// nibble first.
+__device__ __forceinline__ uint2 codes16(const float (&y)[16])
+{
+    return make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8));
+}
+
+// One block from its kVecs raw vectors: the E4M3 scale byte, and the 8 code bytes. The block
+// is widened to fp32 once (fp8: times s8); its maximum |v| is taken with float max on those
+// values (one instruction per value, and the same value as the maximum of the raw magnitudes:
+// fp8 upcasting rounds monotonically), then the codes of v * (1 / (sb * sg)).
 template <int SRC>
 __device__ __forceinline__ uint32_t encode_one(const uint4 *r, float s8, float sg, float t,
                                                float rt, const float *rcp_tab, uint2 &packed)
 {
-    constexpr int V = Enc<SRC>::kVecs;
-    const uint32_t sb = block_scale<SRC>(r, V, s8, sg, t, rt);
-    if constexpr (V == 4) { // fp32: 2 code bytes per vector
-        uint32_t c[4];
+    float v[16];
+    block_to_f32<SRC>(r, s8, v);
+    float m[4];
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-            c[v] = vec_codes<SRC>(r[v], s8, sb, rcp_tab).x;
-        packed = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-    } else if constexpr (V == 2) { // bf16: 4 per vector
-        packed = make_uint2(vec_codes<SRC>(r[0], s8, sb, rcp_tab).x,
-                            vec_codes<SRC>(r[1], s8, sb, rcp_tab).x);
-    } else { // fp8: 8 per vector
-        packed = vec_codes<SRC>(r[0], s8, sb, rcp_tab);
+    for (int i = 0; i < 4; ++i)
+        m[i] = fmaxf(fmaxf(fabsf(v[4 * i]), fabsf(v[4 * i + 1])),
+                     fmaxf(fabsf(v[4 * i + 2]), fabsf(v[4 * i + 3])));
+    const float bmax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+    const uint32_t sb = sg > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
+    packed = make_uint2(0u, 0u);
+    if (sb != 0u) {
+        const float rcp = rcp_tab[sb];
+        const float2 rr = make_float2(rcp, rcp);
+        float y[16];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+            const float2 q = __fmul2_rn(make_float2(v[j], v[j + 1]), rr);
+            y[j] = q.x;
+            y[j + 1] = q.y;
+        }
+        packed = codes16(y);
     }
     return sb;
 }
@@ -512,7 +542,7 @@ __device__ __forceinline__ uint32_t encode_one(const uint4 *r, float s8, float s
 // before waiting on the amax kernel (programmatic dependent launch), so the loads overlap its
 // tail; later items are double-buffered.
 template <int SRC>
-__global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs a)
+__device__ __forceinline__ void encode_body(const QuantArgs &a, int bid, int nblk)
 {
     __shared__ float s_sg;
     __shared__ float s_rcp[128];
@@ -524,8 +554,8 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
     const int runs = (nb + 63) >> 6;  // 64-block runs per row (one per warp item)
     const int apb = (nb + 3) >> 2;    // scale atoms per 128-row band
     const int64_t row_bytes = (int64_t)a.cols * Src<SRC>::kBytes;
-    const int r0 = (int)((int64_t)a.rows * blockIdx.x / gridDim.x);
-    const int r1 = (int)((int64_t)a.rows * (blockIdx.x + 1) / gridDim.x);
+    const int r0 = (int)((int64_t)a.rows * bid / nblk);
+    const int r1 = (int)((int64_t)a.rows * (bid + 1) / nblk);
     const int items = (r1 - r0) * runs;
     const uint8_t *xbase = a.x + (int64_t)r0 * row_bytes;
 
@@ -590,7 +620,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
         if (threadIdx.x == 0) {
             const float sg = __fdiv_rn(g, 2688.0f); // 6 * 448
             s_sg = sg;
-            if (blockIdx.x == 0)
+            if (bid == 0)
                 *a.global_scale = sg;
         }
     }
@@ -633,22 +663,28 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
         // fp32 blocks are 64 bytes: one item in flight keeps the registers in budget
         while (it < items) {
             encode_store(roa, b0a, ra);
-            it += 32;
+            it += kEncThreads / 32;
             load_item(it, ra, roa, b0a);
         }
     } else {
         while (it < items) {
-            load_item(it + 32, rb, rob, b0b);
+            load_item(it + kEncThreads / 32, rb, rob, b0b);
             encode_store(roa, b0a, ra);
-            it += 32;
+            it += kEncThreads / 32;
             if (it >= items)
                 break;
-            load_item(it + 32, ra, roa, b0a);
+            load_item(it + kEncThreads / 32, ra, roa, b0a);
             encode_store(rob, b0b, rb);
-            it += 32;
+            it += kEncThreads / 32;
         }
     }
-    zero_pad_rows(a, apb);
+    zero_pad_rows(a, apb, bid, nblk);
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs a)
+{
+    encode_body<SRC>(a, blockIdx.x, gridDim.x);
 }
 
 // Fused single-pass quantizer for tensors that fit in the CTAs' shared memory (one CTA per
@@ -806,7 +842,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
         if (f0 < nblocks)
             store_lane<SRC>(a, f0, nb, apb, cw, sb0, sb1);
     }
-    zero_pad_rows(a, apb);
+    zero_pad_rows(a, apb, blockIdx.x, gridDim.x);
 }
 
 template <int SRC>
@@ -903,6 +939,97 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
     return cudaLaunchKernelEx(&cfg, encode_kernel<SRC>, qa);
 }
 
+
+// ---------------------------------------------------------------------------------------
+// Batched quantize: several tensors in one amax launch and one encode launch. The grid's
+// CTAs are split over the tensors in proportion to their bytes; a CTA finds its tensor by
+// its index and runs the single-tensor body on its share (its own partial maxima, its own
+// global scale), so the tensors' memory traffic overlaps instead of running back to back.
+// ---------------------------------------------------------------------------------------
+
+struct QuantGroup {
+    int njobs;
+    int src[kMaxQuantJobs];
+    int amax_cta0[kMaxQuantJobs + 1]; // amax CTAs of job j: [amax_cta0[j], amax_cta0[j + 1])
+    int enc_cta0[kMaxQuantJobs + 1];  // encode CTAs of job j
+    QuantArgs job[kMaxQuantJobs];
+};
+
+__device__ __forceinline__ int job_of(const int *cta0, int njobs)
+{
+    int j = 0;
+    while (j + 1 < njobs && (int)blockIdx.x >= cta0[j + 1])
+        ++j;
+    return j;
+}
+
+__global__ void __launch_bounds__(kAmaxThreads, 1) amax_group_kernel(const __grid_constant__ QuantGroup g)
+{
+    extern __shared__ __align__(128) uint8_t ring[];
+    const int j = job_of(g.amax_cta0, g.njobs);
+    const QuantArgs &a = g.job[j];
+    const int bid = blockIdx.x - g.amax_cta0[j], nblk = g.amax_cta0[j + 1] - g.amax_cta0[j];
+    float *part = const_cast<float *>(a.partials);
+    switch (g.src[j]) {
+    case kSrcF32: amax_body<kSrcF32>(a.x, a.nbytes, part, a.status, bid, nblk, ring); break;
+    case kSrcBF16: amax_body<kSrcBF16>(a.x, a.nbytes, part, a.status, bid, nblk, ring); break;
+    default: amax_body<kSrcE4M3>(a.x, a.nbytes, part, a.status, bid, nblk, ring); break;
+    }
+}
+
+__global__ void __launch_bounds__(kEncThreads, 1) encode_group_kernel(const __grid_constant__ QuantGroup g)
+{
+    const int j = job_of(g.enc_cta0, g.njobs);
+    const QuantArgs &a = g.job[j];
+    const int bid = blockIdx.x - g.enc_cta0[j], nblk = g.enc_cta0[j + 1] - g.enc_cta0[j];
+    switch (g.src[j]) {
+    case kSrcF32: encode_body<kSrcF32>(a, bid, nblk); break;
+    case kSrcBF16: encode_body<kSrcBF16>(a, bid, nblk); break;
+    default: encode_body<kSrcE4M3>(a, bid, nblk); break;
+    }
+}
+
+template <int SRC> void fill_args(QuantArgs &qa, const QuantJob &jb)
+{
+    qa.x = reinterpret_cast<const uint8_t *>(jb.x);
+    qa.fp8_scale = jb.fp8_scale;
+    qa.rows = (int)jb.rows;
+    qa.cols = (int)jb.cols;
+    qa.static_amax = jb.static_amax;
+    qa.codes = jb.codes;
+    qa.sf_swz = jb.scales_swz;
+    qa.sf_lin = jb.scales_lin;
+    qa.global_scale = jb.global_scale;
+    qa.nbytes = jb.rows * jb.cols * Src<SRC>::kBytes;
+    const uint64_t nb = (uint64_t)(jb.cols / 16);
+    qa.nb_magic = nb > 1 ? (uint32_t)((((uint64_t)1 << 32) + nb - 1) / nb) : 0u;
+    qa.blocks_fit32 = (uint64_t)jb.rows * nb < ((uint64_t)1 << 32) ? 1 : 0;
+    const uint64_t runs = (nb + 63) / 64;
+    qa.runs_magic = runs > 1 ? (uint32_t)((((uint64_t)1 << 32) + runs - 1) / runs) : 0u;
+    qa.status = device_status_ptr();
+}
+
+// Split `total` CTAs over jobs in proportion to weight[j] (0 = no CTA), at least one each,
+// at most cap[j]; writes the prefix sums to cta0 and returns the CTA count.
+int split_ctas(int n, const int64_t *weight, const int64_t *cap, int total, int *cta0)
+{
+    int64_t wsum = 0;
+    for (int j = 0; j < n; ++j)
+        wsum += weight[j];
+    cta0[0] = 0;
+    for (int j = 0; j < n; ++j) {
+        int64_t c = 0;
+        if (weight[j] > 0) {
+            c = wsum > 0 ? (int64_t)total * weight[j] / wsum : 1;
+            if (c < 1)
+                c = 1;
+            if (c > cap[j])
+                c = cap[j];
+        }
+        cta0[j + 1] = cta0[j] + (int)c;
+    }
+    return cta0[n];
+}
 } // namespace
 
 size_t quantize_workspace_bytes() { return (size_t)kAmaxPartials * sizeof(float); }
@@ -923,6 +1050,69 @@ cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale,
         return launch_typed<kSrcE4M3>(x, fp8_scale, rows, cols, static_amax, codes, scales_swz,
                                       scales_lin, global_scale, ws, s);
     }
+}
+
+cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t s)
+{
+    const int sms = num_sms();
+    QuantGroup g{};
+    g.njobs = njobs;
+    int64_t amax_w[kMaxQuantJobs], amax_cap[kMaxQuantJobs], enc_w[kMaxQuantJobs],
+        enc_cap[kMaxQuantJobs];
+    bool dynamic = false;
+    for (int j = 0; j < njobs; ++j) {
+        const QuantJob &jb = jobs[j];
+        g.src[j] = jb.src;
+        switch (jb.src) {
+        case kSrcF32: fill_args<kSrcF32>(g.job[j], jb); break;
+        case kSrcBF16: fill_args<kSrcBF16>(g.job[j], jb); break;
+        default: fill_args<kSrcE4M3>(g.job[j], jb); break;
+        }
+        const int64_t nbytes = g.job[j].nbytes;
+        const bool dyn = !jb.static_amax && nbytes > 0;
+        dynamic = dynamic || dyn;
+        amax_w[j] = dyn ? nbytes : 0;
+        amax_cap[j] = (nbytes + kChunk - 1) / kChunk;
+        enc_w[j] = nbytes > 0 ? nbytes : 0;
+        enc_cap[j] = jb.rows;
+    }
+    int amax_total = sms < kAmaxPartials ? sms : kAmaxPartials;
+    const int na = split_ctas(njobs, amax_w, amax_cap, amax_total, g.amax_cta0);
+    for (int j = 0; j < njobs; ++j) {
+        g.job[j].partials = reinterpret_cast<const float *>(ws) + g.amax_cta0[j];
+        g.job[j].npartials = g.amax_cta0[j + 1] - g.amax_cta0[j];
+    }
+    const int ne = split_ctas(njobs, enc_w, enc_cap, sms, g.enc_cta0);
+    cudaError_t e;
+    if (dynamic && na > 0) {
+        const size_t smem = (size_t)kRing * kChunk;
+        static std::once_flag attr[64];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaError_t ae = cudaSuccess;
+        std::call_once(attr[dev & 63], [&]() {
+            ae = cudaFuncSetAttribute(amax_group_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        });
+        if (ae != cudaSuccess)
+            return ae;
+        amax_group_kernel<<<na, kAmaxThreads, smem, s>>>(g);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+    }
+    if (ne == 0)
+        return cudaSuccess;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)ne);
+    cfg.blockDim = dim3(kEncThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = (dynamic && na > 0) ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, encode_group_kernel, g);
 }
 
 } // namespace nvfp4

@@ -73,6 +73,42 @@ def test_quantize_single_pass_sizes(kind, rows, cols, static):
     assert_quant_equal(gpu_quantize(x, amax=amax), O.quantize(x, amax=amax))
 
 
+def test_quantize_batch_matches_single_calls():
+    # a weight re-quantized from FP8, bf16 activations, an fp32 tensor with a static amax, a
+    # tiny ragged one: one batched call gives each exactly its own quantization
+    w8, s8 = W.to_fp8_tensorwise(W.normal((3072, 3072), 0.02, 33, 1))
+    xb = W.to_bf16_bits(W.normal((1000, 3072), 1.0, 33, 2))
+    xf = W.normal((300, 1056), 1.0, 33, 3)
+    xt = W.to_bf16_bits(W.normal((7, 96), 1.0, 33, 4))
+    jobs = [{"x": dev_tensor(w8), "fp8_scale": scalar_dev(s8), "linear": True},
+            {"x": dev_tensor(xb), "linear": True},
+            {"x": dev_tensor(xf), "static_amax": scalar_dev(2.5), "linear": True},
+            {"x": dev_tensor(xt), "linear": True}]
+    q = nv.quantize_batch(jobs)
+    torch.cuda.synchronize()
+    assert_quant_equal(q[0], O.quantize(w8, fp8_scale=s8))
+    assert_quant_equal(q[1], O.quantize(xb))
+    assert_quant_equal(q[2], O.quantize(xf, amax=2.5))
+    assert_quant_equal(q[3], O.quantize(xt))
+    assert nv.sync_status() == 0
+
+
+def test_quantize_batch_rejects_bad_jobs():
+    from nvfp4_block_scaled_14_b200 import _lib as L
+    lib = L.load()
+    assert lib.nvfp4_quantize_batch(None, 1, None, 0, None) == L.NVFP4_ERR_INVALID_ARG
+    jobs = (L.QuantJob * 9)()
+    assert lib.nvfp4_quantize_batch(jobs, 9, None, 0, None) == L.NVFP4_ERR_INVALID_ARG
+    x = torch.zeros((4, 48), dtype=torch.bfloat16, device="cuda")  # cols not a multiple of 32
+    q = gpu_quantize(W.to_bf16_bits(W.normal((4, 64), 1.0, 33, 5)))
+    j = (L.QuantJob * 1)()
+    j[0].x, j[0].src, j[0].rows, j[0].cols = x.data_ptr(), L.NVFP4_SRC_BF16, 4, 48
+    j[0].static_amax = q.global_scale.data_ptr()
+    j[0].codes, j[0].scales_swz = q.codes.data_ptr(), q.scales_swz.data_ptr()
+    j[0].global_scale = q.global_scale.data_ptr()
+    assert lib.nvfp4_quantize_batch(j, 1, None, 0, None) == L.NVFP4_ERR_SHAPE
+
+
 def test_quantize_fp8_source_double_quant():
     w8, s8 = W.to_fp8_tensorwise(W.normal((320, 384), 0.02, 22, 1))
     assert_quant_equal(gpu_quantize(w8, fp8_scale=s8), O.quantize(w8, fp8_scale=s8))

@@ -55,43 +55,73 @@ constexpr uint32_t kSpinLimit = 1u << 24;
 
 template <int SRC> struct Src;
 
-// |x| orders like the magnitude bits of x for finite values, so maxima are taken on the bit
-// patterns with SIMD integer max: exact, order-free.
+// Maxima of |x| are folded into a 32-bit container per source type, with native max
+// instructions (exact, order-free): fp32 -> the float max itself; bf16 -> a bf16x2 pair of
+// magnitudes (packed bf16 max, two values an instruction); fp8 -> an f16x2 pair of |e|
+// (E4M3 widens to f16 exactly; packed f16 max). mag_to_f32 gives the maximum as fp32 (fp8:
+// of |e|, before the fp8 scale).
+__device__ __forceinline__ uint32_t hmax2_bf16(uint32_t a, uint32_t b)
+{
+    __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162 *>(&a),
+                               *reinterpret_cast<__nv_bfloat162 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ uint32_t hmax2_f16(uint32_t a, uint32_t b)
+{
+    __half2 r = __hmax2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// two E4M3 bytes -> f16x2 of their magnitudes (exact)
+__device__ __forceinline__ uint32_t e4m3x2_abs_to_f16x2(uint32_t b2)
+{
+    uint32_t h;
+    const uint16_t in = (uint16_t)(b2 & 0x7F7Fu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(in));
+    return h;
+}
+
 template <> struct Src<kSrcF32> {
     static constexpr int kBytes = 4;
-    __device__ static uint32_t vec_magmax(uint4 v) // fp32 magnitude bits
+    __device__ static uint32_t vec_magmax(uint4 v)
     {
-        return max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu),
-                   max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu));
+        return __float_as_uint(fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                                     fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
     }
+    __device__ static uint32_t fold(uint32_t a, uint32_t b) { return max(a, b); }
     __device__ static float mag_to_f32(uint32_t m) { return __uint_as_float(m); }
 };
 
 template <> struct Src<kSrcBF16> {
     static constexpr int kBytes = 2;
-    __device__ static uint32_t vec_magmax(uint4 v) // two 16-bit lanes of magnitude bits
+    __device__ static uint32_t vec_magmax(uint4 v)
     {
         const uint32_t k = 0x7FFF7FFFu;
-        return __vmaxu2(__vmaxu2(v.x & k, v.y & k), __vmaxu2(v.z & k, v.w & k));
+        return hmax2_bf16(hmax2_bf16(v.x & k, v.y & k), hmax2_bf16(v.z & k, v.w & k));
     }
+    __device__ static uint32_t fold(uint32_t a, uint32_t b) { return hmax2_bf16(a, b); }
     __device__ static float mag_to_f32(uint32_t m)
     {
-        return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+        return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
     }
 };
 
 template <> struct Src<kSrcE4M3> {
     static constexpr int kBytes = 1;
-    __device__ static uint32_t vec_magmax(uint4 v) // four 8-bit lanes of magnitude bits
+    __device__ static uint32_t vec_magmax(uint4 v)
     {
-        const uint32_t k = 0x7F7F7F7Fu;
-        return __vmaxu4(__vmaxu4(v.x & k, v.y & k), __vmaxu4(v.z & k, v.w & k));
+        const uint32_t a = hmax2_f16(e4m3x2_abs_to_f16x2(v.x), e4m3x2_abs_to_f16x2(v.x >> 16));
+        const uint32_t b = hmax2_f16(e4m3x2_abs_to_f16x2(v.y), e4m3x2_abs_to_f16x2(v.y >> 16));
+        const uint32_t c = hmax2_f16(e4m3x2_abs_to_f16x2(v.z), e4m3x2_abs_to_f16x2(v.z >> 16));
+        const uint32_t d = hmax2_f16(e4m3x2_abs_to_f16x2(v.w), e4m3x2_abs_to_f16x2(v.w >> 16));
+        return hmax2_f16(hmax2_f16(a, b), hmax2_f16(c, d));
     }
+    __device__ static uint32_t fold(uint32_t a, uint32_t b) { return hmax2_f16(a, b); }
     __device__ static float mag_to_f32(uint32_t m) // |e4m3| (before the fp8 scale)
     {
-        const uint32_t b = max(max(m & 0xFFu, (m >> 8) & 0xFFu),
-                               max((m >> 16) & 0xFFu, m >> 24));
-        return e4m3_to_f32(b);
+        const __half2 h = *reinterpret_cast<const __half2 *>(&m);
+        return fmaxf(__low2float(h), __high2float(h));
     }
 };
 
@@ -114,15 +144,10 @@ __device__ __forceinline__ uint32_t e4m3_of_quotient(float bmax, float t, float 
     return cvt_e4m3(__fdiv_rn(bmax, t));
 }
 
-// Fold a magnitude-bit accumulator (per source type) into another.
+// Fold a magnitude accumulator (per source type) into another.
 template <int SRC> __device__ __forceinline__ uint32_t mag_fold(uint32_t a, uint32_t b)
 {
-    if constexpr (SRC == kSrcF32)
-        return max(a, b);
-    else if constexpr (SRC == kSrcBF16)
-        return __vmaxu2(a, b);
-    else
-        return __vmaxu4(a, b);
+    return Src<SRC>::fold(a, b);
 }
 
 struct QuantArgs {

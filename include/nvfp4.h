@@ -232,6 +232,16 @@ nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_bat
                                          cudaStream_t stream);
 
 /*
+ * Test of the failure-detection path. No counterpart in the paper. Launches one small kernel
+ * whose bounded wait cannot complete (an mbarrier that nothing arrives on); it gives up after
+ * a short poll limit and records NVFP4_ERR_TIMEOUT in the device-side status word, exactly as
+ * a library kernel does when one of its waits runs out, and returns normally (no fault, the
+ * context stays usable). The next nvfp4_sync_status on the stream reports NVFP4_ERR_TIMEOUT.
+ * Returns the launch status.
+ */
+nvfp4_status nvfp4_selftest_wait_timeout(cudaStream_t stream);
+
+/*
  * Synchronize the stream, then report and clear the library's device-side status word
  * (set by a kernel whose bounded wait gave up: NVFP4_ERR_TIMEOUT). Returns NVFP4_ERR_CUDA if
  * the synchronization itself failed.

@@ -72,6 +72,7 @@ _SIGNATURES = {
                              _int),
     "nvfp4_calib_percentile_amax": ([ctypes.POINTER(_vp), _int, _i64, _int, _u32, _u32, _vp,
                                      _vp, _vp, _sz, _vp], _int),
+    "nvfp4_selftest_wait_timeout": ([_vp], _int),
     "nvfp4_sync_status": ([_vp], _int),
 }
 

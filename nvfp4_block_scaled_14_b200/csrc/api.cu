@@ -340,6 +340,14 @@ nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_bat
                                  out_pct, out_max, ws, stream));
 }
 
+nvfp4_status nvfp4_selftest_wait_timeout(cudaStream_t stream)
+{
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    return map_cuda(launch_wait_timeout_selftest(stream));
+}
+
 nvfp4_status nvfp4_sync_status(cudaStream_t stream)
 {
     if (cudaStreamSynchronize(stream) != cudaSuccess)

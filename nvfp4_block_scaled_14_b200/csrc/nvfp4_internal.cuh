@@ -44,6 +44,9 @@ struct QuantJob {
 };
 cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t s);
 
+// Launches a kernel whose bounded wait cannot complete (selftest.cu).
+cudaError_t launch_wait_timeout_selftest(cudaStream_t s);
+
 cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale, int64_t rows,
                             int64_t cols, const float *static_amax, uint8_t *codes,
                             uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,

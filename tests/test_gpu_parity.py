@@ -386,5 +386,21 @@ def test_calib_ragged_element_count():
     assert (float(p.cpu()[0]), float(m.cpu()[0])) == O.percentile_abs(xs)
 
 
+def test_calib_skewed_layout():
+    # every 256th 16-byte vector large, the rest small (the large values sit at the same
+    # offset of every CTA's range): median and p99.9 still exact
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    nvec = sms * 256
+    g = np.random.Generator(np.random.PCG64(35))
+    x = (g.random((nvec, 8), dtype=np.float32) * 0.01).astype(np.float32)
+    x[::256] = 50.0 + g.random((nvec // 256, 8), dtype=np.float32)
+    xb = W.to_bf16_bits(x.reshape(1, -1))
+    for num, den in [(1, 2), (999, 1000)]:
+        p, m = nv.calib_percentile_amax([dev_tensor(xb), dev_tensor(xb)], num, den)
+        torch.cuda.synchronize()
+        f = W.bf16_bits_to_f32(xb)
+        assert (float(p.cpu()[0]), float(m.cpu()[0])) == O.percentile_abs([f, f], num, den)
+
+
 def test_sync_status_clean():
     assert nv.sync_status() == 0

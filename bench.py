@@ -256,7 +256,11 @@ def extras(nv, W, dev, hbm, fp4_peak):
                 ("quantize_x_then_linear", [lambda q=q: (nv.quantize(xd, out=qa),
                                                          nv.linear(qa, q, out=y,
                                                                    resident_weights=True))
-                                            for q in qws])]:
+                                            for q in qws]),
+                # the same decode layer in one call (fused for M <= 16)
+                ("linear_dynamic", [lambda q=q: nv.linear_dynamic(xd, q, out=y,
+                                                                  resident_weights=True)
+                                    for q in qws])]:
             avg, med = op_timer(fns)
             gbs = wbytes / (avg * 1e-3) / 1e9
             row[key] = {"us": avg * 1e3, "GB/s_weights": gbs, "frac_hbm": gbs / hbm,

@@ -57,7 +57,8 @@ typedef enum {
     NVFP4_OP_QUANTIZE = 0,   /* m = rows, k = cols (n ignored) */
     NVFP4_OP_LINEAR = 1,     /* m = M, n = N, k = K */
     NVFP4_OP_CALIB_BF16 = 2, /* m, n, k ignored */
-    NVFP4_OP_CALIB_F32 = 3   /* m, n, k ignored */
+    NVFP4_OP_CALIB_F32 = 3,  /* m, n, k ignored */
+    NVFP4_OP_LINEAR_DYNAMIC = 4 /* m = M, n = N, k = K of nvfp4_linear_dynamic */
 } nvfp4_op;
 
 /* Human-readable name of a status. Never NULL. */
@@ -188,6 +189,26 @@ nvfp4_status nvfp4_linear_ex(const uint8_t *a_codes, const uint8_t *a_scales_swz
                              const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
                              int64_t N, int64_t K, nvfp4_dtype out_dt, void *y, void *ws,
                              size_t ws_bytes, uint32_t flags, cudaStream_t stream);
+
+/*
+ * Linear layer on unquantized activations: Y = dequant(Q(x)) . dequant(W)^T, where Q(x) is
+ * exactly what nvfp4_quantize(x, dynamic per-tensor amax) gives ("Qwen3-VL-8B-Instruct-
+ * heretic-NVFP4", "Quantization Details": activations quantized at runtime from the per-tensor
+ * amax), and the product is nvfp4_linear's. x: M x K of x_dt (NVFP4_F32 or NVFP4_BF16),
+ * row-major, 16-byte aligned; W as in nvfp4_linear. x_gs_out (device fp32, may be NULL)
+ * receives the activations' global scale.
+ * For M <= 16 (decode) one kernel does both: every thread-block cluster takes the tensor amax
+ * itself, each CTA encodes its K range of x straight into the tensor-core operand in shared
+ * memory, and the weights stream as in nvfp4_linear (flags as in nvfp4_linear_ex), so the
+ * quantized activations never go to HBM and no quantize kernels run before the GEMV. Other
+ * shapes run nvfp4_quantize and nvfp4_linear, with the quantized activations in ws.
+ * ws: nvfp4_workspace_bytes(NVFP4_OP_LINEAR_DYNAMIC, M, N, K) bytes (0 for the fused case).
+ */
+nvfp4_status nvfp4_linear_dynamic(const void *x, nvfp4_dtype x_dt, const uint8_t *w_codes,
+                                  const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
+                                  int64_t N, int64_t K, nvfp4_dtype out_dt, void *y,
+                                  float *x_gs_out, void *ws, size_t ws_bytes, uint32_t flags,
+                                  cudaStream_t stream);
 
 /*
  * nvfp4_linear without a caller-supplied workspace. No counterpart in the paper: it exists for

@@ -22,6 +22,7 @@ from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_LINEAR_DEFAULT, NVFP4_LINEAR_RES
                    NVFP4Error, check, load)
 
 __all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "quantize_batch", "dequantize", "linear",
+           "linear_dynamic",
            "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
 
 
@@ -206,6 +207,35 @@ def linear(a: NVFP4Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
                            _ptr(w.codes), _ptr(w.scales_swz), _ptr(w.global_scale), M, N, K, dt,
                            _ptr(out), _ptr(ws), ws_bytes, flags, _stream(dev))
     check(st, "nvfp4_linear_ex")
+    return out
+
+
+def linear_dynamic(x: torch.Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
+                   out: torch.Tensor = None, resident_weights: bool = False,
+                   x_gs_out: torch.Tensor = None) -> torch.Tensor:
+    """Y = dequant(quantize(x)) . dequant(w)^T with the dynamic per-tensor amax, from fp32 / bf16
+    activations x [M x K]; one fused kernel for M <= 16. x_gs_out (1-element fp32 CUDA tensor)
+    receives the activations' global scale."""
+    if x.dtype not in (torch.float32, torch.bfloat16) or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("linear_dynamic expects a 2-D CUDA fp32 or bf16 tensor")
+    x = x.contiguous()
+    M, K = x.shape
+    if K != w.cols:
+        raise ValueError("K mismatch")
+    N = w.rows
+    dev = x.device
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(_lib.NVFP4_OP_LINEAR_DYNAMIC, M, N, K)
+    ws = _workspace(dev, ws_bytes)
+    flags = NVFP4_LINEAR_RESIDENT_WEIGHTS if resident_weights else NVFP4_LINEAR_DEFAULT
+    st = L.nvfp4_linear_dynamic(_ptr(x), NVFP4_F32 if x.dtype == torch.float32 else NVFP4_BF16,
+                                _ptr(w.codes), _ptr(w.scales_swz), _ptr(w.global_scale), M, N, K,
+                                NVFP4_F32 if out.dtype == torch.float32 else NVFP4_BF16,
+                                _ptr(out), _ptr(x_gs_out), _ptr(ws), ws_bytes, flags,
+                                _stream(dev))
+    check(st, "nvfp4_linear_dynamic")
     return out
 
 

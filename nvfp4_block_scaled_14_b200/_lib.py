@@ -30,6 +30,7 @@ NVFP4_OP_QUANTIZE = 0
 NVFP4_OP_LINEAR = 1
 NVFP4_OP_CALIB_BF16 = 2
 NVFP4_OP_CALIB_F32 = 3
+NVFP4_OP_LINEAR_DYNAMIC = 4
 
 HEADER = os.path.join(os.path.dirname(_build.PKG), "include", "nvfp4.h")
 
@@ -68,6 +69,8 @@ _SIGNATURES = {
                      _int),
     "nvfp4_linear_ex": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _sz, _u32,
                          _vp], _int),
+    "nvfp4_linear_dynamic": ([_vp, _int, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _vp,
+                              _sz, _u32, _vp], _int),
     "nvfp4_linear_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp],
                              _int),
     "nvfp4_calib_percentile_amax": ([ctypes.POINTER(_vp), _int, _i64, _int, _u32, _u32, _vp,

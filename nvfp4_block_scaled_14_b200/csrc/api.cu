@@ -134,6 +134,30 @@ nvfp4_status quantize_common(const void *x, int src_type, const float *fp8_scale
                                     scales_swz, scales_lin, global_scale, ws, s));
 }
 
+// Workspace of nvfp4_linear_dynamic when it runs as quantize + linear: the quantized
+// activations (codes, swizzled scales, global scale), the quantize workspace and the linear
+// workspace, each 256-byte aligned. total = 0 when the fused kernel takes the shape.
+struct DynWs {
+    size_t codes, scales, gs, qws, lws, total;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+DynWs linear_dynamic_ws(int64_t M, int64_t N, int64_t K)
+{
+    DynWs d{};
+    LinearPlan pl;
+    if (plan_linear_xq(M, N, K, &pl))
+        return d;
+    d.codes = 0;
+    d.scales = d.codes + align256(nvfp4_codes_bytes(M, K));
+    d.gs = d.scales + align256(nvfp4_scales_bytes(M, K, 1));
+    d.qws = d.gs + 256;
+    d.lws = d.qws + align256(quantize_ws_bytes());
+    d.total = d.lws + align256(plan_linear(M, N, K).ws_bytes);
+    return d;
+}
+
 } // namespace
 
 extern "C" {
@@ -204,6 +228,10 @@ size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
         if (m <= 0 || n <= 0 || k <= 0)
             return 0;
         return plan_linear(m, n, k).ws_bytes;
+    case NVFP4_OP_LINEAR_DYNAMIC:
+        if (m <= 0 || n <= 0 || k <= 0)
+            return 0;
+        return linear_dynamic_ws(m, n, k).total;
     case NVFP4_OP_CALIB_BF16: return calib_workspace_bytes(1);
     case NVFP4_OP_CALIB_F32: return calib_workspace_bytes(0);
     }
@@ -262,6 +290,58 @@ nvfp4_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales_swz, c
 {
     return nvfp4_linear_ex(a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs, M, N, K,
                            out_dt, y, ws, ws_bytes, 0u, stream);
+}
+
+nvfp4_status nvfp4_linear_dynamic(const void *x, nvfp4_dtype x_dt, const uint8_t *w_codes,
+                                  const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
+                                  int64_t N, int64_t K, nvfp4_dtype out_dt, void *y,
+                                  float *x_gs_out, void *ws, size_t ws_bytes, uint32_t flags,
+                                  cudaStream_t stream)
+{
+    if (flags & ~(uint32_t)NVFP4_LINEAR_RESIDENT_WEIGHTS)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || K % 32 != 0)
+        return NVFP4_ERR_SHAPE;
+    if ((out_dt != NVFP4_F32 && out_dt != NVFP4_BF16) ||
+        (x_dt != NVFP4_F32 && x_dt != NVFP4_BF16))
+        return NVFP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (!y)
+        return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    const size_t esz = out_dt == NVFP4_BF16 ? 2 : 4;
+    if (K == 0)
+        return map_cuda(cudaMemsetAsync(y, 0, (size_t)M * N * esz, stream));
+    if (!x || !w_codes || !w_scales_swz || !w_gs)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales_swz) || !aligned16(y) ||
+        !aligned16(ws) || (reinterpret_cast<uintptr_t>(w_gs) & 3u) ||
+        (reinterpret_cast<uintptr_t>(x_gs_out) & 3u))
+        return NVFP4_ERR_ALIGNMENT;
+    LinearPlan pl;
+    if (plan_linear_xq(M, N, K, &pl)) {
+        st = NVFP4_OK;
+        const cudaError_t e =
+            launch_linear_xq(pl, x, x_dt == NVFP4_BF16, w_codes, w_scales_swz, w_gs, M, N, K,
+                             out_dt == NVFP4_BF16, y, x_gs_out, flags, stream, &st);
+        return st != NVFP4_OK ? st : map_cuda(e);
+    }
+    // quantize + linear, the quantized activations in ws
+    const DynWs d = linear_dynamic_ws(M, N, K);
+    if (!ws || ws_bytes < d.total)
+        return NVFP4_ERR_WORKSPACE;
+    uint8_t *w = reinterpret_cast<uint8_t *>(ws);
+    float *gs = x_gs_out ? x_gs_out : reinterpret_cast<float *>(w + d.gs);
+    st = quantize_common(x, x_dt == NVFP4_BF16 ? kSrcBF16 : kSrcF32, nullptr, M, K, nullptr,
+                         w + d.codes, w + d.scales, nullptr, gs, w + d.qws,
+                         quantize_ws_bytes(), stream);
+    if (st != NVFP4_OK)
+        return st;
+    return nvfp4_linear_ex(w + d.codes, w + d.scales, gs, w_codes, w_scales_swz, w_gs, M, N, K,
+                           out_dt, y, w + d.lws, ws_bytes - d.lws, flags, stream);
 }
 
 nvfp4_status nvfp4_linear_ex(const uint8_t *a_codes, const uint8_t *a_scales_swz,

@@ -35,7 +35,9 @@
 #include <cuda.h>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
+#include "nvfp4_encode.cuh"
 #include "nvfp4_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -88,6 +90,7 @@ template <int BN, int STAGES = (BN == 256 ? NVFP4_STAGES_256 : (BN == 128 ? 6 : 
     // instruction descriptor: E2M1 x E2M1, K-major both, UE4M3 scales, M = 128, N = BN
     static constexpr uint32_t kIdesc =
         (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static constexpr bool kResidentB = false;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kUsedCols <= 512, "TMEM budget");
 };
@@ -947,16 +950,49 @@ __global__ void splitk_reduce_kernel(const float *__restrict__ partial, int spli
 // previous kernel of the stream, its global reads and writes wait for that kernel.
 // ---------------------------------------------------------------------------------------
 
-template <int BN> struct SmallCfg {
+// Fused-activation layout (M <= 32): the TMA ring carries W and its scales only; the
+// activations' codes (B operand, 128B-swizzled, one BN x 128-byte tile per k-tile) and scale
+// atoms (2 KB per k-tile) of this CTA's k-range (at most kXqMaxKt k-tiles) stay resident,
+// written by the CTA itself from the bf16 / fp32 activations.
+constexpr int kXqMaxKt = 8;
+template <int BN> struct XqLayout {
+    static constexpr int kStages = BN <= 16 ? 4 : 3;
+    static constexpr int kSfbBands = 1;
+    static constexpr int kABytes = BM * 128;
+    static constexpr int kBBytes = BN * 128; // per resident k-tile
+    static constexpr int kSfaBytes = 4 * 512;
+    static constexpr int kSfbBytes = 4 * 512; // per resident k-tile
+    static constexpr int kOffSfa = kStages * kABytes;
+    static constexpr int kOffB = kOffSfa + kStages * kSfaBytes; // resident B
+    static constexpr int kOffSfb = kOffB + kXqMaxKt * kBBytes;   // resident SFB atoms
+    static constexpr int kOffBar = kOffSfb + kXqMaxKt * kSfbBytes;
+    static constexpr int kSmemBytes = kOffBar + 512;
+    static constexpr uint32_t kTx = kABytes + kSfaBytes; // per stage: W tile and its scales
+    static constexpr int kAccCols = BN < 32 ? 32 : BN;
+    static constexpr int kSfSlots = 4;
+    static constexpr int kSfbColsPerKb = 4;
+    static constexpr int kSlotCols = 32;
+    static constexpr int kSfCol = kAccCols;
+    static constexpr int kUsedCols = kSfCol + kSfSlots * kSlotCols;
+    static constexpr int kTmemCols = kUsedCols <= 128 ? 128 : 256;
+    static constexpr uint32_t kIdesc =
+        (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static constexpr bool kResidentB = true;
+    static_assert(kOffB % 1024 == 0, "swizzled operand alignment");
+};
+
+template <int BN, bool XQ = false> struct SmallCfg {
     // stages that keep one CTA at <= 113 KB of shared memory (two per SM)
     static constexpr int kStages = BN <= 16 ? 5 : BN <= 64 ? 4 : 3;
-    using L = Cfg<BN, kStages>;
+    using L = typename std::conditional<XQ, XqLayout<BN>, Cfg<BN, kStages>>::type;
     static_assert(L::kSmemBytes <= 115712, "two CTAs per SM");
     static_assert(L::kTmemCols <= 256, "two CTAs per SM");
     // partial accumulators of a non-leader CTA, [BN][128] fp32, over the drained stages
     static_assert(BN * 128 * 4 + BN * 128 * 2 <= L::kOffSfa,
                   "partials and bf16 output staging fit in the operand stages");
 };
+
+
 
 struct SmallParams {
     int64_t rows_a, rows_b; // weight rows (N), activation rows (M)
@@ -970,6 +1006,12 @@ struct SmallParams {
     int resident_w; // 1: W is not written by earlier work still running on the stream, so
                     // its first stages load before the programmatic-launch wait
     int *status;
+    // fused activation quantize (XQ kernels): x [M x K] row-major, bf16 (x_bf16) or fp32;
+    // x_gs_out (may be null): receives the activations' global scale
+    const void *x;
+    int x_bf16;
+    int64_t K;
+    float *x_gs_out;
 };
 
 // Output rows [rank*BN/CS, (rank+1)*BN/CS) of the tile, summed over the CS partials of the
@@ -1049,7 +1091,180 @@ __device__ __forceinline__ void reduce_slice(const SmallParams &p, uint8_t *smem
     }
 }
 
-template <int BN>
+
+// Fused activation quantize of the XQ kernels, run by every thread of the CTA before its
+// warp roles: max |x| over the whole M x K activation tensor (each CTA of the cluster folds a
+// share, the shares are combined through distributed shared memory, so every cluster holds
+// the same exact maximum), sg = amax / 2688, and this CTA's k-range of x encoded into the
+// resident B tiles (codes, 128B-swizzled rows, the layout TMA would write) and scale atoms,
+// with the quantizer's arithmetic (the codes equal nvfp4_quantize's). Rows M .. BN-1 and
+// blocks past K stay zero. Returns sg.
+template <int BN, typename L>
+__device__ __forceinline__ float xq_prologue(const SmallParams &p, uint8_t *smem, uint32_t rank,
+                                             int cs, int k0, int k1)
+{
+    __shared__ float s_warp[kThreads / 32];
+    __shared__ float s_part; // this CTA's share of the maximum (read by the cluster)
+    __shared__ float s_sg;
+    __shared__ float s_rcp[128];
+    const int tid = threadIdx.x;
+    const int nk = k1 - k0;
+    // zero the resident operand region of this CTA's k-tiles
+    {
+        uint4 *zb = reinterpret_cast<uint4 *>(smem + L::kOffB);
+        const int nb16 = nk * L::kBBytes / 16;
+        for (int i = tid; i < nb16; i += kThreads)
+            zb[i] = make_uint4(0u, 0u, 0u, 0u);
+        uint4 *zs = reinterpret_cast<uint4 *>(smem + L::kOffSfb);
+        const int ns16 = nk * L::kSfbBytes / 16;
+        for (int i = tid; i < ns16; i += kThreads)
+            zs[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // max |x| over this CTA's share of the tensor (16-byte vectors)
+    const int64_t nvec = p.rows_b * p.K * (p.x_bf16 ? 2 : 4) / 16;
+    const int64_t v0 = nvec * rank / cs, v1 = nvec * (rank + 1) / cs;
+    const uint4 *xv = reinterpret_cast<const uint4 *>(p.x);
+    float m = 0.0f;
+    constexpr int kVin = 8; // loads in flight per thread
+    for (int64_t i0 = v0 + tid; i0 < v1; i0 += (int64_t)kThreads * kVin) {
+        uint4 w[kVin];
+#pragma unroll
+        for (int q = 0; q < kVin; ++q) {
+            const int64_t i = i0 + (int64_t)q * kThreads;
+            w[q] = i < v1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < kVin; ++q) {
+            const uint32_t u[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (p.x_bf16)
+                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(u[j] << 16)),
+                                       fabsf(__uint_as_float(u[j] & 0xFFFF0000u))));
+                else
+                    m = fmaxf(m, fabsf(__uint_as_float(u[j])));
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((tid & 31) == 0)
+        s_warp[tid >> 5] = m;
+    __syncthreads();
+    if (tid == 0) {
+        float f = 0.0f;
+        for (int w = 0; w < kThreads / 32; ++w)
+            f = fmaxf(f, s_warp[w]);
+        s_part = f;
+    }
+    if (cs > 1)
+        cluster_sync(); // every share of the cluster is in place
+    else
+        __syncthreads();
+    if (tid == 0) {
+        float amax = s_part;
+        for (int r = 0; r < cs; ++r)
+            if (r != (int)rank)
+                amax = fmaxf(amax, ld_shared_cluster_f32(mapa_shared(smem_u32(&s_part), r)));
+        const float sg = __fdiv_rn(amax, 2688.0f); // 6 * 448
+        s_sg = sg;
+        if (blockIdx.x == 0 && p.x_gs_out)
+            *p.x_gs_out = sg;
+    }
+    __syncthreads();
+    const float sg = s_sg;
+    const float t = __fmul_rn(sg, 6.0f);
+    const float rt = __frcp_rn(t);
+    if (tid < 128)
+        s_rcp[tid] = __frcp_rn(__fmul_rn(e4m3_to_f32(tid), sg));
+    __syncthreads();
+    // encode rows 0 .. M-1 of k-tiles k0 .. k1-1, two 16-value blocks per thread step (both
+    // blocks' loads in flight together)
+    const int nbk = (int)(p.K >> 4); // blocks per row
+    const int total = (int)p.rows_b * nk * 16;
+    const uint8_t *xb = reinterpret_cast<const uint8_t *>(p.x);
+    const int esz = p.x_bf16 ? 2 : 4;
+    auto locate = [&](int i, int &r, int &j, int &bb, int &kb) {
+        bb = i & 15;          // block inside the k-tile
+        j = (i >> 4) % nk;    // resident k-tile
+        r = (i >> 4) / nk;    // row
+        kb = (k0 + j) * 16 + bb; // block along K
+    };
+    auto load_block = [&](int r, int kb, uint4 (&raw)[4]) {
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(xb + ((int64_t)r * p.K + kb * 16) * esz);
+        raw[0] = __ldg(src);
+        raw[1] = __ldg(src + 1);
+        if (!p.x_bf16) {
+            raw[2] = __ldg(src + 2);
+            raw[3] = __ldg(src + 3);
+        }
+    };
+    auto encode_block = [&](int r, int j, int bb, const uint4 (&raw)[4]) {
+        float v[16];
+        if (p.x_bf16) {
+            const uint32_t u[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w,
+                                   raw[1].x, raw[1].y, raw[1].z, raw[1].w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                v[2 * q] = __uint_as_float(u[q] << 16);
+                v[2 * q + 1] = __uint_as_float(u[q] & 0xFFFF0000u);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                v[4 * q] = __uint_as_float(raw[q].x);
+                v[4 * q + 1] = __uint_as_float(raw[q].y);
+                v[4 * q + 2] = __uint_as_float(raw[q].z);
+                v[4 * q + 3] = __uint_as_float(raw[q].w);
+            }
+        }
+        float bm = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            bm = fmaxf(bm, fabsf(v[q]));
+        const uint32_t sb = sg > 0.0f ? e4m3_of_quotient(bm, t, rt) : 0u;
+        if (sb == 0u)
+            return; // codes and scale stay zero
+        const float rcp = s_rcp[sb];
+        float y[16];
+#pragma unroll
+        for (int q = 0; q < 16; q += 2) {
+            const float2 pr = __fmul2_rn(make_float2(v[q], v[q + 1]), make_float2(rcp, rcp));
+            y[q] = pr.x;
+            y[q + 1] = pr.y;
+        }
+        const uint2 codes = make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8));
+        // B tile j: row r at r * 128 bytes, 16-byte chunk c stored at c ^ (r % 8)
+        uint8_t *bt = smem + L::kOffB + j * L::kBBytes + r * 128;
+        *reinterpret_cast<uint2 *>(bt + (((bb >> 1) ^ (r & 7)) << 4) + (bb & 1) * 8) = codes;
+        // scale atom (r, bb) of k-tile j
+        smem[L::kOffSfb + j * L::kSfbBytes + (bb >> 2) * 512 + 16 * (r & 31) +
+             4 * ((r & 127) >> 5) + (bb & 3)] = (uint8_t)sb;
+    };
+    for (int i = tid; i < total; i += 2 * kThreads) {
+        const int i2 = i + kThreads;
+        int r0, j0, bb0, kb0, r1 = 0, j1 = 0, bb1 = 0, kb1 = nbk;
+        locate(i, r0, j0, bb0, kb0);
+        if (i2 < total)
+            locate(i2, r1, j1, bb1, kb1);
+        uint4 raw0[4], raw1[4];
+        if (kb0 < nbk)
+            load_block(r0, kb0, raw0);
+        if (kb1 < nbk)
+            load_block(r1, kb1, raw1);
+        if (kb0 < nbk)
+            encode_block(r0, j0, bb0, raw0);
+        if (kb1 < nbk)
+            encode_block(r1, j1, bb1, raw1);
+    }
+    fence_proxy_async_smem(); // the tensor cores read the B tiles through the async proxy
+    __syncthreads();
+    return sg;
+}
+
+template <int BN, bool XQ>
 __global__ void __launch_bounds__(kThreads, 2)
     nvfp4_gemm_smallm_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
@@ -1057,7 +1272,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                              const __grid_constant__ CUtensorMap tmSFB,
                              const __grid_constant__ CUtensorMap tmY, const SmallParams p)
 {
-    using C = typename SmallCfg<BN>::L;
+    using C = typename SmallCfg<BN, XQ>::L;
     extern __shared__ __align__(1024) uint8_t smem[];
     if ((smem_u32(smem) & 1023u) != 0) { // same for every CTA: the whole grid returns here
         if (threadIdx.x == 0)
@@ -1109,24 +1324,34 @@ __global__ void __launch_bounds__(kThreads, 2)
     pdl_launch_dependents();
     float alpha = 0.0f; // sgA * sgW, read by the epilogue warps
 
+    // Resident weights: the first stages' W tiles and scales are requested while the
+    // previous kernel may still run (the stages start out free); the activations always
+    // wait for it.
+    const int pre = p.resident_w ? min(k1 - k0, C::kStages) : 0;
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmSFA);
+        if constexpr (!XQ) {
+            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmSFB);
+        }
+        for (int i = 0; i < pre; ++i) {
+            mbar_arrive_expect_tx(&full_bar[i], C::kTx);
+            tma_load_2d(smem + i * C::kABytes, &tmA, &full_bar[i], (k0 + i) * 128,
+                        (int)(ta * BM));
+            tma_load_3d(smem + C::kOffSfa + i * C::kSfaBytes, &tmSFA, &full_bar[i], 0,
+                        (k0 + i) * 4, (int)ta);
+        }
+    }
+    float sg_x = 0.0f; // XQ: the activations' global scale
+    if constexpr (XQ) {
+        pdl_wait(); // the activations may come from the previous kernel
+        sg_x = xq_prologue<BN, C>(p, smem, rank, cs, k0, k1);
+    }
+
     if (warp == 0) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
-            tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB);
-            tma_prefetch_desc(&tmSFA);
-            tma_prefetch_desc(&tmSFB);
-            // Resident weights: the first stages' W tiles and scales are requested while the
-            // previous kernel may still run (the stages start out free); the activations
-            // always wait for it.
-            const int pre = p.resident_w ? min(k1 - k0, C::kStages) : 0;
-            for (int i = 0; i < pre; ++i) {
-                mbar_arrive_expect_tx(&full_bar[i], C::kTx);
-                tma_load_2d(smem + i * C::kABytes, &tmA, &full_bar[i], (k0 + i) * 128,
-                            (int)(ta * BM));
-                tma_load_3d(smem + C::kOffSfa + i * C::kSfaBytes, &tmSFA, &full_bar[i], 0,
-                            (k0 + i) * 4, (int)ta);
-            }
             pdl_wait(); // operands may come from the previous kernel
             int stage = 0;
             uint32_t phase = 0;
@@ -1145,8 +1370,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, (int)(ta * BM));
                     tma_load_3d(ssfa, &tmSFA, &full_bar[stage], 0, kt * 4, (int)ta);
                 }
-                tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, 0);
-                tma_load_3d(ssfb, &tmSFB, &full_bar[stage], 0, kt * 4, 0);
+                if constexpr (!XQ) { // XQ: the activations are resident already
+                    tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, 0);
+                    tma_load_3d(ssfb, &tmSFB, &full_bar[stage], 0, kt * 4, 0);
+                }
                 ++issued;
                 if (++stage == C::kStages) {
                     stage = 0;
@@ -1180,7 +1407,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             tc_fence_after();
             const uint32_t ssfa = smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes);
-            const uint32_t ssfb = smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes);
+            const uint32_t ssfb =
+                smem_u32(smem + C::kOffSfb + (XQ ? kt - k0 : stage) * C::kSfbBytes);
             const uint32_t tslot =
                 tmem + ((uint32_t)(q * 32) << 16) + C::kSfCol + slot * C::kSlotCols;
             uint32_t ra[16], rb[16];
@@ -1231,8 +1459,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t tsfa = tmem + C::kSfCol + slot * C::kSlotCols;
                 const uint64_t adesc = smem_desc(smem_u32(smem + stage * C::kABytes), 16, 1024,
                                                  kLayoutSwizzle128B);
-                const uint64_t bdesc = smem_desc(smem_u32(smem + C::kOffB + stage * C::kBBytes),
-                                                 16, 1024, kLayoutSwizzle128B);
+                const uint64_t bdesc =
+                    smem_desc(smem_u32(smem + C::kOffB + (XQ ? kt - k0 : stage) * C::kBBytes), 16,
+                              1024, kLayoutSwizzle128B);
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb)
                     tc_mma_nvf4(tmem, adesc + (uint64_t)(2 * kb), bdesc + (uint64_t)(2 * kb),
@@ -1269,7 +1498,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         constexpr int NC = BN < 32 ? BN : 32;
         pdl_wait(); // global scales and y belong to the stream's earlier work
-        alpha = __fmul_rn(*p.a_gs, *p.w_gs);
+        alpha = __fmul_rn(XQ ? sg_x : *p.a_gs, *p.w_gs);
         const bool ok = mbar_wait(acc_full, 0, kWaitLimit);
         if (!ok && lane == 0)
             set_timeout(p.status);
@@ -1478,17 +1707,17 @@ cudaError_t launch_pair(const LinearPlan &pl, const uint8_t *a_codes, const uint
     return cudaGetLastError();
 }
 
-template <int BN> cudaError_t smallm_set_smem_attr()
+template <int BN, bool XQ = false> cudaError_t smallm_set_smem_attr()
 {
     static std::once_flag flags[64];
     int dev = 0;
     cudaGetDevice(&dev);
     cudaError_t e = cudaSuccess;
     std::call_once(flags[dev & 63], [&]() {
-        e = cudaFuncSetAttribute(nvfp4_gemm_smallm_kernel<BN>,
+        e = cudaFuncSetAttribute(nvfp4_gemm_smallm_kernel<BN, XQ>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SmallCfg<BN>::L::kSmemBytes);
-        if (e == cudaSuccess)
+                                 SmallCfg<BN, XQ>::L::kSmemBytes);
+        if (e == cudaSuccess && !XQ)
             e = cudaFuncSetAttribute(smallm_occupancy_proxy<BN>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      SmallCfg<BN>::L::kSmemBytes);
@@ -1548,14 +1777,16 @@ const SmallOccupancy &small_occupancy()
 
 int bn_index(int bn) { return bn <= 8 ? 0 : bn <= 16 ? 1 : bn <= 32 ? 2 : bn <= 64 ? 3 : 4; }
 
-template <int BN>
+template <int BN, bool XQ = false>
 cudaError_t launch_smallm(const LinearPlan &pl, const uint8_t *w_codes, const uint8_t *w_sf,
                           const uint8_t *a_codes, const uint8_t *a_sf, int64_t K,
                           const SmallParams &sp, cudaStream_t s, nvfp4_status *st)
 {
-    using C = typename SmallCfg<BN>::L;
+    using C = typename SmallCfg<BN, XQ>::L;
     CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
     memset(&tmY, 0, sizeof(tmY));
+    memset(&tmB, 0, sizeof(tmB));
+    memset(&tmSFB, 0, sizeof(tmSFB));
     SmallParams spl = sp;
     spl.tma_store = 0;
     const int64_t esz = sp.out_bf16 ? 2 : 4;
@@ -1563,13 +1794,13 @@ cudaError_t launch_smallm(const LinearPlan &pl, const uint8_t *w_codes, const ui
         encode_fn() && make_out_map_swap(&tmY, sp.y, pl.rows_b, sp.ldy, sp.out_bf16, BN / pl.csplit))
         spl.tma_store = 1;
     if (!encode_fn() || !make_codes_map(&tmA, w_codes, pl.rows_a, K, BM) ||
-        !make_codes_map(&tmB, a_codes, pl.rows_b, K, BN) ||
         !make_sf_map(&tmSFA, w_sf, pl.rows_a, K, 1) ||
-        !make_sf_map(&tmSFB, a_sf, pl.rows_b, K, 1)) {
+        (!XQ && (!make_codes_map(&tmB, a_codes, pl.rows_b, K, BN) ||
+                 !make_sf_map(&tmSFB, a_sf, pl.rows_b, K, 1)))) {
         *st = NVFP4_ERR_CUDA;
         return cudaErrorInvalidValue;
     }
-    cudaError_t e = smallm_set_smem_attr<BN>();
+    cudaError_t e = smallm_set_smem_attr<BN, XQ>();
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg{};
@@ -1591,8 +1822,8 @@ cudaError_t launch_smallm(const LinearPlan &pl, const uint8_t *w_codes, const ui
     }
     cfg.attrs = at;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_smallm_kernel<BN>, tmA, tmB, tmSFA, tmSFB, tmY,
-                              spl);
+    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_smallm_kernel<BN, XQ>, tmA, tmB, tmSFA, tmSFB,
+                              tmY, spl);
 }
 
 } // namespace
@@ -1726,6 +1957,77 @@ cudaError_t launch_linear(const LinearPlan &pl, const uint8_t *a_codes, const ui
         reinterpret_cast<const float *>(ws), pl.splits, pl.rows_a, pl.rows_b, pl.tiles_a * 128,
         pl.tiles_b * pl.bn, a_gs, w_gs, y, N, out_bf16, pl.swap_ab ? 1 : 0);
     return cudaGetLastError();
+}
+
+// Fused dynamic-activation linear (M <= 16): the small-M plan with a cluster split whose
+// per-CTA k-range holds at most kXqMaxKt k-tiles (the resident activation tiles). Returns
+// false when the shape does not fit that. Above M = 16 the in-kernel quantize (every cluster
+// reads the whole activation tensor for its amax) costs more than a separate quantize: on
+// B200, N12288 K4096, fused vs quantize + linear: M16 14.9 vs 17.5 us, M24 18.5 vs 17.9 us.
+bool plan_linear_xq(int64_t M, int64_t N, int64_t K, LinearPlan *out)
+{
+    if (M < 1 || M > 16 || N < 1 || K < 32)
+        return false;
+    LinearPlan p = plan_linear(M, N, K, 0);
+    if (!p.swap_ab || p.bn > 32)
+        return false;
+    const SmallOccupancy &occ = small_occupancy();
+    const int bi = bn_index(p.bn);
+    const int64_t tiles = p.tiles_a;
+    const int64_t max_ctas = (int64_t)num_sms() * 4 / 3;
+    int csplit = 0;
+    for (int cs = kMaxCsplit; cs >= 1; cs /= 2) {
+        const bool fits = cs <= p.kt && tiles <= occ.clusters[bi][cs] &&
+                          (cs == 1 || tiles * cs <= max_ctas) &&
+                          (p.kt + cs - 1) / cs <= kXqMaxKt;
+        if (fits) {
+            csplit = cs;
+            break;
+        }
+    }
+    if (csplit == 0) { // the k-range would not stay resident: the largest resident split
+        for (int cs = kMaxCsplit; cs >= 1; cs /= 2)
+            if (cs <= p.kt && tiles <= occ.clusters[bi][cs] &&
+                (p.kt + cs - 1) / cs <= kXqMaxKt) {
+                csplit = cs;
+                break;
+            }
+    }
+    if (csplit == 0)
+        return false;
+    p.csplit = csplit;
+    p.ws_bytes = 0;
+    *out = p;
+    return true;
+}
+
+cudaError_t launch_linear_xq(const LinearPlan &pl, const void *x, int x_bf16,
+                             const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,
+                             int64_t M, int64_t N, int64_t K, int out_bf16, void *y,
+                             float *x_gs_out, unsigned flags, cudaStream_t s, nvfp4_status *st)
+{
+    SmallParams sp{};
+    sp.rows_a = pl.rows_a;
+    sp.rows_b = pl.rows_b;
+    sp.kt_total = pl.kt;
+    sp.csplit = pl.csplit;
+    sp.a_gs = nullptr;
+    sp.w_gs = w_gs;
+    sp.y = y;
+    sp.ldy = N;
+    sp.out_bf16 = out_bf16;
+    sp.resident_w = (flags & NVFP4_LINEAR_RESIDENT_WEIGHTS) ? 1 : 0;
+    sp.status = device_status_ptr();
+    sp.x = x;
+    sp.x_bf16 = x_bf16;
+    sp.K = K;
+    sp.x_gs_out = x_gs_out;
+    (void)M;
+    switch (pl.bn) {
+    case 8: return launch_smallm<8, true>(pl, w_codes, w_sf, nullptr, nullptr, K, sp, s, st);
+    case 16: return launch_smallm<16, true>(pl, w_codes, w_sf, nullptr, nullptr, K, sp, s, st);
+    default: return launch_smallm<32, true>(pl, w_codes, w_sf, nullptr, nullptr, K, sp, s, st);
+    }
 }
 
 // ---------------------------------------------------------------------------------------

@@ -85,4 +85,12 @@ cudaError_t launch_linear(const LinearPlan &p, const uint8_t *a_codes, const uin
                           const float *w_gs, int64_t M, int64_t N, int64_t K, int out_bf16,
                           void *y, void *ws, unsigned flags, cudaStream_t s, nvfp4_status *st);
 
+// Fused dynamic-activation linear for M <= 32 (gemm_sm100.cu): plan (false if the shape does
+// not fit the fused kernel) and launch.
+bool plan_linear_xq(int64_t M, int64_t N, int64_t K, LinearPlan *out);
+cudaError_t launch_linear_xq(const LinearPlan &pl, const void *x, int x_bf16,
+                             const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,
+                             int64_t M, int64_t N, int64_t K, int out_bf16, void *y,
+                             float *x_gs_out, unsigned flags, cudaStream_t s, nvfp4_status *st);
+
 } // namespace nvfp4

@@ -317,6 +317,35 @@ def test_linear_rejects_unknown_flag():
     assert not y.float().abs().sum().item()
 
 
+@pytest.mark.parametrize("M,N,K,xkind", [
+    (1, 384, 512, "bf16"), (3, 1004, 2048, "f32"), (8, 1536, 3072, "bf16"),
+    (16, 640, 1792, "bf16"), (32, 2560, 1024, "f32"), (8, 256, 8192, "bf16"),
+    (5, 12288, 4096, "bf16"), (8, 384, 320, "bf16"),
+    (64, 512, 1024, "bf16"), (130, 256, 512, "f32"),  # beyond the fused kernel: two steps
+])
+def test_linear_dynamic_matches_oracle(M, N, K, xkind):
+    # activations quantized with their dynamic amax inside the linear call (one kernel for
+    # M <= 32): the result is the oracle's quantize-then-GEMM, the reported global scale the
+    # oracle's, bit for bit
+    xa = W.normal((M, K), 1.0, 36, M + K)
+    xa[M // 2, K // 3] = 23.0
+    if xkind == "bf16":
+        xa = W.to_bf16_bits(xa)
+    xw = W.to_bf16_bits(W.normal((N, K), 0.02, 37, N))
+    qw = gpu_quantize(xw)
+    gs = torch.zeros(1, dtype=torch.float32, device="cuda")
+    for resident in (False, True):
+        y = nv.linear_dynamic(dev_tensor(xa), qw, x_gs_out=gs, resident_weights=resident)
+        torch.cuda.synchronize()
+        ra, rw = O.quantize(xa), O.quantize(xw)
+        ref = O.gemm(ra, rw)
+        err = np.abs(to_numpy_f64(y) - ref)
+        tol = gemm_tolerance(ref, True)
+        assert np.all(err <= tol), f"max err {err.max()}"
+        assert np.float32(gs.cpu()[0]).tobytes() == np.float32(ra.sg).tobytes()
+    assert nv.sync_status() == 0
+
+
 def test_linear_exact_with_unit_scales():
     # all block scales 1.0 and both global scales 1: 2 * each value is an integer in
     # [-12, 12], the sums are exact in fp32, so the fp32 output must equal the exact product.

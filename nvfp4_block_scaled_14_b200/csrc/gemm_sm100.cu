@@ -887,10 +887,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (threadIdx.x == 64) {
+                // boxes that start past the last row or column of Y hold nothing to store
+                const int64_t yrow = ta * 256 + rank * 128;
 #pragma unroll
                 for (int b = 0; b < 4; ++b)
-                    tma_store_2d(&tmY, smem + C::kOffStaging + b * (128 * 128),
-                                 (int)(tb * 256 + b * 64), (int)(ta * 256 + rank * 128));
+                    if (yrow < p.rows_a && tb * 256 + b * 64 < p.rows_b)
+                        tma_store_2d(&tmY, smem + C::kOffStaging + b * (128 * 128),
+                                     (int)(tb * 256 + b * 64), (int)yrow);
                 bulk_commit_group();
             }
             acc_phase ^= 1;

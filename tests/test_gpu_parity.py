@@ -386,6 +386,35 @@ def test_linear_large_tile_path_sampled():
     assert np.all(np.abs(y[ms, ns] - ref) <= tol)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    # CTA-pair kernel (bf16 out, more than 74 tiles of 128 x 256 on 148 SMs)
+    (1300, 1960, 512),    # ragged M (a CTA with no valid row) and N (the last 256 x 256 tile
+                          # holds 168 columns: one store box lies wholly past the output)
+    (1280, 3072, 1024),
+    (2000, 2296, 2048),   # ragged M and N, 8 k-tiles
+    (4200, 2560, 768),    # two or three tiles per CTA pair (accumulator reuse), ragged M
+])
+def test_linear_pair_kernel_sampled(M, N, K):
+    xa = W.to_bf16_bits(W.normal((M, K), 1.0, 41, M))
+    xw = W.to_bf16_bits(W.normal((N, K), 0.02, 42, N))
+    qa, qw = gpu_quantize(xa), gpu_quantize(xw)
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nv.linear(qa, qw, out=out)
+    torch.cuda.synchronize()
+    y = to_numpy_f64(out)
+    assert np.isfinite(y).all()  # every element written
+    ra, rw = O.quantize(xa), O.quantize(xw)
+    r = np.random.Generator(np.random.PCG64(43))
+    edge_m = [0, 127, 128, 255, 256, M - 1]
+    edge_n = [0, 63, 64, 191, 192, 255, 256, 383, 384, N - 1]
+    ms = np.concatenate([r.integers(0, M, 3000), np.repeat(edge_m, len(edge_n))])
+    ns = np.concatenate([r.integers(0, N, 3000), np.tile(edge_n, len(edge_m))])
+    ref = O.gemm_sampled(ra, rw, ms, ns)
+    full_max = np.abs(y).max()
+    tol = 1e-3 * full_max + np.abs(ref) * 2.0 ** -8
+    assert np.all(np.abs(y[ms, ns] - ref) <= tol)
+
+
 # ---------------------------------------------------------------------------------------
 # calibration percentile
 # ---------------------------------------------------------------------------------------

@@ -11,6 +11,8 @@ Sources of each step (see the header of nvfp4_oracle.c for the full list):
   * "Qwen-Rapid-AIO FP8 -> NVFP4", "1. Double Quantization" -- FP8 upcast, then NVFP4.
   * "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details" -- dynamic per-tensor amax.
   * "Qwen-Rapid-AIO FP8 -> NVFP4", "Recommended Model" -- p99.9 static input scales.
+  * "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details" / "Layer breakdown" -- FP8
+    E4M3 tensorwise round-to-nearest layers (quantize_e4m3, gemm_e4m3).
 """
 import ctypes
 import os
@@ -65,6 +67,12 @@ def lib():
         L.ora_e4m3_encode_array.argtypes = [_f32p, _i64, _u8p]
         L.ora_amax.argtypes = [_f32p, _i64]
         L.ora_amax.restype = ctypes.c_float
+        L.ora_quantize_e4m3.argtypes = [_vp, ctypes.c_int, _i64, _f32p, _u8p, _f32p]
+        L.ora_quantize_e4m3.restype = ctypes.c_int
+        L.ora_gemm_e4m3_f64.argtypes = [_u8p, ctypes.c_float, _u8p, ctypes.c_float, _i64, _i64,
+                                        _i64, _f64p]
+        L.ora_gemm_e4m3_f64_sampled.argtypes = [_u8p, ctypes.c_float, _u8p, ctypes.c_float, _i64,
+                                                _i64p, _i64p, _i64, _f64p]
         _lib = L
     return _lib
 
@@ -213,3 +221,43 @@ def source_to_f32(x: np.ndarray, fp8_scale=None) -> np.ndarray:
     f = lut[x]
     s8 = np.float32(1.0 if fp8_scale is None else fp8_scale)
     return (f * s8).astype(np.float32)
+
+
+# ---- FP8 E4M3 tensorwise layers ----------------------------------------------------------
+def quantize_e4m3(x: np.ndarray, amax=None):
+    """x: float32 or uint16 (bf16 bits), any shape -> (codes uint8 of x's shape, scale s)."""
+    x = np.ascontiguousarray(x)
+    dt = _src_dtype(x)
+    if dt == E4M3:
+        raise TypeError("E4M3 sources are already FP8")
+    codes = np.zeros(x.shape, np.uint8)
+    s = np.zeros(1, np.float32)
+    am = None if amax is None else np.array([amax], np.float32)
+    rc = lib().ora_quantize_e4m3(x.ctypes.data_as(_vp), dt, x.size,
+                                 None if am is None else _p(am, _f32p), _p(codes, _u8p),
+                                 _p(s, _f32p))
+    if rc != 0:
+        raise ValueError(f"oracle quantize_e4m3 failed ({rc})")
+    return codes, float(s[0])
+
+
+def gemm_e4m3(a_codes, sa, w_codes, sw) -> np.ndarray:
+    """Y = sA * sW * eA . eW^T in fp64 from E4M3 codes A [M, K], W [N, K]."""
+    a = np.ascontiguousarray(a_codes, np.uint8)
+    w = np.ascontiguousarray(w_codes, np.uint8)
+    (M, K), (N, K2) = a.shape, w.shape
+    assert K == K2
+    out = np.zeros((M, N), np.float64)
+    lib().ora_gemm_e4m3_f64(_p(a, _u8p), sa, _p(w, _u8p), sw, M, N, K, _p(out, _f64p))
+    return out
+
+
+def gemm_e4m3_sampled(a_codes, sa, w_codes, sw, ms, ns) -> np.ndarray:
+    a = np.ascontiguousarray(a_codes, np.uint8)
+    w = np.ascontiguousarray(w_codes, np.uint8)
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    out = np.zeros(len(ms), np.float64)
+    lib().ora_gemm_e4m3_f64_sampled(_p(a, _u8p), sa, _p(w, _u8p), sw, a.shape[1], _p(ms, _i64p),
+                                    _p(ns, _i64p), len(ms), _p(out, _f64p))
+    return out

@@ -366,6 +366,80 @@ void ora_gemm_f64_sampled(const uint8_t *a_codes, const uint8_t *a_scales_lin, f
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* FP8 E4M3 tensorwise layers                                                                  */
+/* ------------------------------------------------------------------------------------------ */
+/* [QVf] "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details" and "Layer breakdown":
+ *       embed_tokens and lm_head are float8_e4m3fn, tensorwise, round-to-nearest; "Runtime /
+ *       hardware": FP8 layers run as native FP8 on Blackwell.
+ * [QRp] "Qwen-Rapid-AIO FP8 -> NVFP4", the "Solution" table and the paragraph under it: layers
+ *       that are FP8 stay FP8 (no re-quantization through fp32).
+ * Readings where the pages are silent (also in the design notes):
+ *   - one fp32 scale per tensor, s = amax / 448 (fp32 division): the largest |x| maps to the
+ *     largest finite E4M3 value; amax is the tensor's own (dynamic) or a static value, above
+ *     which values saturate.
+ *   - code = sign(x) | E4M3(|x| / s): the quotient is an IEEE fp32 division, rounded to the
+ *     nearest E4M3 value, ties to the even code, saturating at 448; s == 0 gives sign-only codes.
+ *   - the linear layer is W8A8: activations quantized the same way from their dynamic amax, and
+ *     Y[m,n] = sA * sW * sum_k eA[m,k] * eW[n,k].
+ */
+
+/* E4M3 codes of n fp32 values with one tensor scale; returns s. */
+float ora_quantize_e4m3_f32(const float *x, int64_t n, const float *amax_in, uint8_t *codes)
+{
+    float amax = amax_in ? *amax_in : ora_amax(x, n);
+    float s = amax / 448.0f;
+    for (int64_t i = 0; i < n; i++) {
+        uint8_t sign = signbit(x[i]) ? 0x80 : 0x00;
+        uint8_t mag = (s > 0.0f) ? ora_e4m3_encode_nonneg(fabsf(x[i]) / s) : 0;
+        codes[i] = (uint8_t)(sign | mag);
+    }
+    return s;
+}
+
+/* Source of dtype 0 (fp32) or 1 (bf16 bits); returns 0, or -1 for another dtype. */
+int ora_quantize_e4m3(const void *src, int dtype, int64_t n, const float *amax_in,
+                      uint8_t *codes, float *scale_out)
+{
+    if (dtype != 0 && dtype != 1)
+        return -1;
+    float *x = (float *)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    if (!x)
+        return -2;
+    ora_source_to_f32(src, dtype, NULL, n, x);
+    *scale_out = ora_quantize_e4m3_f32(x, n, amax_in, codes);
+    free(x);
+    return 0;
+}
+
+/* One output of the W8A8 product: exact decodes, fp64 accumulation. */
+static double gemm_e4m3_one(const uint8_t *a, float sa, const uint8_t *w, float sw, int64_t m,
+                            int64_t n, int64_t K)
+{
+    double acc = 0.0;
+    for (int64_t k = 0; k < K; k++)
+        acc += ora_e4m3_decode(a[m * K + k]) * ora_e4m3_decode(w[n * K + k]);
+    return (double)sa * (double)sw * acc;
+}
+
+/* Y [M x N] row-major from A codes [M x K] and W codes [N x K] (nn.Linear layout). */
+void ora_gemm_e4m3_f64(const uint8_t *a, float sa, const uint8_t *w, float sw, int64_t M,
+                       int64_t N, int64_t K, double *out)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++)
+            out[m * N + n] = gemm_e4m3_one(a, sa, w, sw, m, n, K);
+}
+
+void ora_gemm_e4m3_f64_sampled(const uint8_t *a, float sa, const uint8_t *w, float sw, int64_t K,
+                               const int64_t *ms, const int64_t *ns, int64_t count, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; i++)
+        out[i] = gemm_e4m3_one(a, sa, w, sw, ms[i], ns[i], K);
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Percentile calibration                                                                      */
 /* ------------------------------------------------------------------------------------------ */
 

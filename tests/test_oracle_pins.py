@@ -337,3 +337,97 @@ def test_percentile_matches_numpy_sort_over_union():
         rank = -(-n * num // den)
         pct, mx = O.percentile_abs(parts, num, den)
         assert pct == allv[rank - 1] and mx == allv[-1]
+
+
+# ---- FP8 E4M3 tensorwise layers ----------------------------------------------------------
+
+def _e4m3_magnitudes():
+    """The 127 finite non-negative E4M3 values in code order, decoded by torch."""
+    return e4m3_torch_decode(np.arange(127))
+
+
+def test_e4m3_tensor_grid_points_are_exact():
+    # amax = 56 -> s = 56 / 448 = 1/8 exactly; x = s * v for every finite E4M3 value v of
+    # either sign must come back as v's own code (scale, sign bit and code order pinned)
+    mags = _e4m3_magnitudes()
+    x = np.concatenate([mags, -mags[1:], [56.0]]).astype(np.float32) * np.float32(0.125)
+    x[-1] = 56.0  # the amax element itself (its own code: 448 = 0x7E)
+    codes, s = O.quantize_e4m3(x.reshape(1, -1))
+    assert s == 0.125
+    want = np.concatenate([np.arange(127), 0x80 | np.arange(1, 127), [0x7E]]).astype(np.uint8)
+    assert np.array_equal(codes.ravel(), want)
+
+
+def test_e4m3_tensor_is_nearest_value_brute_force():
+    # every code decodes to a nearest E4M3 value of the fp32 quotient |x| / s (ties to the
+    # even code), found by scanning all 127 magnitudes; the sign bit is x's
+    g = np.random.Generator(np.random.PCG64(120))
+    x = (g.standard_normal(4000) * np.exp(g.uniform(-8, 3, 4000))).astype(np.float32)
+    x[::97] = 0.0
+    x[1::211] = -0.0
+    codes, s = O.quantize_e4m3(x)
+    assert s == np.float32(np.abs(x).max()) / np.float32(448.0)
+    mags = _e4m3_magnitudes()
+    q = (np.abs(x) / np.float32(s)).astype(np.float64)  # fp32 division, widened exactly
+    for xi, qi, c in zip(x, q, codes):
+        d = np.abs(mags - min(qi, 448.0))
+        best = np.flatnonzero(d == d.min())
+        expect = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        assert (c & 0x7F) == expect and (c >> 7) == int(np.signbit(xi))
+
+
+def test_e4m3_tensor_matches_torch_cast():
+    # a library route to the same codes: fp32 quotient, then torch's RNE float8_e4m3fn cast
+    g = np.random.Generator(np.random.PCG64(121))
+    x = g.standard_normal((37, 48)).astype(np.float32) * np.float32(3.0)
+    codes, s = O.quantize_e4m3(x)
+    ref = torch.from_numpy(x / np.float32(s)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+
+
+def test_e4m3_tensor_bf16_source_and_static_amax():
+    g = np.random.Generator(np.random.PCG64(122))
+    xf = g.standard_normal((8, 40)).astype(np.float32)
+    xb = W.to_bf16_bits(xf)
+    cb, sb = O.quantize_e4m3(xb)
+    cf, sf = O.quantize_e4m3(W.bf16_bits_to_f32(xb))
+    assert sb == sf and np.array_equal(cb, cf)  # bf16 widens exactly
+    # static amax below max|x|: s = amax / 448 and the values above it saturate at 448
+    c, s = O.quantize_e4m3(xf, amax=0.5)
+    assert s == np.float32(0.5) / np.float32(448.0)
+    big = np.abs(xf) > 0.5 * (1 + 2 ** -4)
+    assert np.all((c[big] & 0x7F) == 0x7E) and np.array_equal(c[big] >> 7, np.signbit(xf[big]))
+    # amax 0: sign-only codes; an all-zero tensor: zero codes and s = 0
+    c0, s0 = O.quantize_e4m3(xf, amax=0.0)
+    assert s0 == 0.0 and np.array_equal(c0, np.where(np.signbit(xf), 0x80, 0).astype(np.uint8))
+    cz, sz = O.quantize_e4m3(np.zeros((3, 16), np.float32))
+    assert sz == 0.0 and not cz.any()
+
+
+def test_gemm_e4m3_integer_exact():
+    # E4M3 holds the integers -16..16 exactly: with unit scales the product is numpy's integer
+    # matmul, and the scales multiply it (a transposed operand or a wrong index would differ)
+    g = np.random.Generator(np.random.PCG64(123))
+    M, N, K = 7, 13, 96
+    ai = g.integers(-16, 17, (M, K))
+    wi = g.integers(-16, 17, (N, K))
+    ints = np.arange(-16, 17)
+    enc = {int(v): int(c) for v, c in zip(ints, torch.from_numpy(ints.astype(np.float32))
+                                          .to(torch.float8_e4m3fn).view(torch.uint8).numpy())}
+    ac = np.vectorize(enc.get)(ai).astype(np.uint8)
+    wc = np.vectorize(enc.get)(wi).astype(np.uint8)
+    exact = (ai @ wi.T).astype(np.float64)
+    assert np.array_equal(O.gemm_e4m3(ac, 1.0, wc, 1.0), exact)
+    assert np.array_equal(O.gemm_e4m3(ac, 0.5, wc, 3.0), 1.5 * exact)
+    ms, ns = np.array([0, 6, 3]), np.array([12, 0, 5])
+    assert np.array_equal(O.gemm_e4m3_sampled(ac, 0.5, wc, 3.0, ms, ns), 1.5 * exact[ms, ns])
+
+
+def test_gemm_e4m3_is_dequantized_product():
+    # the product of the layer equals the fp64 product of the dequantized operands
+    g = np.random.Generator(np.random.PCG64(124))
+    a, sa = O.quantize_e4m3(g.standard_normal((5, 64)).astype(np.float32))
+    w, sw = O.quantize_e4m3((g.standard_normal((9, 64)) * 0.02).astype(np.float32))
+    da = e4m3_torch_decode(a) * sa
+    dw = e4m3_torch_decode(w) * sw
+    assert np.allclose(O.gemm_e4m3(a, sa, w, sw), da @ dw.T, rtol=1e-12, atol=0)

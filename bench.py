@@ -41,6 +41,7 @@ FLOPS = 2.0 * M * N * K
 METRIC = "NVFP4 GEMM TFLOPS & quantize GB/s at 1 B200 (fraction of FP4/HBM peak)"
 WORKLOAD = "attn_proj_fp8w_m4096_n3072_k3072"
 FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 ratio (4.5 / 2.25 PFLOP/s)
 # the kernel the linear layer runs for this shape (bf16 output, M > 128, one 256 x 256 tile
 # per CTA pair): the dominant kernel of the step
 GEMM_KERNEL = "nvfp4_gemm_pair_kernel"
@@ -288,6 +289,41 @@ def extras(nv, W, dev, hbm, fp4_peak):
     elems = 12288 * 3072
     gbs = (elems / 2 + elems / 16 + elems * 2) / (avg * 1e-3) / 1e9
     rows["dequantize_12288x3072_bf16"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    del wqs, w1
+    torch.cuda.empty_cache()
+
+    # --- FP8 E4M3 tensorwise W8A8 layers (embed / lm_head path): quantize X, GEMM, both
+    fp8_peak = fp4_peak / FP4_PER_BF16 * FP8_PER_BF16
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(8)
+    fp8 = {}
+    for name, mm, nn, kk in [("m4096_n3072_k3072", 4096, 3072, 3072),
+                             ("m4096_n12288_k3072", 4096, 12288, 3072),
+                             ("m4096_n3072_k12288", 4096, 3072, 12288)]:
+        nset = sets_for(mm * kk * 2)
+        xs = [torch.randn(mm, kk, device=dev, generator=gen).to(torch.bfloat16)
+              for _ in range(nset)]
+        w8 = nv.quantize_e4m3((torch.randn(nn, kk, device=dev, generator=gen) * 0.02)
+                              .to(torch.bfloat16))
+        nsw = sets_for(mm * kk + nn * kk)
+        a8s = [nv.quantize_e4m3(xs[i % nset]) for i in range(nsw)]
+        w8s = [nv.E4M3Tensor(w8.codes.clone(), w8.scale.clone()) for _ in range(nsw)]
+        y = torch.empty((mm, nn), dtype=torch.bfloat16, device=dev)
+        avg_q, _ = op_timer([lambda x=x, a=a8s[0]: nv.quantize_e4m3(x, out=a) for x in xs])
+        avg_g, _ = op_timer([lambda a=a, w=w: nv.linear_e4m3(a, w, out=y)
+                             for a, w in zip(a8s, w8s)])
+        avg_l, _ = op_timer([lambda x=x, a=a8s[i], w=w8s[i]: (nv.quantize_e4m3(x, out=a),
+                                                              nv.linear_e4m3(a, w, out=y))
+                             for i, x in enumerate(xs[:nsw] if nsw <= nset else xs)])
+        qgbs = mm * kk * 3 / (avg_q * 1e-3) / 1e9
+        tf = 2.0 * mm * nn * kk / (avg_g * 1e-3) / 1e12
+        fp8[name] = {"quantize_x_us": avg_q * 1e3, "quantize_x_GB/s": qgbs,
+                     "quantize_x_frac_hbm": qgbs / hbm, "gemm_us": avg_g * 1e3,
+                     "gemm_TFLOP/s": tf, "gemm_frac_fp8": tf / fp8_peak,
+                     "quantize_x_then_gemm_us": avg_l * 1e3}
+        del xs, a8s, w8s, w8, y
+        torch.cuda.empty_cache()
+    rows["fp8_e4m3_w8a8"] = fp8
     return rows
 
 

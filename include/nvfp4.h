@@ -58,7 +58,8 @@ typedef enum {
     NVFP4_OP_LINEAR = 1,     /* m = M, n = N, k = K */
     NVFP4_OP_CALIB_BF16 = 2, /* m, n, k ignored */
     NVFP4_OP_CALIB_F32 = 3,  /* m, n, k ignored */
-    NVFP4_OP_LINEAR_DYNAMIC = 4 /* m = M, n = N, k = K of nvfp4_linear_dynamic */
+    NVFP4_OP_LINEAR_DYNAMIC = 4, /* m = M, n = N, k = K of nvfp4_linear_dynamic */
+    NVFP4_OP_QUANTIZE_E4M3 = 5   /* nvfp4_quantize_e4m3 (m, n, k ignored) */
 } nvfp4_op;
 
 /* Human-readable name of a status. Never NULL. */
@@ -251,6 +252,40 @@ nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_bat
                                          uint32_t pct_num, uint32_t pct_den, float *out_pct,
                                          float *out_max, void *ws, size_t ws_bytes,
                                          cudaStream_t stream);
+
+/*
+ * FP8 E4M3 tensorwise quantization ("Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization
+ * Details" and "Layer breakdown": embed_tokens and lm_head in float8_e4m3fn, tensorwise,
+ * round-to-nearest). One fp32 scale per tensor and one E4M3 code per value:
+ *   s = amax / 448 (fp32 division; amax = max |x| of the tensor, or *static_amax),
+ *   code = sign(x) | E4M3(|x| / s): the IEEE fp32 quotient rounded to the nearest E4M3 value,
+ *   ties to the even code, saturating at 448; s == 0 gives sign-only codes.
+ * Decode: x ~= E4M3(code) * s.
+ * x: rows x cols of dt (NVFP4_F32 or NVFP4_BF16), row-major and contiguous, 16-byte aligned.
+ * codes: rows x cols bytes (device, 16-byte aligned), written. scale: device fp32, written.
+ * static_amax: device fp32 or NULL (dynamic). Values must be finite.
+ * ws: nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_E4M3, 0, 0, 0) bytes, unused with static_amax.
+ * Asynchronous on stream. The caller owns every buffer.
+ */
+nvfp4_status nvfp4_quantize_e4m3(const void *x, nvfp4_dtype dt, int64_t rows, int64_t cols,
+                                 const float *static_amax, uint8_t *codes, float *scale, void *ws,
+                                 size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * FP8 E4M3 tensorwise W8A8 linear layer on the FP8 tensor cores ("Qwen3-VL-8B-Instruct-
+ * heretic-NVFP4", "Runtime / hardware": FP8 layers run as native FP8 on Blackwell; "Qwen-Rapid-
+ * AIO FP8 -> NVFP4", "Solution": FP8 layers stay FP8, so E4M3 weights with their scale are used
+ * as they are):
+ *   Y[m, n] = (sA * sW) * sum_k E4M3(a[m, k]) * E4M3(w[n, k]),
+ * accumulated in fp32 by the tensor cores, scaled by sA * sW (fp32), stored as out_dt (bf16
+ * rounded to nearest even).
+ * a: M x K codes (activations, e.g. from nvfp4_quantize_e4m3), w: N x K codes (nn.Linear
+ * layout), both row-major and 16-byte aligned; a_scale / w_scale: device fp32.
+ * y: M x N of out_dt, row-major. K must be a positive multiple of 16. No workspace.
+ */
+nvfp4_status nvfp4_linear_e4m3(const uint8_t *a, const float *a_scale, const uint8_t *w,
+                               const float *w_scale, int64_t M, int64_t N, int64_t K,
+                               nvfp4_dtype out_dt, void *y, cudaStream_t stream);
 
 /*
  * Test of the failure-detection path. No counterpart in the paper. Launches one small kernel

@@ -9,6 +9,8 @@ device memory and the current stream, nothing else.
     y = linear(q_x, q_w)                      # block-scaled W4A4 GEMM, bf16 out
     pct, mx = calib_percentile_amax(batches)  # static p99.9 input scale
     q_s = quantize(x_bf16, static_amax=pct)
+    e_w = quantize_e4m3(w_bf16)               # FP8 E4M3 tensorwise (embed / lm_head layers)
+    y8 = linear_e4m3(quantize_e4m3(x_bf16), e_w)
 
 The C entry points are also available under their own names (``nvfp4_quantize`` ...).
 """
@@ -22,7 +24,7 @@ from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_LINEAR_DEFAULT, NVFP4_LINEAR_RES
                    NVFP4Error, check, load)
 
 __all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "quantize_batch", "dequantize", "linear",
-           "linear_dynamic",
+           "linear_dynamic", "E4M3Tensor", "quantize_e4m3", "linear_e4m3",
            "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
 
 
@@ -236,6 +238,58 @@ def linear_dynamic(x: torch.Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
                                 _ptr(out), _ptr(x_gs_out), _ptr(ws), ws_bytes, flags,
                                 _stream(dev))
     check(st, "nvfp4_linear_dynamic")
+    return out
+
+
+@dataclass
+class E4M3Tensor:
+    """FP8 E4M3 tensorwise: codes [rows, cols] uint8 and one fp32 scale (device, [1])."""
+    codes: torch.Tensor
+    scale: torch.Tensor
+
+    @property
+    def rows(self):
+        return self.codes.shape[0]
+
+    @property
+    def cols(self):
+        return self.codes.shape[1]
+
+
+def quantize_e4m3(x: torch.Tensor, static_amax: torch.Tensor = None,
+                  out: E4M3Tensor = None) -> E4M3Tensor:
+    """FP8 E4M3 tensorwise quantize of a 2-D fp32 / bf16 CUDA tensor: s = amax / 448,
+    code = sign | E4M3(|x| / s) (nearest, ties to even, saturating)."""
+    if x.dtype not in (torch.float32, torch.bfloat16) or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("quantize_e4m3 expects a 2-D CUDA fp32 or bf16 tensor")
+    x = x.contiguous()
+    rows, cols = x.shape
+    if out is None:
+        out = E4M3Tensor(torch.empty((rows, cols), dtype=torch.uint8, device=x.device),
+                         torch.empty(1, dtype=torch.float32, device=x.device))
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(_lib.NVFP4_OP_QUANTIZE_E4M3, 0, 0, 0)
+    ws = _workspace(x.device, ws_bytes)
+    dt = NVFP4_F32 if x.dtype == torch.float32 else NVFP4_BF16
+    st = L.nvfp4_quantize_e4m3(_ptr(x), dt, rows, cols, _ptr(static_amax), _ptr(out.codes),
+                               _ptr(out.scale), _ptr(ws), ws_bytes, _stream(x.device))
+    check(st, "nvfp4_quantize_e4m3")
+    return out
+
+
+def linear_e4m3(a: E4M3Tensor, w: E4M3Tensor, out_dtype=torch.bfloat16,
+                out: torch.Tensor = None) -> torch.Tensor:
+    """Y = (sA * sW) * A . W^T from E4M3 codes, [a.rows x w.rows], fp32 accumulation."""
+    if a.cols != w.cols:
+        raise ValueError("K mismatch")
+    M, N, K = a.rows, w.rows, a.cols
+    dev = a.codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    dt = NVFP4_F32 if out.dtype == torch.float32 else NVFP4_BF16
+    st = load().nvfp4_linear_e4m3(_ptr(a.codes), _ptr(a.scale), _ptr(w.codes), _ptr(w.scale),
+                                  M, N, K, dt, _ptr(out), _stream(dev))
+    check(st, "nvfp4_linear_e4m3")
     return out
 
 

@@ -232,6 +232,7 @@ size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
         if (m <= 0 || n <= 0 || k <= 0)
             return 0;
         return linear_dynamic_ws(m, n, k).total;
+    case NVFP4_OP_QUANTIZE_E4M3: return quantize_ws_bytes();
     case NVFP4_OP_CALIB_BF16: return calib_workspace_bytes(1);
     case NVFP4_OP_CALIB_F32: return calib_workspace_bytes(0);
     }
@@ -418,6 +419,52 @@ nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_bat
         rank = 1;
     return map_cuda(launch_calib(batches, num_batches, elems_per_batch, bf16, (uint64_t)rank,
                                  out_pct, out_max, ws, stream));
+}
+
+nvfp4_status nvfp4_quantize_e4m3(const void *x, nvfp4_dtype dt, int64_t rows, int64_t cols,
+                                 const float *static_amax, uint8_t *codes, float *scale, void *ws,
+                                 size_t ws_bytes, cudaStream_t stream)
+{
+    if (dt != NVFP4_F32 && dt != NVFP4_BF16)
+        return NVFP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || rows >= kMaxDim || cols >= kMaxDim)
+        return NVFP4_ERR_SHAPE;
+    const int64_t n = rows * cols;
+    if (!scale || (n > 0 && (!x || !codes)))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(scale) & 3u) || (reinterpret_cast<uintptr_t>(static_amax) & 3u))
+        return NVFP4_ERR_ALIGNMENT;
+    if (!static_amax && (!ws || ws_bytes < quantize_ws_bytes()))
+        return NVFP4_ERR_WORKSPACE;
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    return map_cuda(launch_quantize_e4m3(x, dt == NVFP4_F32 ? kSrcF32 : kSrcBF16, n, static_amax,
+                                         codes, scale, ws, stream));
+}
+
+nvfp4_status nvfp4_linear_e4m3(const uint8_t *a, const float *a_scale, const uint8_t *w,
+                               const float *w_scale, int64_t M, int64_t N, int64_t K,
+                               nvfp4_dtype out_dt, void *y, cudaStream_t stream)
+{
+    if (out_dt != NVFP4_F32 && out_dt != NVFP4_BF16)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K <= 0 || M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || K % 16 != 0)
+        return NVFP4_ERR_SHAPE;
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (!a || !w || !a_scale || !w_scale || !y)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(w) || (reinterpret_cast<uintptr_t>(a_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(w_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(y) & (out_dt == NVFP4_F32 ? 3u : 1u)))
+        return NVFP4_ERR_ALIGNMENT;
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    return map_cuda(launch_linear_e4m3(a, a_scale, w, w_scale, M, N, K, out_dt == NVFP4_BF16, y,
+                                       stream));
 }
 
 nvfp4_status nvfp4_selftest_wait_timeout(cudaStream_t stream)

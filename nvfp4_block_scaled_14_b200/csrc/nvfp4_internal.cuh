@@ -47,6 +47,14 @@ cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cud
 // Launches a kernel whose bounded wait cannot complete (selftest.cu).
 cudaError_t launch_wait_timeout_selftest(cudaStream_t s);
 
+// FP8 E4M3 tensorwise quantize of n values (fp32 or bf16, 16-byte aligned) into codes (16-byte
+// aligned) and the tensor scale (device fp32); ws as for launch_quantize.
+cudaError_t launch_quantize_e4m3(const void *x, int src_type, int64_t n, const float *static_amax,
+                                 uint8_t *codes, float *scale_out, void *ws, cudaStream_t s);
+// FP8 E4M3 tensorwise W8A8 GEMM: Y = (a_scale * w_scale) * A . W^T, A [M x K], W [N x K].
+cudaError_t launch_linear_e4m3(const uint8_t *a, const float *a_scale, const uint8_t *w,
+                               const float *w_scale, int64_t M, int64_t N, int64_t K, int out_bf16,
+                               void *y, cudaStream_t s);
 cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale, int64_t rows,
                             int64_t cols, const float *static_amax, uint8_t *codes,
                             uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,

@@ -1038,6 +1038,196 @@ int split_ctas(int n, const int64_t *weight, const int64_t *cap, int total, int 
     }
     return cta0[n];
 }
+// ---------------------------------------------------------------------------------------
+// FP8 E4M3 tensorwise quantization ("Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization
+// Details": embed_tokens / lm_head in float8_e4m3fn, tensorwise, round-to-nearest): one fp32
+// scale s = amax / 448 per tensor, code = sign(x) | E4M3(|x| / s) (RN of the IEEE quotient,
+// ties to even, saturating; s == 0 gives sign-only codes). HBM-bound elementwise pass after
+// the amax kernel (programmatic dependent launch): 8 values per thread-step, 16 or 32 bytes
+// in, 8 bytes out, grid-stride over the flat tensor.
+// ---------------------------------------------------------------------------------------
+constexpr int kE8Threads = 256;
+
+// sign(x) | E4M3(|x| / s) for one value (s > 0 or s == 0), as the helper of the block scales
+// computes it: the reference for the grouped form below and the ragged tail.
+__device__ __forceinline__ uint32_t e4m3_tensor_code(float v, float s, float rs)
+{
+    const uint32_t mag = s > 0.0f ? e4m3_of_quotient(fabsf(v), s, rs) : 0u;
+    return mag | ((__float_as_uint(v) >> 24) & 0x80u);
+}
+
+// Codes of 8 values (first value in the low byte of .x), s > 0. q = x * RN(1/s) in packed fp32
+// multiplies; the hardware pair conversion rounds the signed quotient to nearest (ties to even,
+// saturating), which is sign(x) | E4M3(|q|). q is within 3 fp32 ulps of RN(x / s), and the
+// E4M3 decision can only differ where q lies within 4 ulps of a midpoint (the 20 mantissa bits
+// below the 3 kept ones at 0x80000), in the subnormal E4M3 range, or when q is not finite; if
+// any of the 8 values is in such a case, all 8 take the IEEE quotient.
+__device__ __forceinline__ uint2 e4m3_codes8(const float (&f)[8], float s, uint64_t rs2)
+{
+    float q[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint64_t r;
+        asm("mul.rn.f32x2 %0, %1, %2;"
+            : "=l"(r)
+            : "l"(((uint64_t)__float_as_uint(f[2 * j + 1]) << 32) | __float_as_uint(f[2 * j])),
+              "l"(rs2));
+        q[2 * j] = __uint_as_float((uint32_t)r);
+        q[2 * j + 1] = __uint_as_float((uint32_t)(r >> 32));
+    }
+    bool slow = false;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float a = fabsf(q[j]);
+        const uint32_t mb = __float_as_uint(q[j]) & 0xFFFFFu;
+        slow |= (a < 0.015625f && a != 0.0f) || !(a <= 3.0e38f) || (mb - 0x7FFFCu <= 8u);
+    }
+    if (slow) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            q[j] = __fdiv_rn(f[j], s);
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint16_t h;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(q[2 * j + 1]), "f"(q[2 * j]));
+        w[j] = h;
+    }
+    return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+template <int SRC> __device__ __forceinline__ void load8(const uint8_t *x, int64_t i, float (&f)[8])
+{
+    if constexpr (SRC == kSrcF32) {
+        const uint4 a = __ldcs(reinterpret_cast<const uint4 *>(x + i * 4));
+        const uint4 b = __ldcs(reinterpret_cast<const uint4 *>(x + i * 4 + 16));
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            f[j] = __uint_as_float(w[j]);
+    } else {
+        const uint4 a = __ldcs(reinterpret_cast<const uint4 *>(x + i * 2));
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            f[2 * j] = __uint_as_float(w[j] << 16);
+            f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+template <int SRC> __device__ __forceinline__ float value_at(const uint8_t *x, int64_t i)
+{
+    if constexpr (SRC == kSrcF32)
+        return reinterpret_cast<const float *>(x)[i];
+    else
+        return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(x)[i] << 16);
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(kE8Threads)
+    e4m3_encode_kernel(const uint8_t *__restrict__ x, int64_t n, const float *static_amax,
+                       const float *__restrict__ partials, int npartials,
+                       uint8_t *__restrict__ codes, float *__restrict__ scale_out)
+{
+    __shared__ float s_s;
+    if (!static_amax)
+        pdl_wait(); // the amax kernel's partial maxima are complete and visible
+    if (threadIdx.x < 32) {
+        float g = 0.0f;
+        if (static_amax) {
+            g = *static_amax;
+        } else {
+            for (int i = threadIdx.x; i < npartials; i += 32)
+                g = fmaxf(g, __ldcg(partials + i));
+            // the amax kernel folds whole 16-byte vectors; the values after the last one
+            const int64_t tail0 = ((n * Src<SRC>::kBytes) & ~(int64_t)15) / Src<SRC>::kBytes;
+            for (int64_t i = tail0 + threadIdx.x; i < n; i += 32)
+                g = fmaxf(g, fabsf(value_at<SRC>(x, i)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+        }
+        if (threadIdx.x == 0) {
+            const float sc = __fdiv_rn(g, 448.0f);
+            s_s = sc;
+            if (blockIdx.x == 0)
+                *scale_out = sc;
+        }
+    }
+    __syncthreads();
+    const float sc = s_s;
+    const float rs = __frcp_rn(sc);
+    const uint64_t rs2 = ((uint64_t)__float_as_uint(rs) << 32) | __float_as_uint(rs);
+    const int64_t nvec = n >> 3;
+    const int64_t stride = (int64_t)gridDim.x * kE8Threads;
+    for (int64_t v = (int64_t)blockIdx.x * kE8Threads + threadIdx.x; v < nvec; v += stride) {
+        float f[8];
+        load8<SRC>(x, v * 8, f);
+        uint2 c;
+        if (sc > 0.0f) {
+            c = e4m3_codes8(f, sc, rs2);
+        } else { // s == 0: sign-only codes
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                w[j >> 2] |= ((__float_as_uint(f[j]) >> 24) & 0x80u) << (8 * (j & 3));
+            c = make_uint2(w[0], w[1]);
+        }
+        __stcs(reinterpret_cast<uint2 *>(codes + v * 8), c);
+    }
+    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) { // ragged tail, one value per thread
+        const int64_t i = (nvec << 3) + threadIdx.x;
+        codes[i] = (uint8_t)e4m3_tensor_code(value_at<SRC>(x, i), sc, rs);
+    }
+}
+
+template <int SRC>
+cudaError_t launch_e4m3_typed(const void *x, int64_t n, const float *static_amax,
+                              uint8_t *codes, float *scale_out, void *ws, cudaStream_t s)
+{
+    const int sms = num_sms();
+    int npartials = 0;
+    if (!static_amax) {
+        const int64_t nbytes = n * Src<SRC>::kBytes;
+        int g = sms < kAmaxPartials ? sms : kAmaxPartials;
+        const int64_t need = (nbytes + kChunk - 1) / kChunk;
+        if (need < g)
+            g = need < 1 ? 1 : (int)need;
+        npartials = g;
+        const size_t smem = (size_t)kRing * kChunk;
+        cudaError_t e = cudaFuncSetAttribute(amax_kernel<SRC>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        amax_kernel<SRC><<<g, kAmaxThreads, smem, s>>>(reinterpret_cast<const uint8_t *>(x),
+                                                       nbytes, reinterpret_cast<float *>(ws),
+                                                       device_status_ptr());
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+    }
+    const int64_t nvec = n >> 3;
+    int64_t grid = (nvec + kE8Threads - 1) / kE8Threads;
+    const int64_t max_grid = (int64_t)sms * 8;
+    if (grid > max_grid)
+        grid = max_grid;
+    if (grid < 1)
+        grid = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kE8Threads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = static_amax ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, e4m3_encode_kernel<SRC>, reinterpret_cast<const uint8_t *>(x),
+                              n, static_amax, reinterpret_cast<const float *>(ws), npartials, codes,
+                              scale_out);
+}
+
 } // namespace
 
 size_t quantize_workspace_bytes() { return (size_t)kAmaxPartials * sizeof(float); }
@@ -1058,6 +1248,14 @@ cudaError_t launch_quantize(const void *x, int src_type, const float *fp8_scale,
         return launch_typed<kSrcE4M3>(x, fp8_scale, rows, cols, static_amax, codes, scales_swz,
                                       scales_lin, global_scale, ws, s);
     }
+}
+
+cudaError_t launch_quantize_e4m3(const void *x, int src_type, int64_t n, const float *static_amax,
+                                 uint8_t *codes, float *scale_out, void *ws, cudaStream_t s)
+{
+    if (src_type == kSrcF32)
+        return launch_e4m3_typed<kSrcF32>(x, n, static_amax, codes, scale_out, ws, s);
+    return launch_e4m3_typed<kSrcBF16>(x, n, static_amax, codes, scale_out, ws, s);
 }
 
 cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t s)

@@ -462,3 +462,104 @@ def test_calib_skewed_layout():
 
 def test_sync_status_clean():
     assert nv.sync_status() == 0
+
+
+# ---------------------------------------------------------------------------------------
+# FP8 E4M3 tensorwise layers
+# ---------------------------------------------------------------------------------------
+
+def _gpu_e4m3(x: np.ndarray, amax=None):
+    q = nv.quantize_e4m3(dev_tensor(x), static_amax=None if amax is None else scalar_dev(amax))
+    torch.cuda.synchronize()
+    return q.codes.cpu().numpy(), float(q.scale.cpu()[0])
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 8), (3, 37), (1, 5), (64, 3072), (257, 1000),
+                                       (4096, 3072)])
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+def test_quantize_e4m3_matches_oracle(rows, cols, kind):
+    x = W.normal((rows, cols), 1.0, 50, rows * 7 + cols)
+    x.reshape(-1)[::101] *= np.float32(40.0)   # a spread of magnitudes, subnormal codes too
+    x.reshape(-1)[1::89] *= np.float32(1e-5)
+    x.reshape(-1)[2::97] = -0.0
+    if kind == "bf16":
+        x = W.to_bf16_bits(x)
+    codes, s = _gpu_e4m3(x)
+    rc, rs = O.quantize_e4m3(x)
+    assert s == rs
+    assert np.array_equal(codes, rc)
+
+
+@pytest.mark.parametrize("amax", [0.75, 0.0, 1e-37])
+def test_quantize_e4m3_static_amax(amax):
+    # values above the static amax saturate at 448; amax 0 gives sign-only codes; a tiny amax
+    # makes 1/s overflow (the quotient path must still round correctly)
+    x = W.normal((33, 48), 1.0, 51, 1)
+    codes, s = _gpu_e4m3(x, amax=amax)
+    rc, rs = O.quantize_e4m3(x, amax=amax)
+    assert s == rs and np.array_equal(codes, rc)
+
+
+def test_quantize_e4m3_all_zero():
+    codes, s = _gpu_e4m3(np.zeros((7, 24), np.float32))
+    assert s == 0.0 and not codes.any()
+
+
+def _e4m3_linear(M, N, K, out_dtype, seed):
+    xa = W.to_bf16_bits(W.normal((M, K), 1.0, seed, M))
+    xw = W.to_bf16_bits(W.normal((N, K), 0.02, seed + 1, N))
+    qa = nv.quantize_e4m3(dev_tensor(xa))
+    qw = nv.quantize_e4m3(dev_tensor(xw))
+    out = torch.full((M, N), float("nan"), dtype=out_dtype, device="cuda")
+    nv.linear_e4m3(qa, qw, out=out)
+    torch.cuda.synchronize()
+    ac, sa = O.quantize_e4m3(xa)
+    wc, sw = O.quantize_e4m3(xw)
+    assert np.array_equal(qa.codes.cpu().numpy(), ac) and np.array_equal(qw.codes.cpu().numpy(), wc)
+    return to_numpy_f64(out), ac, sa, wc, sw
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 256, 128), (5, 384, 512), (300, 520, 1056), (256, 264, 512), (129, 256, 256),
+    (130, 1004, 256),   # bf16 rows whose byte stride is not a multiple of 16: direct stores
+    (512, 768, 2048),   # several tiles per CTA pair: both accumulators in turn
+    (40, 200, 16),      # K of one 16-value step (the rest of the k-tile is zero fill)
+])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_linear_e4m3_matches_oracle(M, N, K, out):
+    odt = torch.bfloat16 if out == "bf16" else torch.float32
+    y, ac, sa, wc, sw = _e4m3_linear(M, N, K, odt, 52)
+    assert np.isfinite(y).all()  # every element written
+    ref = O.gemm_e4m3(ac, sa, wc, sw)
+    tol = gemm_tolerance(ref, out == "bf16")
+    assert np.all(np.abs(y - ref) <= tol), f"max err {np.abs(y - ref).max()}"
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 3072, 3072), (1300, 1960, 512)])
+def test_linear_e4m3_large_sampled(M, N, K):
+    y, ac, sa, wc, sw = _e4m3_linear(M, N, K, torch.bfloat16, 53)
+    assert np.isfinite(y).all()
+    r = np.random.Generator(np.random.PCG64(54))
+    edge = [0, 127, 128, 255, 256, M - 1]
+    edge_n = [0, 63, 64, 255, 256, N - 1]
+    ms = np.concatenate([r.integers(0, M, 3000), np.repeat(edge, len(edge_n))])
+    ns = np.concatenate([r.integers(0, N, 3000), np.tile(edge_n, len(edge))])
+    ref = O.gemm_e4m3_sampled(ac, sa, wc, sw, ms, ns)
+    tol = 1e-3 * np.abs(y).max() + np.abs(ref) * 2.0 ** -8
+    assert np.all(np.abs(y[ms, ns] - ref) <= tol)
+
+
+def test_linear_e4m3_integer_exact():
+    # integer codes with unit scales: every partial sum is an integer below 2^24, so the fp32
+    # tensor-core accumulation is exact and equals the oracle bit for bit
+    g = np.random.Generator(np.random.PCG64(55))
+    M, N, K = 300, 520, 1056
+    ints = np.arange(-16, 17).astype(np.float32)
+    enc = torch.from_numpy(ints).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ai = g.integers(0, len(ints), (M, K))
+    wi = g.integers(0, len(ints), (N, K))
+    a = nv.E4M3Tensor(torch.from_numpy(enc[ai]).cuda(), scalar_dev(1.0))
+    w = nv.E4M3Tensor(torch.from_numpy(enc[wi]).cuda(), scalar_dev(1.0))
+    y = nv.linear_e4m3(a, w, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_numpy_f64(y), O.gemm_e4m3(enc[ai], 1.0, enc[wi], 1.0))

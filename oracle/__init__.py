@@ -67,6 +67,15 @@ def lib():
         L.ora_e4m3_encode_array.argtypes = [_f32p, _i64, _u8p]
         L.ora_amax.argtypes = [_f32p, _i64]
         L.ora_amax.restype = ctypes.c_float
+        L.ora_gelu_tanh_f64.argtypes = [ctypes.c_double]
+        L.ora_gelu_tanh_f64.restype = ctypes.c_double
+        L.ora_linear_act_f64_sampled.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p,
+                                                 ctypes.c_float, _i64, ctypes.c_int, _i64p,
+                                                 _i64p, _i64, _f64p]
+        L.ora_linear_quantize_out.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p,
+                                              ctypes.c_float, _i64, _i64, _i64, ctypes.c_float,
+                                              ctypes.c_int, _u8p, _u8p, _u8p, _f32p]
+        L.ora_linear_quantize_out.restype = ctypes.c_int
         L.ora_quantize_e4m3.argtypes = [_vp, ctypes.c_int, _i64, _f32p, _u8p, _f32p]
         L.ora_quantize_e4m3.restype = ctypes.c_int
         L.ora_gemm_e4m3_f64.argtypes = [_u8p, ctypes.c_float, _u8p, ctypes.c_float, _i64, _i64,
@@ -221,6 +230,42 @@ def source_to_f32(x: np.ndarray, fp8_scale=None) -> np.ndarray:
     f = lut[x]
     s8 = np.float32(1.0 if fp8_scale is None else fp8_scale)
     return (f * s8).astype(np.float32)
+
+
+# ---- linear layer with an NVFP4 output (producer epilogue) -------------------------------
+ACT_NONE, ACT_GELU_TANH = 0, 1
+
+
+def gelu_tanh(y: float) -> float:
+    return lib().ora_gelu_tanh_f64(float(y))
+
+
+def linear_act_sampled(a: Quantized, w: Quantized, act, ms, ns) -> np.ndarray:
+    """act(sgA sgW acc) in fp64 at (ms[i], ns[i]): the exact value the fused layer encodes."""
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    out = np.zeros(len(ms), np.float64)
+    lib().ora_linear_act_f64_sampled(_p(a.codes, _u8p), _p(a.scales_lin, _u8p), a.sg,
+                                     _p(w.codes, _u8p), _p(w.scales_lin, _u8p), w.sg, a.cols,
+                                     act, _p(ms, _i64p), _p(ns, _i64p), len(ms), _p(out, _f64p))
+    return out
+
+
+def linear_quantize_out(a: Quantized, w: Quantized, static_amax, act=ACT_NONE) -> Quantized:
+    """NVFP4 (static amax) of act(RN32(RN32(acc) * RN32(sgA sgW))), [a.rows x w.rows]."""
+    assert a.cols == w.cols
+    M, N, K = a.rows, w.rows, a.cols
+    codes = np.zeros((M, N // 2), np.uint8)
+    lin = np.zeros((M, N // 16), np.uint8)
+    swz = np.zeros(max(swizzled_bytes(M, N), 1), np.uint8)
+    sg = np.zeros(1, np.float32)
+    rc = lib().ora_linear_quantize_out(_p(a.codes, _u8p), _p(a.scales_lin, _u8p), a.sg,
+                                       _p(w.codes, _u8p), _p(w.scales_lin, _u8p), w.sg, M, N, K,
+                                       float(static_amax), act, _p(codes, _u8p), _p(lin, _u8p),
+                                       _p(swz, _u8p), _p(sg, _f32p))
+    if rc != 0:
+        raise ValueError(f"oracle linear_quantize_out failed ({rc})")
+    return Quantized(codes, lin, swz, float(sg[0]), M, N)
 
 
 # ---- FP8 E4M3 tensorwise layers ----------------------------------------------------------

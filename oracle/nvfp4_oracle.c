@@ -366,6 +366,71 @@ void ora_gemm_f64_sampled(const uint8_t *a_codes, const uint8_t *a_scales_lin, f
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* Linear layer with an NVFP4 output (a producer epilogue)                                     */
+/* ------------------------------------------------------------------------------------------ */
+/* [QRc] "Recommended Model": with static input scales from calibration, the next layer's input
+ * can be quantized where it is produced. Readings where the pages are silent (design notes):
+ *   - acc = sum_b sA[m,b] sW[n,b] sum_k eA eW (exact), y = RN32(RN32(acc) * RN32(sgA * sgW)):
+ *     the fp32 product the tensor cores accumulate, scaled as the linear layer's epilogue does;
+ *   - activation act: 0 identity; 1 GELU in its tanh form,
+ *     gelu(y) = 0.5 y (1 + tanh(u)) = y / (1 + exp(-2 u)), u = sqrt(2/pi) (y + 0.044715 y^3),
+ *     evaluated in fp64 (the second form: no cancellation for negative y) and rounded to fp32;
+ *   - the activation output is NVFP4-quantized with the static amax (ora_quantize_f32). */
+
+double ora_gelu_tanh_f64(double y)
+{
+    double u = 0.7978845608028654 * (y + 0.044715 * y * y * y);
+    return y / (1.0 + exp(-2.0 * u));
+}
+
+static double act_f64(double y, int act) { return act == 1 ? ora_gelu_tanh_f64(y) : y; }
+
+/* acc without the global scales (see gemm_one). */
+static double block_sum(const uint8_t *a_codes, const uint8_t *a_sc, const uint8_t *w_codes,
+                        const uint8_t *w_sc, int64_t m, int64_t n, int64_t K)
+{
+    return gemm_one(a_codes, a_sc, 1.0f, w_codes, w_sc, 1.0f, m, n, K);
+}
+
+/* fp64 activation of the exact product sgA sgW acc: the value the fused layer approximates. */
+void ora_linear_act_f64_sampled(const uint8_t *a_codes, const uint8_t *a_sc, float a_sg,
+                                const uint8_t *w_codes, const uint8_t *w_sc, float w_sg,
+                                int64_t K, int act, const int64_t *ms, const int64_t *ns,
+                                int64_t count, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; i++)
+        out[i] = act_f64((double)a_sg * (double)w_sg *
+                             block_sum(a_codes, a_sc, w_codes, w_sc, ms[i], ns[i], K),
+                         act);
+}
+
+/* The fused layer's NVFP4 output [M x N]: y as above, v = act(y) in fp32, quantized with the
+ * static amax. Returns 0, or -1 if N is not a multiple of 16, -2 on allocation failure. */
+int ora_linear_quantize_out(const uint8_t *a_codes, const uint8_t *a_sc, float a_sg,
+                            const uint8_t *w_codes, const uint8_t *w_sc, float w_sg, int64_t M,
+                            int64_t N, int64_t K, float static_amax, int act, uint8_t *codes,
+                            uint8_t *scales_lin, uint8_t *scales_swz, float *sg_out)
+{
+    if (N % 16 != 0)
+        return -1;
+    float *v = (float *)malloc((size_t)(M * N > 0 ? M * N : 1) * sizeof(float));
+    if (!v)
+        return -2;
+    const float alpha = a_sg * w_sg;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            float acc = (float)block_sum(a_codes, a_sc, w_codes, w_sc, m, n, K);
+            float y = acc * alpha;
+            v[m * N + n] = act == 1 ? (float)ora_gelu_tanh_f64((double)y) : y;
+        }
+    int rc = ora_quantize_f32(v, M, N, &static_amax, codes, scales_lin, scales_swz, sg_out);
+    free(v);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* FP8 E4M3 tensorwise layers                                                                  */
 /* ------------------------------------------------------------------------------------------ */
 /* [QVf] "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details" and "Layer breakdown":

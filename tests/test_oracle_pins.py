@@ -431,3 +431,53 @@ def test_gemm_e4m3_is_dequantized_product():
     da = e4m3_torch_decode(a) * sa
     dw = e4m3_torch_decode(w) * sw
     assert np.allclose(O.gemm_e4m3(a, sa, w, sw), da @ dw.T, rtol=1e-12, atol=0)
+
+
+# ---- linear layer with an NVFP4 output -------------------------------------------------
+
+def test_gelu_tanh_matches_torch():
+    y = np.concatenate([np.linspace(-12, 12, 2001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]])
+    ref = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
+    ours = np.array([O.gelu_tanh(v) for v in y])
+    assert np.allclose(ours, ref, rtol=1e-13, atol=1e-15)
+    assert O.gelu_tanh(0.0) == 0.0 and O.gelu_tanh(40.0) == 40.0 and O.gelu_tanh(-40.0) == 0.0
+
+
+def _exact_product_operands(M, N, K, seed, a_sg=1.0, w_sg=0.5):
+    # unit block scales (0x38) and power-of-two global scales: every partial sum of
+    # E2M1 x E2M1 products is a multiple of 1/4 below 2^24, so fp32 holds the product exactly
+    g = np.random.Generator(np.random.PCG64(seed))
+    ac = g.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    wc = g.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    a = O.Quantized(ac, np.full((M, K // 16), 0x38, np.uint8), None, a_sg, M, K)
+    w = O.Quantized(wc, np.full((N, K // 16), 0x38, np.uint8), None, w_sg, N, K)
+    return a, w
+
+
+@pytest.mark.parametrize("act", [O.ACT_NONE, O.ACT_GELU_TANH])
+def test_linear_quantize_out_equals_quantize_of_product(act):
+    M, N, K = 5, 64, 96
+    a, w = _exact_product_operands(M, N, K, 130)
+    y = O.gemm(a, w).astype(np.float32)  # exact: power-of-two scales, small integer sums
+    assert np.array_equal(y.astype(np.float64), O.gemm(a, w))
+    if act == O.ACT_GELU_TANH:
+        y = torch.nn.functional.gelu(torch.from_numpy(y.astype(np.float64)),
+                                     approximate="tanh").numpy().astype(np.float32)
+    amax = 0.8 * float(np.abs(y).max())  # some values saturate
+    ref = O.quantize(y, amax=amax)
+    got = O.linear_quantize_out(a, w, amax, act)
+    assert got.sg == ref.sg
+    assert np.array_equal(got.codes, ref.codes)
+    assert np.array_equal(got.scales_lin, ref.scales_lin)
+    assert np.array_equal(got.scales_swz, ref.scales_swz)
+
+
+@pytest.mark.parametrize("act", [O.ACT_NONE, O.ACT_GELU_TANH])
+def test_linear_act_sampled_is_activation_of_gemm(act):
+    a = O.quantize(W.normal((20, 64), 1.0, 131, 1))
+    w = O.quantize(W.normal((30, 64), 0.02, 131, 2))
+    ms, ns = np.array([0, 19, 7, 3]), np.array([29, 0, 15, 3])
+    y = O.gemm_sampled(a, w, ms, ns)
+    if act == O.ACT_GELU_TANH:
+        y = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
+    assert np.allclose(O.linear_act_sampled(a, w, act, ms, ns), y, rtol=1e-14, atol=0)

@@ -253,6 +253,33 @@ nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_bat
                                          float *out_max, void *ws, size_t ws_bytes,
                                          cudaStream_t stream);
 
+/* Activation of nvfp4_linear_nvfp4_out. */
+typedef enum {
+    NVFP4_ACT_IDENTITY = 0,
+    NVFP4_ACT_GELU_TANH = 1 /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) */
+} nvfp4_act;
+
+/*
+ * Linear layer whose output is the next layer's NVFP4 operand: Y as nvfp4_linear defines it
+ * (fp32 tensor-core accumulation, scaled by sgA * sgW in fp32), V = act(Y), then V quantized
+ * exactly as nvfp4_quantize(V, static_amax) would quantize an fp32 V, inside the GEMM's
+ * epilogue, so V never goes to memory in bf16 ("Qwen-Rapid-AIO FP8 -> NVFP4", "Recommended
+ * Model": static input scales from calibration; e.g. the first GEMM of an MLP writing the
+ * second one's activations). act: nvfp4_act; NVFP4_ACT_GELU_TANH uses the hardware's fast
+ * exponential and division (relative error ~1e-6 against the exact formula), so codes can
+ * differ from an exact evaluation only where V lies that close to a rounding boundary.
+ * A: M x K, W: N x K as in nvfp4_linear (swizzled scales). static_amax: device fp32.
+ * Outputs (device, 16-byte aligned): y_codes M x N/2 bytes, y_scales_swz
+ * nvfp4_scales_bytes(M, N, 1) bytes (padding written as zero), y_gs one fp32 (the global scale,
+ * static_amax / 2688). K and N must be multiples of 32. No workspace.
+ */
+nvfp4_status nvfp4_linear_nvfp4_out(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                                    const float *a_gs, const uint8_t *w_codes,
+                                    const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
+                                    int64_t N, int64_t K, int act, const float *static_amax,
+                                    uint8_t *y_codes, uint8_t *y_scales_swz, float *y_gs,
+                                    cudaStream_t stream);
+
 /*
  * FP8 E4M3 tensorwise quantization ("Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization
  * Details" and "Layer breakdown": embed_tokens and lm_head in float8_e4m3fn, tensorwise,

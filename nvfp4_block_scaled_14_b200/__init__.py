@@ -24,7 +24,7 @@ from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_LINEAR_DEFAULT, NVFP4_LINEAR_RES
                    NVFP4Error, check, load)
 
 __all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "quantize_batch", "dequantize", "linear",
-           "linear_dynamic", "E4M3Tensor", "quantize_e4m3", "linear_e4m3",
+           "linear_dynamic", "linear_nvfp4_out", "E4M3Tensor", "quantize_e4m3", "linear_e4m3",
            "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
 
 
@@ -238,6 +238,29 @@ def linear_dynamic(x: torch.Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
                                 _ptr(out), _ptr(x_gs_out), _ptr(ws), ws_bytes, flags,
                                 _stream(dev))
     check(st, "nvfp4_linear_dynamic")
+    return out
+
+
+def linear_nvfp4_out(a: NVFP4Tensor, w: NVFP4Tensor, static_amax: torch.Tensor,
+                     act: str = "identity", out: NVFP4Tensor = None) -> NVFP4Tensor:
+    """NVFP4 (static amax) of act(dequant(a) . dequant(w)^T), quantized in the GEMM's epilogue;
+    act is "identity" or "gelu_tanh". The result feeds linear() as its activation operand."""
+    if a.cols != w.cols:
+        raise ValueError("K mismatch")
+    acts = {"identity": _lib.NVFP4_ACT_IDENTITY, "gelu_tanh": _lib.NVFP4_ACT_GELU_TANH}
+    if act not in acts:
+        raise ValueError(f"act must be one of {sorted(acts)}")
+    M, N, K = a.rows, w.rows, a.cols
+    dev = a.codes.device
+    if out is None:
+        codes, swz, _, gs = _alloc_outputs(M, N, dev, True, False)
+        out = NVFP4Tensor(codes, swz, None, gs, M, N)
+    st = load().nvfp4_linear_nvfp4_out(_ptr(a.codes), _ptr(a.scales_swz), _ptr(a.global_scale),
+                                       _ptr(w.codes), _ptr(w.scales_swz), _ptr(w.global_scale),
+                                       M, N, K, acts[act], _ptr(static_amax), _ptr(out.codes),
+                                       _ptr(out.scales_swz), _ptr(out.global_scale),
+                                       _stream(dev))
+    check(st, "nvfp4_linear_nvfp4_out")
     return out
 
 

@@ -421,6 +421,40 @@ nvfp4_status nvfp4_calib_percentile_amax(const void *const *batches, int num_bat
                                  out_pct, out_max, ws, stream));
 }
 
+nvfp4_status nvfp4_linear_nvfp4_out(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                                    const float *a_gs, const uint8_t *w_codes,
+                                    const uint8_t *w_scales_swz, const float *w_gs, int64_t M,
+                                    int64_t N, int64_t K, int act, const float *static_amax,
+                                    uint8_t *y_codes, uint8_t *y_scales_swz, float *y_gs,
+                                    cudaStream_t stream)
+{
+    if (act != NVFP4_ACT_IDENTITY && act != NVFP4_ACT_GELU_TANH)
+        return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st;
+    if ((st = check_matrix(M, K)) != NVFP4_OK || (st = check_matrix(N, K)) != NVFP4_OK ||
+        (st = check_matrix(M, N)) != NVFP4_OK)
+        return st;
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (K == 0)
+        return NVFP4_ERR_SHAPE;
+    if (!a_codes || !a_scales_swz || !a_gs || !w_codes || !w_scales_swz || !w_gs ||
+        !static_amax || !y_codes || !y_scales_swz || !y_gs)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_scales_swz) || !aligned16(w_codes) ||
+        !aligned16(w_scales_swz) || !aligned16(y_codes) || !aligned16(y_scales_swz) ||
+        (reinterpret_cast<uintptr_t>(a_gs) & 3u) || (reinterpret_cast<uintptr_t>(w_gs) & 3u) ||
+        (reinterpret_cast<uintptr_t>(static_amax) & 3u) || (reinterpret_cast<uintptr_t>(y_gs) & 3u))
+        return NVFP4_ERR_ALIGNMENT;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    st = NVFP4_OK;
+    const cudaError_t e =
+        launch_linear_nvfp4_out(a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs, M, N, K,
+                                act, static_amax, y_codes, y_scales_swz, y_gs, stream, &st);
+    return st != NVFP4_OK ? st : map_cuda(e);
+}
+
 nvfp4_status nvfp4_quantize_e4m3(const void *x, nvfp4_dtype dt, int64_t rows, int64_t cols,
                                  const float *static_amax, uint8_t *codes, float *scale, void *ws,
                                  size_t ws_bytes, cudaStream_t stream)

@@ -107,6 +107,14 @@ struct GemmParams {
     float *partial;            // split-K partials [splits][tiles_a*128][tiles_b*BN]
     int *status;
     int tma_store; // 1: bf16 output through the shared-memory staging + TMA store
+    // NVFP4 output of the pair kernel's quantizing epilogue (nvfp4_linear_nvfp4_out): codes
+    // [rows_a x rows_b / 2], swizzled scales (q_apb atoms per 128-row band, q_rows_pad rows),
+    // global scale from the static amax, activation (0 identity, 1 tanh-form GELU)
+    uint8_t *q_codes, *q_sf;
+    float *q_gs;
+    const float *q_amax;
+    int act, q_apb;
+    int64_t q_rows_pad;
 };
 
 __device__ __forceinline__ void set_timeout(int *status)
@@ -605,11 +613,96 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Activation of the quantizing epilogue: ACT 0 identity; ACT 1 GELU in its tanh form,
+// y / (1 + exp(-2u)) with u = sqrt(2/pi) (y + 0.044715 y^3), as y * rcp(1 + 2^(y * k (1 + c y^2)))
+// with k = -2 sqrt(2/pi) log2(e) and the hardware's approximate base-2 exponential and
+// reciprocal (relative error ~1e-6). The exponent is clamped at 126, where the result is
+// already below 1e-37 |y|: 1 + 2^126 keeps the reciprocal finite and non-zero.
+__device__ __forceinline__ float fast_ex2(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float fast_rcp(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+template <int ACT> __device__ __forceinline__ float epi_act(float y)
+{
+    if constexpr (ACT == 1) {
+        const float z = y * (-2.3022082f * fmaf(0.044715f, y * y, 1.0f));
+        return y * fast_rcp(1.0f + fast_ex2(fminf(z, 126.0f)));
+    } else {
+        return y;
+    }
+}
+
+// One thread's 256-column accumulator row (TMEM address trow) of output row `row`, columns
+// col0..col0+255 -> NVFP4: v = act(acc * alpha); per 16-value block sb = E4M3(bmax / t)
+// (t = 6 sg, the quantizer's exact quotient), codes E2M1(v * s_rcp[sb]) with
+// s_rcp[c] = RN(1 / RN(E4M3(c) * sg)); sb = 0 gives zero codes. Codes go to the row's 32-byte
+// runs, the four scales of each 64-column atom row to the swizzled layout in one 4-byte store.
+// Rows past M and columns past N hold zeros (their operands are TMA zero fill), so the
+// swizzled padding of the last band and atom is written as zero scales.
+template <int ACT>
+__device__ __forceinline__ void quantize_out_row(const GemmParams &p, uint32_t trow, int64_t row,
+                                                 int64_t col0, float alpha, float t, float rt,
+                                                 const float *s_rcp)
+{
+#pragma unroll 1
+    for (int c0 = 0; c0 < 256; c0 += 64) {
+        uint32_t v[64];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            tmem_ld_32x32b_x16(trow + c0 + 16 * i, v + 16 * i);
+        tmem_ld_wait();
+        uint32_t cw[8];
+        uint32_t sw = 0u;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            float y[16];
+            float bmax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                y[j] = epi_act<ACT>(__fmul_rn(__uint_as_float(v[16 * b + j]), alpha));
+                bmax = fmaxf(bmax, fabsf(y[j]));
+            }
+            const uint32_t sb = t > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
+            const float r = s_rcp[sb]; // sb = 0: every code is 0 (selected below)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                y[j] = __fmul_rn(y[j], r);
+            const uint32_t lo = cvt_e2m1x8(y), hi = cvt_e2m1x8(y + 8);
+            cw[2 * b] = sb != 0u ? lo : 0u;
+            cw[2 * b + 1] = sb != 0u ? hi : 0u;
+            sw |= sb << (8 * b);
+        }
+        const int64_t col = col0 + c0;
+        if (row < p.rows_a && col < p.rows_b) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.q_codes + row * (p.rows_b / 2) + col / 2);
+            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            if (col + 32 < p.rows_b)
+                dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        }
+        const int64_t atom = col / 64;
+        if (row < p.q_rows_pad && atom < p.q_apb)
+            *reinterpret_cast<uint32_t *>(p.q_sf + ((row >> 7) * p.q_apb + atom) * 512 +
+                                          16 * (row & 31) + 4 * ((row & 127) >> 5)) = sw;
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // 2-SM variant: a CTA pair (cluster of 2) computes a 256 x 256 tile with
 // tcgen05.mma.cta_group::2 (M256 N256 K64). Each CTA loads its 128 rows of A and its 128
 // rows of B, so the shared-memory traffic per SM per k-tile drops from ~108 KB (1-SM 128x256
-// tile: TMA writes + MMA reads) to ~76 KB. The leader CTA (rank 0) issues the MMAs and
+// tile: TMA writes + MMA reads) to ~76 KB. QOUT: the epilogue quantizes the (activated) tile
+// to NVFP4 with a static global scale instead of storing bf16 (quantize_out_row): the next
+// layer's operand is produced without a bf16 round trip. The leader CTA (rank 0) issues the MMAs and
 // commits to barriers of both CTAs; the other CTA's TMA loads of A / B and its feeder and
 // epilogue warps arrive on the leader's barriers. Scale factors: each CTA's TMEM holds SFA
 // of its own 128 rows and SFB of all 256 columns (its feeders write both). Only the bf16,
@@ -641,6 +734,7 @@ struct Pair {
     static_assert(kSfCol + kSfSlots * kSlotCols <= kTmemCols, "TMEM budget");
 };
 
+template <bool QOUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
@@ -867,6 +961,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
         const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
         uint32_t acc_phase = 0;
+        float q_t = 0.0f, q_rt = 0.0f;
+        float *s_rcp = reinterpret_cast<float *>(smem + C::kOffStaging); // QOUT: no staging
+        if constexpr (QOUT) {
+            const float sg = __fdiv_rn(*p.q_amax, 2688.0f); // 6 * 448, as the quantizer
+            q_t = __fmul_rn(sg, 6.0f);
+            q_rt = __frcp_rn(q_t);
+            const int i = (int)threadIdx.x - 64; // 0..127
+            s_rcp[i] = __frcp_rn(__fmul_rn(e4m3_to_f32((uint32_t)i), sg));
+            if (i == 0 && blockIdx.x == 0)
+                *p.q_gs = sg;
+            named_bar_sync(1, 128);
+        }
         for (int64_t u = cluster_id; u < tiles_ab; u += nclusters) {
             const int64_t ta = u % p.tiles_a, tb = u / p.tiles_a;
             if (!mbar_wait(acc_full, acc_phase, kWaitLimit)) {
@@ -876,6 +982,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+            if constexpr (QOUT) {
+                if (p.act == 1)
+                    quantize_out_row<1>(p, trow, ta * 256 + rank * 128 + q * 32 + lane, tb * 256,
+                                        alpha, q_t, q_rt, s_rcp);
+                else
+                    quantize_out_row<0>(p, trow, ta * 256 + rank * 128 + q * 32 + lane, tb * 256,
+                                        alpha, q_t, q_rt, s_rcp);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_remote(leader_acc_empty); // this CTA's accumulator is drained
+                acc_phase ^= 1;
+                continue;
+            }
             if (threadIdx.x == 64)
                 bulk_wait_group_read0();
             named_bar_sync(1, 128);
@@ -1675,14 +1795,16 @@ cudaError_t launch_bn(const LinearPlan &pl, const uint8_t *a_codes, const uint8_
     return cudaGetLastError();
 }
 
-cudaError_t launch_pair(const LinearPlan &pl, const uint8_t *a_codes, const uint8_t *a_sf,
-                        const uint8_t *w_codes, const uint8_t *w_sf, int64_t M, int64_t N,
-                        int64_t K, GemmParams gp, cudaStream_t s, nvfp4_status *st)
+template <bool QOUT>
+cudaError_t launch_pair(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *w_codes,
+                        const uint8_t *w_sf, int64_t M, int64_t N, int64_t K, GemmParams gp,
+                        cudaStream_t s, nvfp4_status *st)
 {
     CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
+    std::memset(&tmY, 0, sizeof(tmY));
     if (!encode_fn() || !make_codes_map(&tmA, a_codes, M, K, 128) ||
         !make_codes_map(&tmB, w_codes, N, K, 128) || !make_sf_map(&tmSFA, a_sf, M, K, 1) ||
-        !make_sf_map(&tmSFB, w_sf, N, K, 2) || !make_out_map(&tmY, gp.y, M, N)) {
+        !make_sf_map(&tmSFB, w_sf, N, K, 2) || (!QOUT && !make_out_map(&tmY, gp.y, M, N))) {
         *st = NVFP4_ERR_CUDA;
         return cudaErrorInvalidValue;
     }
@@ -1691,7 +1813,7 @@ cudaError_t launch_pair(const LinearPlan &pl, const uint8_t *a_codes, const uint
     cudaGetDevice(&dev);
     cudaError_t attr_err = cudaSuccess;
     std::call_once(flags[dev & 63], [&]() {
-        attr_err = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel,
+        attr_err = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QOUT>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         Pair::kSmemBytes);
     });
@@ -1705,7 +1827,7 @@ cudaError_t launch_pair(const LinearPlan &pl, const uint8_t *a_codes, const uint
         clusters = gp.units;
     if (clusters < 1)
         clusters = 1;
-    nvfp4_gemm_pair_kernel<<<(unsigned)(2 * clusters), kThreads, Pair::kSmemBytes, s>>>(
+    nvfp4_gemm_pair_kernel<QOUT><<<(unsigned)(2 * clusters), kThreads, Pair::kSmemBytes, s>>>(
         tmA, tmB, tmSFA, tmSFB, tmY, gp);
     return cudaGetLastError();
 }
@@ -1889,6 +2011,32 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, unsigned flags)
     return p;
 }
 
+cudaError_t launch_linear_nvfp4_out(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gs,
+                                    const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,
+                                    int64_t M, int64_t N, int64_t K, int act,
+                                    const float *static_amax, uint8_t *y_codes, uint8_t *y_sf,
+                                    float *y_gs, cudaStream_t s, nvfp4_status *st)
+{
+    GemmParams gp{};
+    gp.rows_a = M;
+    gp.rows_b = N;
+    gp.kt_total = (int)((K + 255) / 256);
+    gp.kt_per_split = gp.kt_total;
+    gp.splits = 1;
+    gp.a_gs = a_gs;
+    gp.w_gs = w_gs;
+    gp.ldy = N;
+    gp.status = device_status_ptr();
+    gp.q_codes = y_codes;
+    gp.q_sf = y_sf;
+    gp.q_gs = y_gs;
+    gp.q_amax = static_amax;
+    gp.act = act;
+    gp.q_apb = (int)((N / 16 + 3) / 4);
+    gp.q_rows_pad = (M + 127) / 128 * 128;
+    return launch_pair<true>(a_codes, a_sf, w_codes, w_sf, M, N, K, gp, s, st);
+}
+
 cudaError_t launch_linear(const LinearPlan &pl, const uint8_t *a_codes, const uint8_t *a_sf,
                           const float *a_gs, const uint8_t *w_codes, const uint8_t *w_sf,
                           const float *w_gs, int64_t M, int64_t N, int64_t K, int out_bf16,
@@ -1940,7 +2088,7 @@ cudaError_t launch_linear(const LinearPlan &pl, const uint8_t *a_codes, const ui
     }
     if (!pl.swap_ab && pl.splits == 1 && out_bf16 && N % 8 == 0 &&
         (reinterpret_cast<uintptr_t>(y) & 15u) == 0 && kUsePairKernel)
-        return launch_pair(pl, a_codes, a_sf, w_codes, w_sf, M, N, K, gp, s, st);
+        return launch_pair<false>(a_codes, a_sf, w_codes, w_sf, M, N, K, gp, s, st);
     switch (pl.bn) {
     case 8: e = launch_bn<8>(pl, ca, sa, cb, sb, K, gp, s, st); break;
     case 16: e = launch_bn<16>(pl, ca, sa, cb, sb, K, gp, s, st); break;

@@ -51,6 +51,13 @@ cudaError_t launch_wait_timeout_selftest(cudaStream_t s);
 // aligned) and the tensor scale (device fp32); ws as for launch_quantize.
 cudaError_t launch_quantize_e4m3(const void *x, int src_type, int64_t n, const float *static_amax,
                                  uint8_t *codes, float *scale_out, void *ws, cudaStream_t s);
+// Block-scaled GEMM whose epilogue applies act (0 identity, 1 tanh-form GELU) and quantizes
+// the [M x N] result to NVFP4 with the static amax: codes, swizzled scales, global scale.
+cudaError_t launch_linear_nvfp4_out(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gs,
+                                    const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,
+                                    int64_t M, int64_t N, int64_t K, int act,
+                                    const float *static_amax, uint8_t *y_codes, uint8_t *y_sf,
+                                    float *y_gs, cudaStream_t s, nvfp4_status *st);
 // FP8 E4M3 tensorwise W8A8 GEMM: Y = (a_scale * w_scale) * A . W^T, A [M x K], W [N x K].
 cudaError_t launch_linear_e4m3(const uint8_t *a, const float *a_scale, const uint8_t *w,
                                const float *w_scale, int64_t M, int64_t N, int64_t K, int out_bf16,

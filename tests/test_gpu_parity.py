@@ -563,3 +563,93 @@ def test_linear_e4m3_integer_exact():
     y = nv.linear_e4m3(a, w, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert np.array_equal(to_numpy_f64(y), O.gemm_e4m3(enc[ai], 1.0, enc[wi], 1.0))
+
+
+# ---------------------------------------------------------------------------------------
+# linear layer with an NVFP4 output (quantizing epilogue, static amax)
+# ---------------------------------------------------------------------------------------
+
+def _unit_scale_operand(rows, K, seed, sg):
+    """Random E2M1 codes with every block scale 1.0 (0x38) and a power-of-two global scale:
+    all partial sums of the product are exact in fp32. Oracle copy and device copy."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    codes = g.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    nb = K // 16
+    lin = np.full((rows, nb), 0x38, np.uint8)
+    swz = np.zeros(O.swizzled_bytes(rows, K), np.uint8)
+    for r in range(rows):
+        for b in range(nb):
+            swz[O.swizzled_offset(r, b, nb)] = 0x38
+    q = O.Quantized(codes, lin, swz, sg, rows, K)
+    d = nv.NVFP4Tensor(torch.from_numpy(codes).cuda(), torch.from_numpy(swz).cuda(), None,
+                       scalar_dev(sg), rows, K)
+    return q, d
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 320, 256), (129, 96, 512), (64, 64, 96),
+                                   (1100, 2080, 256), (4100, 544, 128)])
+def test_linear_nvfp4_out_exact_identity(M, N, K):
+    # exact products: the epilogue's codes, swizzled scales (padding included) and global
+    # scale equal the oracle's bit for bit
+    qa, da = _unit_scale_operand(M, K, 60 + M, 1.0)
+    qw, dw = _unit_scale_operand(N, K, 61 + N, 0.5)
+    amax = 0.7 * float(np.abs(O.gemm_sampled(qa, qw, np.arange(M).repeat(4),
+                                              np.tile([0, N // 3, N // 2, N - 1], M))).max())
+    out = nv.linear_nvfp4_out(da, dw, scalar_dev(amax), "identity")
+    torch.cuda.synchronize()
+    ref = O.linear_quantize_out(qa, qw, amax, O.ACT_NONE)
+    assert float(out.global_scale.cpu()[0]) == ref.sg
+    assert np.array_equal(out.codes.cpu().numpy(), ref.codes)
+    assert np.array_equal(out.scales_swz.cpu().numpy(), ref.scales_swz)
+
+
+def _e2m1_value(code):
+    mag = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0][code & 7]
+    return -mag if code & 8 else mag
+
+
+@pytest.mark.parametrize("act", ["identity", "gelu_tanh"])
+@pytest.mark.parametrize("M,N,K", [(500, 640, 1024), (4096, 3072, 3072)])
+def test_linear_nvfp4_out_within_error_bound(M, N, K, act):
+    # realistic operands: the fp32 accumulation (and the fast GELU) move the encoded values by
+    # a little, so a code may differ from an exact evaluation where a value sits that close to
+    # a rounding boundary. Each sampled block's scale must be the E4M3 rounding of some block
+    # maximum within the error bound of the exact one, and each code (with that scale) the E2M1
+    # rounding of some value within the bound of the exact value.
+    xa = W.to_bf16_bits(W.normal((M, K), 1.0, 62, M))
+    xw = W.to_bf16_bits(W.normal((N, K), 0.02, 63, N))
+    qa_h, qw_h = O.quantize(xa), O.quantize(xw)
+    qa, qw = gpu_quantize(xa), gpu_quantize(xw)
+    a_act = O.ACT_GELU_TANH if act == "gelu_tanh" else O.ACT_NONE
+    r = np.random.Generator(np.random.PCG64(64))
+    nb = N // 16
+    rows = np.concatenate([r.integers(0, M, 300), [0, M - 1]])
+    blks = np.concatenate([r.integers(0, nb, 300), [nb - 1, 0]])
+    ms = np.repeat(rows, 16)
+    ns = (blks[:, None] * 16 + np.arange(16)).ravel()
+    v = O.linear_act_sampled(qa_h, qw_h, a_act, ms, ns).reshape(-1, 16)
+    amax = 0.9 * float(np.abs(v).max())
+    out = nv.linear_nvfp4_out(qa, qw, scalar_dev(amax), act)
+    torch.cuda.synchronize()
+    codes = out.codes.cpu().numpy()
+    swz = out.scales_swz.cpu().numpy()
+    sg = np.float32(amax) / np.float32(2688.0)
+    assert float(out.global_scale.cpu()[0]) == sg
+    t = np.float64(np.float32(sg * np.float32(6.0)))
+    delta = 2e-5 * np.abs(v).max() + 2e-5 * np.abs(v)
+    for i, (row, b) in enumerate(zip(rows, blks)):
+        sb = int(swz[O.swizzled_offset(int(row), int(b), nb)])
+        lo = np.maximum(np.abs(v[i]) - delta[i], 0.0).max()
+        hi = (np.abs(v[i]) + delta[i]).max()
+        assert O.e4m3_encode(lo / t) <= sb <= O.e4m3_encode(hi / t), (row, b, sb)
+        got = codes[row, b * 8:(b + 1) * 8]
+        got = np.stack([got & 15, got >> 4], -1).ravel()
+        if sb == 0:
+            assert not got.any()
+            continue
+        rcp = np.float32(1.0) / (np.float32(O.e4m3_decode(sb)) * sg)
+        for j in range(16):
+            c_lo = O.e2m1_encode(float(np.float32(v[i, j] - delta[i, j]) * rcp))
+            c_hi = O.e2m1_encode(float(np.float32(v[i, j] + delta[i, j]) * rcp))
+            assert _e2m1_value(c_lo) <= _e2m1_value(int(got[j])) <= _e2m1_value(c_hi), \
+                (row, b, j, v[i, j], got[j])

@@ -642,57 +642,97 @@ template <int ACT> __device__ __forceinline__ float epi_act(float y)
     }
 }
 
-// One thread's 256-column accumulator row (TMEM address trow) of output row `row`, columns
-// col0..col0+255 -> NVFP4: v = act(acc * alpha); per 16-value block sb = E4M3(bmax / t)
-// (t = 6 sg, the quantizer's exact quotient), codes E2M1(v * s_rcp[sb]) with
-// s_rcp[c] = RN(1 / RN(E4M3(c) * sg)); sb = 0 gives zero codes. Codes go to the row's 32-byte
-// runs, the four scales of each 64-column atom row to the swizzled layout in one 4-byte store.
-// Rows past M and columns past N hold zeros (their operands are TMA zero fill), so the
-// swizzled padding of the last band and atom is written as zero scales.
+// 64 accumulator values (fp32 bits) of output row `row`, columns col..col+63 -> NVFP4:
+// v = act(acc * alpha); per 16-value block sb = E4M3(bmax / t) (t = 6 sg, the quantizer's exact
+// quotient), codes E2M1(v * s_rcp[sb]) with s_rcp[c] = RN(1 / RN(E4M3(c) * sg)); sb = 0 gives
+// zero codes. The codes go to the row's 32-byte run, the four scales (one 64-column atom row)
+// to the swizzled layout in one 4-byte store. Rows past M and columns past N hold zeros (their
+// operands are TMA zero fill), so the swizzled padding of the last band and atom is written as
+// zero scales.
 template <int ACT>
-__device__ __forceinline__ void quantize_out_row(const GemmParams &p, uint32_t trow, int64_t row,
-                                                 int64_t col0, float alpha, float t, float rt,
-                                                 const float *s_rcp)
+__device__ __forceinline__ void quantize_out_chunk(const GemmParams &p, const uint32_t (&v)[64],
+                                                   int64_t row, int64_t col, float alpha, float t,
+                                                   float rt, const float *s_rcp)
+{
+    uint32_t cw[8];
+    uint32_t sw = 0u;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        float y[16];
+        float bmax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            y[j] = epi_act<ACT>(__fmul_rn(__uint_as_float(v[16 * b + j]), alpha));
+            bmax = fmaxf(bmax, fabsf(y[j]));
+        }
+        const uint32_t sb = t > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
+        const float r = s_rcp[sb]; // sb = 0: every code is 0 (selected below)
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            y[j] = __fmul_rn(y[j], r);
+        const uint32_t lo = cvt_e2m1x8(y), hi = cvt_e2m1x8(y + 8);
+        cw[2 * b] = sb != 0u ? lo : 0u;
+        cw[2 * b + 1] = sb != 0u ? hi : 0u;
+        sw |= sb << (8 * b);
+    }
+    if (row < p.rows_a && col < p.rows_b) {
+        uint4 *dst = reinterpret_cast<uint4 *>(p.q_codes + row * (p.rows_b / 2) + col / 2);
+        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        if (col + 32 < p.rows_b)
+            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    }
+    const int64_t atom = col / 64;
+    if (row < p.q_rows_pad && atom < p.q_apb)
+        *reinterpret_cast<uint32_t *>(p.q_sf + ((row >> 7) * p.q_apb + atom) * 512 +
+                                      16 * (row & 31) + 4 * ((row & 127) >> 5)) = sw;
+}
+
+// One thread's 256-column accumulator row (TMEM address trow, row r of the CTA's 128) of
+// output row `row`, columns col0.. -> NVFP4. Columns 128..255 are first copied to the staging
+// tile as fp32 (column-major in 16-byte groups: a warp's stores and loads are conflict-free,
+// and each thread reads back only its own row), columns 0..127 are quantized from TMEM, then
+// the accumulator is handed back (release()) and the saved half is quantized while the next
+// tile's MMAs run.
+template <int ACT, typename Release>
+__device__ __forceinline__ void quantize_out_row(const GemmParams &p, uint32_t trow, uint32_t stg,
+                                                 int r, int64_t row, int64_t col0, float alpha,
+                                                 float t, float rt, const float *s_rcp,
+                                                 Release release)
 {
 #pragma unroll 1
-    for (int c0 = 0; c0 < 256; c0 += 64) {
+    for (int c0 = 128; c0 < 256; c0 += 64) {
         uint32_t v[64];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             tmem_ld_32x32b_x16(trow + c0 + 16 * i, v + 16 * i);
         tmem_ld_wait();
-        uint32_t cw[8];
-        uint32_t sw = 0u;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            float y[16];
-            float bmax = 0.0f;
+        for (int g = 0; g < 16; ++g)
+            sts128(stg + ((((c0 - 128) >> 2) + g) * 128 + r) * 16, v[4 * g], v[4 * g + 1],
+                   v[4 * g + 2], v[4 * g + 3]);
+    }
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 64) {
+        uint32_t v[64];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                y[j] = epi_act<ACT>(__fmul_rn(__uint_as_float(v[16 * b + j]), alpha));
-                bmax = fmaxf(bmax, fabsf(y[j]));
-            }
-            const uint32_t sb = t > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
-            const float r = s_rcp[sb]; // sb = 0: every code is 0 (selected below)
+        for (int i = 0; i < 4; ++i)
+            tmem_ld_32x32b_x16(trow + c0 + 16 * i, v + 16 * i);
+        tmem_ld_wait();
+        quantize_out_chunk<ACT>(p, v, row, col0 + c0, alpha, t, rt, s_rcp);
+    }
+    release();
+#pragma unroll 1
+    for (int c0 = 128; c0 < 256; c0 += 64) {
+        uint32_t v[64];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                y[j] = __fmul_rn(y[j], r);
-            const uint32_t lo = cvt_e2m1x8(y), hi = cvt_e2m1x8(y + 8);
-            cw[2 * b] = sb != 0u ? lo : 0u;
-            cw[2 * b + 1] = sb != 0u ? hi : 0u;
-            sw |= sb << (8 * b);
+        for (int g = 0; g < 16; ++g) {
+            const uint4 w = lds128(stg + ((((c0 - 128) >> 2) + g) * 128 + r) * 16);
+            v[4 * g] = w.x;
+            v[4 * g + 1] = w.y;
+            v[4 * g + 2] = w.z;
+            v[4 * g + 3] = w.w;
         }
-        const int64_t col = col0 + c0;
-        if (row < p.rows_a && col < p.rows_b) {
-            uint4 *dst = reinterpret_cast<uint4 *>(p.q_codes + row * (p.rows_b / 2) + col / 2);
-            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            if (col + 32 < p.rows_b)
-                dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-        }
-        const int64_t atom = col / 64;
-        if (row < p.q_rows_pad && atom < p.q_apb)
-            *reinterpret_cast<uint32_t *>(p.q_sf + ((row >> 7) * p.q_apb + atom) * 512 +
-                                          16 * (row & 31) + 4 * ((row & 127) >> 5)) = sw;
+        quantize_out_chunk<ACT>(p, v, row, col0 + c0, alpha, t, rt, s_rcp);
     }
 }
 
@@ -721,7 +761,8 @@ struct Pair {
     static constexpr int kOffStaging = kOffSfb + kStages * kSfbBytes;
     static constexpr int kStagingBytes = 128 * 256 * 2;
     static constexpr int kOffBar = kOffStaging + kStagingBytes;
-    static constexpr int kSmemBytes = kOffBar + 512;
+    static constexpr int kOffRcp = kOffBar + 512; // quantizing epilogue: 128 reciprocals
+    static constexpr int kSmemBytes = kOffRcp + 512;
     static constexpr uint32_t kTxAB = 2 * (kABytes + kBBytes); // both CTAs, on the leader
     static constexpr uint32_t kTxSf = kSfaBytes + kSfbBytes;   // own CTA
     static constexpr int kSfSlots = 4;
@@ -962,7 +1003,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
         uint32_t acc_phase = 0;
         float q_t = 0.0f, q_rt = 0.0f;
-        float *s_rcp = reinterpret_cast<float *>(smem + C::kOffStaging); // QOUT: no staging
+        float *s_rcp = reinterpret_cast<float *>(smem + C::kOffRcp);
         if constexpr (QOUT) {
             const float sg = __fdiv_rn(*p.q_amax, 2688.0f); // 6 * 448, as the quantizer
             q_t = __fmul_rn(sg, 6.0f);
@@ -983,16 +1024,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
             if constexpr (QOUT) {
+                auto release = [&]() {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive_remote(leader_acc_empty); // this CTA's accumulator is read
+                };
+                const uint32_t stg = smem_u32(smem + C::kOffStaging);
+                const int64_t row = ta * 256 + rank * 128 + q * 32 + lane;
                 if (p.act == 1)
-                    quantize_out_row<1>(p, trow, ta * 256 + rank * 128 + q * 32 + lane, tb * 256,
-                                        alpha, q_t, q_rt, s_rcp);
+                    quantize_out_row<1>(p, trow, stg, q * 32 + lane, row, tb * 256, alpha, q_t,
+                                        q_rt, s_rcp, release);
                 else
-                    quantize_out_row<0>(p, trow, ta * 256 + rank * 128 + q * 32 + lane, tb * 256,
-                                        alpha, q_t, q_rt, s_rcp);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive_remote(leader_acc_empty); // this CTA's accumulator is drained
+                    quantize_out_row<0>(p, trow, stg, q * 32 + lane, row, tb * 256, alpha, q_t,
+                                        q_rt, s_rcp, release);
                 acc_phase ^= 1;
                 continue;
             }

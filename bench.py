@@ -231,6 +231,23 @@ def extras(nv, W, dev, hbm, fp4_peak):
         avg, med = op_timer([lambda p=p, y=y: nv.linear(p[0], p[1], out=y) for p in sets])
         tf = 2.0 * 4096 * nn * kk / (avg * 1e-3) / 1e12
         rows[name] = {"us": avg * 1e3, "TFLOP/s": tf, "frac_fp4": tf / fp4_peak}
+        if name.startswith("gemm1"):
+            # the same GEMM writing GEMM2's NVFP4 operand from its epilogue (static amax of
+            # the activation), against GEMM1 in bf16 followed by the static-scale quantize
+            amax = torch.tensor([float(X2.float().abs().max())], device=dev)
+            outs = [nv.linear_nvfp4_out(p[0], p[1], amax) for p in sets]
+            for act in ("identity", "gelu_tanh"):
+                avg_f, _ = op_timer([lambda p=p, o=o: nv.linear_nvfp4_out(p[0], p[1], amax, act,
+                                                                           out=o)
+                                     for p, o in zip(sets, outs)])
+                rows[name][f"nvfp4_out_{act}_us"] = avg_f * 1e3
+            y_sets = [Y1] + [torch.empty_like(Y1) for _ in range(sets_for(Y1.numel() * 2) - 1)]
+            for yy in y_sets:
+                yy.copy_(X2[:, :12288] if X2.shape[1] >= 12288 else Y1)
+            avg_q, _ = op_timer([lambda yy=yy: nv.quantize(yy, static_amax=amax, out=qx2)
+                                 for yy in y_sets])
+            rows[name]["then_quantize_static_us"] = avg_q * 1e3
+            del outs, y_sets
         del sets
     del X2s, W1, W2, X1, X2, Y1, Y2, q1, q2, qx1, qx2
     torch.cuda.empty_cache()

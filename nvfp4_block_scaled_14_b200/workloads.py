@@ -136,3 +136,11 @@ def calib_batch(b: int, M=4096, K=3072) -> np.ndarray:
 
 def calib_weight(N=3072, K=3072) -> np.ndarray:
     return to_bf16_bits(normal((N, K), 0.02, 5, 1))
+
+
+def lowrank_factors(N=3072, K=3072, r=128, std=0.02, workload=2):
+    """BF16 low-rank branch of a linear layer (FP4 layers with BF16 rank-128 branches): down
+    D [r x K] and up U [N x r], both N(0, std^2), bf16 bits. With x ~ N(0, 1) and K = 3072
+    the branch's output has about a fifth of the FP4 product's standard deviation."""
+    return (to_bf16_bits(normal((r, K), std, workload, 7)),
+            to_bf16_bits(normal((N, r), std, workload, 8)))

@@ -13,6 +13,8 @@ Sources of each step (see the header of nvfp4_oracle.c for the full list):
   * "Qwen-Rapid-AIO FP8 -> NVFP4", "Recommended Model" -- p99.9 static input scales.
   * "Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization Details" / "Layer breakdown" -- FP8
     E4M3 tensorwise round-to-nearest layers (quantize_e4m3, gemm_e4m3).
+  * "Qwen Image 2.1: INT4 + FP4", "What I quantized" -- FP4 layers with BF16 rank-128
+    branches (lowrank_down, linear_lowrank).
 """
 import ctypes
 import os
@@ -78,6 +80,18 @@ def lib():
         L.ora_linear_quantize_out.restype = ctypes.c_int
         L.ora_quantize_e4m3.argtypes = [_vp, ctypes.c_int, _i64, _f32p, _u8p, _f32p]
         L.ora_quantize_e4m3.restype = ctypes.c_int
+        _u16p = ctypes.POINTER(ctypes.c_uint16)
+        L.ora_f64_to_bf16.argtypes = [ctypes.c_double]
+        L.ora_f64_to_bf16.restype = ctypes.c_uint16
+        L.ora_lowrank_down_bf16.argtypes = [_u16p, _u16p, _i64, _i64, _i64, _u16p]
+        L.ora_linear_lowrank_f64.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p,
+                                             ctypes.c_float, _u16p, _u16p, _u16p, _i64, _i64,
+                                             _i64, _i64, _f64p]
+        L.ora_linear_lowrank_f64.restype = ctypes.c_int
+        L.ora_linear_lowrank_f64_sampled.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p,
+                                                     ctypes.c_float, _u16p, _u16p, _u16p, _i64,
+                                                     _i64, _i64p, _i64p, _i64, _f64p]
+        L.ora_linear_lowrank_f64_sampled.restype = ctypes.c_int
         L.ora_gemm_e4m3_f64.argtypes = [_u8p, ctypes.c_float, _u8p, ctypes.c_float, _i64, _i64,
                                         _i64, _f64p]
         L.ora_gemm_e4m3_f64_sampled.argtypes = [_u8p, ctypes.c_float, _u8p, ctypes.c_float, _i64,
@@ -305,4 +319,64 @@ def gemm_e4m3_sampled(a_codes, sa, w_codes, sw, ms, ns) -> np.ndarray:
     out = np.zeros(len(ms), np.float64)
     lib().ora_gemm_e4m3_f64_sampled(_p(a, _u8p), sa, _p(w, _u8p), sw, a.shape[1], _p(ms, _i64p),
                                     _p(ns, _i64p), len(ms), _p(out, _f64p))
+    return out
+
+
+# ---- FP4 linear layer with a BF16 low-rank branch ------------------------------------------
+_u16 = ctypes.c_uint16
+
+
+def f64_to_bf16(v: float) -> int:
+    """Nearest bf16 (ties to even) of a double, in one rounding, as bits."""
+    return int(lib().ora_f64_to_bf16(float(v)))
+
+
+def _bits16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, "bf16 operands are passed as uint16 bit patterns"
+    return a
+
+
+def lowrank_down(x_bits, d_bits) -> np.ndarray:
+    """T = bf16(x . D^T) as uint16 bits [M x r]; x [M x K], D [r x K] bf16 bits."""
+    x, d = _bits16(x_bits), _bits16(d_bits)
+    (M, K), (r, K2) = x.shape, d.shape
+    assert K == K2
+    t = np.zeros((M, r), np.uint16)
+    u16p = ctypes.POINTER(_u16)
+    lib().ora_lowrank_down_bf16(_p(x, u16p), _p(d, u16p), M, K, r, _p(t, u16p))
+    return t
+
+
+def linear_lowrank(a: Quantized, w: Quantized, x_bits, d_bits, u_bits) -> np.ndarray:
+    """Y = dequant(A) . dequant(W)^T + bf16(x . D^T) . U^T in fp64, [M x N]."""
+    x, d, u = _bits16(x_bits), _bits16(d_bits), _bits16(u_bits)
+    M, N, K = a.rows, w.rows, a.cols
+    r = d.shape[0]
+    assert a.cols == w.cols == x.shape[1] == d.shape[1] and x.shape[0] == M
+    assert u.shape == (N, r)
+    out = np.zeros((M, N), np.float64)
+    u16p = ctypes.POINTER(_u16)
+    rc = lib().ora_linear_lowrank_f64(_p(a.codes, _u8p), _p(a.scales_lin, _u8p), a.sg,
+                                      _p(w.codes, _u8p), _p(w.scales_lin, _u8p), w.sg,
+                                      _p(x, u16p), _p(d, u16p), _p(u, u16p), M, N, K, r,
+                                      _p(out, _f64p))
+    if rc != 0:
+        raise MemoryError("oracle linear_lowrank")
+    return out
+
+
+def linear_lowrank_sampled(a: Quantized, w: Quantized, x_bits, d_bits, u_bits, ms, ns):
+    x, d, u = _bits16(x_bits), _bits16(d_bits), _bits16(u_bits)
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    out = np.zeros(len(ms), np.float64)
+    u16p = ctypes.POINTER(_u16)
+    rc = lib().ora_linear_lowrank_f64_sampled(_p(a.codes, _u8p), _p(a.scales_lin, _u8p), a.sg,
+                                              _p(w.codes, _u8p), _p(w.scales_lin, _u8p), w.sg,
+                                              _p(x, u16p), _p(d, u16p), _p(u, u16p), a.cols,
+                                              d.shape[0], _p(ms, _i64p), _p(ns, _i64p), len(ms),
+                                              _p(out, _f64p))
+    if rc != 0:
+        raise MemoryError("oracle linear_lowrank_sampled")
     return out

@@ -540,3 +540,108 @@ int ora_percentile_abs(const float *const *arrays, const int64_t *lengths, int c
     free(v);
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Linear layer with a BF16 low-rank branch                                                    */
+/* ------------------------------------------------------------------------------------------ */
+/* "Qwen Image 2.1: INT4 + FP4", section "What I quantized": the transformer's linear layers
+ * run in native FP4 on Blackwell together with BF16 rank-128 branches. Readings where the
+ * page is silent (each also listed in the design notes):
+ *   - a branch is a rank-r factorization U . D of a correction to the layer's weight, applied
+ *     to the layer's unquantized bf16 input x:
+ *       Y = dequant(A) . dequant(W)^T + (x . D^T) . U^T,  D [r x K] ("down"), U [N x r] ("up");
+ *   - the branch runs in BF16: its intermediate T = x . D^T is a bf16 tensor, each element the
+ *     exact sum rounded once to the nearest bf16 (ties to even);
+ *   - the up product T . U^T and its sum with the FP4 product are exact (fp64) here; the
+ *     tensor cores approximate them with fp32 accumulation. The caller rounds Y. */
+
+/* fp64 -> nearest bf16 (ties to even) in one rounding, as bits. Finite inputs whose rounded
+ * magnitude is below 2^128. bf16 keeps 8 significant bits; below 2^-126 the spacing stays
+ * 2^-133 (subnormals). */
+uint16_t ora_f64_to_bf16(double v)
+{
+    if (v == 0.0)
+        return signbit(v) ? 0x8000u : 0u;
+    int e;
+    frexp(v, &e); /* |v| in [2^(e-1), 2^e) */
+    if (e < -125)
+        e = -125;
+    double q = rint(ldexp(v, 8 - e)); /* round to a multiple of 2^(e-8); default mode: ties even */
+    float f = (float)ldexp(q, e - 8);  /* exact: at most 9 significant bits, in range */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+/* T [M x r] (bf16 bits) = RNE_bf16(sum_k x[m,k] * d[j,k]), x [M x K], d [r x K] bf16 bits. */
+static uint16_t lowrank_t(const uint16_t *x, const uint16_t *d, int64_t K, int64_t m, int64_t j)
+{
+    double s = 0.0;
+    for (int64_t k = 0; k < K; k++)
+        s += (double)ora_bf16_to_f32(x[m * K + k]) * (double)ora_bf16_to_f32(d[j * K + k]);
+    return ora_f64_to_bf16(s);
+}
+
+void ora_lowrank_down_bf16(const uint16_t *x, const uint16_t *d, int64_t M, int64_t K,
+                           int64_t r, uint16_t *t)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t j = 0; j < r; j++)
+            t[m * r + j] = lowrank_t(x, d, K, m, j);
+}
+
+/* One output: the FP4 product (gemm_one) plus sum_j T[m,j] * U[n,j], T from row t_row. */
+static double lowrank_one(const uint8_t *a_codes, const uint8_t *a_sc, float a_sg,
+                          const uint8_t *w_codes, const uint8_t *w_sc, float w_sg,
+                          const uint16_t *t_row, const uint16_t *u, int64_t m, int64_t n,
+                          int64_t K, int64_t r)
+{
+    double lr = 0.0;
+    for (int64_t j = 0; j < r; j++)
+        lr += (double)ora_bf16_to_f32(t_row[j]) * (double)ora_bf16_to_f32(u[n * r + j]);
+    return gemm_one(a_codes, a_sc, a_sg, w_codes, w_sc, w_sg, m, n, K) + lr;
+}
+
+/* Full output Y [M x N] in fp64. Returns 0, or -2 on allocation failure. */
+int ora_linear_lowrank_f64(const uint8_t *a_codes, const uint8_t *a_sc, float a_sg,
+                           const uint8_t *w_codes, const uint8_t *w_sc, float w_sg,
+                           const uint16_t *x, const uint16_t *d, const uint16_t *u, int64_t M,
+                           int64_t N, int64_t K, int64_t r, double *out)
+{
+    uint16_t *t = (uint16_t *)malloc((size_t)(M * r > 0 ? M * r : 1) * 2);
+    if (!t)
+        return -2;
+    ora_lowrank_down_bf16(x, d, M, K, r, t);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++)
+            out[m * N + n] = lowrank_one(a_codes, a_sc, a_sg, w_codes, w_sc, w_sg, t + m * r, u,
+                                         m, n, K, r);
+    free(t);
+    return 0;
+}
+
+/* Selected outputs (ms[i], ns[i]); the needed row of T is recomputed per output. */
+int ora_linear_lowrank_f64_sampled(const uint8_t *a_codes, const uint8_t *a_sc, float a_sg,
+                                   const uint8_t *w_codes, const uint8_t *w_sc, float w_sg,
+                                   const uint16_t *x, const uint16_t *d, const uint16_t *u,
+                                   int64_t K, int64_t r, const int64_t *ms, const int64_t *ns,
+                                   int64_t count, double *out)
+{
+    int err = 0;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; i++) {
+        uint16_t *t_row = (uint16_t *)malloc((size_t)(r > 0 ? r : 1) * 2);
+        if (!t_row) {
+            err = -2;
+            continue;
+        }
+        for (int64_t j = 0; j < r; j++)
+            t_row[j] = lowrank_t(x, d, K, ms[i], j);
+        out[i] = lowrank_one(a_codes, a_sc, a_sg, w_codes, w_sc, w_sg, t_row, u, ms[i], ns[i],
+                             K, r);
+        free(t_row);
+    }
+    return err;
+}

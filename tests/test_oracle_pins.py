@@ -481,3 +481,116 @@ def test_linear_act_sampled_is_activation_of_gemm(act):
     if act == O.ACT_GELU_TANH:
         y = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
     assert np.allclose(O.linear_act_sampled(a, w, act, ms, ns), y, rtol=1e-14, atol=0)
+
+
+# ---- FP4 linear layer with a BF16 low-rank branch ("What I quantized") ---------------------
+
+def _bf16(vals) -> np.ndarray:
+    """Exactly representable values -> bf16 bits (checked to be exact)."""
+    v = np.asarray(vals, np.float32)
+    bits = W.to_bf16_bits(v)
+    assert np.array_equal(W.bf16_bits_to_f32(bits), v), "value is not a bf16"
+    return bits
+
+
+def _lowrank_operands(M, N, K, seed):
+    g = np.random.default_rng(seed)
+    x = (g.standard_normal((M, K)) * 0.5).astype(np.float32)
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    xb = W.to_bf16_bits(x)
+    return O.quantize(W.bf16_bits_to_f32(xb)), O.quantize(w), xb
+
+
+def test_f64_to_bf16_rounds_once():
+    # values exact in fp32 round as torch's fp32 -> bf16 cast does (nearest, ties to even)
+    g = np.random.default_rng(7)
+    v = (g.standard_normal(4000) * np.exp2(g.integers(-40, 40, 4000))).astype(np.float32)
+    v = np.concatenate([v, np.float32([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2 ** -130,
+                                       3 * 2 ** -134, 0.0])])
+    ref = W.to_bf16_bits(v)
+    got = np.array([O.f64_to_bf16(float(t)) for t in v], np.uint16)
+    assert np.array_equal(got, ref)
+    # one rounding from fp64: 1 + 2^-8 + 2^-30 lies above the tie, so it rounds up, whereas
+    # rounding through fp32 first (to the tie 1 + 2^-8) would give 1.0
+    assert O.f64_to_bf16(1 + 2 ** -8 + 2 ** -30) == 0x3F81
+    assert O.f64_to_bf16(-(1 + 2 ** -8 + 2 ** -30)) == 0xBF81
+
+
+def test_lowrank_zero_up_is_the_fp4_gemm():
+    M, N, K, r = 12, 20, 64, 16
+    a, w, xb = _lowrank_operands(M, N, K, 1)
+    d = W.to_bf16_bits(np.random.default_rng(2).standard_normal((r, K)).astype(np.float32))
+    u = np.zeros((N, r), np.uint16)
+    assert np.array_equal(O.linear_lowrank(a, w, xb, d, u), O.gemm(a, w))
+
+
+def test_lowrank_one_hot_factors_select_entries():
+    # D[j] = e_{sel[j]} makes T = x[:, sel] exactly; U[n] = e_{pick[n]} * c[n] then makes the
+    # branch c[n] * x[m, sel[pick[n]]]. Swapping D / U, transposing either or dropping the
+    # branch gives other entries.
+    M, N, K, r = 9, 14, 96, 8
+    a, w, xb = _lowrank_operands(M, N, K, 3)
+    sel = np.array([5, 77, 0, 31, 95, 12, 64, 40])
+    pick = np.arange(N) % r
+    c = np.float32([1, -2, 0.5, 4, -0.25, 8, 1, -1, 2, 0.125, -4, 1, 0.5, 16])
+    d = np.zeros((r, K), np.float32)
+    d[np.arange(r), sel] = 1.0
+    u = np.zeros((N, r), np.float32)
+    u[np.arange(N), pick] = c
+    y = O.linear_lowrank(a, w, xb, _bf16(d), _bf16(u))
+    x = W.bf16_bits_to_f32(xb).astype(np.float64)
+    expect = O.gemm(a, w) + x[:, sel[pick]] * c.astype(np.float64)[None, :]
+    np.testing.assert_allclose(y, expect, rtol=0, atol=1e-12 * np.abs(expect).max())
+    # the branch against a library product on exact small integers: any summation order
+    g = np.random.default_rng(4)
+    xi = g.integers(-2, 3, (M, K)).astype(np.float32)
+    di = g.integers(-1, 2, (r, K)).astype(np.float32)
+    ui = g.integers(-3, 4, (N, r)).astype(np.float32)
+    xib = _bf16(xi)
+    zero_a = O.quantize(np.zeros((M, K), np.float32))
+    lr = O.linear_lowrank(zero_a, w, xib, _bf16(di), _bf16(ui))
+    t = torch.from_numpy(xi.astype(np.float64)) @ torch.from_numpy(di.astype(np.float64)).T
+    assert torch.all(t.abs() <= 256)  # |T| <= 2 * 96: integers this small are bf16s
+    ref = (t @ torch.from_numpy(ui.astype(np.float64)).T).numpy()
+    assert np.array_equal(lr, ref)
+
+
+def test_lowrank_intermediate_is_rounded_once_to_bf16():
+    # T = x . D^T with D = ones: each row's sum is set by hand; U = identity reads T back.
+    K, r = 32, 6
+    rows = [
+        ([1.0, 2.0 ** -9], 1.0),                             # below half an ulp: down
+        ([1.0, 2.0 ** -8], 1.0),                             # tie, even neighbour 1.0
+        ([1.0, 2.0 ** -7, 2.0 ** -8], 1.0 + 2.0 ** -6),      # tie, even neighbour 1 + 2^-6
+        ([1.0, 2.0 ** -8, 2.0 ** -30], 1.0 + 2.0 ** -7),     # just above the tie: up
+        ([-1.0, -(2.0 ** -7), -(2.0 ** -8)], -(1.0 + 2.0 ** -6)),
+        ([3.0, 2.0 ** -7], 3.0),                             # ulp of 3 is 2^-6
+    ]
+    x = np.zeros((len(rows), K), np.float32)
+    for i, (vals, _) in enumerate(rows):
+        x[i, :len(vals)] = vals
+    d = np.zeros((r, K), np.float32)
+    d[:, :] = 1.0
+    zero_a = O.quantize(np.zeros((len(rows), K), np.float32))
+    zero_w = O.quantize(np.zeros((r, K), np.float32))
+    u = np.eye(r, dtype=np.float32)
+    y = O.linear_lowrank(zero_a, zero_w, _bf16(x), _bf16(d), _bf16(u))
+    for i, (_, t) in enumerate(rows):
+        assert np.all(y[i] == t), (i, y[i], t)
+    t_bits = O.lowrank_down(_bf16(x), _bf16(d))
+    assert np.array_equal(W.bf16_bits_to_f32(t_bits)[:, 0], np.float32([t for _, t in rows]))
+
+
+def test_lowrank_sampled_matches_full_and_scales_linearly():
+    M, N, K, r = 10, 24, 128, 16
+    a, w, xb = _lowrank_operands(M, N, K, 5)
+    g = np.random.default_rng(6)
+    d = W.to_bf16_bits((g.standard_normal((r, K)) * 0.05).astype(np.float32))
+    u = W.to_bf16_bits((g.standard_normal((N, r)) * 0.05).astype(np.float32))
+    y = O.linear_lowrank(a, w, xb, d, u)
+    ms, ns = g.integers(0, M, 40), g.integers(0, N, 40)
+    assert np.array_equal(O.linear_lowrank_sampled(a, w, xb, d, u, ms, ns), y[ms, ns])
+    # doubling U doubles the branch exactly (a power-of-two scale of every term)
+    u2 = W.to_bf16_bits(W.bf16_bits_to_f32(u) * 2)
+    base = O.gemm(a, w)
+    assert np.array_equal(O.linear_lowrank(a, w, xb, d, u2) - base, 2 * (y - base))

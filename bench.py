@@ -37,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 M, N, K = 4096, 3072, 3072
+LOWRANK_R = 128  # rank of the BF16 low-rank branch (FP4 layers with rank-128 BF16 branches)
 FLOPS = 2.0 * M * N * K
 METRIC = "NVFP4 GEMM TFLOPS & quantize GB/s at 1 B200 (fraction of FP4/HBM peak)"
 WORKLOAD = "attn_proj_fp8w_m4096_n3072_k3072"
@@ -341,6 +342,31 @@ def extras(nv, W, dev, hbm, fp4_peak):
         del xs, a8s, w8s, w8, y
         torch.cuda.empty_cache()
     rows["fp8_e4m3_w8a8"] = fp8
+
+    # --- FP4 linear with a BF16 rank-128 branch on the attention projection (4096x3072x3072):
+    #     the down projection of the bf16 input plus the GEMM with the low-rank k-tiles,
+    #     against the plain FP4 linear on the same operands
+    wl = W.attn_proj()
+    xb = t(wl.X_bf16)
+    d_bits, u_bits = W.lowrank_factors(N=N, K=K, r=LOWRANK_R)
+    dd, uu = t(d_bits), t(u_bits)
+    qw0 = nv.quantize_fp8(torch.from_numpy(wl.W_e4m3).to(dev),
+                          torch.tensor([wl.w_scale], dtype=torch.float32, device=dev))
+    nset = sets_for(M * K * 2 + N * K // 2)
+    xs = [xb.clone() for _ in range(nset)]
+    qxs = [nv.quantize(x) for x in xs]
+    qws = [clone_q(qw0) for _ in range(nset)]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    avg_p, _ = op_timer([lambda a=a, w=w: nv.linear(a, w, out=y) for a, w in zip(qxs, qws)])
+    avg_l, _ = op_timer([lambda a=a, w=w, x=x: nv.linear_lowrank(a, w, x, dd, uu, out=y)
+                         for a, w, x in zip(qxs, qws, xs)])
+    flops = 2.0 * M * N * K + 2.0 * M * K * LOWRANK_R + 2.0 * M * N * LOWRANK_R
+    rows[f"lowrank_r{LOWRANK_R}_m{M}_n{N}_k{K}"] = {
+        "linear_us": avg_p * 1e3, "linear_lowrank_us": avg_l * 1e3,
+        "branch_extra_us": (avg_l - avg_p) * 1e3,
+        "TFLOP/s": flops / (avg_l * 1e-3) / 1e12}
+    del xs, qxs, qws, y, xb, dd, uu, qw0
+    torch.cuda.empty_cache()
     return rows
 
 

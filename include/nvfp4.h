@@ -59,7 +59,8 @@ typedef enum {
     NVFP4_OP_CALIB_BF16 = 2, /* m, n, k ignored */
     NVFP4_OP_CALIB_F32 = 3,  /* m, n, k ignored */
     NVFP4_OP_LINEAR_DYNAMIC = 4, /* m = M, n = N, k = K of nvfp4_linear_dynamic */
-    NVFP4_OP_QUANTIZE_E4M3 = 5   /* nvfp4_quantize_e4m3 (m, n, k ignored) */
+    NVFP4_OP_QUANTIZE_E4M3 = 5,  /* nvfp4_quantize_e4m3 (m, n, k ignored) */
+    NVFP4_OP_LINEAR_LOWRANK = 6  /* nvfp4_linear_lowrank: m = M, n = rank (k ignored) */
 } nvfp4_op;
 
 /* Human-readable name of a status. Never NULL. */
@@ -279,6 +280,32 @@ nvfp4_status nvfp4_linear_nvfp4_out(const uint8_t *a_codes, const uint8_t *a_sca
                                     int64_t N, int64_t K, int act, const float *static_amax,
                                     uint8_t *y_codes, uint8_t *y_scales_swz, float *y_gs,
                                     cudaStream_t stream);
+
+/*
+ * Linear layer with a BF16 low-rank branch ("Qwen Image 2.1: INT4 + FP4", section "What I
+ * quantized": the transformer's layers run in native FP4 on Blackwell with BF16 rank-128
+ * branches):
+ *   Y = dequant(A) . dequant(W)^T + (x . D^T) . U^T
+ * A, W, a_gs, w_gs: the FP4 operands as in nvfp4_linear (A is normally nvfp4_quantize(x)).
+ * x: M x K bf16, the layer's unquantized input. lr_down D: rank x K bf16; lr_up U: N x rank
+ * bf16; all row-major, 16-byte aligned. y: M x N bf16.
+ * How it is computed: one kernel forms T' = bf16((x . D^T) / alpha) with fp32 tensor-core
+ * accumulation, alpha = sgA * sgW in fp32 (1 when that product is 0), into ws; the FP4 GEMM
+ * then adds T' . U^T (bf16 tensor-core MMAs) into the same fp32 accumulator as the FP4
+ * product, and its epilogue multiplies by alpha and rounds to bf16. Against the branch taken
+ * exactly with its intermediate rounded once to bf16 (bf16(x . D^T) . U^T), each term
+ * T[m,j] U[n,j] can differ by up to 2^-7 |T[m,j] U[n,j]| (two bf16 roundings instead of one),
+ * on top of nvfp4_linear's fp32 accumulation. |x . D^T| / alpha must stay below the bf16
+ * range (3.4e38).
+ * K: multiple of 32, > 0. N: multiple of 8. rank: multiple of 16, 16..256.
+ * ws: nvfp4_workspace_bytes(NVFP4_OP_LINEAR_LOWRANK, M, rank, 0) bytes (M * rank * 2).
+ */
+nvfp4_status nvfp4_linear_lowrank(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                                  const float *a_gs, const uint8_t *w_codes,
+                                  const uint8_t *w_scales_swz, const float *w_gs,
+                                  const void *x_bf16, const void *lr_down, const void *lr_up,
+                                  int64_t M, int64_t N, int64_t K, int64_t rank, void *y,
+                                  void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
  * FP8 E4M3 tensorwise quantization ("Qwen3-VL-8B-Instruct-heretic-NVFP4", "Quantization

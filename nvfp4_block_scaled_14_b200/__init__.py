@@ -11,6 +11,7 @@ device memory and the current stream, nothing else.
     q_s = quantize(x_bf16, static_amax=pct)
     e_w = quantize_e4m3(w_bf16)               # FP8 E4M3 tensorwise (embed / lm_head layers)
     y8 = linear_e4m3(quantize_e4m3(x_bf16), e_w)
+    y_lr = linear_lowrank(q_x, q_w, x_bf16, down, up)  # FP4 + BF16 rank-r branch
 
 The C entry points are also available under their own names (``nvfp4_quantize`` ...).
 """
@@ -24,7 +25,7 @@ from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_LINEAR_DEFAULT, NVFP4_LINEAR_RES
                    NVFP4Error, check, load)
 
 __all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "quantize_batch", "dequantize", "linear",
-           "linear_dynamic", "linear_nvfp4_out", "E4M3Tensor", "quantize_e4m3", "linear_e4m3",
+           "linear_dynamic", "linear_nvfp4_out", "linear_lowrank", "E4M3Tensor", "quantize_e4m3", "linear_e4m3",
            "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
 
 
@@ -261,6 +262,36 @@ def linear_nvfp4_out(a: NVFP4Tensor, w: NVFP4Tensor, static_amax: torch.Tensor,
                                        _ptr(out.scales_swz), _ptr(out.global_scale),
                                        _stream(dev))
     check(st, "nvfp4_linear_nvfp4_out")
+    return out
+
+
+def linear_lowrank(a: NVFP4Tensor, w: NVFP4Tensor, x: torch.Tensor, down: torch.Tensor,
+                   up: torch.Tensor, out: torch.Tensor = None) -> torch.Tensor:
+    """Y = dequant(a) . dequant(w)^T + (x . down^T) . up^T, bf16 [a.rows x w.rows].
+
+    x: the layer's bf16 input [M, K] (a is its NVFP4 quantization); down: bf16 [rank, K];
+    up: bf16 [N, rank]. The branch's intermediate is kept in bf16 (divided by the FP4 product's
+    global scales, so that both parts share one fp32 tensor-core accumulator)."""
+    if a.cols != w.cols:
+        raise ValueError("K mismatch")
+    M, N, K = a.rows, w.rows, a.cols
+    if x.dtype != torch.bfloat16 or down.dtype != torch.bfloat16 or up.dtype != torch.bfloat16:
+        raise TypeError("x, down and up must be bfloat16")
+    rank = down.shape[0]
+    if tuple(x.shape) != (M, K) or tuple(down.shape) != (rank, K) or tuple(up.shape) != (N, rank):
+        raise ValueError("shape mismatch: x [M, K], down [rank, K], up [N, rank]")
+    x, down, up = x.contiguous(), down.contiguous(), up.contiguous()
+    dev = a.codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    L = load()
+    ws_bytes = L.nvfp4_workspace_bytes(_lib.NVFP4_OP_LINEAR_LOWRANK, M, rank, 0)
+    ws = _workspace(dev, ws_bytes)
+    st = L.nvfp4_linear_lowrank(_ptr(a.codes), _ptr(a.scales_swz), _ptr(a.global_scale),
+                                _ptr(w.codes), _ptr(w.scales_swz), _ptr(w.global_scale),
+                                _ptr(x), _ptr(down), _ptr(up), M, N, K, rank, _ptr(out), _ptr(ws),
+                                ws_bytes, _stream(dev))
+    check(st, "nvfp4_linear_lowrank")
     return out
 
 

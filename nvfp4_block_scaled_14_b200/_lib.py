@@ -32,6 +32,7 @@ NVFP4_OP_CALIB_BF16 = 2
 NVFP4_OP_CALIB_F32 = 3
 NVFP4_OP_LINEAR_DYNAMIC = 4
 NVFP4_OP_QUANTIZE_E4M3 = 5
+NVFP4_OP_LINEAR_LOWRANK = 6
 NVFP4_ACT_IDENTITY = 0
 NVFP4_ACT_GELU_TANH = 1
 
@@ -81,6 +82,8 @@ _SIGNATURES = {
     "nvfp4_linear_nvfp4_out": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp,
                                 _vp, _vp, _vp], _int),
     "nvfp4_quantize_e4m3": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp], _int),
+    "nvfp4_linear_lowrank": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                              _vp, _vp, _sz, _vp], _int),
     "nvfp4_linear_e4m3": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp], _int),
     "nvfp4_selftest_wait_timeout": ([_vp], _int),
     "nvfp4_sync_status": ([_vp], _int),

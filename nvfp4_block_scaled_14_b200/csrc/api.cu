@@ -233,6 +233,10 @@ size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
             return 0;
         return linear_dynamic_ws(m, n, k).total;
     case NVFP4_OP_QUANTIZE_E4M3: return quantize_ws_bytes();
+    case NVFP4_OP_LINEAR_LOWRANK:
+        if (m <= 0 || n <= 0 || m >= kMaxDim || n > 256)
+            return 0;
+        return (size_t)m * (size_t)n * 2;
     case NVFP4_OP_CALIB_BF16: return calib_workspace_bytes(1);
     case NVFP4_OP_CALIB_F32: return calib_workspace_bytes(0);
     }
@@ -452,6 +456,39 @@ nvfp4_status nvfp4_linear_nvfp4_out(const uint8_t *a_codes, const uint8_t *a_sca
     const cudaError_t e =
         launch_linear_nvfp4_out(a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs, M, N, K,
                                 act, static_amax, y_codes, y_scales_swz, y_gs, stream, &st);
+    return st != NVFP4_OK ? st : map_cuda(e);
+}
+
+nvfp4_status nvfp4_linear_lowrank(const uint8_t *a_codes, const uint8_t *a_scales_swz,
+                                  const float *a_gs, const uint8_t *w_codes,
+                                  const uint8_t *w_scales_swz, const float *w_gs,
+                                  const void *x_bf16, const void *lr_down, const void *lr_up,
+                                  int64_t M, int64_t N, int64_t K, int64_t rank, void *y,
+                                  void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    nvfp4_status st;
+    if ((st = check_matrix(M, K)) != NVFP4_OK || (st = check_matrix(N, K)) != NVFP4_OK)
+        return st;
+    if (K == 0 || N % 8 != 0 || rank < 16 || rank > 256 || rank % 16 != 0)
+        return NVFP4_ERR_SHAPE;
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (!a_codes || !a_scales_swz || !a_gs || !w_codes || !w_scales_swz || !w_gs || !x_bf16 ||
+        !lr_down || !lr_up || !y)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_scales_swz) || !aligned16(w_codes) ||
+        !aligned16(w_scales_swz) || !aligned16(x_bf16) || !aligned16(lr_down) ||
+        !aligned16(lr_up) || !aligned16(y) || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(a_gs) & 3u) || (reinterpret_cast<uintptr_t>(w_gs) & 3u))
+        return NVFP4_ERR_ALIGNMENT;
+    if (!ws || ws_bytes < (size_t)M * (size_t)rank * 2)
+        return NVFP4_ERR_WORKSPACE;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    st = NVFP4_OK;
+    const cudaError_t e =
+        launch_linear_lowrank(a_codes, a_scales_swz, a_gs, w_codes, w_scales_swz, w_gs, x_bf16,
+                              lr_down, lr_up, M, N, K, (int)rank, y, ws, stream, &st);
     return st != NVFP4_OK ? st : map_cuda(e);
 }
 

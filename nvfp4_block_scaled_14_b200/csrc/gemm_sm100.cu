@@ -115,6 +115,9 @@ struct GemmParams {
     const float *q_amax;
     int act, q_apb;
     int64_t q_rows_pad;
+    // low-rank branch of the pair kernel (nvfp4_linear_lowrank): 64-wide k-tiles of bf16
+    // T' [rows_a x r] and U [rows_b x r] after the FP4 k-tiles of each tile (0 = none)
+    int lr_kt;
 };
 
 __device__ __forceinline__ void set_timeout(int *status)
@@ -771,17 +774,36 @@ struct Pair {
     static constexpr int kTmemCols = 512;
     static constexpr uint32_t kIdesc =
         (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+    // low-rank k-tiles: kind::f16 with D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9 and
+    // 10-12 = 1), K-major, M256 x N256; a 64-wide bf16 k-tile fills the same 128-byte smem
+    // rows as a 256-wide FP4 k-tile, so it reuses the stage buffers and their byte counts
+    static constexpr uint32_t kIdescLr = (1u << 4) | (1u << 7) | (1u << 10) |
+                                         ((uint32_t)(256 >> 3) << 17) |
+                                         ((uint32_t)(256 >> 4) << 24);
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kSfCol + kSfSlots * kSlotCols <= kTmemCols, "TMEM budget");
 };
 
-template <bool QOUT>
+// 2-SM bf16 MMA issued by the leader CTA (the low-rank k-tiles): D (+)= A x B^T, fp32.
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+template <bool QOUT, bool LR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSFA,
                            const __grid_constant__ CUtensorMap tmSFB,
-                           const __grid_constant__ CUtensorMap tmY, const GemmParams p)
+                           const __grid_constant__ CUtensorMap tmY,
+                           const __grid_constant__ CUtensorMap tmT,
+                           const __grid_constant__ CUtensorMap tmU, const GemmParams p)
 {
     using C = Pair;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -831,6 +853,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     const int64_t tiles_ab = p.tiles_a * p.tiles_b; // tiles_a counts 256-row pairs
     const int64_t cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int kt_tile = p.kt_total + (LR ? p.lr_kt : 0); // stage uses per tile
 
     if (warp == 0) {
         // ------------------------------- TMA producer (both CTAs) ---------------------
@@ -839,6 +862,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmB);
             tma_prefetch_desc(&tmSFA);
             tma_prefetch_desc(&tmSFB);
+            if constexpr (LR) {
+                tma_prefetch_desc(&tmT);
+                tma_prefetch_desc(&tmU);
+            }
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -846,7 +873,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int64_t ta = u % p.tiles_a, tb = u / p.tiles_a;
                 const int arow = (int)(ta * 256 + rank * 128);
                 const int brow = (int)(tb * 256 + rank * 128);
-                for (int kt = 0; kt < p.kt_total; ++kt) {
+                for (int kt = 0; kt < kt_tile; ++kt) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimit)) {
                         set_timeout(p.status);
                         ok = false;
@@ -855,6 +882,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t leader_full = mapa_shared(smem_u32(&full_bar[stage]), 0);
                     if (leader)
                         mbar_arrive_expect_tx(&full_bar[stage], C::kTxAB);
+                    if (LR && kt >= p.kt_total) {
+                        // low-rank k-tile: 64 ranks of T' (A side) and U (B side), 16 KB each;
+                        // no scales, and sfdata[stage] is left alone: its phases count the
+                        // stage's FP4 uses only (the feeders track them per stage)
+                        const int x = (kt - p.kt_total) * 64;
+                        tma_load_2d_pair(smem + stage * C::kABytes, &tmT, leader_full, x, arow);
+                        tma_load_2d_pair(smem + C::kOffB + stage * C::kBBytes, &tmU, leader_full,
+                                         x, brow);
+                        if (++stage == C::kStages) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
+                        continue;
+                    }
                     mbar_arrive_expect_tx(&sfdata[stage], C::kTxSf);
                     tma_load_2d_pair(smem + stage * C::kABytes, &tmA, leader_full, kt * 128, arow);
                     tma_load_2d_pair(smem + C::kOffB + stage * C::kBBytes, &tmB, leader_full,
@@ -876,10 +917,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t leader_sf_full0 = mapa_shared(smem_u32(&sf_full[0]), 0);
         int stage = 0, slot = 0;
         uint32_t phase = 0, sphase = 0;
+        // LR: per-stage parity of sfdata, which completes a phase per FP4 use of the stage
+        // only. The next FP4 use of a stage is armed after the MMA warp has consumed this one
+        // (which needs these warps' slot), so sfdata never runs two phases ahead of them.
+        uint32_t sfbits = 0;
         bool ok = true;
         for (int64_t u = cluster_id; u < tiles_ab && ok; u += nclusters) {
-            for (int kt = 0; kt < p.kt_total; ++kt) {
-                if (!mbar_wait(&sfdata[stage], phase, kWaitLimit) ||
+            for (int kt = 0; kt < kt_tile; ++kt) {
+                if (LR && kt >= p.kt_total) { // low-rank k-tile: no scales to feed
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                    continue;
+                }
+                const uint32_t sfpar = LR ? ((sfbits >> stage) & 1u) : phase;
+                if (LR)
+                    sfbits ^= 1u << stage;
+                if (!mbar_wait(&sfdata[stage], sfpar, kWaitLimit) ||
                     !mbar_wait(&sf_empty[slot], sphase ^ 1, kWaitLimit)) {
                     if (lane == 0)
                         set_timeout(p.status);
@@ -947,7 +1002,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int kt = 0; kt < p.kt_total; ++kt) {
+                for (int kt = 0; kt < kt_tile; ++kt) {
+                    if (LR && kt >= p.kt_total) {
+                        if (!mbar_wait(&full_bar[stage], phase, kWaitLimit)) {
+                            if (lane == 0)
+                                set_timeout(p.status);
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (lane == 0) {
+                            const uint64_t adesc = smem_desc(smem_u32(smem + stage * C::kABytes),
+                                                             16, 1024, kLayoutSwizzle128B);
+                            const uint64_t bdesc =
+                                smem_desc(smem_u32(smem + C::kOffB + stage * C::kBBytes), 16,
+                                          1024, kLayoutSwizzle128B);
+#pragma unroll
+                            for (int kb = 0; kb < 4; ++kb) // K16 bf16 = 32 bytes per MMA
+                                tc_mma_bf16_pair(tmem, adesc + (uint64_t)(2 * kb),
+                                                 bdesc + (uint64_t)(2 * kb), C::kIdescLr,
+                                                 (kt > 0 || kb > 0) ? 1u : 0u);
+                            tc_commit_pair_mc(&empty_bar[stage], 0x3);
+                        }
+                        __syncwarp();
+                        if (++stage == C::kStages) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
+                        continue;
+                    }
                     if (!mbar_wait(&full_bar[stage], phase, kWaitLimit) ||
                         !mbar_wait(&sf_full[slot], sphase, kWaitLimit)) {
                         if (lane == 0)
@@ -999,7 +1082,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------- epilogue (both CTAs, warps 2..5) -------------
         const int q = warp & 3;
-        const float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
+        float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
+        if (LR && alpha == 0.0f)
+            alpha = 1.0f; // the FP4 product is zero; T' was not divided either
         const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
         uint32_t acc_phase = 0;
         float q_t = 0.0f, q_rt = 0.0f;
@@ -1840,25 +1925,32 @@ cudaError_t launch_bn(const LinearPlan &pl, const uint8_t *a_codes, const uint8_
     return cudaGetLastError();
 }
 
-template <bool QOUT>
+// LR: lr_t (T' [M x lr_rank] bf16) and lr_u (U [N x lr_rank] bf16) feed the low-rank k-tiles.
+template <bool QOUT, bool LR = false>
 cudaError_t launch_pair(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *w_codes,
                         const uint8_t *w_sf, int64_t M, int64_t N, int64_t K, GemmParams gp,
-                        cudaStream_t s, nvfp4_status *st)
+                        cudaStream_t s, nvfp4_status *st, const void *lr_t = nullptr,
+                        const void *lr_u = nullptr, int lr_rank = 0)
 {
-    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY, tmT, tmU;
     std::memset(&tmY, 0, sizeof(tmY));
+    std::memset(&tmT, 0, sizeof(tmT));
+    std::memset(&tmU, 0, sizeof(tmU));
     if (!encode_fn() || !make_codes_map(&tmA, a_codes, M, K, 128) ||
         !make_codes_map(&tmB, w_codes, N, K, 128) || !make_sf_map(&tmSFA, a_sf, M, K, 1) ||
-        !make_sf_map(&tmSFB, w_sf, N, K, 2) || (!QOUT && !make_out_map(&tmY, gp.y, M, N))) {
+        !make_sf_map(&tmSFB, w_sf, N, K, 2) || (!QOUT && !make_out_map(&tmY, gp.y, M, N)) ||
+        (LR && (!make_bf16_kmajor_map(&tmT, lr_t, M, lr_rank, 128) ||
+                !make_bf16_kmajor_map(&tmU, lr_u, N, lr_rank, 128)))) {
         *st = NVFP4_ERR_CUDA;
         return cudaErrorInvalidValue;
     }
+    gp.lr_kt = LR ? (lr_rank + 63) / 64 : 0;
     static std::once_flag flags[64];
     int dev = 0;
     cudaGetDevice(&dev);
     cudaError_t attr_err = cudaSuccess;
     std::call_once(flags[dev & 63], [&]() {
-        attr_err = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QOUT>,
+        attr_err = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QOUT, LR>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         Pair::kSmemBytes);
     });
@@ -1872,8 +1964,8 @@ cudaError_t launch_pair(const uint8_t *a_codes, const uint8_t *a_sf, const uint8
         clusters = gp.units;
     if (clusters < 1)
         clusters = 1;
-    nvfp4_gemm_pair_kernel<QOUT><<<(unsigned)(2 * clusters), kThreads, Pair::kSmemBytes, s>>>(
-        tmA, tmB, tmSFA, tmSFB, tmY, gp);
+    nvfp4_gemm_pair_kernel<QOUT, LR><<<(unsigned)(2 * clusters), kThreads, Pair::kSmemBytes,
+                                       s>>>(tmA, tmB, tmSFA, tmSFB, tmY, tmT, tmU, gp);
     return cudaGetLastError();
 }
 
@@ -2195,6 +2287,33 @@ bool plan_linear_xq(int64_t M, int64_t N, int64_t K, LinearPlan *out)
     p.ws_bytes = 0;
     *out = p;
     return true;
+}
+
+// Linear layer with a BF16 low-rank branch: T' = bf16(x . D^T / alpha) into t_ws (the down
+// kernel), then the pair GEMM with the low-rank k-tiles appended to every tile. bf16 output.
+cudaError_t launch_linear_lowrank(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gs,
+                                  const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,
+                                  const void *x, const void *lr_down, const void *lr_up,
+                                  int64_t M, int64_t N, int64_t K, int rank, void *y, void *t_ws,
+                                  cudaStream_t s, nvfp4_status *st)
+{
+    cudaError_t e = launch_lowrank_down(x, lr_down, M, K, rank, a_gs, w_gs, t_ws, s, st);
+    if (e != cudaSuccess || *st != NVFP4_OK)
+        return e;
+    GemmParams gp{};
+    gp.rows_a = M;
+    gp.rows_b = N;
+    gp.kt_total = (int)((K + 255) / 256);
+    gp.kt_per_split = gp.kt_total;
+    gp.splits = 1;
+    gp.a_gs = a_gs;
+    gp.w_gs = w_gs;
+    gp.y = y;
+    gp.ldy = N;
+    gp.out_bf16 = 1;
+    gp.status = device_status_ptr();
+    return launch_pair<false, true>(a_codes, a_sf, w_codes, w_sf, M, N, K, gp, s, st, t_ws, lr_up,
+                                    rank);
 }
 
 cudaError_t launch_linear_xq(const LinearPlan &pl, const void *x, int x_bf16,

@@ -1,6 +1,7 @@
 // nvfp4_internal.cuh -- declarations shared by the library's translation units.
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -107,5 +108,22 @@ cudaError_t launch_linear_xq(const LinearPlan &pl, const void *x, int x_bf16,
                              const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,
                              int64_t M, int64_t N, int64_t K, int out_bf16, void *y,
                              float *x_gs_out, unsigned flags, cudaStream_t s, nvfp4_status *st);
+
+// ---- lowrank_sm100.cu ----------------------------------------------------------------
+// bf16 [rows x cols] row-major tensor map: box 64 columns x box_rows rows, 128B swizzle.
+bool make_bf16_kmajor_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                          int box_rows);
+// T' [M x r] = bf16((x . D^T) / alpha), alpha = sgA * sgW (1 if that is 0); x [M x K] and
+// D [r x K] bf16, r a multiple of 16 in 16..256, K > 0.
+cudaError_t launch_lowrank_down(const void *x, const void *d, int64_t M, int64_t K, int r,
+                                const float *a_gs, const float *w_gs, void *t, cudaStream_t s,
+                                nvfp4_status *st);
+// Y = FP4 product + T . U^T (bf16 out): launch_lowrank_down into t_ws (M x rank bf16), then the
+// pair GEMM with the low-rank k-tiles.
+cudaError_t launch_linear_lowrank(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gs,
+                                  const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,
+                                  const void *x, const void *lr_down, const void *lr_up,
+                                  int64_t M, int64_t N, int64_t K, int rank, void *y, void *t_ws,
+                                  cudaStream_t s, nvfp4_status *st);
 
 } // namespace nvfp4

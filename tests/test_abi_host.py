@@ -124,3 +124,22 @@ def test_product_path_never_imports_oracle():
                 text = open(os.path.join(root, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
                 assert "nvfp4_oracle" not in text, f
+
+
+def test_linear_lowrank_checks(lib):
+    lr = lib.nvfp4_linear_lowrank
+    ops = [FAKE] * 9  # a codes / scales / gs, w codes / scales / gs, x, down, up
+    ws = 256 * 128 * 2
+    assert lr(*ops, 256, 256, 48, 128, FAKE, FAKE, ws, None) == L.NVFP4_ERR_SHAPE  # K % 32
+    assert lr(*ops, 256, 256, 0, 128, FAKE, FAKE, ws, None) == L.NVFP4_ERR_SHAPE   # K == 0
+    assert lr(*ops, 256, 260, 64, 128, FAKE, FAKE, ws, None) == L.NVFP4_ERR_SHAPE  # N % 8
+    assert lr(*ops, 256, 256, 64, 24, FAKE, FAKE, ws, None) == L.NVFP4_ERR_SHAPE   # rank % 16
+    assert lr(*ops, 256, 256, 64, 272, FAKE, FAKE, ws, None) == L.NVFP4_ERR_SHAPE  # rank > 256
+    assert lr(*ops, 0, 256, 64, 128, None, None, 0, None) == L.NVFP4_OK            # empty
+    assert lr(*([FAKE] * 6), None, FAKE, FAKE, 256, 256, 64, 128, FAKE, FAKE, ws, None) == \
+        L.NVFP4_ERR_INVALID_ARG
+    assert lr(*ops, 256, 256, 64, 128, FAKE + 8, FAKE, ws, None) == L.NVFP4_ERR_ALIGNMENT
+    assert lr(*ops, 256, 256, 64, 128, FAKE, FAKE, ws - 2, None) == L.NVFP4_ERR_WORKSPACE
+    assert lr(*ops, 256, 256, 64, 128, FAKE, None, 0, None) == L.NVFP4_ERR_WORKSPACE
+    assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_LINEAR_LOWRANK, 4096, 128, 0) == 4096 * 128 * 2
+    assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_LINEAR_LOWRANK, 4096, 512, 0) == 0

@@ -653,3 +653,116 @@ def test_linear_nvfp4_out_within_error_bound(M, N, K, act):
             c_hi = O.e2m1_encode(float(np.float32(v[i, j] + delta[i, j]) * rcp))
             assert _e2m1_value(c_lo) <= _e2m1_value(int(got[j])) <= _e2m1_value(c_hi), \
                 (row, b, j, v[i, j], got[j])
+
+
+# ---------------------------------------------------------------------------------------
+# linear layer with a BF16 low-rank branch
+# ---------------------------------------------------------------------------------------
+
+def _lowrank_case(M, N, K, r, seed, w_std=0.02, lr_std=0.02):
+    xb = W.to_bf16_bits(W.normal((M, K), 1.0, 70, seed))
+    wb = W.to_bf16_bits(W.normal((N, K), w_std, 71, seed)) if w_std else \
+        np.zeros((N, K), np.uint16)
+    d = W.to_bf16_bits(W.normal((r, K), lr_std, 72, seed))
+    u = W.to_bf16_bits(W.normal((N, r), lr_std, 73, seed))
+    return xb, wb, d, u
+
+
+def _lowrank_per_term(xb, d, t_bits):
+    """[rows x r] allowance per unit of |U| for the rows of t_bits (= the rows of xb): each term
+    T[m,j] U[n,j] may carry two bf16 roundings (T / alpha on the GPU, T in the oracle: 2^-7 |T|)
+    and the fp32 accumulation of T over K (below 2^-12 sum_k |x d|)."""
+    x = np.abs(W.bf16_bits_to_f32(xb).astype(np.float64))
+    df = np.abs(W.bf16_bits_to_f32(d).astype(np.float64))
+    t = np.abs(W.bf16_bits_to_f32(t_bits).astype(np.float64))
+    return 2.0 ** -7 * t + 2.0 ** -12 * (x @ df.T)
+
+
+def _lowrank_bound(xb, d, u, t_bits):
+    """Allowance of the branch for every output [M x N]."""
+    uf = np.abs(W.bf16_bits_to_f32(u).astype(np.float64))
+    return _lowrank_per_term(xb, d, t_bits) @ uf.T
+
+
+def _assert_lowrank_close(y, ref, branch, bound):
+    """Every output within the sound bound (FP4 product's tolerance + the branch's allowance);
+    and, since that allowance sums |T U| over the rank, an aggregate check that the error has
+    the size of rounding noise: RMS error at most 2^-8 RMS(Y) (bf16 output) + 1 % RMS(branch)
+    (its two bf16 roundings leave ~0.3 %) + 1e-4 max|Y| (fp32 accumulation)."""
+    err = np.abs(y - ref)
+    tol = gemm_tolerance(ref, True) + bound
+    assert np.all(err <= tol), f"max err {err.max()} at {np.unravel_index(err.argmax(), err.shape)}"
+    rms = lambda a: float(np.sqrt(np.mean(np.square(a))))
+    limit = 2.0 ** -8 * rms(ref) + 0.01 * rms(branch) + 1e-4 * float(np.abs(ref).max())
+    assert rms(y - ref) <= limit, (rms(y - ref), limit)
+
+
+def _run_lowrank(xb, wb, d, u):
+    qa, qw = gpu_quantize(xb), gpu_quantize(wb)
+    y = nv.linear_lowrank(qa, qw, dev_tensor(xb), dev_tensor(d), dev_tensor(u))
+    torch.cuda.synchronize()
+    assert nv.sync_status() == 0
+    return to_numpy_f64(y)
+
+
+@pytest.mark.parametrize("M,N,K,r", [(256, 256, 256, 128), (300, 520, 224, 48),
+                                     (130, 264, 512, 256), (512, 768, 3072, 128),
+                                     (40, 1032, 96, 16)])
+def test_linear_lowrank_matches_oracle(M, N, K, r):
+    xb, wb, d, u = _lowrank_case(M, N, K, r, seed=M + N + r)
+    y = _run_lowrank(xb, wb, d, u)
+    qa_h, qw_h = O.quantize(xb), O.quantize(wb)
+    ref = O.linear_lowrank(qa_h, qw_h, xb, d, u)
+    bound = _lowrank_bound(xb, d, u, O.lowrank_down(xb, d))
+    branch = ref - O.gemm(qa_h, qw_h)
+    _assert_lowrank_close(y, ref, branch, bound)
+    # the branch is a real part of the output: without it the check fails
+    assert np.abs(branch).max() > 0.05 * np.abs(ref).max()
+    assert not np.all(np.abs(y - (ref - branch)) <= gemm_tolerance(ref, True) + bound)
+
+
+def test_linear_lowrank_zero_up_is_the_linear_layer():
+    # a shape nvfp4_linear runs on the same pair kernel (enough tiles for no K split)
+    M, N, K, r = 2560, 2048, 1024, 128
+    xb, wb, d, _ = _lowrank_case(M, N, K, r, seed=5)
+    u = np.zeros((N, r), np.uint16)
+    qa, qw = gpu_quantize(xb), gpu_quantize(wb)
+    y = nv.linear_lowrank(qa, qw, dev_tensor(xb), dev_tensor(d), dev_tensor(u))
+    y0 = nv.linear(qa, qw)
+    torch.cuda.synchronize()
+    assert torch.equal(y.float(), y0.float())  # adding zero terms leaves the fp32 sums as they are
+
+
+def test_linear_lowrank_zero_weight_is_the_branch_alone():
+    # sgW = 0: the FP4 product vanishes and alpha is taken as 1, so T' is T rounded once
+    M, N, K, r = 256, 264, 512, 64
+    xb, wb, d, u = _lowrank_case(M, N, K, r, seed=6, w_std=0.0)
+    y = _run_lowrank(xb, wb, d, u)
+    ref = O.linear_lowrank(O.quantize(xb), O.quantize(wb), xb, d, u)
+    bound = _lowrank_bound(xb, d, u, O.lowrank_down(xb, d))
+    _assert_lowrank_close(y, ref, ref, bound)
+
+
+def test_linear_lowrank_full_size_sampled():
+    # the attention projection with a rank-128 branch: M4096 N3072 K3072, sampled outputs
+    wl = W.attn_proj()
+    M, K = wl.X_bf16.shape
+    w32 = W.bf16_bits_to_f32(W.to_bf16_bits(W.normal((3072, K), 0.02, 2, 1)))
+    wb = W.to_bf16_bits(w32)
+    d, u = W.lowrank_factors(N=3072, K=K, r=128)
+    y = _run_lowrank(wl.X_bf16, wb, d, u)
+    g = np.random.Generator(np.random.PCG64(74))
+    ms = np.concatenate([g.integers(0, M, 1500), [0, M - 1, M - 1]])
+    ns = np.concatenate([g.integers(0, 3072, 1500), [0, 3071, 0]])
+    qa_h, qw_h = O.quantize(wl.X_bf16), O.quantize(wb)
+    ref = O.linear_lowrank_sampled(qa_h, qw_h, wl.X_bf16, d, u, ms, ns)
+    rows = np.unique(ms)
+    per = _lowrank_per_term(wl.X_bf16[rows], d, O.lowrank_down(wl.X_bf16[rows], d))
+    uf = np.abs(W.bf16_bits_to_f32(u).astype(np.float64))
+    bound = np.einsum("ij,ij->i", per[np.searchsorted(rows, ms)], uf[ns])
+    full_max = float(np.abs(y).max())
+    tol = 1e-3 * full_max + np.abs(ref) * 2.0 ** -8 + bound
+    assert np.all(np.abs(y[ms, ns] - ref) <= tol)
+    branch = ref - O.gemm_sampled(qa_h, qw_h, ms, ns)
+    rms = lambda a: float(np.sqrt(np.mean(np.square(a))))
+    assert rms(y[ms, ns] - ref) <= 2.0 ** -8 * rms(ref) + 0.01 * rms(branch) + 1e-4 * full_max

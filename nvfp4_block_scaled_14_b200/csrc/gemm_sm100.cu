@@ -866,6 +866,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tma_prefetch_desc(&tmT);
                 tma_prefetch_desc(&tmU);
             }
+            pdl_wait(); // operands come from the stream's earlier kernels
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -1082,6 +1083,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------- epilogue (both CTAs, warps 2..5) -------------
         const int q = warp & 3;
+        pdl_wait(); // global scales (and Y's previous readers) belong to earlier kernels
         float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
         if (LR && alpha == 0.0f)
             alpha = 1.0f; // the FP4 product is zero; T' was not divided either
@@ -1964,9 +1966,21 @@ cudaError_t launch_pair(const uint8_t *a_codes, const uint8_t *a_sf, const uint8
         clusters = gp.units;
     if (clusters < 1)
         clusters = 1;
-    nvfp4_gemm_pair_kernel<QOUT, LR><<<(unsigned)(2 * clusters), kThreads, Pair::kSmemBytes,
-                                       s>>>(tmA, tmB, tmSFA, tmSFB, tmY, tmT, tmU, gp);
-    return cudaGetLastError();
+    // programmatic dependent launch: barrier set-up, TMEM allocation and the cluster barrier
+    // overlap the previous kernel's tail; the producer and the epilogue wait for it before
+    // touching its outputs
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Pair::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QOUT, LR>, tmA, tmB, tmSFA, tmSFB, tmY,
+                              tmT, tmU, gp);
 }
 
 template <int BN, bool XQ = false> cudaError_t smallm_set_smem_attr()

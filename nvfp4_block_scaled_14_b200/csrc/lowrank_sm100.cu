@@ -10,12 +10,12 @@
 //
 // Shape of the work: M x r outputs (r <= 256) over K = 3072 is little arithmetic next to the
 // bytes of x, so the kernel is HBM-bound on x. Each 128-row band of x is split along K over a
-// thread-block cluster of up to 4 CTAs (one CTA per SM for the 4096-row case: 128 CTAs),
-// each streaming its K range of x and D through a 4-stage TMA ring into one M128 x N=r MMA
-// accumulator in TMEM. The partial accumulators meet in shared memory: every CTA stages its
-// partial, and after a cluster barrier each CTA sums a quarter of the band's rows over the
-// cluster's partials in rank order (distributed shared memory, deterministic), divides by
-// alpha, rounds to bf16 and stores.
+// thread-block cluster of up to 4 CTAs (128 CTAs for 4096 rows, one per SM), each streaming
+// its K range of x and D through a 4-stage TMA ring into one M128 x N=r MMA accumulator in
+// TMEM. The partial accumulators meet in shared memory: every CTA stages its partial, and
+// after a cluster barrier each CTA sums its share of the band's rows over the cluster's
+// partials in rank order (distributed shared memory, deterministic), divides by alpha, rounds
+// to bf16 and stores.
 #include <cuda.h>
 #include <cstring>
 #include <mutex>
@@ -27,8 +27,18 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kDnThreads = 192; // warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 epilogue
-constexpr int kDnStages = 4;
-constexpr int kDnMaxSplit = 4;
+// K split (CTAs per cluster, a power of two <= 8) and TMA ring depth. Measured on
+// M4096 K3072 r128: a split of 4 with 4 stages (one CTA per SM) beats 8 with 3 stages (two
+// CTAs per SM).
+#ifndef NVFP4_DN_SPLIT
+#define NVFP4_DN_SPLIT 4
+#endif
+#ifndef NVFP4_DN_STAGES
+#define NVFP4_DN_STAGES 4
+#endif
+constexpr int kDnStages = NVFP4_DN_STAGES;
+constexpr int kDnMaxSplit = NVFP4_DN_SPLIT;
+static_assert(kDnStages >= 3, "the fp32 partial must fit in the drained stage buffers");
 constexpr int kDnABytes = 128 * 128; // 128 rows of x x 64 bf16 (one 128-byte swizzle row)
 constexpr uint32_t kDnWaitLimit = 1u << 20;
 
@@ -82,7 +92,7 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b)
 
 // grid (S, ceil(M / 128)), cluster (S, 1, 1): CTA (rank, band) takes k-tiles
 // [kt_total * rank / S, kt_total * (rank + 1) / S) of rows [128 band, 128 band + 128).
-__global__ void __launch_bounds__(kDnThreads, 1)
+__global__ void __launch_bounds__(kDnThreads, kDnStages <= 3 ? 2 : 1)
     lowrank_down_kernel(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmD, const DownParams p)
 {
@@ -199,6 +209,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
     tc_fence_before();
     __syncwarp();
     cluster_sync(); // every partial of the cluster is in shared memory
+    pdl_launch_dependents(); // the GEMM may set up while the partials are reduced
 
     if (aligned) {
         float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
@@ -315,7 +326,11 @@ cudaError_t launch_lowrank_down(const void *x, const void *d, int64_t M, int64_t
     p.w_gs = w_gs;
     p.t = reinterpret_cast<__nv_bfloat16 *>(t);
     p.status = device_status_ptr();
-    const int S = p.kt_total >= kDnMaxSplit ? kDnMaxSplit : (p.kt_total >= 2 ? 2 : 1);
+    // the largest power-of-two split (<= 8, so a band's 128 rows divide evenly) that leaves
+    // every CTA at least one k-tile
+    int S = 1;
+    while (S * 2 <= kDnMaxSplit && S * 2 <= p.kt_total)
+        S *= 2;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)S, (unsigned)((M + 127) / 128), 1);
     cfg.blockDim = dim3(kDnThreads, 1, 1);

@@ -549,7 +549,7 @@ __device__ __forceinline__ uint32_t encode_one(const uint4 *r, float s8, float s
 // one 16-byte store and the two scale bytes as one 16-bit store. The first item is loaded
 // before waiting on the amax kernel (programmatic dependent launch), so the loads overlap its
 // tail; later items are double-buffered.
-template <int SRC>
+template <int SRC, int NT = kEncThreads>
 __device__ __forceinline__ void encode_body(const QuantArgs &a, int bid, int nblk)
 {
     __shared__ float s_sg;
@@ -639,6 +639,7 @@ __device__ __forceinline__ void encode_body(const QuantArgs &a, int bid, int nbl
     if (threadIdx.x < 128)
         s_rcp[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
     __syncthreads();
+    pdl_launch_dependents(); // a dependent GEMM may set up while this grid encodes
 
     // blocks b0, b0 + 1 of row r0 + ro: codes, scales; atom padding blocks get zero scales
     auto encode_store = [&](int ro, int b0, const uint4 (&r)[8]) {
@@ -671,19 +672,19 @@ __device__ __forceinline__ void encode_body(const QuantArgs &a, int bid, int nbl
         // fp32 blocks are 64 bytes: one item in flight keeps the registers in budget
         while (it < items) {
             encode_store(roa, b0a, ra);
-            it += kEncThreads / 32;
+            it += NT / 32;
             load_item(it, ra, roa, b0a);
         }
     } else {
         while (it < items) {
-            load_item(it + kEncThreads / 32, rb, rob, b0b);
+            load_item(it + NT / 32, rb, rob, b0b);
             encode_store(roa, b0a, ra);
-            it += kEncThreads / 32;
+            it += NT / 32;
             if (it >= items)
                 break;
-            load_item(it + kEncThreads / 32, ra, roa, b0a);
+            load_item(it + NT / 32, ra, roa, b0a);
             encode_store(rob, b0b, rb);
-            it += kEncThreads / 32;
+            it += NT / 32;
         }
     }
     zero_pad_rows(a, apb, bid, nblk);
@@ -703,13 +704,94 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
 // the tensor is read from HBM once and no second kernel is launched. Static amax: no
 // barrier, each item is encoded as soon as its copy lands. Lanes read their 64 (32) bytes
 // in an order rotated by lane so that a warp's shared-memory reads are conflict-free.
-template <int SRC>
-__global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const QuantArgs a)
+//
+// With SS >= 0 the same launch also quantizes a second, smaller tensor b (source type SS)
+// that is held in registers: each CTA takes a contiguous range of b's blocks, every thread
+// loads whole blocks of it (kPairRegVecs 16-byte vectors: 6 blocks of fp8, 3 of bf16, 1 of
+// fp32) with plain loads issued right after a's bulk copies, folds max |b| as they arrive,
+// keeps them across the grid-wide barrier (b's partials meet a's there) and encodes them
+// before a's shared-memory encode. Two tensors then cost one launch, one barrier and one HBM
+// read each, with all of both in flight at once (nvfp4_quantize_batch of, e.g., a layer's FP8
+// weight and its activations).
+constexpr int kPairThreads = 768; // 85 registers a thread: b's 24 plus the encode's
+constexpr int kPairRegVecs = 6;
+
+// b's part of the pair kernel after the grid-wide barrier: its global scale from the partial
+// maxima (or its static amax), then each thread's register-held blocks encoded and stored
+// (codes 8 bytes a block; scales in the linear and / or swizzled layout, a row's last atom
+// padded with zeros; padding rows of the last band zeroed).
+template <int SS, int BPT>
+__device__ __forceinline__ void pair_encode_regs(const QuantArgs &b, const uint4 *bv, int64_t bk0,
+                                                 int64_t bk1, float s8, float static_amax)
+{
+    __shared__ float s_sgb;
+    __shared__ float s_rcpb[128];
+    constexpr int BV = Enc<SS>::kVecs;
+    if (threadIdx.x < 32) {
+        float g = 0.0f;
+        if (b.static_amax) {
+            g = static_amax;
+        } else {
+            float pv[5]; // gridDim <= 160: one L2 round trip
+#pragma unroll
+            for (int u = 0; u < 5; ++u) {
+                const int i = threadIdx.x + 32 * u;
+                pv[u] = i < (int)gridDim.x ? __ldcg(b.partials_out + i) : 0.0f;
+            }
+            g = fmaxf(fmaxf(fmaxf(pv[0], pv[1]), fmaxf(pv[2], pv[3])), pv[4]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+            if (SS == kSrcE4M3)
+                g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
+        }
+        if (threadIdx.x == 0) {
+            const float sg = __fdiv_rn(g, 2688.0f); // 6 * 448
+            s_sgb = sg;
+            if (blockIdx.x == 0)
+                *b.global_scale = sg;
+        }
+    }
+    __syncthreads();
+    const float sg = s_sgb;
+    const float t = __fmul_rn(sg, 6.0f);
+    const float rt = __frcp_rn(t);
+    if (threadIdx.x < 128)
+        s_rcpb[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
+    __syncthreads();
+    const uint32_t nb = (uint32_t)(b.cols >> 4);
+    const int apb = (int)((nb + 3) >> 2);
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+        const int64_t blk = bk0 + (int64_t)j * blockDim.x + threadIdx.x;
+        if (blk >= bk1)
+            continue;
+        uint2 codes;
+        const uint32_t sb = encode_one<SS>(bv + j * BV, s8, sg, t, rt, s_rcpb, codes);
+        *reinterpret_cast<uint2 *>(b.codes + blk * 8) = codes;
+        if (b.sf_lin)
+            b.sf_lin[blk] = (uint8_t)sb;
+        if (b.sf_swz) {
+            const int64_t row = blk / nb;
+            const uint32_t c = (uint32_t)(blk - row * nb);
+            uint8_t *q = b.sf_swz + swz_offset(row, c, apb);
+            q[0] = (uint8_t)sb;
+            if (c + 1 == nb) // the row's last block: the rest of its atom row is padding
+                for (uint32_t e = (c & 3u) + 1u; e < 4u; ++e)
+                    q[e - (c & 3u)] = 0u;
+        }
+    }
+    zero_pad_rows(b, apb, blockIdx.x, gridDim.x);
+}
+
+template <int SRC, int NT, int SS>
+__device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &b, uint8_t *buf)
 {
     using E = Enc<SRC>;
-    extern __shared__ __align__(128) uint8_t buf[];
+    constexpr bool kPair = SS >= 0;
     __shared__ uint64_t bars[kFusedMaxChunks];
-    __shared__ float s_red[kFusedThreads / 32];
+    __shared__ float s_red[NT / 32];
+    __shared__ float s_red_b[NT / 32];
     __shared__ float s_sg;
     __shared__ float s_rcp[128];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -720,11 +802,25 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
     const int64_t byte0 = c0 * E::kItem;
     const int64_t nbytes = max((int64_t)0, min(a.nbytes, c1 * E::kItem) - byte0);
     const int nch = (int)((nbytes + kFusedChunk - 1) / kFusedChunk);
-    __shared__ float s_scalars[2];
+    // b's blocks: a contiguous range per CTA, block j * NT + tid of it per thread
+    using EB = Enc<kPair ? SS : SRC>;
+    constexpr int BV = EB::kVecs;                 // 16-byte vectors per block of b
+    constexpr int BPT = kPairRegVecs / BV;        // b's blocks per thread
+    const int64_t b_nblk = kPair ? (int64_t)b.rows * (b.cols >> 4) : 0;
+    const int64_t b_per = (b_nblk + gridDim.x - 1) / gridDim.x;
+    const int64_t bk0 = min(b_nblk, b_per * (int64_t)blockIdx.x);
+    const int64_t bk1 = min(b_nblk, bk0 + b_per);
+    const bool b_dyn = kPair && !b.static_amax;
+    uint4 bv[kPair ? kPairRegVecs : 1];
+    __shared__ float s_scalars[4];
     if (threadIdx.x == 0) {
         // the scalar inputs go out ahead of the bulk copies, not behind them in the queue
         s_scalars[0] = (SRC == kSrcE4M3 && a.fp8_scale) ? *a.fp8_scale : 1.0f;
         s_scalars[1] = a.static_amax ? *a.static_amax : 0.0f;
+        if constexpr (kPair) {
+            s_scalars[2] = (SS == kSrcE4M3 && b.fp8_scale) ? *b.fp8_scale : 1.0f;
+            s_scalars[3] = b.static_amax ? *b.static_amax : 0.0f;
+        }
         for (int i = 0; i < nch; ++i)
             mbar_init(&bars[i], 1);
         fence_barrier_init();
@@ -735,12 +831,23 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
             bulk_load_1d(buf + off, a.x + byte0 + off, n, &bars[i]);
         }
     }
+    if constexpr (kPair) {
+        // all of this thread's blocks of b in flight at once
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) {
+            const int64_t blk = bk0 + (int64_t)j * NT + threadIdx.x;
+            const uint4 *q = reinterpret_cast<const uint4 *>(b.x + blk * EB::kBlk);
+#pragma unroll
+            for (int v = 0; v < BV; ++v)
+                bv[j * BV + v] = blk < bk1 ? ldg_stream(q + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
     __syncthreads();
     const float s8 = s_scalars[0];
     // rotation: bf16 / fp32 lanes read 64 bytes (4 vectors), fp8 lanes 32 bytes (2 vectors)
     const uint32_t k = SRC == kSrcE4M3 ? (uint32_t)(lane >> 2) & 1u : (uint32_t)(lane >> 1) & 3u;
     constexpr int NVL = E::kBpl * E::kVecs;
-    constexpr int kWarps = kFusedThreads / 32;
+    constexpr int kWarps = NT / 32;
     constexpr int MIW = kFusedCap / E::kItem / kWarps; // items per warp at most
     const int items = (int)(c1 - c0);
     auto load_lane = [&](int j, uint4 (&r)[NVL]) -> bool {
@@ -756,6 +863,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
         if (!mbar_wait(&bars[(j * E::kItem) / kFusedChunk], 0, kSpinLimit) && lane == 0)
             atomicExch(a.status, (int)NVFP4_ERR_TIMEOUT);
     };
+    if constexpr (kPair) {
+        // b's maxima first: its loads were issued right behind a's copies
+        if (b_dyn) {
+            uint32_t m = 0; // blocks past the range were loaded as zeros
+#pragma unroll
+            for (int i = 0; i < BPT * BV; ++i)
+                m = mag_fold<SS>(m, Src<SS>::vec_magmax(bv[i]));
+            float f = Src<SS>::mag_to_f32(m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
+            if (lane == 0)
+                s_red_b[warp] = f;
+        }
+    }
+    const bool need_barrier = !a.static_amax || b_dyn;
     float bm0[MIW], bm1[MIW]; // block maxima of this lane's blocks, item by item
     if (!a.static_amax) {
         // block maxima as the copies land; the CTA maximum is their maximum
@@ -777,19 +900,38 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
             lm = fmaxf(lm, __shfl_xor_sync(0xFFFFFFFFu, lm, o));
         if (lane == 0)
             s_red[warp] = lm;
+    }
+    float g = 0.0f;
+    if (need_barrier) {
         __syncthreads();
-        float g = 0.0f;
         if (threadIdx.x < 32) {
-            g = s_red[threadIdx.x];
+            if (!a.static_amax) {
+                g = threadIdx.x < kWarps ? s_red[threadIdx.x] : 0.0f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
-            if (threadIdx.x == 0 && gridDim.x > 1)
-                a.partials_out[blockIdx.x] = g;
+                for (int o = 16; o > 0; o >>= 1)
+                    g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+                if (threadIdx.x == 0 && gridDim.x > 1)
+                    a.partials_out[blockIdx.x] = g;
+            }
+            if (b_dyn) {
+                float gb = threadIdx.x < kWarps ? s_red_b[threadIdx.x] : 0.0f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    gb = fmaxf(gb, __shfl_xor_sync(0xFFFFFFFFu, gb, o));
+                if (threadIdx.x == 0)
+                    b.partials_out[blockIdx.x] = gb;
+            }
         }
-        if (gridDim.x > 1) { // a single CTA already holds the tensor's maximum
-            cooperative_groups::this_grid().sync(); // every CTA's partial is visible
-            if (threadIdx.x < 32) {
+        // every CTA's partials are visible after the barrier (a single CTA already holds
+        // the maxima)
+        if (gridDim.x > 1)
+            cooperative_groups::this_grid().sync();
+    }
+    if constexpr (kPair)
+        pair_encode_regs<SS, BPT>(b, bv, bk0, bk1, s_scalars[2], s_scalars[3]);
+    if (!a.static_amax) {
+        if (threadIdx.x < 32) {
+            if (gridDim.x > 1) {
                 // all loads in flight at once (gridDim <= 160): one L2 round trip
                 float pv[5];
 #pragma unroll
@@ -802,8 +944,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
                 for (int o = 16; o > 0; o >>= 1)
                     g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
             }
-        }
-        if (threadIdx.x < 32) {
             if (SRC == kSrcE4M3)
                 g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
             if (threadIdx.x == 0) {
@@ -826,6 +966,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
     if (threadIdx.x < 128)
         s_rcp[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
     __syncthreads();
+    pdl_launch_dependents(); // a dependent GEMM may set up while this grid encodes
 
     const uint32_t nb = (uint32_t)(a.cols >> 4);
     const int apb = (int)((nb + 3) >> 2);
@@ -851,6 +992,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const 
             store_lane<SRC>(a, f0, nb, apb, cw, sb0, sb1);
     }
     zero_pad_rows(a, apb, blockIdx.x, gridDim.x);
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(kFusedThreads, 1) fused_quantize_kernel(const QuantArgs a)
+{
+    extern __shared__ __align__(128) uint8_t buf[];
+    fused_body<SRC, kFusedThreads, -1>(a, a, buf);
+}
+
+// a held in shared memory, b streamed (see fused_body).
+template <int SA, int SB>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    fused_pair_quantize_kernel(const QuantArgs a, const QuantArgs b)
+{
+    extern __shared__ __align__(128) uint8_t buf[];
+    fused_body<SA, kPairThreads, SB>(a, b, buf);
 }
 
 template <int SRC>
@@ -1258,6 +1415,84 @@ cudaError_t launch_quantize_e4m3(const void *x, int src_type, int64_t n, const f
     return launch_e4m3_typed<kSrcBF16>(x, n, static_amax, codes, scale_out, ws, s);
 }
 
+// Two tensors in one cooperative launch (fused_pair_quantize_kernel): a, the larger, held in
+// shared memory, b in registers. Taken when a's share per SM fits at kPairThreads, b's share
+// fits the threads' registers (about 10.9 MB of fp8 or bf16, 7.3 MB of fp32 on 148 SMs) and
+// the pair is large enough for the single pass to pay (16 MB, the single-tensor fused
+// kernel's floor). Returns false when the pair does not qualify (nothing launched).
+template <int SA, int SB>
+cudaError_t launch_fused_pair_typed(const QuantArgs &a, const QuantArgs &b, int grid, bool coop,
+                                    cudaStream_t s)
+{
+    constexpr int kSmem = kFusedCap;
+    static std::once_flag fattr[64];
+    static cudaError_t fe[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::call_once(fattr[dev & 63], [&]() {
+        fe[dev & 63] = cudaFuncSetAttribute(fused_pair_quantize_kernel<SA, SB>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    });
+    if (fe[dev & 63] != cudaSuccess)
+        return fe[dev & 63];
+    cudaLaunchConfig_t fc{};
+    fc.gridDim = dim3((unsigned)grid);
+    fc.blockDim = dim3(kPairThreads);
+    fc.dynamicSmemBytes = kSmem;
+    fc.stream = s;
+    cudaLaunchAttribute fa[1];
+    fa[0].id = cudaLaunchAttributeCooperative;
+    fa[0].val.cooperative = coop ? 1 : 0;
+    fc.attrs = fa;
+    fc.numAttrs = 1;
+    return cudaLaunchKernelEx(&fc, fused_pair_quantize_kernel<SA, SB>, a, b);
+}
+
+template <int SA>
+cudaError_t launch_fused_pair_b(int sb, const QuantArgs &a, const QuantArgs &b, int grid,
+                                bool coop, cudaStream_t s)
+{
+    switch (sb) {
+    case kSrcF32: return launch_fused_pair_typed<SA, kSrcF32>(a, b, grid, coop, s);
+    case kSrcBF16: return launch_fused_pair_typed<SA, kSrcBF16>(a, b, grid, coop, s);
+    default: return launch_fused_pair_typed<SA, kSrcE4M3>(a, b, grid, coop, s);
+    }
+}
+
+int64_t enc_item_bytes(int src) { return src == kSrcF32 ? 2048 : src == kSrcBF16 ? 2048 : 1024; }
+
+bool try_fused_pair(const QuantGroup &g, void *ws, cudaStream_t s, cudaError_t *err)
+{
+    if (g.njobs != 2)
+        return false;
+    const int ia = g.job[0].nbytes >= g.job[1].nbytes ? 0 : 1, ib = 1 - ia;
+    QuantArgs a = g.job[ia], b = g.job[ib];
+    const int grid = num_sms();
+    // b must fit in registers: kPairRegVecs 16-byte vectors a thread (whole blocks of it)
+    const int64_t b_blocks = (int64_t)b.rows * (b.cols / 16);
+    const int64_t b_bpt = kPairRegVecs / (g.src[ib] == kSrcF32 ? 4 : g.src[ib] == kSrcBF16 ? 2 : 1);
+    if (grid > 160 || 2 * grid > kAmaxPartials || a.nbytes + b.nbytes < kFusedMinBytes ||
+        b.nbytes <= 0 || b_blocks > (int64_t)grid * kPairThreads * b_bpt)
+        return false;
+    // warp items of a (Enc<>: 32 blocks of fp32, 64 of bf16 / fp8; 2 KB / 2 KB / 1 KB)
+    const int64_t item_blocks = g.src[ia] == kSrcF32 ? 32 : 64;
+    const int64_t item = enc_item_bytes(g.src[ia]);
+    const int64_t nitems = ((int64_t)a.rows * (a.cols / 16) + item_blocks - 1) / item_blocks;
+    const int64_t items_per_warp_max = kFusedCap / item / (kPairThreads / 32);
+    if ((nitems + grid - 1) / grid > items_per_warp_max * (kPairThreads / 32))
+        return false;
+    float *part = reinterpret_cast<float *>(ws);
+    a.partials_out = part;
+    b.partials_out = part + grid;
+    const bool coop = !a.static_amax || !b.static_amax;
+    switch (g.src[ia]) {
+    case kSrcF32: *err = launch_fused_pair_b<kSrcF32>(g.src[ib], a, b, grid, coop, s); break;
+    case kSrcBF16: *err = launch_fused_pair_b<kSrcBF16>(g.src[ib], a, b, grid, coop, s); break;
+    default: *err = launch_fused_pair_b<kSrcE4M3>(g.src[ib], a, b, grid, coop, s); break;
+    }
+    return true;
+}
+
 cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t s)
 {
     const int sms = num_sms();
@@ -1281,6 +1516,11 @@ cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cud
         amax_cap[j] = (nbytes + kChunk - 1) / kChunk;
         enc_w[j] = nbytes > 0 ? nbytes : 0;
         enc_cap[j] = jb.rows;
+    }
+    {
+        cudaError_t fe = cudaSuccess;
+        if (try_fused_pair(g, ws, s, &fe))
+            return fe;
     }
     int amax_total = sms < kAmaxPartials ? sms : kAmaxPartials;
     const int na = split_ctas(njobs, amax_w, amax_cap, amax_total, g.amax_cta0);

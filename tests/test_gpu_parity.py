@@ -93,6 +93,45 @@ def test_quantize_batch_matches_single_calls():
     assert nv.sync_status() == 0
 
 
+@pytest.mark.parametrize("case", ["dynamic", "x_static", "w_static", "both_static",
+                                  "fp32_ragged", "b_bf16_ragged", "b_fp32_ragged"])
+def test_quantize_batch_single_launch_pair(case):
+    # two tensors that take the one-launch pair kernel (the larger held in shared memory, the
+    # smaller in registers): each gets exactly its single-call result
+    w8, s8 = W.to_fp8_tensorwise(W.normal((3072, 3072), 0.02, 34, 1))
+    if case == "fp32_ragged":
+        xa = W.normal((2050, 3104), 1.0, 34, 3)                 # 25.4 MB fp32, ragged rows
+    else:
+        xa = W.to_bf16_bits(W.normal((4096, 3072), 1.0, 34, 2))  # the attention projection
+    ax = 3.5 if case in ("x_static", "both_static") else None
+    aw = 0.05 if case in ("w_static", "both_static") else None
+    jobs = [{"x": dev_tensor(xa), "linear": True}]
+    if case == "b_bf16_ragged":   # pad blocks (66 per row) and pad rows (1000 rows)
+        xb = W.to_bf16_bits(W.normal((1000, 1056), 0.5, 34, 4))
+        jobs.append({"x": dev_tensor(xb), "linear": True})
+    elif case == "b_fp32_ragged":
+        xb = W.normal((300, 1056), 0.5, 34, 5)
+        jobs.append({"x": dev_tensor(xb), "linear": True})
+    else:
+        jobs.append({"x": dev_tensor(w8), "fp8_scale": scalar_dev(s8), "linear": True})
+    if ax is not None:
+        jobs[0]["static_amax"] = scalar_dev(ax)
+    if aw is not None:
+        jobs[1]["static_amax"] = scalar_dev(aw)
+    if case == "w_static":
+        jobs = jobs[::-1]  # order of the jobs does not matter
+    q = nv.quantize_batch(jobs)
+    torch.cuda.synchronize()
+    assert nv.sync_status() == 0
+    if case == "w_static":
+        q = q[::-1]
+    assert_quant_equal(q[0], O.quantize(xa, amax=ax))
+    if case.startswith("b_"):
+        assert_quant_equal(q[1], O.quantize(xb))
+    else:
+        assert_quant_equal(q[1], O.quantize(w8, amax=aw, fp8_scale=s8))
+
+
 def test_quantize_batch_rejects_bad_jobs():
     from nvfp4_block_scaled_14_b200 import _lib as L
     lib = L.load()

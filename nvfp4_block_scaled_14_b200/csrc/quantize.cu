@@ -707,58 +707,29 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
 //
 // With SS >= 0 the same launch also quantizes a second, smaller tensor b (source type SS)
 // that is held in registers: each CTA takes a contiguous range of b's blocks, every thread
-// loads whole blocks of it (kPairRegVecs 16-byte vectors: 6 blocks of fp8, 3 of bf16, 1 of
+// loads whole blocks of it (kPairRegVecs 16-byte vectors: 4 blocks of fp8, 2 of bf16, 1 of
 // fp32) with plain loads issued right after a's bulk copies, folds max |b| as they arrive,
 // keeps them across the grid-wide barrier (b's partials meet a's there) and encodes them
 // before a's shared-memory encode. Two tensors then cost one launch, one barrier and one HBM
 // read each, with all of both in flight at once (nvfp4_quantize_batch of, e.g., a layer's FP8
-// weight and its activations).
-constexpr int kPairThreads = 768; // 85 registers a thread: b's 24 plus the encode's
-constexpr int kPairRegVecs = 6;
+// weight and its activations). Measured on W 3072x3072 FP8 + X 4096x3072 bf16 (globaltimer
+// stamps in an instrumented copy): loads and maxima ~7-8 us, grid barrier ~2 us, partials +
+// W's encode ~6 us, X's encode ~3.5 us; 1024 threads x 4 vectors beat 768 x 6 by ~0.5 us.
+constexpr int kPairThreads = 1024; // 64 registers a thread: b's 16 plus the encode's
+constexpr int kPairRegVecs = 4;
 
-// b's part of the pair kernel after the grid-wide barrier: its global scale from the partial
-// maxima (or its static amax), then each thread's register-held blocks encoded and stored
-// (codes 8 bytes a block; scales in the linear and / or swizzled layout, a row's last atom
-// padded with zeros; padding rows of the last band zeroed).
+// b's part of the pair kernel after the grid-wide barrier and its global scale sg: each
+// thread's register-held blocks encoded and stored (codes 8 bytes a block; scales in the linear
+// and / or swizzled layout, a row's last atom padded with zeros; padding rows of the last band
+// zeroed). rcp_tab: 1 / (E4M3(c) * sg) for the 128 non-negative codes.
 template <int SS, int BPT>
 __device__ __forceinline__ void pair_encode_regs(const QuantArgs &b, const uint4 *bv, int64_t bk0,
-                                                 int64_t bk1, float s8, float static_amax)
+                                                 int64_t bk1, float s8, float sg,
+                                                 const float *rcp_tab)
 {
-    __shared__ float s_sgb;
-    __shared__ float s_rcpb[128];
     constexpr int BV = Enc<SS>::kVecs;
-    if (threadIdx.x < 32) {
-        float g = 0.0f;
-        if (b.static_amax) {
-            g = static_amax;
-        } else {
-            float pv[5]; // gridDim <= 160: one L2 round trip
-#pragma unroll
-            for (int u = 0; u < 5; ++u) {
-                const int i = threadIdx.x + 32 * u;
-                pv[u] = i < (int)gridDim.x ? __ldcg(b.partials_out + i) : 0.0f;
-            }
-            g = fmaxf(fmaxf(fmaxf(pv[0], pv[1]), fmaxf(pv[2], pv[3])), pv[4]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
-            if (SS == kSrcE4M3)
-                g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
-        }
-        if (threadIdx.x == 0) {
-            const float sg = __fdiv_rn(g, 2688.0f); // 6 * 448
-            s_sgb = sg;
-            if (blockIdx.x == 0)
-                *b.global_scale = sg;
-        }
-    }
-    __syncthreads();
-    const float sg = s_sgb;
     const float t = __fmul_rn(sg, 6.0f);
     const float rt = __frcp_rn(t);
-    if (threadIdx.x < 128)
-        s_rcpb[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
-    __syncthreads();
     const uint32_t nb = (uint32_t)(b.cols >> 4);
     const int apb = (int)((nb + 3) >> 2);
 #pragma unroll
@@ -767,13 +738,21 @@ __device__ __forceinline__ void pair_encode_regs(const QuantArgs &b, const uint4
         if (blk >= bk1)
             continue;
         uint2 codes;
-        const uint32_t sb = encode_one<SS>(bv + j * BV, s8, sg, t, rt, s_rcpb, codes);
+        const uint32_t sb = encode_one<SS>(bv + j * BV, s8, sg, t, rt, rcp_tab, codes);
         *reinterpret_cast<uint2 *>(b.codes + blk * 8) = codes;
         if (b.sf_lin)
             b.sf_lin[blk] = (uint8_t)sb;
         if (b.sf_swz) {
-            const int64_t row = blk / nb;
-            const uint32_t c = (uint32_t)(blk - row * nb);
+            uint32_t row, c; // blk / nb by multiply-high (exact or one too large), as store_lane
+            if (b.blocks_fit32) {
+                row = __umulhi((uint32_t)blk, b.nb_magic);
+                if (row * nb > (uint32_t)blk)
+                    --row;
+                c = (uint32_t)blk - row * nb;
+            } else {
+                row = (uint32_t)(blk / nb);
+                c = (uint32_t)(blk - (int64_t)row * nb);
+            }
             uint8_t *q = b.sf_swz + swz_offset(row, c, apb);
             q[0] = (uint8_t)sb;
             if (c + 1 == nb) // the row's last block: the rest of its atom row is padding
@@ -792,8 +771,9 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
     __shared__ uint64_t bars[kFusedMaxChunks];
     __shared__ float s_red[NT / 32];
     __shared__ float s_red_b[NT / 32];
-    __shared__ float s_sg;
+    __shared__ float s_sg, s_sgb;
     __shared__ float s_rcp[128];
+    __shared__ float s_rcpb[kPair ? 128 : 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nblocks = (int64_t)a.rows * (a.cols >> 4);
     const int64_t nitems = (nblocks + E::kItemBlocks - 1) / E::kItemBlocks;
@@ -927,37 +907,46 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
         if (gridDim.x > 1)
             cooperative_groups::this_grid().sync();
     }
-    if constexpr (kPair)
-        pair_encode_regs<SS, BPT>(b, bv, bk0, bk1, s_scalars[2], s_scalars[3]);
-    if (!a.static_amax) {
-        if (threadIdx.x < 32) {
-            if (gridDim.x > 1) {
-                // all loads in flight at once (gridDim <= 160): one L2 round trip
-                float pv[5];
+    // the global scales; the partial maxima of both tensors in one L2 round trip (gridDim <=
+    // 160: five loads a lane each)
+    if (threadIdx.x < 32) {
+        const bool a_round = !a.static_amax && gridDim.x > 1;
+        float pa[5], pb[5];
 #pragma unroll
-                for (int u = 0; u < 5; ++u) {
-                    const int i = threadIdx.x + 32 * u;
-                    pv[u] = i < (int)gridDim.x ? __ldcg(a.partials_out + i) : 0.0f;
-                }
-                g = fmaxf(fmaxf(fmaxf(pv[0], pv[1]), fmaxf(pv[2], pv[3])), pv[4]);
+        for (int u = 0; u < 5; ++u) {
+            const int i = threadIdx.x + 32 * u;
+            pa[u] = (a_round && i < (int)gridDim.x) ? __ldcg(a.partials_out + i) : 0.0f;
+            pb[u] = (b_dyn && i < (int)gridDim.x) ? __ldcg(b.partials_out + i) : 0.0f;
+        }
+        if (a_round) {
+            g = fmaxf(fmaxf(fmaxf(pa[0], pa[1]), fmaxf(pa[2], pa[3])), pa[4]);
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
-            }
-            if (SRC == kSrcE4M3)
-                g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
-            if (threadIdx.x == 0) {
-                const float sg = __fdiv_rn(g, 2688.0f); // 6 * 448
-                s_sg = sg;
+            for (int o = 16; o > 0; o >>= 1)
+                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+        }
+        float gb = 0.0f;
+        if (b_dyn) {
+            gb = fmaxf(fmaxf(fmaxf(pb[0], pb[1]), fmaxf(pb[2], pb[3])), pb[4]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                gb = fmaxf(gb, __shfl_xor_sync(0xFFFFFFFFu, gb, o));
+            if (SS == kSrcE4M3)
+                gb = __fmul_rn(gb, s_scalars[2]); // max |e| * s8 == max |e * s8|
+        }
+        if (!a.static_amax && SRC == kSrcE4M3)
+            g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
+        if (threadIdx.x == 0) {
+            const float sg = __fdiv_rn(a.static_amax ? s_scalars[1] : g, 2688.0f); // 6 * 448
+            s_sg = sg;
+            if (blockIdx.x == 0)
+                *a.global_scale = sg;
+            if constexpr (kPair) {
+                const float sgb = __fdiv_rn(b.static_amax ? s_scalars[3] : gb, 2688.0f);
+                s_sgb = sgb;
                 if (blockIdx.x == 0)
-                    *a.global_scale = sg;
+                    *b.global_scale = sgb;
             }
         }
-    } else if (threadIdx.x == 0) {
-        const float sg = __fdiv_rn(s_scalars[1], 2688.0f);
-        s_sg = sg;
-        if (blockIdx.x == 0)
-            *a.global_scale = sg;
     }
     __syncthreads();
     const float sg = s_sg;
@@ -965,8 +954,12 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
     const float rt = __frcp_rn(t);
     if (threadIdx.x < 128)
         s_rcp[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
+    if (kPair && threadIdx.x >= 128 && threadIdx.x < 256)
+        s_rcpb[threadIdx.x - 128] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x - 128), s_sgb));
     __syncthreads();
     pdl_launch_dependents(); // a dependent GEMM may set up while this grid encodes
+    if constexpr (kPair)
+        pair_encode_regs<SS, BPT>(b, bv, bk0, bk1, s_scalars[2], s_sgb, s_rcpb);
 
     const uint32_t nb = (uint32_t)(a.cols >> 4);
     const int apb = (int)((nb + 3) >> 2);
@@ -1417,7 +1410,7 @@ cudaError_t launch_quantize_e4m3(const void *x, int src_type, int64_t n, const f
 
 // Two tensors in one cooperative launch (fused_pair_quantize_kernel): a, the larger, held in
 // shared memory, b in registers. Taken when a's share per SM fits at kPairThreads, b's share
-// fits the threads' registers (about 10.9 MB of fp8 or bf16, 7.3 MB of fp32 on 148 SMs) and
+// fits the threads' registers (about 9.7 MB of fp8, bf16 or fp32 on 148 SMs) and
 // the pair is large enough for the single pass to pay (16 MB, the single-tensor fused
 // kernel's floor). Returns false when the pair does not qualify (nothing launched).
 template <int SA, int SB>

@@ -27,24 +27,26 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kDnThreads = 192; // warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 epilogue
-// K split (CTAs per cluster, a power of two <= 8) and TMA ring depth. Measured on
-// M4096 K3072 r128: a split of 4 with 4 stages (one CTA per SM) beats 8 with 3 stages (two
-// CTAs per SM).
+// K split (CTAs per cluster, a power of two <= 8) and the most TMA ring stages (as many as the
+// shared memory holds, up to this). Measured on M4096 K3072 r128: a split of 4 with one CTA per
+// SM beats 8 with two CTAs per SM (3 stages each) and 8 with 4 stages; the loads are
+// latency-bound, so the deepest ring that fits is taken.
 #ifndef NVFP4_DN_SPLIT
 #define NVFP4_DN_SPLIT 4
 #endif
 #ifndef NVFP4_DN_STAGES
-#define NVFP4_DN_STAGES 4
+#define NVFP4_DN_STAGES 6
 #endif
-constexpr int kDnStages = NVFP4_DN_STAGES;
+constexpr int kDnMaxStages = NVFP4_DN_STAGES;
 constexpr int kDnMaxSplit = NVFP4_DN_SPLIT;
-static_assert(kDnStages >= 3, "the fp32 partial must fit in the drained stage buffers");
+constexpr int kDnSmemMax = 232448; // per-CTA shared memory limit
 constexpr int kDnABytes = 128 * 128; // 128 rows of x x 64 bf16 (one 128-byte swizzle row)
 constexpr uint32_t kDnWaitLimit = 1u << 20;
 
 struct DownParams {
     int64_t M;
     int r;        // rank: multiple of 16, 16..256
+    int stages;   // TMA ring depth (3 .. kDnMaxStages; the fp32 partial fits in 3 or more)
     int kt_total; // 64-wide k-tiles of K
     const float *a_gs, *w_gs;
     __nv_bfloat16 *t; // [M x r], row stride r
@@ -56,7 +58,22 @@ __host__ __device__ constexpr uint32_t dn_tmem_cols(int r)
 {
     return r <= 32 ? 32u : r <= 64 ? 64u : r <= 128 ? 128u : 256u;
 }
-constexpr int dn_smem_bytes(int r) { return kDnStages * dn_stage_bytes(r) + 256; }
+constexpr int dn_stages(int r)
+{
+    return (kDnSmemMax - 256) / dn_stage_bytes(r) < kDnMaxStages
+               ? (kDnSmemMax - 256) / dn_stage_bytes(r)
+               : kDnMaxStages;
+}
+constexpr int dn_smem_bytes(int r) { return dn_stages(r) * dn_stage_bytes(r) + 256; }
+static_assert(dn_stages(256) >= 3 && dn_stages(16) >= 3, "ring depth");
+constexpr int dn_smem_max()
+{
+    int m = 0;
+    for (int r = 16; r <= 256; r += 16)
+        m = dn_smem_bytes(r) > m ? dn_smem_bytes(r) : m;
+    return m;
+}
+static_assert(dn_smem_max() <= kDnSmemMax, "shared memory");
 
 __device__ __forceinline__ void dn_timeout(int *status)
 {
@@ -92,7 +109,7 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b)
 
 // grid (S, ceil(M / 128)), cluster (S, 1, 1): CTA (rank, band) takes k-tiles
 // [kt_total * rank / S, kt_total * (rank + 1) / S) of rows [128 band, 128 band + 128).
-__global__ void __launch_bounds__(kDnThreads, kDnStages <= 3 ? 2 : 1)
+__global__ void __launch_bounds__(kDnThreads, 1)
     lowrank_down_kernel(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmD, const DownParams p)
 {
@@ -103,9 +120,10 @@ __global__ void __launch_bounds__(kDnThreads, kDnStages <= 3 ? 2 : 1)
     const uint32_t S = gridDim.x;
     const uint32_t rank = cluster_ctarank();
     const int64_t band = blockIdx.y;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDnStages * stage_bytes);
-    uint64_t *empty = full + kDnStages;
-    uint64_t *acc_full = empty + kDnStages;
+    const int nst = p.stages;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + nst * stage_bytes);
+    uint64_t *empty = full + kDnMaxStages;
+    uint64_t *acc_full = empty + kDnMaxStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
     const bool aligned = (smem_u32(smem) & 1023u) == 0; // uniform over the cluster
     const int kt0 = (int)((int64_t)p.kt_total * rank / S);
@@ -113,7 +131,7 @@ __global__ void __launch_bounds__(kDnThreads, kDnStages <= 3 ? 2 : 1)
     const uint32_t tcols = dn_tmem_cols(r);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kDnStages; ++s) {
+        for (int s = 0; s < nst; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -138,8 +156,8 @@ __global__ void __launch_bounds__(kDnThreads, kDnStages <= 3 ? 2 : 1)
             tma_prefetch_desc(&tmX);
             tma_prefetch_desc(&tmD);
             for (int i = 0; i < nk; ++i) {
-                const int s = i % kDnStages;
-                const uint32_t ph = (uint32_t)(i / kDnStages) & 1u;
+                const int s = i % nst;
+                const uint32_t ph = (uint32_t)(i / nst) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, kDnWaitLimit)) {
                     dn_timeout(p.status);
                     break;
@@ -156,8 +174,8 @@ __global__ void __launch_bounds__(kDnThreads, kDnStages <= 3 ? 2 : 1)
         const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(r >> 3) << 17) |
                                ((uint32_t)(128 >> 4) << 24);
         for (int i = 0; i < nk; ++i) {
-            const int s = i % kDnStages;
-            const uint32_t ph = (uint32_t)(i / kDnStages) & 1u;
+            const int s = i % nst;
+            const uint32_t ph = (uint32_t)(i / nst) & 1u;
             if (!mbar_wait(&full[s], ph, kDnWaitLimit)) {
                 if (lane == 0)
                     dn_timeout(p.status);
@@ -314,13 +332,14 @@ cudaError_t launch_lowrank_down(const void *x, const void *d, int64_t M, int64_t
     std::call_once(flags[dev & 63], [&]() {
         attr_err[dev & 63] = cudaFuncSetAttribute(lowrank_down_kernel,
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  dn_smem_bytes(256));
+                                                  dn_smem_max());
     });
     if (attr_err[dev & 63] != cudaSuccess)
         return attr_err[dev & 63];
     DownParams p{};
     p.M = M;
     p.r = r;
+    p.stages = dn_stages(r);
     p.kt_total = (int)((K + 63) / 64);
     p.a_gs = a_gs;
     p.w_gs = w_gs;

@@ -161,10 +161,13 @@ __device__ __forceinline__ void amax_body(const uint8_t *__restrict__ x, int64_t
 {
     __shared__ uint64_t bars[kRing];
     __shared__ float s_red[kAmaxThreads / 32];
+    // whole 16-byte vectors only (bulk copies move multiples of 16 bytes); a tensor's last
+    // nbytes % 16 bytes are folded by the kernel that reads the partials
     const int64_t nvec = nbytes >> 4;
+    const int64_t nfull = nvec << 4;
     const int64_t per = ((nvec + nblk - 1) / nblk) << 4;
-    const int64_t b0 = min(nbytes, per * (int64_t)bid);
-    const int64_t b1 = min(nbytes, b0 + per);
+    const int64_t b0 = min(nfull, per * (int64_t)bid);
+    const int64_t b1 = min(nfull, b0 + per);
     const int nchunks = (int)((b1 - b0 + kChunk - 1) / kChunk);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i)
@@ -1333,12 +1336,164 @@ __global__ void __launch_bounds__(kE8Threads)
     }
 }
 
+// Single-pass FP8 tensorwise quantize for dynamic amax (tensors of 16 MB up to what the CTAs'
+// shared memory holds): one CTA per SM bulk-loads its contiguous share of the flat tensor in
+// 32 KB copies and folds max |x| as they land, publishes one partial, meets the other CTAs at
+// a grid-wide barrier (cooperative launch), reduces the partials to s = amax / 448 and encodes
+// from shared memory, 8 values per thread-step (one 8-byte code store; consecutive threads,
+// consecutive vectors: conflict-free shared-memory reads and coalesced stores). The tensor is
+// read from HBM once and no second kernel runs. n: a multiple of 8.
+constexpr int kE8FusedThreads = 1024;
+
+template <int SRC>
+__global__ void __launch_bounds__(kE8FusedThreads, 1)
+    e4m3_fused_kernel(const uint8_t *__restrict__ x, int64_t n, float *__restrict__ partials,
+                      uint8_t *__restrict__ codes, float *__restrict__ scale_out, int *status)
+{
+    extern __shared__ __align__(128) uint8_t buf[];
+    __shared__ uint64_t bars[kFusedMaxChunks];
+    __shared__ float s_red[kE8FusedThreads / 32];
+    __shared__ float s_s;
+    constexpr int G = 16 / Src<SRC>::kBytes >= 8 ? 1 : 2; // 16-byte vectors per 8 values
+    const int64_t ngroups = n >> 3;
+    const int64_t g0 = ngroups * blockIdx.x / gridDim.x;
+    const int64_t g1 = ngroups * (blockIdx.x + 1) / gridDim.x;
+    const int64_t byte0 = g0 * 16 * G;
+    const int64_t nbytes = (g1 - g0) * 16 * G;
+    const int nch = (int)((nbytes + kFusedChunk - 1) / kFusedChunk);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < nch; ++i)
+            mbar_init(&bars[i], 1);
+        fence_barrier_init();
+        for (int i = 0; i < nch; ++i) {
+            const int64_t off = (int64_t)i * kFusedChunk;
+            const uint32_t nb = (uint32_t)min((int64_t)kFusedChunk, nbytes - off);
+            mbar_arrive_expect_tx(&bars[i], nb);
+            bulk_load_1d(buf + off, x + byte0 + off, nb, &bars[i]);
+        }
+    }
+    __syncthreads();
+    const uint32_t base = smem_u32(buf);
+    uint32_t m = 0;
+    for (int c = 0; c < nch; ++c) {
+        if (!mbar_wait(&bars[c], 0, kSpinLimit) && (threadIdx.x & 31) == 0)
+            atomicExch(status, (int)NVFP4_ERR_TIMEOUT);
+        const int nv = (int)(min((int64_t)kFusedChunk, nbytes - (int64_t)c * kFusedChunk) >> 4);
+        const uint32_t cb = base + (uint32_t)c * kFusedChunk;
+        for (int i = threadIdx.x; i < nv; i += kE8FusedThreads)
+            m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(lds128(cb + 16 * i)));
+    }
+    float f = Src<SRC>::mag_to_f32(m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
+    if ((threadIdx.x & 31) == 0)
+        s_red[threadIdx.x >> 5] = f;
+    __syncthreads();
+    float g = 0.0f;
+    if (threadIdx.x < 32) {
+        g = s_red[threadIdx.x];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+        if (threadIdx.x == 0)
+            partials[blockIdx.x] = g;
+    }
+    cooperative_groups::this_grid().sync(); // every CTA's partial is visible
+    if (threadIdx.x < 32) {
+        float pv[5]; // gridDim <= 160: one L2 round trip
+#pragma unroll
+        for (int u = 0; u < 5; ++u) {
+            const int i = threadIdx.x + 32 * u;
+            pv[u] = i < (int)gridDim.x ? __ldcg(partials + i) : 0.0f;
+        }
+        g = fmaxf(fmaxf(fmaxf(pv[0], pv[1]), fmaxf(pv[2], pv[3])), pv[4]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+        if (threadIdx.x == 0) {
+            const float sc = __fdiv_rn(g, 448.0f);
+            s_s = sc;
+            if (blockIdx.x == 0)
+                *scale_out = sc;
+        }
+    }
+    __syncthreads();
+    pdl_launch_dependents(); // a dependent GEMM may set up while this grid encodes
+    const float sc = s_s;
+    const float rs = __frcp_rn(sc);
+    const uint64_t rs2 = ((uint64_t)__float_as_uint(rs) << 32) | __float_as_uint(rs);
+    const int ng = (int)(g1 - g0);
+    for (int q = threadIdx.x; q < ng; q += kE8FusedThreads) {
+        float fv[8];
+        if constexpr (SRC == kSrcF32) {
+            const uint4 a = lds128(base + 32 * q), b = lds128(base + 32 * q + 16);
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                fv[j] = __uint_as_float(w[j]);
+        } else {
+            const uint4 a = lds128(base + 16 * q);
+            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                fv[2 * j] = __uint_as_float(w[j] << 16);
+                fv[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+        }
+        uint2 c;
+        if (sc > 0.0f) {
+            c = e4m3_codes8(fv, sc, rs2);
+        } else { // s == 0: sign-only codes
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                w[j >> 2] |= ((__float_as_uint(fv[j]) >> 24) & 0x80u) << (8 * (j & 3));
+            c = make_uint2(w[0], w[1]);
+        }
+        __stcs(reinterpret_cast<uint2 *>(codes + (g0 + q) * 8), c);
+    }
+}
+
 template <int SRC>
 cudaError_t launch_e4m3_typed(const void *x, int64_t n, const float *static_amax,
                               uint8_t *codes, float *scale_out, void *ws, cudaStream_t s)
 {
     const int sms = num_sms();
     int npartials = 0;
+    {
+        // single pass when every CTA's share fits in its shared memory (16 MB and up, as the
+        // NVFP4 fused kernel; n a multiple of 8)
+        const int64_t nbytes = n * Src<SRC>::kBytes;
+        const int64_t per = ((n >> 3) + sms - 1) / sms * 8 * Src<SRC>::kBytes;
+        if (!static_amax && (n & 7) == 0 && nbytes >= kFusedMinBytes && per <= kFusedCap &&
+            sms <= 160) {
+            static std::once_flag fattr[64];
+            static cudaError_t fe[64];
+            int dev = 0;
+            cudaGetDevice(&dev);
+            std::call_once(fattr[dev & 63], [&]() {
+                fe[dev & 63] = cudaFuncSetAttribute(
+                    e4m3_fused_kernel<SRC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedCap);
+            });
+            if (fe[dev & 63] != cudaSuccess)
+                return fe[dev & 63];
+            cudaLaunchConfig_t fc{};
+            fc.gridDim = dim3((unsigned)sms);
+            fc.blockDim = dim3(kE8FusedThreads);
+            fc.dynamicSmemBytes = kFusedCap;
+            fc.stream = s;
+            cudaLaunchAttribute fa[1];
+            fa[0].id = cudaLaunchAttributeCooperative;
+            fa[0].val.cooperative = 1;
+            fc.attrs = fa;
+            fc.numAttrs = 1;
+            return cudaLaunchKernelEx(&fc, e4m3_fused_kernel<SRC>,
+                                      reinterpret_cast<const uint8_t *>(x), n,
+                                      reinterpret_cast<float *>(ws), codes, scale_out,
+                                      device_status_ptr());
+        }
+    }
     if (!static_amax) {
         const int64_t nbytes = n * Src<SRC>::kBytes;
         int g = sms < kAmaxPartials ? sms : kAmaxPartials;

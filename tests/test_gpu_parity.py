@@ -510,13 +510,16 @@ def test_sync_status_clean():
 def _gpu_e4m3(x: np.ndarray, amax=None):
     q = nv.quantize_e4m3(dev_tensor(x), static_amax=None if amax is None else scalar_dev(amax))
     torch.cuda.synchronize()
+    st = nv.sync_status()
+    assert st == 0, f"device status {st}"
     return q.codes.cpu().numpy(), float(q.scale.cpu()[0])
 
 
 @pytest.mark.parametrize("rows,cols", [(1, 8), (3, 37), (1, 5), (64, 3072), (257, 1000),
-                                       (4096, 3072)])
+                                       (4096, 3072), (2050, 3104), (2731, 3072), (2731, 3073)])
 @pytest.mark.parametrize("kind", ["f32", "bf16"])
 def test_quantize_e4m3_matches_oracle(rows, cols, kind):
+    # 16 MB and up (n a multiple of 8, within the CTAs' shared memory): the single-pass kernel
     x = W.normal((rows, cols), 1.0, 50, rows * 7 + cols)
     x.reshape(-1)[::101] *= np.float32(40.0)   # a spread of magnitudes, subnormal codes too
     x.reshape(-1)[1::89] *= np.float32(1e-5)
@@ -539,9 +542,13 @@ def test_quantize_e4m3_static_amax(amax):
     assert s == rs and np.array_equal(codes, rc)
 
 
-def test_quantize_e4m3_all_zero():
-    codes, s = _gpu_e4m3(np.zeros((7, 24), np.float32))
-    assert s == 0.0 and not codes.any()
+@pytest.mark.parametrize("shape", [(7, 24), (4096, 3072)])
+def test_quantize_e4m3_all_zero(shape):
+    x = np.zeros(shape, np.float32)
+    x.reshape(-1)[1::3] = -0.0
+    codes, s = _gpu_e4m3(W.to_bf16_bits(x))
+    assert s == 0.0
+    assert np.array_equal(codes, O.quantize_e4m3(W.to_bf16_bits(x))[0])  # sign-only codes
 
 
 def _e4m3_linear(M, N, K, out_dtype, seed):

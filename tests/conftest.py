@@ -27,3 +27,19 @@ def read_golden(name):
 
 def golden_dict(name):
     return {r[0]: r[1] for r in read_golden(name)}
+
+
+@pytest.fixture(autouse=True)
+def _device_status_clean(request):
+    """After every GPU test: the library's device status word is clean (a bounded wait that
+    gave up inside any kernel of the test would otherwise go unnoticed)."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import nvfp4_block_scaled_14_b200 as nv
+    torch.cuda.synchronize()
+    st = nv.sync_status()
+    assert st == 0, f"device status {st} left by the test"

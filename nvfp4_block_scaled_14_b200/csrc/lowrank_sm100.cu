@@ -214,7 +214,17 @@ __global__ void __launch_bounds__(kDnThreads, 1)
             tc_fence_after();
             fence_proxy_async_smem();
             const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-            for (int c = 0; c < r; c += 16) {
+            int c = 0;
+            for (; c + 32 <= r; c += 32) { // two 16-column loads per wait
+                uint32_t v[32];
+                tmem_ld_32x32b_x16(trow + (uint32_t)c, v);
+                tmem_ld_32x32b_x16(trow + (uint32_t)c + 16u, v + 16);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    sts128(prow + (uint32_t)((c + j) * 4), v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+            if (c < r) { // r % 32 == 16
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(trow + (uint32_t)c, v);
                 tmem_ld_wait();
@@ -243,22 +253,30 @@ __global__ void __launch_bounds__(kDnThreads, 1)
             if (m >= p.M)
                 continue;
             const uint32_t off = base + (uint32_t)((lr * (r + 4) + c) * 4);
+            // every rank's loads in flight before the sum (one remote round trip, not S)
+            float4 lo[kDnMaxSplit], hi[kDnMaxSplit];
+#pragma unroll
+            for (int s = 0; s < kDnMaxSplit; ++s)
+                if (s < (int)S) {
+                    lo[s] = ld_shared_cluster_f32x4(mapa_shared(off, (uint32_t)s));
+                    hi[s] = ld_shared_cluster_f32x4(mapa_shared(off + 16, (uint32_t)s));
+                }
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 acc[j] = 0.0f;
-            for (uint32_t s = 0; s < S; ++s) { // rank order: the same sum on every run
-                const float4 lo = ld_shared_cluster_f32x4(mapa_shared(off, s));
-                const float4 hi = ld_shared_cluster_f32x4(mapa_shared(off + 16, s));
-                acc[0] += lo.x;
-                acc[1] += lo.y;
-                acc[2] += lo.z;
-                acc[3] += lo.w;
-                acc[4] += hi.x;
-                acc[5] += hi.y;
-                acc[6] += hi.z;
-                acc[7] += hi.w;
-            }
+#pragma unroll
+            for (int s = 0; s < kDnMaxSplit; ++s) // rank order: the same sum on every run
+                if (s < (int)S) {
+                    acc[0] += lo[s].x;
+                    acc[1] += lo[s].y;
+                    acc[2] += lo[s].z;
+                    acc[3] += lo[s].w;
+                    acc[4] += hi[s].x;
+                    acc[5] += hi[s].y;
+                    acc[6] += hi[s].z;
+                    acc[7] += hi[s].w;
+                }
             uint4 o;
             o.x = bf16x2_bits(__fdiv_rn(acc[0], alpha), __fdiv_rn(acc[1], alpha));
             o.y = bf16x2_bits(__fdiv_rn(acc[2], alpha), __fdiv_rn(acc[3], alpha));

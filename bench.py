@@ -401,6 +401,21 @@ def cpu_baseline(seconds=10.0):
                       f"Y[0:{ms},0:{ns}] in fp64; {reps} repetitions, {dt:.3f} s each"}
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over all ranks (every rank gets it); x itself without a process group."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, ms_per_step: float, flops_per_rank_step: float) -> float:
+    """Whole-job throughput: every rank runs its own step on its own inputs (weak scaling), so
+    the job does world x the work of one rank in the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -468,10 +483,7 @@ def run_ours(args):
     gemm_ms, _ = op_timer([lambda i=i: nv.linear(qxs[i], qws[i], out=st.Y) for i in range(n_sets)])
     del qws, qxs
 
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist, dev)
 
     # e2e: host inputs in pinned memory, copies inside the timed region
     e2e_steps = max(3, min(args.steps, 50))
@@ -495,11 +507,7 @@ def run_ours(args):
         y_host.copy_(st.Y.view(torch.int16), non_blocking=True)
     b.record()
     b.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, dist, dev)
 
     rows = None
     if not args.no_extras and rank == 0:
@@ -512,7 +520,7 @@ def run_ours(args):
         return
 
     ms_step = ms_max / args.steps
-    value = world * FLOPS / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, ms_step, FLOPS)
     gemm_tf = FLOPS / (gemm_ms * 1e-3) / 1e12
     qx_bytes = M * K * (2 + 0.5 + 1 / 16) + 4
     qw_bytes = N * K * (1 + 0.5 + 1 / 16) + 4
@@ -542,7 +550,7 @@ def run_ours(args):
                      "frac": gemm_tf / fp4_peak, "traffic": traffic,
                      "peak_note": f"{peak_kind} bf16 burst {bf16} TFLOP/s x {FP4_PER_BF16} "
                                   "(nominal FP4/BF16 ratio)"},
-        "e2e": {"value": FLOPS / (e2e_ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
+        "e2e": {"value": job_tflops(world, e2e_ms, FLOPS), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(wl.W_e4m3.nbytes + wl.X_bf16.nbytes),
                 "d2h_bytes_per_step": int(M * N * 2)},
         "gpu_launches": launches_per_step(nv) * args.steps,

@@ -298,7 +298,26 @@ def extras(nv, W, dev, hbm, fp4_peak):
     nbytes = 53 * 4096 * 3072 * 2
     gbs = nbytes / (avg * 1e-3) / 1e9
     rows["calib_p999_53x4096x3072_bf16"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
-    del distinct, batches
+    # static input scales from the p99.9 percentile and from the max over the batches, each used
+    # to quantize an evaluation batch (the 54th draw) for the GEMM against a 3072x3072 NVFP4
+    # weight; error of Y against the fp64 dense product of the unquantized operands on every
+    # 64th row
+    pct, mx = nv.calib_percentile_amax(batches)
+    pct, mx = float(pct.cpu()[0]), float(mx.cpu()[0])
+    ev_host, wt_host = W.calib_batch(53), W.calib_weight()
+    ev, wt = t(ev_host), t(wt_host)
+    qwt = nv.quantize(wt)
+    sel = np.arange(0, 4096, 64)
+    dense = (W.bf16_bits_to_f32(ev_host)[sel].astype(np.float64)
+             @ W.bf16_bits_to_f32(wt_host).astype(np.float64).T)
+    cal = {"p999": pct, "max": mx, "p999_over_max": pct / mx, "max_over_p999": mx / pct,
+           "batches": "8 distinct seeded batches, each counted 53/8 times"}
+    for name, amax in (("p999", pct), ("max", mx)):
+        qa = nv.quantize(ev, static_amax=torch.tensor([amax], device=dev))
+        y = nv.linear(qa, qwt, out_dtype=torch.float32)[sel].double().cpu().numpy()
+        cal[f"rel_err_{name}"] = float(np.linalg.norm(y - dense) / np.linalg.norm(dense))
+    rows["calib_p999_53x4096x3072_bf16"]["static_scales"] = cal
+    del distinct, batches, ev, wt, qwt
 
     # --- dequantize 12288x3072 to bf16
     w1 = nv.quantize(t(W.mlp_pair(M=8).W1), linear=True)

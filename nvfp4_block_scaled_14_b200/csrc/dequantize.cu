@@ -11,7 +11,8 @@
 // l + 96: every load instruction reads contiguous codes (256 B) or scales (32 B) across the
 // warp and every pair of 16-byte stores writes a contiguous 1 KB (bf16) run; the four blocks'
 // loads, and the next step's, are in flight together, enough bytes to cover HBM latency.
-// Write-dominated, HBM-bound.
+// Write-dominated, HBM-bound. With a 32-byte-aligned output each block leaves as 256-bit
+// stores (one for bf16, two for fp32), so every store instruction covers whole sectors.
 #include "nvfp4_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -20,8 +21,16 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// Decode one block (8 code bytes, scale sb as fp32) and store its 16 values at `o`.
-template <bool BF16>
+__device__ __forceinline__ void st_v8(void *p, const uint32_t (&v)[8])
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+// Decode one block (8 code bytes, scale sb as fp32) and store its 16 values at `o` (32-byte
+// aligned when V8: 256-bit stores).
+template <bool BF16, bool V8>
 __device__ __forceinline__ void decode_store(uint2 c, float fsb, float sg, void *o)
 {
     float v[16];
@@ -41,9 +50,22 @@ __device__ __forceinline__ void decode_store(uint2 c, float fsb, float sg, void 
             __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
             p[j] = *reinterpret_cast<uint32_t *>(&h);
         }
-        uint4 *q = reinterpret_cast<uint4 *>(o);
-        q[0] = make_uint4(p[0], p[1], p[2], p[3]);
-        q[1] = make_uint4(p[4], p[5], p[6], p[7]);
+        if constexpr (V8) {
+            st_v8(o, p);
+        } else {
+            uint4 *q = reinterpret_cast<uint4 *>(o);
+            q[0] = make_uint4(p[0], p[1], p[2], p[3]);
+            q[1] = make_uint4(p[4], p[5], p[6], p[7]);
+        }
+    } else if constexpr (V8) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t u[8] = {__float_as_uint(v[8 * i]), __float_as_uint(v[8 * i + 1]),
+                                   __float_as_uint(v[8 * i + 2]), __float_as_uint(v[8 * i + 3]),
+                                   __float_as_uint(v[8 * i + 4]), __float_as_uint(v[8 * i + 5]),
+                                   __float_as_uint(v[8 * i + 6]), __float_as_uint(v[8 * i + 7])};
+            st_v8(reinterpret_cast<uint8_t *>(o) + 32 * i, u);
+        }
     } else {
         float4 *q = reinterpret_cast<float4 *>(o);
 #pragma unroll
@@ -52,7 +74,7 @@ __device__ __forceinline__ void decode_store(uint2 c, float fsb, float sg, void 
     }
 }
 
-template <bool BF16>
+template <bool BF16, bool V8>
 __global__ void __launch_bounds__(kThreads)
     dequant_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ sf_lin,
                    const float *__restrict__ global_scale, int64_t nblocks_total,
@@ -88,7 +110,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int j = 0; j < 4; ++j) {
             const int64_t b = st * 128 + lane + 32 * j;
             if (b < nblocks_total)
-                decode_store<BF16>(c[j], e4m3_to_f32(s4[j]), sg, ob + b * kOutBlk);
+                decode_store<BF16, V8>(c[j], e4m3_to_f32(s4[j]), sg, ob + b * kOutBlk);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -114,12 +136,19 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales_lin,
         g = cap;
     if (g < 1)
         g = 1;
-    if (out_bf16)
-        dequant_kernel<true><<<(unsigned)g, kThreads, 0, s>>>(codes, scales_lin, global_scale,
-                                                              nblk, out);
+    const bool v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+    if (out_bf16 && v8)
+        dequant_kernel<true, true><<<(unsigned)g, kThreads, 0, s>>>(codes, scales_lin,
+                                                                    global_scale, nblk, out);
+    else if (out_bf16)
+        dequant_kernel<true, false><<<(unsigned)g, kThreads, 0, s>>>(codes, scales_lin,
+                                                                     global_scale, nblk, out);
+    else if (v8)
+        dequant_kernel<false, true><<<(unsigned)g, kThreads, 0, s>>>(codes, scales_lin,
+                                                                     global_scale, nblk, out);
     else
-        dequant_kernel<false><<<(unsigned)g, kThreads, 0, s>>>(codes, scales_lin, global_scale,
-                                                               nblk, out);
+        dequant_kernel<false, false><<<(unsigned)g, kThreads, 0, s>>>(codes, scales_lin,
+                                                                      global_scale, nblk, out);
     return cudaGetLastError();
 }
 

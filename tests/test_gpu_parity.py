@@ -274,6 +274,30 @@ def test_dequantize_bit_exact(rows, cols):
     assert np.array_equal(b, O.dequantize(ref, "bf16"))
 
 
+@pytest.mark.parametrize("offset", [0, 16])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_dequantize_output_alignment(offset, out):
+    # a 32-byte-aligned output takes 256-bit stores, a 16-byte-aligned one 128-bit stores:
+    # both give the oracle's bits (through the C ABI, at an offset into a larger buffer)
+    rows, cols = 300, 1056
+    x = W.normal((rows, cols), 0.02, 24, rows)
+    ref = O.dequantize(O.quantize(x), out)
+    q = gpu_quantize(x)
+    esz = 4 if out == "f32" else 2
+    buf = torch.zeros(rows * cols * esz + 64, dtype=torch.uint8, device="cuda")
+    base = buf.data_ptr()
+    base += (-base) % 32 + offset
+    st = nv.nvfp4_dequantize(q.codes.data_ptr(), q.scales_lin.data_ptr(), q.global_scale.data_ptr(),
+                             rows, cols, 0 if out == "f32" else 1, base,
+                             torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    start = base - buf.data_ptr()
+    got = buf[start:start + rows * cols * esz].cpu().numpy()
+    want = ref.view(np.uint8).reshape(-1)
+    assert np.array_equal(got, want)
+
+
 # ---------------------------------------------------------------------------------------
 # GEMM
 # ---------------------------------------------------------------------------------------

@@ -570,9 +570,18 @@ __device__ __forceinline__ void encode_body(const QuantArgs &a, int bid, int nbl
     const int items = (r1 - r0) * runs;
     const uint8_t *xbase = a.x + (int64_t)r0 * row_bytes;
 
-    // item -> (row offset, first block of this lane). The quotient by multiply-high is exact
-    // or one too large (item < 2^31, runs < 2^26); one correction.
-    auto item_rb = [&](int it, int &ro, int &b0) {
+    // item -> (row offset, first block of this lane). Items are taken from the end of the
+    // CTA's rows backwards: the amax pass read the tensor front to back, so the last part of
+    // each CTA's range is the part still in L2 (for tensors too large for the fused kernel
+    // most of the re-read then hits L2). The quotient by multiply-high is exact or one too
+    // large (item < 2^31, runs < 2^26); one correction.
+    auto item_rb = [&](int it_fwd, int &ro, int &b0) {
+        if (it_fwd >= items) { // past this CTA's items: nothing to load or store
+            ro = 0;
+            b0 = nb;
+            return;
+        }
+        const int it = items - 1 - it_fwd;
         if (runs == 1) {
             ro = it;
             b0 = 2 * lane;

@@ -780,6 +780,9 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
 {
     using E = Enc<SRC>;
     constexpr bool kPair = SS >= 0;
+    // launched with programmatic dependent launch: set-up may overlap the previous kernel's
+    // tail; nothing it writes is touched before this wait
+    pdl_wait();
     __shared__ uint64_t bars[kFusedMaxChunks];
     __shared__ float s_red[NT / 32];
     __shared__ float s_red_b[NT / 32];
@@ -1066,11 +1069,13 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
             fc.blockDim = dim3(kFusedThreads);
             fc.dynamicSmemBytes = kFusedCap;
             fc.stream = s;
-            cudaLaunchAttribute fa[1];
+            cudaLaunchAttribute fa[2];
             fa[0].id = cudaLaunchAttributeCooperative;
             fa[0].val.cooperative = static_amax ? 0 : 1;
+            fa[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            fa[1].val.programmaticStreamSerializationAllowed = 1;
             fc.attrs = fa;
-            fc.numAttrs = 1;
+            fc.numAttrs = 2;
             return cudaLaunchKernelEx(&fc, fused_quantize_kernel<SRC>, qa);
         }
     }
@@ -1360,6 +1365,7 @@ __global__ void __launch_bounds__(kE8FusedThreads, 1)
                       uint8_t *__restrict__ codes, float *__restrict__ scale_out, int *status)
 {
     extern __shared__ __align__(128) uint8_t buf[];
+    pdl_wait(); // programmatic dependent launch: the previous kernel's writes are visible
     __shared__ uint64_t bars[kFusedMaxChunks];
     __shared__ float s_red[kE8FusedThreads / 32];
     __shared__ float s_s;
@@ -1492,11 +1498,13 @@ cudaError_t launch_e4m3_typed(const void *x, int64_t n, const float *static_amax
             fc.blockDim = dim3(kE8FusedThreads);
             fc.dynamicSmemBytes = kFusedCap;
             fc.stream = s;
-            cudaLaunchAttribute fa[1];
+            cudaLaunchAttribute fa[2];
             fa[0].id = cudaLaunchAttributeCooperative;
             fa[0].val.cooperative = 1;
+            fa[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            fa[1].val.programmaticStreamSerializationAllowed = 1;
             fc.attrs = fa;
-            fc.numAttrs = 1;
+            fc.numAttrs = 2;
             return cudaLaunchKernelEx(&fc, e4m3_fused_kernel<SRC>,
                                       reinterpret_cast<const uint8_t *>(x), n,
                                       reinterpret_cast<float *>(ws), codes, scale_out,
@@ -1597,11 +1605,13 @@ cudaError_t launch_fused_pair_typed(const QuantArgs &a, const QuantArgs &b, int 
     fc.blockDim = dim3(kPairThreads);
     fc.dynamicSmemBytes = kSmem;
     fc.stream = s;
-    cudaLaunchAttribute fa[1];
+    cudaLaunchAttribute fa[2];
     fa[0].id = cudaLaunchAttributeCooperative;
     fa[0].val.cooperative = coop ? 1 : 0;
+    fa[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    fa[1].val.programmaticStreamSerializationAllowed = 1;
     fc.attrs = fa;
-    fc.numAttrs = 1;
+    fc.numAttrs = 2;
     return cudaLaunchKernelEx(&fc, fused_pair_quantize_kernel<SA, SB>, a, b);
 }
 

@@ -1152,6 +1152,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     }
 
+    pdl_launch_dependents(); // all of this CTA's work is issued: the next kernel may launch
     if (threadIdx.x == 64)
         bulk_wait_group0();
     tc_fence_before();

@@ -188,6 +188,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
+            pdl_wait(); // operands come from the stream's earlier kernels
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -275,6 +276,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
     } else {
         // ------------------------------- epilogue (both CTAs, warps 2..5) -------------
         const int q = warp & 3;
+        pdl_wait(); // tensor scales (and Y's previous readers) belong to earlier kernels
         const float alpha = __fmul_rn(*p.a_scale, *p.w_scale);
         uint32_t acc_phases = 0u;
         int buf = 0;
@@ -320,6 +322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
         }
     }
 
+    pdl_launch_dependents(); // all of this CTA's work is issued: the next kernel may launch
     if (threadIdx.x == 64)
         bulk_wait_group0();
     tc_fence_before();
@@ -420,9 +423,19 @@ cudaError_t launch_linear_e4m3(const uint8_t *a, const float *a_scale, const uin
         clusters = tiles;
     if (clusters < 1)
         clusters = 1;
-    fp8_gemm_pair_kernel<<<(unsigned)(2 * clusters), kF8Threads, F8::kSmemBytes, s>>>(tmA, tmB, tmY,
-                                                                                    p);
-    return cudaGetLastError();
+    // programmatic dependent launch: set-up overlaps the previous kernel's tail; the producer
+    // and the epilogue wait for it before touching its outputs
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    cfg.blockDim = dim3(kF8Threads, 1, 1);
+    cfg.dynamicSmemBytes = F8::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fp8_gemm_pair_kernel, tmA, tmB, tmY, p);
 }
 
 } // namespace nvfp4

@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                         const __grid_constant__ CUtensorMap tmD, const DownParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
+    pdl_wait(); // programmatic dependent launch: x and the global scales come from earlier kernels
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = p.r;
     const int stage_bytes = dn_stage_bytes(r);
@@ -373,13 +374,15 @@ cudaError_t launch_lowrank_down(const void *x, const void *d, int64_t M, int64_t
     cfg.blockDim = dim3(kDnThreads, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = s;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = (unsigned)S;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, lowrank_down_kernel, tmX, tmD, p);
 }
 

@@ -110,3 +110,46 @@ def test_calibration_full_53_batches():
         assert_quant_equal(qa, ra)
         y = to_numpy_f64(nv.linear(qa, qw))
         _sampled_check(y, ra, rw, 1000, 44)
+
+
+def test_step_in_cuda_graph_matches_eager():
+    # the attention-projection step as the bench replays it: W (FP8) and X quantized in one
+    # launch, then the GEMM, captured in a CUDA graph over two input sets (the kernels overlap
+    # through programmatic dependent launch) -- bit for bit the eager results
+    wl = W.attn_proj()
+    w8 = torch.from_numpy(wl.W_e4m3).cuda()
+    s8 = torch.tensor([wl.w_scale], dtype=torch.float32, device="cuda")
+    xs = [dev_tensor(wl.X_bf16), dev_tensor(W.to_bf16_bits(W.normal((4096, 3072), 1.0, 80, 1)))]
+    ws = [w8, w8.clone()]
+    ref = []
+    for w, x in zip(ws, xs):
+        qw, qx = nv.quantize_batch([{"x": w, "fp8_scale": s8}, {"x": x}])
+        ref.append(nv.linear(qx, qw).clone())
+    qw, qx = nv.quantize_batch([{"x": ws[0], "fp8_scale": s8}, {"x": xs[0]}])
+    y = torch.empty_like(ref[0])
+    outs = [torch.empty_like(ref[0]) for _ in range(2)]
+
+    def step(i):
+        nv.quantize_batch([{"x": ws[i], "fp8_scale": s8, "out": qw}, {"x": xs[i], "out": qx}])
+        nv.linear(qx, qw, out=y)
+        outs[i].copy_(y)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(0)
+        step(1)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(0)
+        step(1)
+    for _ in range(2):
+        outs[0].zero_()
+        outs[1].zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for i in range(2):
+            assert torch.equal(outs[i].view(torch.int16), ref[i].view(torch.int16)), i
+    del g

@@ -135,6 +135,9 @@ typedef struct {
  * counterpart in the paper: the per-tensor method above, batched so that the tensors share one
  * amax launch and one encode launch (CTAs split in proportion to the bytes) and their memory
  * traffic overlaps, e.g. a weight re-quantized from FP8 and the activations of the same layer.
+ * Two tensors whose larger fits the CTAs' shared memory (up to about 28 MB) and whose smaller
+ * fits their registers (up to about 9.7 MB) are quantized in a single launch instead, each read
+ * from HBM once.
  * jobs: HOST array of njobs (1 .. NVFP4_MAX_QUANT_JOBS) descriptors, each checked as its own
  * call would be (first failure returned, nothing launched). ws: one workspace of
  * nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, ...) bytes serves the whole batch.

@@ -178,10 +178,14 @@ def quantize_batch(jobs) -> list:
     return outs
 
 
-def dequantize(q: NVFP4Tensor, out_dtype=torch.float32) -> torch.Tensor:
+def dequantize(q: NVFP4Tensor, out_dtype=torch.float32, out: torch.Tensor = None) -> torch.Tensor:
+    """fp32 / bf16 values of q [rows, cols]; out: an optional preallocated contiguous output."""
     if q.scales_lin is None:
         raise ValueError("dequantize needs the linear scales (quantize(..., linear=True))")
-    out = torch.empty((q.rows, q.cols), dtype=out_dtype, device=q.codes.device)
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=out_dtype, device=q.codes.device)
+    elif out.dtype != out_dtype or tuple(out.shape) != (q.rows, q.cols) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous [rows, cols] tensor of out_dtype")
     dt = NVFP4_F32 if out_dtype == torch.float32 else NVFP4_BF16
     st = load().nvfp4_dequantize(_ptr(q.codes), _ptr(q.scales_lin), _ptr(q.global_scale),
                                  q.rows, q.cols, dt, _ptr(out), _stream(q.codes.device))

@@ -292,7 +292,7 @@ nvfp4_status nvfp4_linear_nvfp4_out(const uint8_t *a_codes, const uint8_t *a_sca
  * A, W, a_gs, w_gs: the FP4 operands as in nvfp4_linear (A is normally nvfp4_quantize(x)).
  * x: M x K bf16, the layer's unquantized input. lr_down D: rank x K bf16; lr_up U: N x rank
  * bf16; all row-major, 16-byte aligned. y: M x N bf16.
- * How it is computed: one kernel forms T' = bf16((x . D^T) / alpha) with fp32 tensor-core
+ * How it is computed: one kernel forms T' = bf16((x . D^T) * RN(1 / alpha)) with fp32 tensor-core
  * accumulation, alpha = sgA * sgW in fp32 (1 when that product is 0), into ws; the FP4 GEMM
  * then adds T' . U^T (bf16 tensor-core MMAs) into the same fp32 accumulator as the FP4
  * product, and its epilogue multiplies by alpha and rounds to bf16. Against the branch taken

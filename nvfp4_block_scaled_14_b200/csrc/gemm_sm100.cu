@@ -2304,7 +2304,7 @@ bool plan_linear_xq(int64_t M, int64_t N, int64_t K, LinearPlan *out)
     return true;
 }
 
-// Linear layer with a BF16 low-rank branch: T' = bf16(x . D^T / alpha) into t_ws (the down
+// Linear layer with a BF16 low-rank branch: T' = bf16(x . D^T * RN(1 / alpha)) into t_ws (the down
 // kernel), then the pair GEMM with the low-rank k-tiles appended to every tile. bf16 output.
 cudaError_t launch_linear_lowrank(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gs,
                                   const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gs,

@@ -4,7 +4,7 @@
 // in native FP4 on Blackwell next to BF16 rank-128 branches, Y = FP4 product + (x . D^T) . U^T
 // with D [r x K] and U [N x r]. This file computes the branch's intermediate T = x . D^T from
 // the layer's bf16 input on the tensor cores (tcgen05 kind::f16, fp32 accumulation) and stores
-// it as bf16 divided by alpha = sgA * sgW (1 when that product is 0): the FP4 GEMM then adds
+// it as bf16 of T * RN(1 / alpha), alpha = sgA * sgW (1 when that product is 0): the FP4 GEMM then adds
 // T . U^T into its own accumulator, which its epilogue multiplies by alpha (gemm_sm100.cu,
 // nvfp4_gemm_pair_kernel with the low-rank k-tiles).
 //
@@ -14,8 +14,8 @@
 // its K range of x and D through a 4-stage TMA ring into one M128 x N=r MMA accumulator in
 // TMEM. The partial accumulators meet in shared memory: every CTA stages its partial, and
 // after a cluster barrier each CTA sums its share of the band's rows over the cluster's
-// partials in rank order (distributed shared memory, deterministic), divides by alpha, rounds
-// to bf16 and stores.
+// partials in rank order (distributed shared memory, deterministic), multiplies by 1 / alpha,
+// rounds to bf16 and stores.
 #include <cuda.h>
 #include <cstring>
 #include <mutex>
@@ -26,7 +26,10 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kDnThreads = 192; // warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 epilogue
+// warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 epilogue; all 8 warps reduce the
+// cluster's partials (globaltimer stamps put that reduce at ~4.3 us of ~13 us with 6 warps, one
+// item in flight a thread and an IEEE division per value)
+constexpr int kDnThreads = 256;
 // K split (CTAs per cluster, a power of two <= 8) and the most TMA ring stages (as many as the
 // shared memory holds, up to this). Measured on M4096 K3072 r128: a split of 4 with one CTA per
 // SM beats 8 with two CTAs per SM (3 stages each) and 8 with 4 stages; the loads are
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
         if (lane == 0)
             tc_commit(acc_full); // also after a timeout, once the issued MMAs complete
         __syncwarp();
-    } else {
+    } else if (warp < 6) {
         // epilogue: this warp's 32 TMEM lanes = rows q*32 .. q*32+31 of the band
         const int q = warp & 3;
         const int row = q * 32 + lane;
@@ -244,46 +247,62 @@ __global__ void __launch_bounds__(kDnThreads, 1)
         float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
         if (alpha == 0.0f)
             alpha = 1.0f; // the FP4 product is zero then; the GEMM scales by 1 as well
+        const float ralpha = __frcp_rn(alpha);
         const int rows_per = 128 / (int)S;
         const int v8 = r / 8;
+        const int nitems = rows_per * v8;
         const uint32_t base = smem_u32(smem);
-        for (int idx = threadIdx.x; idx < rows_per * v8; idx += kDnThreads) {
-            const int lr = (int)rank * rows_per + idx / v8;
-            const int c = (idx % v8) * 8;
-            const int64_t m = band * 128 + lr;
-            if (m >= p.M)
-                continue;
-            const uint32_t off = base + (uint32_t)((lr * (r + 4) + c) * 4);
-            // every rank's loads in flight before the sum (one remote round trip, not S)
-            float4 lo[kDnMaxSplit], hi[kDnMaxSplit];
+        // two items a thread per pass, every rank's loads of both in flight before the sums
+        for (int i0 = threadIdx.x; i0 < nitems; i0 += 2 * kDnThreads) {
+            float4 lo[2][kDnMaxSplit], hi[2][kDnMaxSplit];
 #pragma unroll
-            for (int s = 0; s < kDnMaxSplit; ++s)
-                if (s < (int)S) {
-                    lo[s] = ld_shared_cluster_f32x4(mapa_shared(off, (uint32_t)s));
-                    hi[s] = ld_shared_cluster_f32x4(mapa_shared(off + 16, (uint32_t)s));
-                }
-            float acc[8];
+            for (int h = 0; h < 2; ++h) {
+                const int idx = i0 + h * kDnThreads;
+                if (idx >= nitems)
+                    break;
+                const int lr = (int)rank * rows_per + idx / v8;
+                const uint32_t off =
+                    base + (uint32_t)((lr * (r + 4) + (idx % v8) * 8) * 4);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                acc[j] = 0.0f;
+                for (int s = 0; s < kDnMaxSplit; ++s)
+                    if (s < (int)S) {
+                        lo[h][s] = ld_shared_cluster_f32x4(mapa_shared(off, (uint32_t)s));
+                        hi[h][s] = ld_shared_cluster_f32x4(mapa_shared(off + 16, (uint32_t)s));
+                    }
+            }
 #pragma unroll
-            for (int s = 0; s < kDnMaxSplit; ++s) // rank order: the same sum on every run
-                if (s < (int)S) {
-                    acc[0] += lo[s].x;
-                    acc[1] += lo[s].y;
-                    acc[2] += lo[s].z;
-                    acc[3] += lo[s].w;
-                    acc[4] += hi[s].x;
-                    acc[5] += hi[s].y;
-                    acc[6] += hi[s].z;
-                    acc[7] += hi[s].w;
-                }
-            uint4 o;
-            o.x = bf16x2_bits(__fdiv_rn(acc[0], alpha), __fdiv_rn(acc[1], alpha));
-            o.y = bf16x2_bits(__fdiv_rn(acc[2], alpha), __fdiv_rn(acc[3], alpha));
-            o.z = bf16x2_bits(__fdiv_rn(acc[4], alpha), __fdiv_rn(acc[5], alpha));
-            o.w = bf16x2_bits(__fdiv_rn(acc[6], alpha), __fdiv_rn(acc[7], alpha));
-            *reinterpret_cast<uint4 *>(p.t + m * r + c) = o;
+            for (int h = 0; h < 2; ++h) {
+                const int idx = i0 + h * kDnThreads;
+                if (idx >= nitems)
+                    break;
+                const int lr = (int)rank * rows_per + idx / v8;
+                const int c = (idx % v8) * 8;
+                const int64_t m = band * 128 + lr;
+                if (m >= p.M)
+                    continue;
+                float acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    acc[j] = 0.0f;
+#pragma unroll
+                for (int s = 0; s < kDnMaxSplit; ++s) // rank order: the same sum on every run
+                    if (s < (int)S) {
+                        acc[0] += lo[h][s].x;
+                        acc[1] += lo[h][s].y;
+                        acc[2] += lo[h][s].z;
+                        acc[3] += lo[h][s].w;
+                        acc[4] += hi[h][s].x;
+                        acc[5] += hi[h][s].y;
+                        acc[6] += hi[h][s].z;
+                        acc[7] += hi[h][s].w;
+                    }
+                uint4 o;
+                o.x = bf16x2_bits(__fmul_rn(acc[0], ralpha), __fmul_rn(acc[1], ralpha));
+                o.y = bf16x2_bits(__fmul_rn(acc[2], ralpha), __fmul_rn(acc[3], ralpha));
+                o.z = bf16x2_bits(__fmul_rn(acc[4], ralpha), __fmul_rn(acc[5], ralpha));
+                o.w = bf16x2_bits(__fmul_rn(acc[6], ralpha), __fmul_rn(acc[7], ralpha));
+                *reinterpret_cast<uint4 *>(p.t + m * r + c) = o;
+            }
         }
     }
     __syncwarp();

@@ -113,7 +113,7 @@ cudaError_t launch_linear_xq(const LinearPlan &pl, const void *x, int x_bf16,
 // bf16 [rows x cols] row-major tensor map: box 64 columns x box_rows rows, 128B swizzle.
 bool make_bf16_kmajor_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
                           int box_rows);
-// T' [M x r] = bf16((x . D^T) / alpha), alpha = sgA * sgW (1 if that is 0); x [M x K] and
+// T' [M x r] = bf16((x . D^T) * RN(1 / alpha)), alpha = sgA * sgW (1 if that is 0); x [M x K] and
 // D [r x K] bf16, r a multiple of 16 in 16..256, K > 0.
 cudaError_t launch_lowrank_down(const void *x, const void *d, int64_t M, int64_t K, int r,
                                 const float *a_gs, const float *w_gs, void *t, cudaStream_t s,

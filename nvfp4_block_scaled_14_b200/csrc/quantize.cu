@@ -8,20 +8,25 @@
 // quantization): "Qwen-Rapid-AIO FP8 -> NVFP4", "1. Double Quantization".
 //
 // Tensors of 16 MB up to what the CTAs' shared memory holds (148 x 192 KB) take one fused
-// single-pass kernel (fused_quantize_kernel, below). Every other size takes two kernels, both
-// HBM-bound, chained by programmatic dependent launch:
+// single-pass kernel (fused_quantize_kernel, below); two tensors of a batch, the larger of that
+// size and the smaller up to what the threads' registers hold, take one fused launch together
+// (fused_pair_quantize_kernel). Every other size takes two kernels, both HBM-bound, chained by
+// programmatic dependent launch:
 //   amax_kernel   (dynamic amax only) -- one CTA per SM streams a contiguous byte range of
-//                 the tensor through a 4 x 32 KB shared-memory ring of 1-D bulk copies and
-//                 reduces max |x| with SIMD integer max on the magnitude bits (exact,
+//                 the tensor (whole 16-byte vectors) through a 4 x 32 KB shared-memory ring of
+//                 1-D bulk copies and reduces max |x| with native packed max (exact,
 //                 order-free); one partial per CTA, no atomics, nothing to zero.
-//   encode_kernel -- one CTA per SM owns a contiguous range of rows; each warp takes a
+//   encode_kernel -- one CTA per SM owns a contiguous range of rows, taken from its end
+//                 backwards (the part the amax pass left in L2 first); each warp takes a
 //                 64-block run of one row (1024 values, fully coalesced), two 16-value blocks
 //                 per lane. It loads its first items before griddepcontrol.wait, so the loads
-//                 overlap the amax kernel's tail (the tensor is then mostly in L2), reduces the
-//                 partial maxima to the global scale, and fills a 128-entry table of
-//                 1 / (E4M3(c) * sg). Per block: block amax, E4M3 scale, E2M1 codes by the
-//                 hardware cvt, a 16-byte code store (a warp writes 512 contiguous bytes) and
-//                 16-bit stores of the swizzled and / or linear scales; atom padding is zeroed.
+//                 overlap the amax kernel's tail, reduces the partial maxima to the global
+//                 scale, and fills a 128-entry table of 1 / (E4M3(c) * sg). Per block: block
+//                 amax, E4M3 scale, E2M1 codes by the hardware cvt, a 16-byte code store (a warp
+//                 writes 512 contiguous bytes) and 16-bit stores of the swizzled and / or linear
+//                 scales; atom padding is zeroed.
+// The FP8 E4M3 tensorwise quantizer at the end of the file follows the same plan (a single
+// pass for 16 MB and up, amax + encode otherwise).
 // Code-deciding arithmetic is IEEE fp32 round-to-nearest in a fixed order (__fdiv_rn,
 // __fmul_rn, __frcp_rn): sg = amax / 2688, sb = E4M3(bmax / (sg * 6)),
 // code = E2M1(x * (1 / (sb * sg))).

@@ -1,22 +1,25 @@
 #!/usr/bin/env python
 """Benchmark of the NVFP4 quantized linear layer on B200.
 
-One step = the whole hot path on the double-quant diffusion attention projection
-(W 3072x3072 stored as FP8 E4M3 with a per-tensor scale, X 4096x3072 bf16 with 0.1 %
-outlier channels): NVFP4-quantize W from FP8 (double quantization), quantize X with its
-dynamic per-tensor amax, and run the block-scaled W4A4 GEMM to a bf16 Y.
+One step = the hot path on the largest single-GPU workload, the diffusion-transformer MLP
+pair at a 64x64 latent (4096 tokens, hidden 3072, MLP 12288): quantize the activations X1
+(4096x3072 bf16, dynamic per-tensor amax) to NVFP4, GEMM1 Y1 = X1 . W1^T (N 12288, K 3072),
+quantize the GELU-like activations X2 (4096x12288 bf16, dynamic amax), GEMM2
+Y2 = X2 . W2^T (N 3072, K 12288); bf16 outputs. The weights (bf16 12288x3072 and 3072x12288)
+are quantized to NVFP4 once, before timing, as a deployed layer keeps them.
 
-The headline `value` is the linear layer's throughput in TFLOP/s (2*M*N*K per step over the
-whole step, quantization included), summed over ranks. Each rank runs its own independent
-batch (weak scaling, no collective on the data path). Inputs rotate over enough buffer sets
-that every step reads them cold from HBM (more than 3x the L2 size in flight). Steps are
-replayed from CUDA graphs (one graph per rotation of the input sets). Per-op durations come
-from CUDA events around graph loops of each op alone over the same rotating inputs, on the
-launching stream (event nodes inside the step graph would break the kernels' programmatic
-dependent launch and add ~15 us per step).
+The headline `value` is the step's throughput in TFLOP/s (2*M*N*K of both GEMMs per step
+over the whole step, activation quantization included), summed over ranks. Each rank runs its
+own independent batch (weak scaling, no collective on the data path). Inputs rotate over
+enough buffer sets that every step reads them cold from HBM (more than 3x the L2 size in
+flight). Steps are replayed from CUDA graphs (one graph per rotation of the input sets).
+Per-op durations come from CUDA events around graph loops of each op alone over the same
+rotating inputs, on the launching stream (event nodes inside the step graph would break the
+kernels' programmatic dependent launch and add ~15 us per step).
 
-The other rows of the hot path (MLP-pair GEMMs, small-M decode GEMV, p99.9 calibration,
-dequantize) are measured after the timed region and reported under "rows".
+The other rows of the hot path (the double-quant attention projection step, the MLP GEMM with
+the NVFP4-output epilogue, the small-M decode GEMV, p99.9 calibration, dequantize, the FP8
+and low-rank layers) are measured after the timed region and reported under "rows".
 
 `--impl reference` times the CPU oracle on a bounded sample of the same workload.
 """
@@ -36,16 +39,23 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# the headline workload: the MLP pair
+T, H, F = 4096, 3072, 12288
+GEMM_FLOPS = 2.0 * T * F * H          # each of the two GEMMs
+FLOPS = 2 * GEMM_FLOPS                # per step
+WORKLOAD = "dit_mlp_pair_m4096_h3072_f12288"
+# the double-quant attention projection (a row)
 M, N, K = 4096, 3072, 3072
+A_FLOPS = 2.0 * M * N * K
+A_WORKLOAD = "attn_proj_fp8w_m4096_n3072_k3072"
 LOWRANK_R = 128  # rank of the BF16 low-rank branch (FP4 layers with rank-128 BF16 branches)
-FLOPS = 2.0 * M * N * K
 METRIC = "NVFP4 GEMM TFLOPS & quantize GB/s at 1 B200 (fraction of FP4/HBM peak)"
-WORKLOAD = "attn_proj_fp8w_m4096_n3072_k3072"
 FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 ratio (4.5 / 2.25 PFLOP/s)
-# the kernel the linear layer runs for this shape (bf16 output, M > 128, one 256 x 256 tile
-# per CTA pair): the dominant kernel of the step
+# the kernel the linear layer runs for M > 128 with a bf16 output (one 256 x 256 tile per CTA
+# pair): the dominant kernel of the step (both GEMMs)
 GEMM_KERNEL = "nvfp4_gemm_pair_kernel"
+QBYTES_BF16 = 2 + 0.5 + 1 / 16        # quantize: read bf16, write codes and E4M3 scales
 
 
 def parse():
@@ -56,6 +66,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None, choices=sorted(PROFILE_CASES),
+                    help="run one op of the hot path --reps times, untimed (for ncu), and exit")
+    ap.add_argument("--reps", type=int, default=4)
     return ap.parse_args()
 
 
@@ -127,8 +140,9 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------------------
 
-class Step:
-    """Preallocated buffers of one step over several input sets."""
+class AttnStep:
+    """The double-quant attention projection step over several input sets: W (FP8 source)
+    and X (bf16, dynamic amax) quantized in one launch, then the GEMM."""
 
     def __init__(self, nv, wl, n_sets, dev):
         self.nv = nv
@@ -144,18 +158,74 @@ class Step:
 
     def run(self, i):
         nv = self.nv
-        # W (FP8 source) and X (bf16, dynamic amax) in one quantize launch, then the GEMM
         nv.quantize_batch([{"x": self.W[i], "fp8_scale": self.s8, "out": self.qw},
                            {"x": self.X[i], "out": self.qx}])
         nv.linear(self.qx, self.qw, out=self.Y)
 
 
+def bf16_dev(a, dev):
+    return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def clone_q(nv, q):
+    return nv.NVFP4Tensor(q.codes.clone(), q.scales_swz.clone(), None, q.global_scale.clone(),
+                          q.rows, q.cols)
+
+
+class MlpStep:
+    """The MLP pair over several input sets: quantize X1, GEMM1, quantize X2, GEMM2. Each set
+    holds its own X1, X2 and its own copy of the quantized weights, so every step reads all of
+    its operands from HBM."""
+
+    def __init__(self, nv, mp, n_sets, dev):
+        self.nv = nv
+        x1, x2 = bf16_dev(mp.X1, dev), bf16_dev(mp.X2, dev)
+        q1, q2 = nv.quantize(bf16_dev(mp.W1, dev)), nv.quantize(bf16_dev(mp.W2, dev))
+        self.X1 = [x1.clone() for _ in range(n_sets)]
+        self.X2 = [x2.clone() for _ in range(n_sets)]
+        self.Q1 = [clone_q(nv, q1) for _ in range(n_sets)]
+        self.Q2 = [clone_q(nv, q2) for _ in range(n_sets)]
+        del x1, x2, q1, q2
+        self.qx1 = nv.quantize(self.X1[0])
+        self.qx2 = nv.quantize(self.X2[0])
+        self.Y1 = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
+        self.Y2 = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        wq = lambda q: q.codes.numel() + q.scales_swz.numel()
+        self.set_bytes = ((self.X1[0].numel() + self.X2[0].numel()) * 2 + wq(self.Q1[0]) +
+                          wq(self.Q2[0]))
+
+    def quantize1(self, i, x=None):
+        self.nv.quantize(self.X1[i] if x is None else x, out=self.qx1)
+
+    def gemm1(self, i):
+        self.nv.linear(self.qx1, self.Q1[i], out=self.Y1)
+
+    def quantize2(self, i, x=None):
+        self.nv.quantize(self.X2[i] if x is None else x, out=self.qx2)
+
+    def gemm2(self, i, y=None):
+        self.nv.linear(self.qx2, self.Q2[i], out=self.Y2 if y is None else y)
+
+    def run(self, i):
+        self.quantize1(i)
+        self.gemm1(i)
+        self.quantize2(i)
+        self.gemm2(i)
+
+
+def quantize_launches(nv, nbytes):
+    """Kernel launches of one dynamic-amax quantize of a tensor of nbytes: the single-pass
+    kernel (one launch) from 16 MB up to what the CTAs' shared memory holds, two (amax, encode)
+    otherwise."""
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return 1 if (16 << 20) <= nbytes <= sms * 192 * 1024 else 2
+
+
 def launches_per_step(nv):
     L = nv.load()
-    ws = L.nvfp4_workspace_bytes(nv.NVFP4_OP_LINEAR, M, N, K)
-    # W and X: one launch (X held in shared memory, W streamed and re-read from L2); the GEMM
-    # (+ split-K reduce)
-    return 1 + (2 if ws > 0 else 1)
+    gemm = lambda m, n, k: 2 if L.nvfp4_workspace_bytes(nv.NVFP4_OP_LINEAR, m, n, k) > 0 else 1
+    return (quantize_launches(nv, T * H * 2) + gemm(T, F, H) +
+            quantize_launches(nv, T * F * 2) + gemm(T, H, F))
 
 
 def capture(fns):
@@ -198,77 +268,23 @@ def op_timer(fns, reps=3):
     return us / 1e3, us / 1e3
 
 
-def extras(nv, W, dev, hbm, fp4_peak):
-    """The other hot-path rows: MLP-pair GEMMs, small-M decode, calibration, dequantize."""
-    rows = {}
+def small_m_rows(nv, W, dev, hbm, Ms=(1, 8, 32, 128)):
+    """Small-M decode: W 12288x4096 packed (rotating copies larger than L2), per M: back-to-back
+    linears (plain), the same with the resident-weights flag (each call starts reading W while
+    the previous one finishes), a decode layer that quantizes the activations (dynamic amax)
+    then runs the linear, and the same layer in one call (fused for M <= 16)."""
     L2 = torch.cuda.get_device_properties(dev).L2_cache_size
-
-    def sets_for(nbytes):
-        return max(2, math.ceil(3 * L2 / max(nbytes, 1)))
-
-    # --- MLP pair (4096x3072 -> 12288 -> 3072), weights pre-quantized
-    mp = W.mlp_pair()
-    t = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-    W1, W2, X1, X2 = t(mp.W1), t(mp.W2), t(mp.X1), t(mp.X2)
-    q1, q2 = nv.quantize(W1), nv.quantize(W2)
-    n_x2 = sets_for(X2.numel() * 2)
-    X2s = [X2.clone() for _ in range(n_x2)]
-    qx2 = nv.quantize(X2)
-    qx1 = nv.quantize(X1)
-    Y1 = torch.empty((4096, 12288), dtype=torch.bfloat16, device=dev)
-    Y2 = torch.empty((4096, 3072), dtype=torch.bfloat16, device=dev)
-    avg, med = op_timer([lambda x=x: nv.quantize(x, out=qx2) for x in X2s])
-    elems = X2.numel()
-    gbs = (elems * 2 + elems / 2 + elems / 16 + 4) / (avg * 1e-3) / 1e9
-    rows["quantize_x2_bf16_4096x12288"] = {"us": avg * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
-    def clone_q(q):
-        return nv.NVFP4Tensor(q.codes.clone(), q.scales_swz.clone(), None,
-                              q.global_scale.clone(), q.rows, q.cols)
-
-    for name, a, w, y, kk, nn in [("gemm1_m4096_n12288_k3072", qx1, q1, Y1, 3072, 12288),
-                                  ("gemm2_m4096_n3072_k12288", qx2, q2, Y2, 12288, 3072)]:
-        # rotate over copies of the quantized operands so each call reads them from HBM
-        nset = sets_for(a.codes.numel() + w.codes.numel())
-        sets = [(clone_q(a), clone_q(w)) for _ in range(nset)]
-        avg, med = op_timer([lambda p=p, y=y: nv.linear(p[0], p[1], out=y) for p in sets])
-        tf = 2.0 * 4096 * nn * kk / (avg * 1e-3) / 1e12
-        rows[name] = {"us": avg * 1e3, "TFLOP/s": tf, "frac_fp4": tf / fp4_peak}
-        if name.startswith("gemm1"):
-            # the same GEMM writing GEMM2's NVFP4 operand from its epilogue (static amax of
-            # the activation), against GEMM1 in bf16 followed by the static-scale quantize
-            amax = torch.tensor([float(X2.float().abs().max())], device=dev)
-            outs = [nv.linear_nvfp4_out(p[0], p[1], amax) for p in sets]
-            for act in ("identity", "gelu_tanh"):
-                avg_f, _ = op_timer([lambda p=p, o=o: nv.linear_nvfp4_out(p[0], p[1], amax, act,
-                                                                           out=o)
-                                     for p, o in zip(sets, outs)])
-                rows[name][f"nvfp4_out_{act}_us"] = avg_f * 1e3
-            y_sets = [Y1] + [torch.empty_like(Y1) for _ in range(sets_for(Y1.numel() * 2) - 1)]
-            for yy in y_sets:
-                yy.copy_(X2[:, :12288] if X2.shape[1] >= 12288 else Y1)
-            avg_q, _ = op_timer([lambda yy=yy: nv.quantize(yy, static_amax=amax, out=qx2)
-                                 for yy in y_sets])
-            rows[name]["then_quantize_static_us"] = avg_q * 1e3
-            del outs, y_sets
-        del sets
-    del X2s, W1, W2, X1, X2, Y1, Y2, q1, q2, qx1, qx2
-    torch.cuda.empty_cache()
-
-    # --- small-M decode: W 12288x4096 packed, M in {1, 8, 32, 128}
-    dc = W.decode()
-    Wd = t(dc.W)
+    dc = W.decode(Ms=Ms)
+    Wd = bf16_dev(dc.W, dev)
     wbytes = 12288 * 4096 // 2 + 12288 * 4096 // 16
-    n_w = sets_for(wbytes)
+    n_w = max(2, math.ceil(3 * L2 / wbytes))
     qws = [nv.quantize(Wd) for _ in range(n_w)]
     small = {}
     for m, xa in dc.X.items():
-        xd = t(xa)
+        xd = bf16_dev(xa, dev)
         qa = nv.quantize(xd)
         y = torch.empty((m, 12288), dtype=torch.bfloat16, device=dev)
         row = {}
-        # back-to-back linears over the rotating weight copies; then the same with the
-        # resident-weights flag (each call starts reading W while the previous finishes);
-        # then a decode layer: quantize the activations (dynamic amax), linear (resident W)
         for key, fns in [
                 ("plain", [lambda q=q: nv.linear(qa, q, out=y) for q in qws]),
                 ("resident", [lambda q=q: nv.linear(qa, q, out=y, resident_weights=True)
@@ -277,7 +293,6 @@ def extras(nv, W, dev, hbm, fp4_peak):
                                                          nv.linear(qa, q, out=y,
                                                                    resident_weights=True))
                                             for q in qws]),
-                # the same decode layer in one call (fused for M <= 16)
                 ("linear_dynamic", [lambda q=q: nv.linear_dynamic(xd, q, out=y,
                                                                   resident_weights=True)
                                     for q in qws])]:
@@ -286,9 +301,75 @@ def extras(nv, W, dev, hbm, fp4_peak):
             row[key] = {"us": avg * 1e3, "GB/s_weights": gbs, "frac_hbm": gbs / hbm,
                         "TFLOP/s": 2.0 * m * 12288 * 4096 / (avg * 1e-3) / 1e12}
         small[f"M{m}"] = row
-    rows["small_m_n12288_k4096"] = small
     del qws, Wd
     torch.cuda.empty_cache()
+    return small
+
+
+def extras(nv, W, dev, hbm, fp4_peak, mlp):
+    """The other hot-path rows: the attention projection step, the MLP GEMM with the
+    NVFP4-output epilogue, small-M decode, calibration, dequantize, FP8 and low-rank layers."""
+    rows = {}
+    L2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def sets_for(nbytes):
+        return max(2, math.ceil(3 * L2 / max(nbytes, 1)))
+
+    t = lambda a: bf16_dev(a, dev)
+
+    # --- the double-quant attention projection: W from FP8 and X in one quantize launch, then
+    #     the GEMM, as one step; and each op alone
+    wl = W.attn_proj()
+    n_a = max(3, math.ceil(3 * L2 / (wl.W_e4m3.nbytes + wl.X_bf16.nbytes)))
+    st = AttnStep(nv, wl, n_a, dev)
+    step_ms, _ = op_timer([lambda i=i: st.run(i) for i in range(n_a)])
+    qw_ms, _ = op_timer([lambda i=i: nv.quantize_fp8(st.W[i], st.s8, out=st.qw)
+                         for i in range(n_a)])
+    qx_ms, _ = op_timer([lambda i=i: nv.quantize(st.X[i], out=st.qx) for i in range(n_a)])
+    qb_ms, _ = op_timer([lambda i=i: nv.quantize_batch([{"x": st.W[i], "fp8_scale": st.s8,
+                                                         "out": st.qw},
+                                                        {"x": st.X[i], "out": st.qx}])
+                         for i in range(n_a)])
+    qws = [nv.quantize_fp8(st.W[i], st.s8) for i in range(n_a)]
+    qxs = [nv.quantize(st.X[i]) for i in range(n_a)]
+    g_ms, _ = op_timer([lambda i=i: nv.linear(qxs[i], qws[i], out=st.Y) for i in range(n_a)])
+    qx_bytes = M * K * QBYTES_BF16 + 4
+    qw_bytes = N * K * (1 + 0.5 + 1 / 16) + 4
+    g_tf = A_FLOPS / (g_ms * 1e-3) / 1e12
+    rows[A_WORKLOAD] = {
+        "step_us": step_ms * 1e3, "step_TFLOP/s": A_FLOPS / (step_ms * 1e-3) / 1e12,
+        "gemm_us": g_ms * 1e3, "gemm_TFLOP/s": g_tf, "gemm_frac_fp4": g_tf / fp4_peak,
+        "quantize_w_fp8_us": qw_ms * 1e3, "quantize_x_bf16_us": qx_ms * 1e3,
+        "quantize_batch_w_x_us": qb_ms * 1e3,
+        "quantize_x_GB/s": qx_bytes / (qx_ms * 1e-3) / 1e9,
+        "quantize_x_frac_hbm": qx_bytes / (qx_ms * 1e-3) / 1e9 / hbm,
+        "quantize_batch_GB/s": (qx_bytes + qw_bytes) / (qb_ms * 1e-3) / 1e9,
+        "quantize_batch_frac_hbm": (qx_bytes + qw_bytes) / (qb_ms * 1e-3) / 1e9 / hbm}
+    del st, qws, qxs
+    torch.cuda.empty_cache()
+
+    # --- the MLP's GEMM1 writing GEMM2's NVFP4 operand from its epilogue (static amax of the
+    #     activation), against GEMM1 in bf16 followed by the static-scale quantize
+    amax = torch.tensor([float(mlp.X2[0].float().abs().max())], device=dev)
+    n_m = len(mlp.X1)
+    sets = list(zip([mlp.qx1] * n_m, mlp.Q1))
+    for i in range(n_m):
+        mlp.quantize1(i)
+    outs = [nv.linear_nvfp4_out(p[0], p[1], amax) for p in sets]
+    row = {}
+    for act in ("identity", "gelu_tanh"):
+        avg_f, _ = op_timer([lambda p=p, o=o: nv.linear_nvfp4_out(p[0], p[1], amax, act, out=o)
+                             for p, o in zip(sets, outs)])
+        row[f"nvfp4_out_{act}_us"] = avg_f * 1e3
+    avg_q, _ = op_timer([lambda i=i: nv.quantize(mlp.X2[i], static_amax=amax, out=mlp.qx2)
+                         for i in range(n_m)])
+    row["quantize_x2_static_us"] = avg_q * 1e3
+    rows["gemm1_m4096_n12288_k3072_nvfp4_out"] = row
+    del outs, sets
+    torch.cuda.empty_cache()
+
+    # --- small-M decode: W 12288x4096 packed, M in {1, 8, 32, 128}
+    rows["small_m_n12288_k4096"] = small_m_rows(nv, W, dev, hbm)
 
     # --- p99.9 calibration over 53 batches of 4096x3072 bf16 (8 distinct seeded batches,
     #     each read several times; 8 x 25 MB exceeds L2, so every read comes from HBM)
@@ -378,7 +459,7 @@ def extras(nv, W, dev, hbm, fp4_peak):
     nset = sets_for(M * K * 2 + N * K // 2)
     xs = [xb.clone() for _ in range(nset)]
     qxs = [nv.quantize(x) for x in xs]
-    qws = [clone_q(qw0) for _ in range(nset)]
+    qws = [clone_q(nv, qw0) for _ in range(nset)]
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     avg_p, _ = op_timer([lambda a=a, w=w: nv.linear(a, w, out=y) for a, w in zip(qxs, qws)])
     avg_l, _ = op_timer([lambda a=a, w=w, x=x: nv.linear_lowrank(a, w, x, dd, uu, out=y)
@@ -393,47 +474,58 @@ def extras(nv, W, dev, hbm, fp4_peak):
     return rows
 
 
+def oracle_sample(O, W):
+    """A bounded sample of the MLP step for the CPU oracle: the weights quantized once (as the
+    GPU step keeps them); per call, quantize X1 rows 0..63 and X2 rows 0..15 with their
+    whole-tensor amax, and compute Y1[0:64, 0:512] and Y2[0:16, 0:512] in fp64. Returns (one
+    call, its GEMM flops, a description)."""
+    mp = W.mlp_pair()
+    m1, m2, n1 = 64, 16, 512
+    amax1 = float(np.abs(W.bf16_bits_to_f32(mp.X1)).max())
+    amax2 = float(np.abs(W.bf16_bits_to_f32(mp.X2)).max())
+    qw1 = O.quantize(mp.W1[:n1])
+    qw2 = O.quantize(mp.W2[:n1])
+    x1, x2 = mp.X1[:m1].copy(), mp.X2[:m2].copy()
+
+    def call():
+        O.gemm(O.quantize(x1, amax=amax1), qw1)
+        O.gemm(O.quantize(x2, amax=amax2), qw2)
+
+    flops = 2.0 * m1 * n1 * H + 2.0 * m2 * n1 * F
+    desc = (f"quantize X1[0:{m1}] and X2[0:{m2}] (whole-tensor amax), Y1[0:{m1},0:{n1}] "
+            f"(K {H}) and Y2[0:{m2},0:{n1}] (K {F}) in fp64; weight rows 0..{n1 - 1} "
+            "quantized once")
+    return call, flops, desc
+
+
 def cpu_baseline(seconds=10.0):
-    """The oracle, as it stands, on a bounded sample of the step: quantize W rows 0..511
-    (FP8 source, with the full-tensor amax), X rows 0..63 (full-tensor amax), and the
-    64 x 512 outputs of Y in fp64. Repeated for about `seconds`; TFLOP/s of the GEMM part
-    over the whole sample time."""
+    """The oracle, as it stands, on a bounded sample of the step (oracle_sample), repeated for
+    about `seconds`; TFLOP/s of the sample's GEMM part over the whole sample time."""
     import oracle as O
     from nvfp4_block_scaled_14_b200 import workloads as W
-    wl = W.attn_proj()
-    ms, ns = 64, 512
-    x_all = wl.X_bf16
-    w8 = wl.W_e4m3
+    call, flops, desc = oracle_sample(O, W)
     reps, t0 = 0, time.time()
     while True:
-        w_f32 = O.source_to_f32(w8, wl.w_scale)
-        amax_w = float(np.abs(w_f32).max())
-        amax_x = float(np.abs(W.bf16_bits_to_f32(x_all)).max())
-        qw = O.quantize(w8[:ns], amax=amax_w, fp8_scale=wl.w_scale)
-        qx = O.quantize(x_all[:ms], amax=amax_x)
-        O.gemm(qx, qw)
+        call()
         reps += 1
         if time.time() - t0 >= seconds:
             break
     dt = (time.time() - t0) / reps
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": 2.0 * ms * ns * K / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
-            "kind": "oracle",
-            "sample": f"quantize W[0:{ns}] (fp8 source) and X[0:{ms}] with full-tensor amax, "
-                      f"Y[0:{ms},0:{ns}] in fp64; {reps} repetitions, {dt:.3f} s each"}
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{desc}; {reps} repetitions, {dt:.3f} s each"}
 
 
-def e2e_pipelined_ms(nv, st, w_host, x_host, steps):
-    """Device time per step with every step's inputs copied in from pinned host memory and its
-    output copied back, overlapped across steps as a serving loop would run them: step i+1's
-    inputs upload on one stream while step i computes on a second and step i-1's output
-    downloads on a third (two device slots for inputs and outputs, events between them)."""
+def e2e_pipelined_ms(st, x1_host, x2_host, steps):
+    """Device time per step with every step's inputs (X1, X2) copied in from pinned host
+    memory and its output Y2 copied back, overlapped across steps as a serving loop would run
+    them: step i+1's inputs upload on one stream while step i computes on a second and step
+    i-1's output downloads on a third (two device slots for inputs and outputs, events between
+    them)."""
     nslot = 2
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    wd = [st.W[k] for k in range(nslot)]
-    xd = [st.X[k] for k in range(nslot)]
-    yd = [torch.empty_like(st.Y) for _ in range(nslot)]
-    yh = [torch.empty((M, N), dtype=torch.int16).pin_memory() for _ in range(nslot)]
+    yd = [torch.empty_like(st.Y2) for _ in range(nslot)]
+    yh = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(nslot)]
     ev_in = [torch.cuda.Event() for _ in range(nslot)]
     ev_comp = [torch.cuda.Event() for _ in range(nslot)]
     ev_out = [torch.cuda.Event() for _ in range(nslot)]
@@ -443,16 +535,17 @@ def e2e_pipelined_ms(nv, st, w_host, x_host, steps):
         if i >= nslot:
             s_in.wait_event(ev_comp[k])  # step i-2 has finished reading slot k's inputs
         with torch.cuda.stream(s_in):
-            wd[k].copy_(w_host, non_blocking=True)
-            xd[k].view(torch.int16).copy_(x_host, non_blocking=True)
+            st.X1[k].view(torch.int16).copy_(x1_host, non_blocking=True)
+            st.X2[k].view(torch.int16).copy_(x2_host, non_blocking=True)
         ev_in[k].record(s_in)
         s_comp.wait_event(ev_in[k])
         if i >= nslot:
             s_comp.wait_event(ev_out[k])  # step i-2's output has left slot k
         with torch.cuda.stream(s_comp):
-            nv.quantize_batch([{"x": wd[k], "fp8_scale": st.s8, "out": st.qw},
-                               {"x": xd[k], "out": st.qx}])
-            nv.linear(st.qx, st.qw, out=yd[k])
+            st.quantize1(k)
+            st.gemm1(k)
+            st.quantize2(k)
+            st.gemm2(k, yd[k])
         ev_comp[k].record(s_comp)
         s_out.wait_event(ev_comp[k])
         with torch.cuda.stream(s_out):
@@ -507,11 +600,12 @@ def run_ours(args):
     hbm, bf16, peak_kind = peaks()
     fp4_peak = bf16 * FP4_PER_BF16
 
-    wl = W.attn_proj(x_tensor=2 + 100 * rank)
+    # every rank its own activations (its own seed), the same weights
+    mp = W.mlp_pair(x_tensor=3 + 100 * rank)
     L2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    set_bytes = wl.W_e4m3.nbytes + wl.X_bf16.nbytes
-    n_sets = max(3, math.ceil(3 * L2 / set_bytes))
-    st = Step(nv, wl, n_sets, dev)
+    act_bytes = (mp.X1.nbytes + mp.X2.nbytes)
+    n_sets = max(3, math.ceil(3 * L2 / act_bytes))
+    st = MlpStep(nv, mp, n_sets, dev)
 
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
@@ -544,46 +638,42 @@ def run_ours(args):
     del plan, full, part
 
     # per-op device durations: each op alone, over the rotating input sets
-    qw_ms, _ = op_timer([lambda i=i: nv.quantize_fp8(st.W[i], st.s8, out=st.qw)
-                         for i in range(n_sets)])
-    qx_ms, _ = op_timer([lambda i=i: nv.quantize(st.X[i], out=st.qx) for i in range(n_sets)])
-    qb_ms, _ = op_timer([lambda i=i: nv.quantize_batch([{"x": st.W[i], "fp8_scale": st.s8,
-                                                         "out": st.qw},
-                                                        {"x": st.X[i], "out": st.qx}])
-                         for i in range(n_sets)])
-    qws = [nv.quantize_fp8(st.W[i], st.s8) for i in range(n_sets)]
-    qxs = [nv.quantize(st.X[i]) for i in range(n_sets)]
-    gemm_ms, _ = op_timer([lambda i=i: nv.linear(qxs[i], qws[i], out=st.Y) for i in range(n_sets)])
-    del qws, qxs
+    for i in range(n_sets):
+        st.quantize1(i)
+    q1_ms, _ = op_timer([lambda i=i: st.quantize1(i) for i in range(n_sets)])
+    g1_ms, _ = op_timer([lambda i=i: st.gemm1(i) for i in range(n_sets)])
+    q2_ms, _ = op_timer([lambda i=i: st.quantize2(i) for i in range(n_sets)])
+    g2_ms, _ = op_timer([lambda i=i: st.gemm2(i) for i in range(n_sets)])
 
     ms_max = max_over_ranks(ms, dist, dev)
 
     # e2e: host inputs in pinned memory, copies inside the timed region
-    e2e_steps = max(3, min(args.steps, 50))
-    w_host = torch.from_numpy(wl.W_e4m3).pin_memory()
-    x_host = torch.from_numpy(wl.X_bf16.view(np.int16)).pin_memory()
-    y_host = torch.empty((M, N), dtype=torch.int16).pin_memory()
-    for _ in range(2):
-        st.W[0].copy_(w_host, non_blocking=True)
-        st.X[0].view(torch.int16).copy_(x_host, non_blocking=True)
+    e2e_steps = max(3, min(args.steps, 30))
+    x1_host = torch.from_numpy(mp.X1.view(np.int16)).pin_memory()
+    x2_host = torch.from_numpy(mp.X2.view(np.int16)).pin_memory()
+    y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
+
+    def e2e_serial_step():
+        st.X1[0].view(torch.int16).copy_(x1_host, non_blocking=True)
+        st.X2[0].view(torch.int16).copy_(x2_host, non_blocking=True)
         st.run(0)
-        y_host.copy_(st.Y.view(torch.int16), non_blocking=True)
+        y_host.copy_(st.Y2.view(torch.int16), non_blocking=True)
+
+    for _ in range(2):
+        e2e_serial_step()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for i in range(e2e_steps):
-        st.W[0].copy_(w_host, non_blocking=True)
-        st.X[0].view(torch.int16).copy_(x_host, non_blocking=True)
-        st.run(0)
-        y_host.copy_(st.Y.view(torch.int16), non_blocking=True)
+    for _ in range(e2e_steps):
+        e2e_serial_step()
     b.record()
     b.synchronize()
     e2e_serial_ms = a.elapsed_time(b) / e2e_steps
     e2e_mode = "overlapped: step i+1 uploads and step i-1 downloads while step i computes"
     try:
-        e2e_local = e2e_pipelined_ms(nv, st, w_host, x_host, e2e_steps)
+        e2e_local = e2e_pipelined_ms(st, x1_host, x2_host, e2e_steps)
     except Exception as exc:  # measured serially instead; the line says which
         print(f"e2e pipelined measurement failed ({exc}); serial copies reported",
               file=sys.stderr)
@@ -591,9 +681,13 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e2e_local, dist, dev)
     e2e_serial_ms = max_over_ranks(e2e_serial_ms, dist, dev)
 
-    rows = None
-    if not args.no_extras and rank == 0:
-        rows = extras(nv, W, dev, hbm, fp4_peak)
+    rows, small = None, None
+    if rank == 0:
+        if not args.no_extras:
+            rows = extras(nv, W, dev, hbm, fp4_peak, st)
+            small = rows["small_m_n12288_k4096"]
+        else:
+            small = small_m_rows(nv, W, dev, hbm, Ms=(8,))
 
     if dist is not None:
         dist.barrier()
@@ -603,40 +697,61 @@ def run_ours(args):
 
     ms_step = ms_max / args.steps
     value = job_tflops(world, ms_step, FLOPS)
-    gemm_tf = FLOPS / (gemm_ms * 1e-3) / 1e12
-    qx_bytes = M * K * (2 + 0.5 + 1 / 16) + 4
-    qw_bytes = N * K * (1 + 0.5 + 1 / 16) + 4
+    g1_tf = GEMM_FLOPS / (g1_ms * 1e-3) / 1e12
+    g2_tf = GEMM_FLOPS / (g2_ms * 1e-3) / 1e12
+    gemm_avg_ms = (g1_ms + g2_ms) / 2
+    gemm_tf = GEMM_FLOPS / (gemm_avg_ms * 1e-3) / 1e12
+    qb1, qb2 = T * H * QBYTES_BF16 + 4, T * F * QBYTES_BF16 + 4
+    q1_gbs, q2_gbs = qb1 / (q1_ms * 1e-3) / 1e9, qb2 / (q2_ms * 1e-3) / 1e9
     traffic = None
     tp = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if os.path.exists(tp):
         traffic = json.load(open(tp)).get(GEMM_KERNEL, {}).get(WORKLOAD)
+    m8 = small["M8"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4-e2m1",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K,
-                   "weights": "fp8 e4m3 tensorwise -> nvfp4 each step", "activations":
-                   "bf16, dynamic per-tensor amax", "out": "bf16",
+        "config": {"workload": WORKLOAD, "tokens": T, "hidden": H, "mlp": F,
+                   "gemm1": {"M": T, "N": F, "K": H}, "gemm2": {"M": T, "N": H, "K": F},
+                   "weights": "bf16 -> nvfp4 once, before timing",
+                   "activations": "bf16, dynamic per-tensor amax, quantized every step",
+                   "out": "bf16",
                    "l2": f"inputs rotate over {n_sets} buffer sets "
-                         f"({n_sets * set_bytes / 1e6:.0f} MB > 3x L2)",
+                         f"({n_sets * st.set_bytes / 1e6:.0f} MB > 3x L2)",
                    "parallelism": f"{world} independent ranks"},
-        "gemm_tflops": gemm_tf,
-        "quantize_gbs": {"x_bf16": qx_bytes / (qx_ms * 1e-3) / 1e9,
-                         "w_fp8": qw_bytes / (qw_ms * 1e-3) / 1e9,
-                         "batch_w_x": (qx_bytes + qw_bytes) / (qb_ms * 1e-3) / 1e9},
-        "op_us": {"quantize_w_fp8": qw_ms * 1e3, "quantize_x_bf16": qx_ms * 1e3,
-                  "quantize_batch_w_x": qb_ms * 1e3, "gemm": gemm_ms * 1e3},
+        "gemm_tflops": {"gemm1": g1_tf, "gemm2": g2_tf},
+        "quantize_gbs": {"x1_bf16_4096x3072": q1_gbs, "x2_bf16_4096x12288": q2_gbs},
+        "op_us": {"quantize_x1": q1_ms * 1e3, "gemm1": g1_ms * 1e3,
+                  "quantize_x2": q2_ms * 1e3, "gemm2": g2_ms * 1e3},
         "roofline": {"bound": "tensor", "kernel": GEMM_KERNEL,
                      "achieved": gemm_tf, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_tf / fp4_peak, "traffic": traffic,
+                     "per_launch": "2*4096*12288*3072 flops (both GEMMs) over the mean of the "
+                                   "two GEMMs' durations",
                      "peak_note": f"{peak_kind} bf16 burst {bf16} TFLOP/s x {FP4_PER_BF16} "
                                   "(nominal FP4/BF16 ratio)"},
+        "roofline_quantize": {
+            "bound": "hbm", "unit": "GB/s", "peak": hbm, "peak_note": f"{peak_kind} HBM copy",
+            "x1_bf16_4096x3072": {"achieved": q1_gbs, "frac": q1_gbs / hbm, "us": q1_ms * 1e3,
+                                  "kernel": "fused_quantize_kernel"},
+            "x2_bf16_4096x12288": {"achieved": q2_gbs, "frac": q2_gbs / hbm, "us": q2_ms * 1e3,
+                                   "kernel": "amax_kernel + encode_kernel"},
+            "bytes": "read 2 B + write 0.5 + 1/16 B per value"},
+        "roofline_small_m": {
+            "bound": "hbm", "unit": "GB/s", "peak": hbm, "kernel": "nvfp4_gemm_smallm_kernel",
+            "workload": "decode M8 N12288 K4096 (packed weights + scales 28.3 MB)",
+            "achieved": m8["plain"]["GB/s_weights"], "frac": m8["plain"]["frac_hbm"],
+            "us": m8["plain"]["us"],
+            "resident_weights": {"achieved": m8["resident"]["GB/s_weights"],
+                                 "frac": m8["resident"]["frac_hbm"],
+                                 "us": m8["resident"]["us"]}},
         "e2e": {"value": job_tflops(world, e2e_ms, FLOPS), "unit": "TFLOP/s",
                 "copies": e2e_mode,
                 "serial_value": job_tflops(world, e2e_serial_ms, FLOPS),
-                "h2d_bytes_per_step": int(wl.W_e4m3.nbytes + wl.X_bf16.nbytes),
-                "d2h_bytes_per_step": int(M * N * 2)},
+                "h2d_bytes_per_step": int(mp.X1.nbytes + mp.X2.nbytes),
+                "d2h_bytes_per_step": int(T * H * 2)},
         "gpu_launches": launches_per_step(nv) * args.steps,
         "clocks": clk,
     }
@@ -653,41 +768,101 @@ def run_reference(args):
         return
     import oracle as O
     from nvfp4_block_scaled_14_b200 import workloads as W
-    wl = W.attn_proj()
-    ms, ns = 16, 256
-    amax_x = float(np.abs(W.bf16_bits_to_f32(wl.X_bf16)).max())
-
-    def step():
-        amax_w = float(np.abs(O.source_to_f32(wl.W_e4m3, wl.w_scale)).max())
-        qw = O.quantize(wl.W_e4m3[:ns], amax=amax_w, fp8_scale=wl.w_scale)
-        qx = O.quantize(wl.X_bf16[:ms], amax=amax_x)
-        O.gemm(qx, qw)
-
+    call, flops, desc = oracle_sample(O, W)
     for _ in range(args.warmup):
-        step()
+        call()
     t0 = time.time()
     for _ in range(args.steps):
-        step()
+        call()
     dt = (time.time() - t0) / args.steps
-    value = 2.0 * ms * ns * K / dt / 1e12
+    value = flops / dt / 1e12
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    sample = (f"per step: quantize W[0:{ns}] (fp8 source, full-tensor amax) and X[0:{ms}], "
-              f"Y[0:{ms},0:{ns}] in fp64 over K={K}")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K},
+        "config": {"workload": WORKLOAD, "tokens": T, "hidden": H, "mlp": F},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": f"per step: {desc}"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
+def profile_case(name, reps):
+    """One op of the hot path on its workload, run `reps` times over rotating inputs, without
+    timing: the program ncu captures. Inputs are a few hundred MB at most."""
+    import nvfp4_block_scaled_14_b200 as nv
+    from nvfp4_block_scaled_14_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    nv.load()
+    if name in ("mlp_step", "quantize_x1", "quantize_x2", "gemm1", "gemm2", "nvfp4_out_gelu",
+                "nvfp4_out_identity"):
+        st = MlpStep(nv, W.mlp_pair(), 3, dev)
+        amax = torch.tensor([float(st.X2[0].float().abs().max())], device=dev)
+        outs = [nv.linear_nvfp4_out(st.qx1, st.Q1[i], amax) for i in range(3)] \
+            if name.startswith("nvfp4_out") else None
+        st.quantize1(0)
+        st.quantize2(0)
+        torch.cuda.synchronize()
+        # the GEMM cases launch only their own GEMM (after the operands' quantize above)
+        op3 = {"mlp_step": st.run, "quantize_x1": st.quantize1, "gemm1": st.gemm1,
+              "quantize_x2": st.quantize2, "gemm2": st.gemm2,
+              "nvfp4_out_gelu": lambda i: nv.linear_nvfp4_out(st.qx1, st.Q1[i], amax,
+                                                              "gelu_tanh", out=outs[i]),
+              "nvfp4_out_identity": lambda i: nv.linear_nvfp4_out(st.qx1, st.Q1[i], amax,
+                                                                  "identity", out=outs[i])}[name]
+        op = lambda i: op3(i % 3)
+    elif name in ("smallm_m8", "smallm_m8_resident", "linear_dynamic_m8"):
+        dc = W.decode(Ms=(8,))
+        wd = bf16_dev(dc.W, dev)
+        qws = [nv.quantize(wd) for _ in range(6)]
+        xd = bf16_dev(dc.X[8], dev)
+        qa = nv.quantize(xd)
+        y = torch.empty((8, 12288), dtype=torch.bfloat16, device=dev)
+        op = {"smallm_m8": lambda i: nv.linear(qa, qws[i % 6], out=y),
+              "smallm_m8_resident": lambda i: nv.linear(qa, qws[i % 6], out=y,
+                                                        resident_weights=True),
+              "linear_dynamic_m8": lambda i: nv.linear_dynamic(xd, qws[i % 6], out=y,
+                                                               resident_weights=True)}[name]
+    elif name == "calib":
+        distinct = [bf16_dev(W.calib_batch(b), dev) for b in range(8)]
+        batches = [distinct[b % 8] for b in range(53)]
+        op = lambda i: nv.calib_percentile_amax(batches)
+    elif name in ("attn_step", "lowrank"):
+        wl = W.attn_proj()
+        if name == "attn_step":
+            st = AttnStep(nv, wl, 3, dev)
+            op = lambda i: st.run(i % 3)
+        else:
+            xb = bf16_dev(wl.X_bf16, dev)
+            d_bits, u_bits = W.lowrank_factors(N=N, K=K, r=LOWRANK_R)
+            dd, uu = bf16_dev(d_bits, dev), bf16_dev(u_bits, dev)
+            qw = nv.quantize_fp8(torch.from_numpy(wl.W_e4m3).to(dev),
+                                 torch.tensor([wl.w_scale], dtype=torch.float32, device=dev))
+            xs = [xb.clone() for _ in range(3)]
+            qxs = [nv.quantize(x) for x in xs]
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            op = lambda i: nv.linear_lowrank(qxs[i % 3], qw, xs[i % 3], dd, uu, out=y)
+    else:
+        raise ValueError(name)
+    for i in range(reps):
+        op(i)
+    torch.cuda.synchronize()
+    assert nv.sync_status() == 0
+
+
+PROFILE_CASES = ("mlp_step", "quantize_x1", "quantize_x2", "gemm1", "gemm2", "nvfp4_out_gelu",
+                 "nvfp4_out_identity", "smallm_m8", "smallm_m8_resident", "linear_dynamic_m8",
+                 "calib", "attn_step", "lowrank")
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        profile_case(args.profile_case, args.reps)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -231,7 +231,7 @@ nvfp4_status nvfp4_linear_dynamic(const void *x, nvfp4_dtype x_dt, const uint8_t
  * overlaps (other streams, or concurrent host threads) race on the array: serialize them.
  * The first call on each device that needs the scratch resolves its address
  * (cudaGetSymbolAddress) with that device current; make that first call before any stream
- * capture.
+ * capture. A lookup that fails returns NVFP4_ERR_CUDA and is tried again by the next call.
  */
 nvfp4_status nvfp4_linear_noalloc(const uint8_t *a_codes, const uint8_t *a_scales_swz,
                                   const float *a_gs, const uint8_t *w_codes,

@@ -2372,13 +2372,14 @@ constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20; // 4 MiB
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 constexpr int kNoAllocMaxDevices = 64;
-std::once_flag g_noalloc_once[kNoAllocMaxDevices];
-void *g_noalloc_ptr[kNoAllocMaxDevices];
-cudaError_t g_noalloc_err[kNoAllocMaxDevices];
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kNoAllocMaxDevices]; // null until an address was resolved on that device
 
 // Device address of the scratch array on the current device. In host code the array's name
 // only stands for the symbol; the address kernels may use comes from cudaGetSymbolAddress,
-// resolved once per device with that device current.
+// resolved with that device current. Only a successful lookup is kept: a failed one (for
+// example a first call made while the stream is being captured) returns its error and the
+// next call tries again.
 cudaError_t noalloc_scratch(void **out)
 {
     int dev = 0;
@@ -2387,13 +2388,14 @@ cudaError_t noalloc_scratch(void **out)
         return e;
     if (dev < 0 || dev >= kNoAllocMaxDevices)
         return cudaErrorInvalidDevice;
-    std::call_once(g_noalloc_once[dev], [dev]() {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
         void *p = nullptr;
-        g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess)
+            return e;
         g_noalloc_ptr[dev] = p;
-    });
-    if (g_noalloc_err[dev] != cudaSuccess)
-        return g_noalloc_err[dev];
+    }
     *out = g_noalloc_ptr[dev];
     return cudaSuccess;
 }

@@ -96,12 +96,14 @@ class MlpPair:
     name: str = "dit_mlp_m4096_h3072_f12288"
 
 
-def mlp_pair(M=4096, H=3072, F=12288) -> MlpPair:
-    z = normal((M, F), 1.0, 3, 4)
+def mlp_pair(M=4096, H=3072, F=12288, x_tensor=3) -> MlpPair:
+    """x_tensor: the seed's tensor id of X1 (X2 takes the next one); other values give other
+    activations for the same weights."""
+    z = normal((M, F), 1.0, 3, x_tensor + 1)
     x2 = torch.nn.functional.gelu(torch.from_numpy(z)).numpy()
     return MlpPair(W1=to_bf16_bits(normal((F, H), 0.02, 3, 1)),
                    W2=to_bf16_bits(normal((H, F), 0.02, 3, 2)),
-                   X1=to_bf16_bits(normal((M, H), 1.0, 3, 3)),
+                   X1=to_bf16_bits(normal((M, H), 1.0, 3, x_tensor)),
                    X2=to_bf16_bits(x2))
 
 

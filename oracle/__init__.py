@@ -74,6 +74,7 @@ def lib():
         L.ora_linear_act_f64_sampled.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p,
                                                  ctypes.c_float, _i64, ctypes.c_int, _i64p,
                                                  _i64p, _i64, _f64p]
+        L.ora_act_f64_array.argtypes = [_f64p, _i64, ctypes.c_int, _f64p]
         L.ora_linear_quantize_out.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p,
                                               ctypes.c_float, _i64, _i64, _i64, ctypes.c_float,
                                               ctypes.c_int, _u8p, _u8p, _u8p, _f32p]
@@ -262,6 +263,14 @@ def linear_act_sampled(a: Quantized, w: Quantized, act, ms, ns) -> np.ndarray:
     lib().ora_linear_act_f64_sampled(_p(a.codes, _u8p), _p(a.scales_lin, _u8p), a.sg,
                                      _p(w.codes, _u8p), _p(w.scales_lin, _u8p), w.sg, a.cols,
                                      act, _p(ms, _i64p), _p(ns, _i64p), len(ms), _p(out, _f64p))
+    return out
+
+
+def act_array(y: np.ndarray, act) -> np.ndarray:
+    """act applied in fp64 to every value of y (e.g. the exact product from gemm)."""
+    y = np.ascontiguousarray(y, np.float64)
+    out = np.zeros(y.shape, np.float64)
+    lib().ora_act_f64_array(_p(y, _f64p), y.size, act, _p(out, _f64p))
     return out
 
 

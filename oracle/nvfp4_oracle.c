@@ -405,6 +405,14 @@ void ora_linear_act_f64_sampled(const uint8_t *a_codes, const uint8_t *a_sc, flo
                          act);
 }
 
+/* act applied in fp64 to each of n values (y = an exact product from ora_gemm_f64, whose
+ * scaling sgA * sgW * acc is the same expression as above). */
+void ora_act_f64_array(const double *y, int64_t n, int act, double *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = act_f64(y[i], act);
+}
+
 /* The fused layer's NVFP4 output [M x N]: y as above, v = act(y) in fp32, quantized with the
  * static amax. Returns 0, or -1 if N is not a multiple of 16, -2 on allocation failure. */
 int ora_linear_quantize_out(const uint8_t *a_codes, const uint8_t *a_sc, float a_sg,

@@ -1,14 +1,17 @@
 """GPU parity at the workloads' full sizes, in the launch configuration bench.py times:
-codes / scales / global scales bit-exact against the oracle over the whole tensors, GEMM
-outputs on sampled positions (the oracle computes them one by one), calibration by the
-nearest-rank property that holds at any size."""
+codes / scales / global scales bit-exact against the oracle over the whole tensors; the
+attention projection's GEMM (the CTA-pair kernel) element by element against the oracle's full
+product, the other GEMMs on sampled positions (the oracle computes them one by one);
+dequantize bit-exact over a whole 12288 x 3072 weight; calibration by the nearest-rank property
+that holds at any size."""
 import numpy as np
 import pytest
 import torch
 
 import nvfp4_block_scaled_14_b200 as nv
 import oracle as O
-from gpu_helpers import assert_quant_equal, dev_tensor, gpu_quantize, to_numpy_f64
+from gpu_helpers import (assert_gemm_close, assert_nvfp4_out_valid, assert_quant_equal,
+                         dev_tensor, gpu_quantize, scalar_dev, to_numpy_f64)
 from nvfp4_block_scaled_14_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -28,21 +31,48 @@ def _sampled_check(y, ra, rw, n_samples, seed, bf16=True, extra=()):
     ns = np.concatenate([g.integers(0, Nr, n_samples), [Nr - 1, 0] + [e[1] for e in extra]])
     ref = O.gemm_sampled(ra, rw, ms, ns)
     # tolerance from the oracle's own values (max over the samples <= max over all of Y)
-    tol = 1e-3 * np.abs(ref).max() + (np.abs(ref) * 2.0 ** -8 if bf16 else 0.0)
-    err = np.abs(y[ms, ns] - ref)
-    assert np.all(err <= tol), f"max err {err.max()} (tol {np.max(tol)})"
+    assert_gemm_close(y[ms, ns], ref, bf16, what=f"sampled {Mr}x{Nr}")
 
 
-def test_attn_proj_double_quant_full():
+@pytest.fixture(scope="module")
+def attn_proj():
+    """The attention projection's operands (W re-quantized from FP8, X bf16 with outlier
+    channels), their oracle quantization, and the oracle's full product Y = X W^T in fp64
+    (4096 x 3072 x 3072: about a minute on the host cores), shared by the tests below."""
     wl = W.attn_proj()
-    qw = gpu_quantize(wl.W_e4m3, fp8_scale=wl.w_scale)
-    qx = gpu_quantize(wl.X_bf16)
     rw = O.quantize(wl.W_e4m3, fp8_scale=wl.w_scale)
     rx = O.quantize(wl.X_bf16)
+    return wl, rx, rw, O.gemm(rx, rw)
+
+
+def test_attn_proj_double_quant_full(attn_proj):
+    # the bench's workload: both quantizations bit-exact, and every one of the 12.6 M outputs
+    # of the CTA-pair GEMM within the tolerance of the oracle's exact product
+    wl, rx, rw, ref = attn_proj
+    qw = gpu_quantize(wl.W_e4m3, fp8_scale=wl.w_scale)
+    qx = gpu_quantize(wl.X_bf16)
     assert_quant_equal(qw, rw)
     assert_quant_equal(qx, rx)
-    y = to_numpy_f64(nv.linear(qx, qw))
-    _sampled_check(y, rx, rw, 2000, 40, extra=[(4095, 3071), (128, 256), (127, 255)])
+    out = torch.full((4096, 3072), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nv.linear(qx, qw, out=out)
+    y = to_numpy_f64(out)
+    assert np.isfinite(y).all()
+    assert_gemm_close(y, ref, True, what="attention projection 4096x3072x3072")
+
+
+@pytest.mark.parametrize("act", ["identity", "gelu_tanh"])
+def test_attn_proj_nvfp4_out_every_block(attn_proj, act):
+    # the GEMM with the NVFP4-output epilogue on the same operands: all 786,432 blocks of the
+    # 4096 x 3072 output against the exact product's bounds
+    wl, rx, rw, ref = attn_proj
+    qw = gpu_quantize(wl.W_e4m3, fp8_scale=wl.w_scale)
+    qx = gpu_quantize(wl.X_bf16)
+    a_act = O.ACT_GELU_TANH if act == "gelu_tanh" else O.ACT_NONE
+    amax = 0.9 * float(np.abs(O.act_array(ref, a_act)).max())
+    out = nv.linear_nvfp4_out(qx, qw, scalar_dev(amax), act)
+    torch.cuda.synchronize()
+    assert_nvfp4_out_valid(out.codes.cpu().numpy(), out.scales_swz.cpu().numpy(),
+                           float(out.global_scale.cpu()[0]), rx, rw, ref, a_act, amax)
 
 
 def test_mlp_pair_full():
@@ -70,10 +100,8 @@ def test_decode_small_m_full():
         qa, ra = gpu_quantize(x), O.quantize(x)
         assert_quant_equal(qa, ra)
         y = to_numpy_f64(nv.linear(qa, qw))
-        if m <= 8:
-            ref = O.gemm(ra, rw)
-            tol = 1e-3 * np.abs(ref).max() + np.abs(ref) * 2.0 ** -8
-            assert np.all(np.abs(y - ref) <= tol), m
+        if m <= 32:
+            assert_gemm_close(y, O.gemm(ra, rw), True, what=f"decode M{m}")
         else:
             _sampled_check(y, ra, rw, 1500, 43 + m)
 
@@ -153,3 +181,30 @@ def test_step_in_cuda_graph_matches_eager():
         for i in range(2):
             assert torch.equal(outs[i].view(torch.int16), ref[i].view(torch.int16)), i
     del g
+
+
+@pytest.mark.parametrize("offset", [0, 16])
+def test_dequantize_full_weight(offset):
+    # the MLP's 12288 x 3072 weight, as the bench times it: every warp of the grid takes several
+    # grid-stride steps (2.36 M blocks), with the next step's loads in flight; fp32 and bf16,
+    # into a 32-byte-aligned output (256-bit stores) and a 16-byte-aligned one (128-bit stores)
+    xw = W.mlp_pair(M=8).W1
+    rows, cols = xw.shape
+    ref = O.quantize(xw)
+    q = gpu_quantize(xw)
+    assert_quant_equal(q, ref)
+    stream = torch.cuda.current_stream().cuda_stream
+    for out, esz, code in (("f32", 4, 0), ("bf16", 2, 1)):
+        want = O.dequantize(ref, out).view(np.uint8).reshape(-1)
+        buf = torch.zeros(rows * cols * esz + 64, dtype=torch.uint8, device="cuda")
+        base = buf.data_ptr()
+        base += (-base) % 32 + offset
+        assert nv.nvfp4_dequantize(q.codes.data_ptr(), q.scales_lin.data_ptr(),
+                                   q.global_scale.data_ptr(), rows, cols, code, base,
+                                   stream) == 0
+        torch.cuda.synchronize()
+        start = base - buf.data_ptr()
+        got = buf[start:start + rows * cols * esz].cpu().numpy()
+        bad = np.flatnonzero(got != want)
+        assert bad.size == 0, f"{out}: {bad.size} bytes differ, first at {bad[0]}"
+        del buf

@@ -214,11 +214,10 @@ class MlpStep:
 
 
 def quantize_launches(nv, nbytes):
-    """Kernel launches of one dynamic-amax quantize of a tensor of nbytes: the single-pass
-    kernel (one launch) from 16 MB up to what the CTAs' shared memory holds, two (amax, encode)
-    otherwise."""
-    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    return 1 if (16 << 20) <= nbytes <= sms * 192 * 1024 else 2
+    """Kernel launches of one dynamic-amax quantize of a tensor of nbytes: one from 16 MB up
+    (the single-pass kernel, or the streamed one beyond shared memory), two (amax, encode)
+    below."""
+    return 1 if nbytes >= (16 << 20) else 2
 
 
 def launches_per_step(nv):
@@ -737,7 +736,7 @@ def run_ours(args):
             "x1_bf16_4096x3072": {"achieved": q1_gbs, "frac": q1_gbs / hbm, "us": q1_ms * 1e3,
                                   "kernel": "fused_quantize_kernel"},
             "x2_bf16_4096x12288": {"achieved": q2_gbs, "frac": q2_gbs / hbm, "us": q2_ms * 1e3,
-                                   "kernel": "amax_kernel + encode_kernel"},
+                                   "kernel": "stream_quantize_kernel"},
             "bytes": "read 2 B + write 0.5 + 1/16 B per value"},
         "roofline_small_m": {
             "bound": "hbm", "unit": "GB/s", "peak": hbm, "kernel": "nvfp4_gemm_smallm_kernel",
@@ -799,9 +798,11 @@ def profile_case(name, reps):
     nv.load()
     if name in ("mlp_step", "quantize_x1", "quantize_x2", "gemm1", "gemm2", "nvfp4_out_gelu",
                 "nvfp4_out_identity"):
-        st = MlpStep(nv, W.mlp_pair(), 3, dev)
+        # one input set (~170 MB on the device): ncu saves and restores device memory around
+        # each replay pass of a captured launch, so the case keeps it small
+        st = MlpStep(nv, W.mlp_pair(), 1, dev)
         amax = torch.tensor([float(st.X2[0].float().abs().max())], device=dev)
-        outs = [nv.linear_nvfp4_out(st.qx1, st.Q1[i], amax) for i in range(3)] \
+        outs = [nv.linear_nvfp4_out(st.qx1, st.Q1[0], amax)] \
             if name.startswith("nvfp4_out") else None
         st.quantize1(0)
         st.quantize2(0)
@@ -813,7 +814,7 @@ def profile_case(name, reps):
                                                               "gelu_tanh", out=outs[i]),
               "nvfp4_out_identity": lambda i: nv.linear_nvfp4_out(st.qx1, st.Q1[i], amax,
                                                                   "identity", out=outs[i])}[name]
-        op = lambda i: op3(i % 3)
+        op = lambda i: op3(0)
     elif name in ("smallm_m8", "smallm_m8_resident", "linear_dynamic_m8"):
         dc = W.decode(Ms=(8,))
         wd = bf16_dev(dc.W, dev)

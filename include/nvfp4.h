@@ -355,6 +355,26 @@ nvfp4_status nvfp4_linear_e4m3(const uint8_t *a, const float *a_scale, const uin
 nvfp4_status nvfp4_selftest_wait_timeout(cudaStream_t stream);
 
 /*
+ * Test of the single-pass quantizers' grid-wide exchange. No counterpart in the paper. Those
+ * kernels (nvfp4_quantize of 16 MB and more with a dynamic amax, the two-tensor
+ * nvfp4_quantize_batch, nvfp4_quantize_e4m3) meet once all their CTAs have folded their
+ * share of the tensor: each CTA writes its partial maximum and a token naming the launch into
+ * a 16-byte slot of the workspace, then polls every slot until all carry that token, at most
+ * a bounded number of rounds. This call runs the exchange alone, on a cooperative grid of nblk
+ * (1..160) CTAs of one warp: CTA i contributes vals[i] (device fp32; and vals[i] / 2 as the
+ * second value); CTA skip_cta (-1: none) never arrives; CTA late_cta (-1: none) arrives after
+ * spinning late_ns nanoseconds; poll_limit bounds the rounds. If every CTA arrived, out[0..1]
+ * (device fp32) get max vals and max vals / 2; otherwise the waiting CTAs give up after
+ * poll_limit rounds, record NVFP4_ERR_TIMEOUT in the status word (see nvfp4_sync_status) and
+ * return, leaving out untouched. ws: nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, ...) bytes,
+ * any contents. Returns the launch status.
+ */
+nvfp4_status nvfp4_selftest_grid_exchange(int nblk, const float *vals, int skip_cta,
+                                          int late_cta, uint32_t late_ns, uint32_t poll_limit,
+                                          float *out, void *ws, size_t ws_bytes,
+                                          cudaStream_t stream);
+
+/*
  * Synchronize the stream, then report and clear the library's device-side status word
  * (set by a kernel whose bounded wait gave up: NVFP4_ERR_TIMEOUT). Returns NVFP4_ERR_CUDA if
  * the synchronization itself failed.

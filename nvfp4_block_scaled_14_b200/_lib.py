@@ -86,6 +86,8 @@ _SIGNATURES = {
                               _vp, _vp, _sz, _vp], _int),
     "nvfp4_linear_e4m3": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp], _int),
     "nvfp4_selftest_wait_timeout": ([_vp], _int),
+    "nvfp4_selftest_grid_exchange": ([_int, _vp, _int, _int, ctypes.c_uint32, ctypes.c_uint32,
+                                      _vp, _vp, ctypes.c_size_t, _vp], _int),
     "nvfp4_sync_status": ([_vp], _int),
 }
 

@@ -3,7 +3,10 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <thread>
+#include <unordered_map>
 
+#include "grid_exchange.cuh"
 #include "nvfp4_internal.cuh"
 
 namespace nvfp4 {
@@ -50,6 +53,66 @@ int *device_status_ptr()
     const int d = current_device();
     init_device(d);
     return g_status_ptr[d];
+}
+
+// Grid barriers of the single-pass kernels (grid_exchange.cuh): one per stream for launches
+// outside graph capture, a fresh one for every launch captured into a graph (round robin over
+// the pool). Zero when the library loads.
+constexpr int kEagerBarriers = 1024;
+constexpr int kCaptureBarriers = 7168;
+__device__ GridBarrier g_grid_barriers[kEagerBarriers + kCaptureBarriers];
+
+namespace {
+std::mutex g_barrier_mutex;
+GridBarrier *g_barrier_base[kMaxDevices];
+std::unordered_map<uint64_t, int> g_stream_barrier[kMaxDevices];
+int g_next_eager[kMaxDevices];
+int g_next_capture[kMaxDevices];
+
+GridBarrier *barrier_base(int d) // with g_barrier_mutex held
+{
+    if (!g_barrier_base[d]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_grid_barriers) != cudaSuccess)
+            return nullptr;
+        g_barrier_base[d] = reinterpret_cast<GridBarrier *>(p);
+    }
+    return g_barrier_base[d];
+}
+} // namespace
+
+GridBarrier *grid_barrier_for(cudaStream_t s)
+{
+    const int d = current_device();
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+        (void)cudaGetLastError();
+        cs = cudaStreamCaptureStatusNone;
+    }
+    std::lock_guard<std::mutex> lock(g_barrier_mutex);
+    GridBarrier *base = barrier_base(d);
+    if (!base)
+        return nullptr;
+    if (cs == cudaStreamCaptureStatusActive)
+        return base + kEagerBarriers + (g_next_capture[d]++ % kCaptureBarriers);
+    // the per-thread default stream is a different stream in every host thread
+    uint64_t key = reinterpret_cast<uint64_t>(s);
+    if (s == cudaStreamPerThread)
+        key ^= (uint64_t)std::hash<std::thread::id>()(std::this_thread::get_id()) << 8;
+    auto it = g_stream_barrier[d].find(key);
+    if (it == g_stream_barrier[d].end())
+        it = g_stream_barrier[d].emplace(key, g_next_eager[d]++ % kEagerBarriers).first;
+    return base + it->second;
+}
+
+cudaError_t reset_grid_barriers()
+{
+    const int d = current_device();
+    std::lock_guard<std::mutex> lock(g_barrier_mutex);
+    GridBarrier *base = barrier_base(d);
+    if (!base)
+        return cudaErrorInvalidValue;
+    return cudaMemset(base, 0, sizeof(GridBarrier) * (kEagerBarriers + kCaptureBarriers));
 }
 
 } // namespace nvfp4
@@ -546,6 +609,23 @@ nvfp4_status nvfp4_selftest_wait_timeout(cudaStream_t stream)
     return map_cuda(launch_wait_timeout_selftest(stream));
 }
 
+nvfp4_status nvfp4_selftest_grid_exchange(int nblk, const float *vals, int skip_cta,
+                                          int late_cta, uint32_t late_ns, uint32_t poll_limit,
+                                          float *out, void *ws, size_t ws_bytes,
+                                          cudaStream_t stream)
+{
+    nvfp4_status st;
+    if ((st = check_device()) != NVFP4_OK)
+        return st;
+    if (nblk < 1 || nblk > 160 || !vals || !out || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(vals) & 3u) || (reinterpret_cast<uintptr_t>(out) & 3u))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < quantize_ws_bytes())
+        return NVFP4_ERR_WORKSPACE;
+    return map_cuda(launch_exchange_selftest(nblk, vals, skip_cta, late_cta, late_ns, poll_limit,
+                                             out, ws, stream));
+}
+
 nvfp4_status nvfp4_sync_status(cudaStream_t stream)
 {
     if (cudaStreamSynchronize(stream) != cudaSuccess)
@@ -560,6 +640,9 @@ nvfp4_status nvfp4_sync_status(cudaStream_t stream)
         const int zero = 0;
         cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
     }
+    // a grid barrier that gave up is left unbalanced: start every barrier afresh
+    if (v == NVFP4_ERR_TIMEOUT && reset_grid_barriers() != cudaSuccess)
+        return NVFP4_ERR_CUDA;
     return (nvfp4_status)v;
 }
 

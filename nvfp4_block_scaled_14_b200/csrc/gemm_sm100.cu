@@ -195,29 +195,54 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t *v)
     }
 }
 
-// This thread's accumulator row (256 fp32 columns of its TMEM lane) x alpha -> bf16 into the
-// shared staging tile: four 128-row x 128-byte boxes, 16-byte chunks swizzled by row % 8 (the
-// TMA store's 128B swizzle). Four TMEM loads are in flight per wait.
-__device__ __forceinline__ void stage_tile_bf16(uint32_t trow, uint32_t stg, int r, float alpha)
+// 64 accumulator columns (registers v) x alpha -> bf16 into box `box` of the shared staging
+// tile: four 128-row x 128-byte boxes, 16-byte chunks swizzled by row % 8 (the TMA store's 128B
+// swizzle).
+__device__ __forceinline__ void stage_box_bf16(const uint32_t (&v)[64], uint32_t stg, int box,
+                                               int r, float alpha)
 {
-#pragma unroll 1
-    for (int c0 = 0; c0 < 256; c0 += 64) {
-        uint32_t v[64];
+    const uint32_t base = stg + box * (128 * 128) + r * 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            tmem_ld_32x32b_x16(trow + c0 + 16 * i, v + 16 * i);
-        tmem_ld_wait();
-        const uint32_t box = stg + (c0 >> 6) * (128 * 128) + r * 128;
+    for (int ch = 0; ch < 8; ++ch) {
+        uint32_t w[4];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                w[j] = pack_bf16x2(__uint_as_float(v[8 * ch + 2 * j]) * alpha,
-                                   __uint_as_float(v[8 * ch + 2 * j + 1]) * alpha);
-            sts128(box + ((ch ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
-        }
+        for (int j = 0; j < 4; ++j)
+            w[j] = pack_bf16x2(__uint_as_float(v[8 * ch + 2 * j]) * alpha,
+                               __uint_as_float(v[8 * ch + 2 * j + 1]) * alpha);
+        sts128(base + ((ch ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
     }
+}
+
+__device__ __forceinline__ void tmem_ld_64cols(uint32_t taddr, uint32_t (&v)[64])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        tmem_ld_32x32b_x16(taddr + 16 * i, v + 16 * i);
+}
+
+// This thread's accumulator row (256 fp32 columns of its TMEM lane) x alpha -> bf16 into the
+// shared staging tile, 64 columns at a time with the next 64 columns' TMEM loads in flight while
+// the current ones are converted and stored. `release` runs once every TMEM load of the row has
+// completed, before the last 64 columns are converted: the MMA warp may then start the next
+// tile while this thread finishes staging.
+template <typename Release>
+__device__ __forceinline__ void stage_tile_bf16(uint32_t trow, uint32_t stg, int r, float alpha,
+                                                Release release)
+{
+    uint32_t va[64], vb[64];
+    tmem_ld_64cols(trow, va);
+    tmem_ld_wait();
+    tmem_ld_64cols(trow + 64, vb);
+    stage_box_bf16(va, stg, 0, r, alpha);
+    tmem_ld_wait();
+    tmem_ld_64cols(trow + 128, va);
+    stage_box_bf16(vb, stg, 1, r, alpha);
+    tmem_ld_wait();
+    tmem_ld_64cols(trow + 192, vb);
+    stage_box_bf16(va, stg, 2, r, alpha);
+    tmem_ld_wait();
+    release();
+    stage_box_bf16(vb, stg, 3, r, alpha);
 }
 
 // Whole accumulator row of this thread -> bf16 pairs in registers (alpha applied).
@@ -558,11 +583,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (threadIdx.x == 64)
                         bulk_wait_group_read0();
                     named_bar_sync(1, 128);
-                    stage_tile_bf16(trow, smem_u32(smem + C::kOffStaging), q * 32 + lane, alpha);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(acc_empty); // accumulator free: next tile's MMAs may start
+                    stage_tile_bf16(trow, smem_u32(smem + C::kOffStaging), q * 32 + lane, alpha,
+                                    [&]() {
+                                        tc_fence_before();
+                                        __syncwarp();
+                                        if (lane == 0) // next tile's MMAs may start
+                                            mbar_arrive(acc_empty);
+                                    });
                     fence_proxy_async_smem();
                     named_bar_sync(1, 128);
                     if (threadIdx.x == 64) {
@@ -1131,11 +1158,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (threadIdx.x == 64)
                 bulk_wait_group_read0();
             named_bar_sync(1, 128);
-            stage_tile_bf16(trow, smem_u32(smem + C::kOffStaging), q * 32 + lane, alpha);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive_remote(leader_acc_empty); // this CTA's accumulator is drained
+            stage_tile_bf16(trow, smem_u32(smem + C::kOffStaging), q * 32 + lane, alpha, [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_remote(leader_acc_empty); // this CTA's accumulator is read
+            });
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (threadIdx.x == 64) {

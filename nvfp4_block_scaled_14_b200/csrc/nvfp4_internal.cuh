@@ -47,6 +47,10 @@ cudaError_t launch_quantize_batch(const QuantJob *jobs, int njobs, void *ws, cud
 
 // Launches a kernel whose bounded wait cannot complete (selftest.cu).
 cudaError_t launch_wait_timeout_selftest(cudaStream_t s);
+// Runs the quantizers' grid-wide exchange alone (selftest.cu).
+cudaError_t launch_exchange_selftest(int nblk, const float *vals, int skip, int late,
+                                     uint32_t late_ns, uint32_t limit, float *out, void *ws,
+                                     cudaStream_t s);
 
 // FP8 E4M3 tensorwise quantize of n values (fp32 or bf16, 16-byte aligned) into codes (16-byte
 // aligned) and the tensor scale (device fp32); ws as for launch_quantize.

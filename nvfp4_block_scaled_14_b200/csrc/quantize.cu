@@ -30,9 +30,10 @@
 // Code-deciding arithmetic is IEEE fp32 round-to-nearest in a fixed order (__fdiv_rn,
 // __fmul_rn, __frcp_rn): sg = amax / 2688, sb = E4M3(bmax / (sg * 6)),
 // code = E2M1(x * (1 / (sb * sg))).
-#include <cooperative_groups.h>
 #include <mutex>
 
+#include "encode_lean.cuh"
+#include "grid_exchange.cuh"
 #include "nvfp4_internal.cuh"
 #include "nvfp4_encode.cuh"
 #include "sm100_ptx.cuh"
@@ -58,6 +59,9 @@ constexpr int kEncThreads = 768;
 // 14.1 vs 14.9 us) and behind below (bf16 6.3 MB: 8.6 vs 7.3 us).
 constexpr int64_t kFusedMinBytes = (int64_t)16 << 20;
 constexpr uint32_t kSpinLimit = 1u << 24;
+// poll rounds of the fused kernels' grid exchange (each an L2 round trip, ~0.5-1 us): about
+// a second before a missing CTA is reported as a timeout
+constexpr uint32_t kExchangeLimit = 1u << 21;
 
 template <int SRC> struct Src;
 
@@ -147,7 +151,8 @@ struct QuantArgs {
     uint8_t *codes, *sf_swz, *sf_lin;
     float *global_scale;
     const float *partials; // one max |x| per amax CTA (dynamic amax)
-    float *partials_out;   // the fused kernel's per-CTA maxima (same workspace)
+    float *slots;          // the fused kernels' grid exchange: one slot per CTA (same workspace)
+    GridBarrier *barrier;  // ... and the launch's grid barrier (library-owned)
     int npartials;
     uint32_t nb_magic;     // ceil(2^32 / blocks per row): block / nb by multiply-high
     uint32_t runs_magic;   // ceil(2^32 / runs) for runs >= 2: item / runs by multiply-high
@@ -240,192 +245,118 @@ template <int SRC> struct Enc {
     static constexpr int kItem = kItemBlocks * kBlk;          // bytes per warp item
 };
 
-// One block of raw vectors -> 16 fp32 values (bf16 widening exact; fp8 times s8).
-template <int SRC>
-__device__ __forceinline__ void block_to_f32(const uint4 *r, float s8, float (&v)[16])
+// Maxima of one block from its raw vectors (fp8: of |e|, before the fp8 scale).
+template <int SRC> __device__ __forceinline__ float block_maximum(const uint4 *r)
 {
-    if constexpr (SRC == kSrcF32) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[4 * i] = __uint_as_float(r[i].x);
-            v[4 * i + 1] = __uint_as_float(r[i].y);
-            v[4 * i + 2] = __uint_as_float(r[i].z);
-            v[4 * i + 3] = __uint_as_float(r[i].w);
-        }
-    } else if constexpr (SRC == kSrcBF16) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const uint32_t u[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[8 * i + 2 * j] = __uint_as_float(u[j] << 16);
-                v[8 * i + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
-            }
-        }
-    } else {
-        const uint32_t u[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
-        const float2 ss = make_float2(s8, s8);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 a = __fmul2_rn(e4m3x2_to_f32x2(u[j] & 0xFFFFu), ss);
-            const float2 b = __fmul2_rn(e4m3x2_to_f32x2(u[j] >> 16), ss);
-            v[4 * j] = a.x;
-            v[4 * j + 1] = a.y;
-            v[4 * j + 2] = b.x;
-            v[4 * j + 3] = b.y;
-        }
-    }
+    if constexpr (SRC == kSrcBF16)
+        return block_absmax_bf16(r[0], r[1]);
+    else if constexpr (SRC == kSrcF32)
+        return block_absmax_f32(r);
+    else
+        return block_absmax_e4m3(r[0]);
 }
 
-// E4M3 scale byte of a block from its nv raw vectors.
+// The two code words of one block from its raw vectors, times rcp (fp8: times s8 first); zero
+// when the block's scale is zero.
 template <int SRC>
-__device__ __forceinline__ uint32_t block_scale(const uint4 *r, int nv, float s8, float sg,
-                                                float t, float rt)
+__device__ __forceinline__ uint2 block_codes(const uint4 *r, float s8, uint32_t sb, float rcp)
 {
-    uint32_t m = Src<SRC>::vec_magmax(r[0]);
-    for (int i = 1; i < nv; ++i)
-        m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(r[i]));
-    float bmax = Src<SRC>::mag_to_f32(m);
-    if constexpr (SRC == kSrcE4M3)
-        bmax = __fmul_rn(bmax, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
-    return sg > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
-}
-
-// E2M1 codes of one 16-byte vector times rcp, low nibble first: 2 (fp32), 4 (bf16) or 8
-// (fp8) bytes; all zero when the block's scale is zero.
-template <int SRC>
-__device__ __forceinline__ uint2 vec_codes(uint4 u, float s8, uint32_t sb, const float *rcp_tab)
-{
-    if (sb == 0u)
-        return make_uint2(0u, 0u);
-    constexpr int NV = 16 / Src<SRC>::kBytes;
-    float v[16];
-    const uint4 r[4] = {u, u, u, u};
-    if constexpr (SRC == kSrcF32) {
-        v[0] = __uint_as_float(u.x);
-        v[1] = __uint_as_float(u.y);
-        v[2] = __uint_as_float(u.z);
-        v[3] = __uint_as_float(u.w);
-    } else if constexpr (SRC == kSrcBF16) {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[2 * j] = __uint_as_float(w[j] << 16);
-            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
-    } else {
-        block_to_f32<SRC>(r, s8, v);
-    }
-    const float rcp = rcp_tab[sb];
-    const float2 rr = make_float2(rcp, rcp);
-    float y[16];
-#pragma unroll
-    for (int j = 0; j < NV; j += 2) {
-        const float2 q = __fmul2_rn(make_float2(v[j], v[j + 1]), rr);
-        y[j] = q.x;
-        y[j + 1] = q.y;
-    }
-    if constexpr (NV == 4) {
-        y[4] = y[5] = y[6] = y[7] = 0.0f;
-        return make_uint2(cvt_e2m1x8(y) & 0xFFFFu, 0u);
-    } else if constexpr (NV == 8) {
-        return make_uint2(cvt_e2m1x8(y), 0u);
-    } else {
-        return make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8));
-    }
-}
-
-// Maxima |x| (fp8: of |e|, before the fp8 scale) of a lane's kBpl blocks, in natural block
-// order, from its vectors read in rotated order: r[v] holds the lane's vector v ^ k (k = 0:
-// natural order; the rotation keeps each block's vectors together).
-template <int SRC>
-__device__ __forceinline__ void lane_block_max(const uint4 *r, uint32_t k, float &m0, float &m1)
-{
-    using S = Src<SRC>;
+    uint2 c;
     if constexpr (SRC == kSrcBF16) {
-        const float ma = S::mag_to_f32(mag_fold<SRC>(S::vec_magmax(r[0]), S::vec_magmax(r[1])));
-        const float mb = S::mag_to_f32(mag_fold<SRC>(S::vec_magmax(r[2]), S::vec_magmax(r[3])));
-        const bool sw = (k & 2u) != 0;
-        m0 = sw ? mb : ma;
-        m1 = sw ? ma : mb;
+        c = make_uint2(codes8_bf16(r[0], rcp), codes8_bf16(r[1], rcp));
     } else if constexpr (SRC == kSrcF32) {
-        m0 = S::mag_to_f32(mag_fold<SRC>(mag_fold<SRC>(S::vec_magmax(r[0]), S::vec_magmax(r[1])),
-                                         mag_fold<SRC>(S::vec_magmax(r[2]), S::vec_magmax(r[3]))));
+        c = make_uint2(codes4_f32(r[0], rcp) | (codes4_f32(r[1], rcp) << 16),
+                       codes4_f32(r[2], rcp) | (codes4_f32(r[3], rcp) << 16));
+    } else {
+        c = make_uint2(codes8_e4m3(r[0].x, r[0].y, s8, rcp), codes8_e4m3(r[0].z, r[0].w, s8, rcp));
+    }
+    return sb != 0u ? c : make_uint2(0u, 0u);
+}
+
+// Scale bytes of two blocks with maxima m0, m1 (fp8: of |e|; the fp8 scale applied here):
+// sb0 | sb1 << 8; all zero when sg is zero.
+template <int SRC>
+__device__ __forceinline__ uint32_t scales_of_pair(float m0, float m1, float s8, float sg, float t,
+                                                   float rt)
+{
+    if (!(sg > 0.0f))
+        return 0u;
+    if constexpr (SRC == kSrcE4M3) { // max |e| * s8 == max |e * s8| (rounding is monotone)
+        m0 = __fmul_rn(m0, s8);
+        m1 = __fmul_rn(m1, s8);
+    }
+    return scale_pair(m0, m1, t, rt);
+}
+
+// Shared-memory reads of a lane's blocks in rotated order: lane reads its vector v ^ k at step v
+// (k = (lane / 2) % 4 for bf16 / fp32 with 4 vectors a lane, (lane / 4) % 2 for fp8 with 2),
+// so the 8 lanes of a quarter-warp hit 8 different 16-byte bank groups. r[v] then holds the
+// lane's natural vector v ^ k.
+template <int SRC> __device__ __forceinline__ uint32_t lane_rotation(int lane)
+{
+    return SRC == kSrcE4M3 ? (uint32_t)(lane >> 2) & 1u : (uint32_t)(lane >> 1) & 3u;
+}
+
+// Natural-order maxima of a lane's blocks from rotated vectors (see lane_rotation).
+template <int SRC>
+__device__ __forceinline__ void lane_maxima_rot(const uint4 *r, uint32_t k, float &m0, float &m1)
+{
+    if constexpr (SRC == kSrcF32) {
+        m0 = block_absmax_f32(r); // one block: the vector order does not matter
         m1 = 0.0f;
     } else {
-        const float ma = S::mag_to_f32(S::vec_magmax(r[0]));
-        const float mb = S::mag_to_f32(S::vec_magmax(r[1]));
-        const bool sw = (k & 1u) != 0;
+        constexpr int V = Enc<SRC>::kVecs;
+        // a block's vectors stay together; the rotation's top bit swaps the two blocks
+        const float ma = block_maximum<SRC>(r), mb = block_maximum<SRC>(r + V);
+        const bool sw = SRC == kSrcE4M3 ? (k & 1u) != 0 : (k & 2u) != 0;
         m0 = sw ? mb : ma;
         m1 = sw ? ma : mb;
     }
 }
 
-// E4M3 scale byte of a block from its maximum (fp8: times s8 first).
+// Scales and natural-order code words of a lane's blocks from rotated vectors and natural
+// maxima: the codes are computed in the rotated order and put back in place with selects.
 template <int SRC>
-__device__ __forceinline__ uint32_t scale_of(float m, float s8, float sg, float t, float rt)
+__device__ __forceinline__ void lane_encode_rot(const uint4 *r, uint32_t k, float m0, float m1,
+                                                float s8, float sg, float t, float rt,
+                                                const float *rcp_tab,
+                                                uint32_t (&cw)[2 * Enc<SRC>::kBpl],
+                                                uint32_t &sb0, uint32_t &sb1)
 {
-    const float bmax = SRC == kSrcE4M3 ? __fmul_rn(m, s8) : m;
-    return sg > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
-}
-
-// Natural-order code bytes (8 per block, as 32-bit words) of a lane's blocks with natural
-// scale bytes sb0, sb1, from its vectors read in rotated order (r[v] = vector v ^ k).
-template <int SRC>
-__device__ __forceinline__ void lane_codes(const uint4 *r, uint32_t k, uint32_t sb0,
-                                           uint32_t sb1, float s8, const float *rcp_tab,
-                                           uint32_t (&cw)[2 * Enc<SRC>::kBpl])
-{
-    if constexpr (SRC == kSrcBF16) {
-        const bool sw = (k & 2u) != 0;
-        const uint32_t sa = sw ? sb1 : sb0, sbb = sw ? sb0 : sb1; // scales of r[0..1], r[2..3]
-        uint32_t c[4];
+    if constexpr (SRC == kSrcF32) {
+        sb0 = sg > 0.0f ? e4m3_of_quotient(m0, t, rt) : 0u;
+        sb1 = 0u;
+        const float rcp = rcp_tab[sb0];
+        uint32_t h[4]; // h[v]: codes of natural vector v ^ k
 #pragma unroll
         for (int v = 0; v < 4; ++v)
-            c[v] = vec_codes<SRC>(r[v], s8, v < 2 ? sa : sbb, rcp_tab).x;
-        const uint32_t a0 = (k & 1u) ? c[1] : c[0], a1 = (k & 1u) ? c[0] : c[1];
-        const uint32_t a2 = (k & 1u) ? c[3] : c[2], a3 = (k & 1u) ? c[2] : c[3];
-        cw[0] = sw ? a2 : a0;
-        cw[1] = sw ? a3 : a1;
-        cw[2] = sw ? a0 : a2;
-        cw[3] = sw ? a1 : a3;
-    } else if constexpr (SRC == kSrcF32) {
-        uint32_t h[4];
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-            h[v] = vec_codes<SRC>(r[v], s8, sb0, rcp_tab).x;
-        uint32_t o[4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            const uint32_t lo = (k & 1u) ? h[n ^ 1] : h[n];
-            const uint32_t hi = (k & 1u) ? h[n ^ 3] : h[n ^ 2];
-            o[n] = (k & 2u) ? hi : lo;
-        }
-        cw[0] = o[0] | (o[1] << 16);
-        cw[1] = o[2] | (o[3] << 16);
+            h[v] = codes4_f32(r[v], rcp);
+        const bool b0 = (k & 1u) != 0, b1 = (k & 2u) != 0;
+        const uint32_t d0 = b0 ? h[1] : h[0], d1 = b0 ? h[0] : h[1];
+        const uint32_t d2 = b0 ? h[3] : h[2], d3 = b0 ? h[2] : h[3];
+        const uint32_t o0 = b1 ? d2 : d0, o1 = b1 ? d3 : d1, o2 = b1 ? d0 : d2, o3 = b1 ? d1 : d3;
+        cw[0] = sb0 ? (o0 | (o1 << 16)) : 0u;
+        cw[1] = sb0 ? (o2 | (o3 << 16)) : 0u;
     } else {
-        const bool sw = (k & 1u) != 0;
-        const uint2 ca = vec_codes<SRC>(r[0], s8, sw ? sb1 : sb0, rcp_tab);
-        const uint2 cb = vec_codes<SRC>(r[1], s8, sw ? sb0 : sb1, rcp_tab);
+        constexpr int V = Enc<SRC>::kVecs;
+        const uint32_t s2 = scales_of_pair<SRC>(m0, m1, s8, sg, t, rt);
+        sb0 = s2 & 0xFFu;
+        sb1 = s2 >> 8;
+        const bool sw = SRC == kSrcE4M3 ? (k & 1u) != 0 : (k & 2u) != 0;
+        const uint32_t sa = sw ? sb1 : sb0, sbb = sw ? sb0 : sb1; // scales of r[0..V), r[V..2V)
+        uint2 ca = block_codes<SRC>(r, s8, sa, rcp_tab[sa]);
+        uint2 cb = block_codes<SRC>(r + V, s8, sbb, rcp_tab[sbb]);
+        if constexpr (SRC == kSrcBF16) { // within a block, the rotation's low bit swaps halves
+            if (k & 1u) {
+                ca = make_uint2(ca.y, ca.x);
+                cb = make_uint2(cb.y, cb.x);
+            }
+        }
         cw[0] = sw ? cb.x : ca.x;
         cw[1] = sw ? cb.y : ca.y;
         cw[2] = sw ? ca.x : cb.x;
         cw[3] = sw ? ca.y : cb.y;
     }
-}
-
-// Scales and codes of a lane's blocks (vectors in rotated order, see lane_block_max).
-template <int SRC>
-__device__ __forceinline__ void lane_encode(const uint4 *r, uint32_t k, float s8, float sg,
-                                            float t, float rt, const float *rcp_tab,
-                                            uint32_t (&cw)[2 * Enc<SRC>::kBpl], uint32_t &sb0,
-                                            uint32_t &sb1)
-{
-    float m0, m1;
-    lane_block_max<SRC>(r, k, m0, m1);
-    sb0 = scale_of<SRC>(m0, s8, sg, t, rt);
-    sb1 = Enc<SRC>::kBpl == 2 ? scale_of<SRC>(m1, s8, sg, t, rt) : 0u;
-    lane_codes<SRC>(r, k, sb0, sb1, s8, rcp_tab, cw);
 }
 
 // Store a lane's codes (blocks f0 .. f0 + kBpl - 1) and scales in the linear and / or
@@ -509,46 +440,6 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4 *p)
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
-}
-
-// E2M1 codes of 16 fp32 values (already multiplied by the block's 1 / (sb * sg)), low
-// nibble first.
-__device__ __forceinline__ uint2 codes16(const float (&y)[16])
-{
-    return make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8));
-}
-
-// One block from its kVecs raw vectors: the E4M3 scale byte, and the 8 code bytes. The block
-// is widened to fp32 once (fp8: times s8); its maximum |v| is taken with float max on those
-// values (one instruction per value, and the same value as the maximum of the raw magnitudes:
-// fp8 upcasting rounds monotonically), then the codes of v * (1 / (sb * sg)).
-template <int SRC>
-__device__ __forceinline__ uint32_t encode_one(const uint4 *r, float s8, float sg, float t,
-                                               float rt, const float *rcp_tab, uint2 &packed)
-{
-    float v[16];
-    block_to_f32<SRC>(r, s8, v);
-    float m[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        m[i] = fmaxf(fmaxf(fabsf(v[4 * i]), fabsf(v[4 * i + 1])),
-                     fmaxf(fabsf(v[4 * i + 2]), fabsf(v[4 * i + 3])));
-    const float bmax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-    const uint32_t sb = sg > 0.0f ? e4m3_of_quotient(bmax, t, rt) : 0u;
-    packed = make_uint2(0u, 0u);
-    if (sb != 0u) {
-        const float rcp = rcp_tab[sb];
-        const float2 rr = make_float2(rcp, rcp);
-        float y[16];
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-            const float2 q = __fmul2_rn(make_float2(v[j], v[j + 1]), rr);
-            y[j] = q.x;
-            y[j + 1] = q.y;
-        }
-        packed = codes16(y);
-    }
-    return sb;
 }
 
 // K2: encode (tensors above the fused kernel's size). One CTA per SM owns a contiguous range
@@ -662,16 +553,16 @@ __device__ __forceinline__ void encode_body(const QuantArgs &a, int bid, int nbl
     auto encode_store = [&](int ro, int b0, const uint4 (&r)[8]) {
         const int row = r0 + ro;
         uint32_t sb0 = 0, sb1 = 0;
-        uint2 p0 = make_uint2(0u, 0u), p1 = make_uint2(0u, 0u);
         if (b0 < nb) {
-            sb0 = encode_one<SRC>(r, s8, sg, t, rt, s_rcp, p0);
+            // b0 is even and nb is even (cols % 32 == 0): both blocks lie in the row
+            const uint32_t s2 = scales_of_pair<SRC>(block_maximum<SRC>(r),
+                                                    block_maximum<SRC>(r + V), s8, sg, t, rt);
+            sb0 = s2 & 0xFFu;
+            sb1 = s2 >> 8;
+            const uint2 c0 = block_codes<SRC>(r, s8, sb0, s_rcp[sb0]);
+            const uint2 c1 = block_codes<SRC>(r + V, s8, sb1, s_rcp[sb1]);
             uint8_t *c = a.codes + (int64_t)row * (a.cols >> 1) + b0 * 8;
-            if (b0 + 1 < nb) {
-                sb1 = encode_one<SRC>(r + V, s8, sg, t, rt, s_rcp, p1);
-                *reinterpret_cast<uint4 *>(c) = make_uint4(p0.x, p0.y, p1.x, p1.y);
-            } else {
-                *reinterpret_cast<uint2 *>(c) = p0;
-            }
+            *reinterpret_cast<uint4 *>(c) = make_uint4(c0.x, c0.y, c1.x, c1.y);
             if (a.sf_lin) {
                 uint8_t *l = a.sf_lin + (int64_t)row * nb + b0;
                 if (b0 + 1 < nb)
@@ -719,8 +610,8 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
 // one partial, meets the other CTAs at a grid-wide barrier (cooperative launch: all CTAs are
 // co-resident), reduces the partials to the global scale and encodes from shared memory, so
 // the tensor is read from HBM once and no second kernel is launched. Static amax: no
-// barrier, each item is encoded as soon as its copy lands. Lanes read their 64 (32) bytes
-// in an order rotated by lane so that a warp's shared-memory reads are conflict-free.
+// barrier, each item is encoded as soon as its copy lands. Each lane reads its 64 (fp8: 32)
+// contiguous bytes as 16-byte vectors in a rotated order (lane_rotation): conflict-free.
 //
 // With SS >= 0 the same launch also quantizes a second, smaller tensor b (source type SS)
 // that is held in registers: each CTA takes a contiguous range of b's blocks, every thread
@@ -749,32 +640,49 @@ __device__ __forceinline__ void pair_encode_regs(const QuantArgs &b, const uint4
     const float rt = __frcp_rn(t);
     const uint32_t nb = (uint32_t)(b.cols >> 4);
     const int apb = (int)((nb + 3) >> 2);
+    // two blocks at a time: their scales with one pair conversion (blocks past the range were
+    // loaded as zeros)
+    constexpr int STEP = BPT >= 2 ? 2 : 1;
 #pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-        const int64_t blk = bk0 + (int64_t)j * blockDim.x + threadIdx.x;
-        if (blk >= bk1)
-            continue;
-        uint2 codes;
-        const uint32_t sb = encode_one<SS>(bv + j * BV, s8, sg, t, rt, rcp_tab, codes);
-        *reinterpret_cast<uint2 *>(b.codes + blk * 8) = codes;
-        if (b.sf_lin)
-            b.sf_lin[blk] = (uint8_t)sb;
-        if (b.sf_swz) {
-            uint32_t row, c; // blk / nb by multiply-high (exact or one too large), as store_lane
-            if (b.blocks_fit32) {
-                row = __umulhi((uint32_t)blk, b.nb_magic);
-                if (row * nb > (uint32_t)blk)
-                    --row;
-                c = (uint32_t)blk - row * nb;
-            } else {
-                row = (uint32_t)(blk / nb);
-                c = (uint32_t)(blk - (int64_t)row * nb);
+    for (int j0 = 0; j0 < BPT; j0 += STEP) {
+        uint32_t sbs[STEP];
+        if constexpr (STEP == 2) {
+            const uint32_t s2 = scales_of_pair<SS>(block_maximum<SS>(bv + j0 * BV),
+                                                   block_maximum<SS>(bv + (j0 + 1) * BV), s8, sg,
+                                                   t, rt);
+            sbs[0] = s2 & 0xFFu;
+            sbs[1] = s2 >> 8;
+        } else {
+            sbs[0] = sg > 0.0f ? e4m3_of_quotient(block_maximum<SS>(bv + j0 * BV), t, rt) : 0u;
+        }
+#pragma unroll
+        for (int jj = 0; jj < STEP; ++jj) {
+            const int j = j0 + jj;
+            const int64_t blk = bk0 + (int64_t)j * blockDim.x + threadIdx.x;
+            if (blk >= bk1)
+                continue;
+            const uint32_t sb = sbs[jj];
+            const uint2 codes = block_codes<SS>(bv + j * BV, s8, sb, rcp_tab[sb]);
+            *reinterpret_cast<uint2 *>(b.codes + blk * 8) = codes;
+            if (b.sf_lin)
+                b.sf_lin[blk] = (uint8_t)sb;
+            if (b.sf_swz) {
+                uint32_t row, c; // blk / nb by multiply-high (exact or one too large)
+                if (b.blocks_fit32) {
+                    row = __umulhi((uint32_t)blk, b.nb_magic);
+                    if (row * nb > (uint32_t)blk)
+                        --row;
+                    c = (uint32_t)blk - row * nb;
+                } else {
+                    row = (uint32_t)(blk / nb);
+                    c = (uint32_t)(blk - (int64_t)row * nb);
+                }
+                uint8_t *q = b.sf_swz + swz_offset(row, c, apb);
+                q[0] = (uint8_t)sb;
+                if (c + 1 == nb) // the row's last block: the rest of its atom row is padding
+                    for (uint32_t e = (c & 3u) + 1u; e < 4u; ++e)
+                        q[e - (c & 3u)] = 0u;
             }
-            uint8_t *q = b.sf_swz + swz_offset(row, c, apb);
-            q[0] = (uint8_t)sb;
-            if (c + 1 == nb) // the row's last block: the rest of its atom row is padding
-                for (uint32_t e = (c & 3u) + 1u; e < 4u; ++e)
-                    q[e - (c & 3u)] = 0u;
         }
     }
     zero_pad_rows(b, apb, blockIdx.x, gridDim.x);
@@ -844,8 +752,7 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
     }
     __syncthreads();
     const float s8 = s_scalars[0];
-    // rotation: bf16 / fp32 lanes read 64 bytes (4 vectors), fp8 lanes 32 bytes (2 vectors)
-    const uint32_t k = SRC == kSrcE4M3 ? (uint32_t)(lane >> 2) & 1u : (uint32_t)(lane >> 1) & 3u;
+    const uint32_t k = lane_rotation<SRC>(lane);
     constexpr int NVL = E::kBpl * E::kVecs;
     constexpr int kWarps = NT / 32;
     constexpr int MIW = kFusedCap / E::kItem / kWarps; // items per warp at most
@@ -891,7 +798,7 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
                 wait_item(j);
                 uint4 r[NVL];
                 load_lane(j, r);
-                lane_block_max<SRC>(r, k, bm0[jj], bm1[jj]);
+                lane_maxima_rot<SRC>(r, k, bm0[jj], bm1[jj]);
                 lm = fmaxf(lm, fmaxf(bm0[jj], bm1[jj]));
             }
         }
@@ -901,58 +808,35 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
         if (lane == 0)
             s_red[warp] = lm;
     }
-    float g = 0.0f;
-    if (need_barrier) {
+    // the global scales: every CTA's maxima of both tensors exchanged through the workspace
+    // in one bounded grid-wide exchange (a single CTA already holds the maxima)
+    if (need_barrier)
         __syncthreads();
-        if (threadIdx.x < 32) {
-            if (!a.static_amax) {
-                g = threadIdx.x < kWarps ? s_red[threadIdx.x] : 0.0f;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
-                if (threadIdx.x == 0 && gridDim.x > 1)
-                    a.partials_out[blockIdx.x] = g;
-            }
-            if (b_dyn) {
-                float gb = threadIdx.x < kWarps ? s_red_b[threadIdx.x] : 0.0f;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    gb = fmaxf(gb, __shfl_xor_sync(0xFFFFFFFFu, gb, o));
-                if (threadIdx.x == 0)
-                    b.partials_out[blockIdx.x] = gb;
-            }
-        }
-        // every CTA's partials are visible after the barrier (a single CTA already holds
-        // the maxima)
-        if (gridDim.x > 1)
-            cooperative_groups::this_grid().sync();
-    }
-    // the global scales; the partial maxima of both tensors in one L2 round trip (gridDim <=
-    // 160: five loads a lane each)
     if (threadIdx.x < 32) {
-        const bool a_round = !a.static_amax && gridDim.x > 1;
-        float pa[5], pb[5];
-#pragma unroll
-        for (int u = 0; u < 5; ++u) {
-            const int i = threadIdx.x + 32 * u;
-            pa[u] = (a_round && i < (int)gridDim.x) ? __ldcg(a.partials_out + i) : 0.0f;
-            pb[u] = (b_dyn && i < (int)gridDim.x) ? __ldcg(b.partials_out + i) : 0.0f;
-        }
-        if (a_round) {
-            g = fmaxf(fmaxf(fmaxf(pa[0], pa[1]), fmaxf(pa[2], pa[3])), pa[4]);
+        float g = 0.0f, gb = 0.0f;
+        if (!a.static_amax) {
+            g = threadIdx.x < kWarps ? s_red[threadIdx.x] : 0.0f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
         }
-        float gb = 0.0f;
         if (b_dyn) {
-            gb = fmaxf(fmaxf(fmaxf(pb[0], pb[1]), fmaxf(pb[2], pb[3])), pb[4]);
+            gb = threadIdx.x < kWarps ? s_red_b[threadIdx.x] : 0.0f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 gb = fmaxf(gb, __shfl_xor_sync(0xFFFFFFFFu, gb, o));
-            if (SS == kSrcE4M3)
-                gb = __fmul_rn(gb, s_scalars[2]); // max |e| * s8 == max |e * s8|
         }
+        if (need_barrier && gridDim.x > 1) {
+            float ga_all, gb_all;
+            if (!grid_exchange_max(a.slots, a.barrier, (int)gridDim.x, (int)blockIdx.x, g, gb,
+                                   kExchangeLimit, ga_all, gb_all) &&
+                threadIdx.x == 0)
+                atomicExch(a.status, (int)NVFP4_ERR_TIMEOUT);
+            g = ga_all;
+            gb = gb_all;
+        }
+        if (b_dyn && SS == kSrcE4M3)
+            gb = __fmul_rn(gb, s_scalars[2]); // max |e| * s8 == max |e * s8|
         if (!a.static_amax && SRC == kSrcE4M3)
             g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
         if (threadIdx.x == 0) {
@@ -992,15 +876,13 @@ __device__ __forceinline__ void fused_body(const QuantArgs &a, const QuantArgs &
         if (a.static_amax) { // the copy may still be in flight; maxima not taken yet
             wait_item(j);
             load_lane(j, r);
-            lane_block_max<SRC>(r, k, bm0[jj], bm1[jj]);
+            lane_maxima_rot<SRC>(r, k, bm0[jj], bm1[jj]);
         } else {
             load_lane(j, r);
         }
         const int64_t f0 = (c0 + j) * E::kItemBlocks + lane * E::kBpl;
-        const uint32_t sb0 = scale_of<SRC>(bm0[jj], s8, sg, t, rt);
-        const uint32_t sb1 = E::kBpl == 2 ? scale_of<SRC>(bm1[jj], s8, sg, t, rt) : 0u;
-        uint32_t cw[2 * E::kBpl];
-        lane_codes<SRC>(r, k, sb0, sb1, s8, s_rcp, cw);
+        uint32_t cw[2 * E::kBpl], sb0, sb1;
+        lane_encode_rot<SRC>(r, k, bm0[jj], bm1[jj], s8, sg, t, rt, s_rcp, cw, sb0, sb1);
         if (f0 < nblocks)
             store_lane<SRC>(a, f0, nb, apb, cw, sb0, sb1);
     }
@@ -1021,6 +903,172 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 {
     extern __shared__ __align__(128) uint8_t buf[];
     fused_body<SA, kPairThreads, SB>(a, b, buf);
+}
+
+// Single-launch quantizer for tensors larger than the CTAs' shared memory. One CTA per SM owns
+// a contiguous range of warp items and streams it through a ring of kStreamSlots chunks (one
+// warp item per warp per chunk) with 1-D bulk copies. Dynamic amax: pass 1 folds max |x| over
+// the range front to back; the grid-wide exchange gives sg; pass 2 walks the range back to
+// front, so it starts on the chunks pass 1 left in the ring (no second read) and continues on
+// the ones read last, which L2 still holds; each warp encodes its item of the chunk (block
+// maxima, E4M3 scales, E2M1 codes) and the chunk's slot is refilled with the chunk kStreamSlots
+// further down. Static amax: pass 2 alone. The tensor leaves HBM once and one kernel runs.
+constexpr int kStreamThreads = 1024;
+constexpr int kStreamSlots = 3;
+
+template <int SRC> struct StreamCfg {
+    static constexpr int kWarps = kStreamThreads / 32;
+    static constexpr int kChunkItems = kWarps; // one warp item per warp per chunk
+    static constexpr int kChunkBytes = kChunkItems * Enc<SRC>::kItem; // 64 KB (fp8: 32 KB)
+    static constexpr int kSmem = kStreamSlots * kChunkBytes;
+};
+
+template <int SRC>
+__global__ void __launch_bounds__(kStreamThreads, 1) stream_quantize_kernel(const QuantArgs a)
+{
+    using E = Enc<SRC>;
+    using C = StreamCfg<SRC>;
+    constexpr int S = kStreamSlots;
+    constexpr int NVL = E::kBpl * E::kVecs; // 16-byte vectors of a lane's blocks
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ uint64_t full[S];
+    __shared__ float s_red[C::kWarps];
+    __shared__ float s_sg;
+    __shared__ float s_rcp[128];
+    pdl_wait(); // the tensor and the outputs belong to the stream's earlier work
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t k = lane_rotation<SRC>(lane);
+    const bool dyn = a.static_amax == nullptr;
+    const int64_t nblocks = (int64_t)a.rows * (a.cols >> 4);
+    const int64_t nitems = (nblocks + E::kItemBlocks - 1) / E::kItemBlocks;
+    const int64_t c0 = nitems * blockIdx.x / gridDim.x;
+    const int64_t c1 = nitems * (blockIdx.x + 1) / gridDim.x;
+    const int64_t byte0 = c0 * E::kItem;
+    const int64_t nbytes = max((int64_t)0, min(a.nbytes, c1 * E::kItem) - byte0);
+    const int nch = (int)((nbytes + C::kChunkBytes - 1) / C::kChunkBytes);
+    const float s8 = (SRC == kSrcE4M3 && a.fp8_scale) ? *a.fp8_scale : 1.0f;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s)
+            mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // fills issued per slot (the same count in every thread); a wait for the latest fill of
+    // slot s uses the parity of its number
+    int nfill[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s)
+        nfill[s] = 0;
+    auto issue = [&](int c) {
+        const int s = c % S;
+        if (threadIdx.x == 0) {
+            const int64_t off = (int64_t)c * C::kChunkBytes;
+            const uint32_t n = (uint32_t)min((int64_t)C::kChunkBytes, nbytes - off);
+            mbar_arrive_expect_tx(&full[s], n);
+            bulk_load_1d(ring + s * C::kChunkBytes, a.x + byte0 + off, n, &full[s]);
+        }
+#pragma unroll
+        for (int t = 0; t < S; ++t)
+            nfill[t] += t == s ? 1 : 0;
+    };
+    auto wait_chunk = [&](int c) {
+        const int s = c % S;
+        int parity = 0;
+#pragma unroll
+        for (int t = 0; t < S; ++t)
+            parity = t == s ? (nfill[t] - 1) & 1 : parity;
+        if (!mbar_wait(&full[s], (uint32_t)parity, kSpinLimit) && lane == 0)
+            atomicExch(a.status, (int)NVFP4_ERR_TIMEOUT);
+    };
+
+    float g = 0.0f;
+    if (dyn) {
+        // pass 1: max |x| over the range, front to back
+        for (int c = 0; c < min(nch, S); ++c)
+            issue(c);
+        uint32_t m = 0;
+        for (int c = 0; c < nch; ++c) {
+            wait_chunk(c);
+            const int nv = (int)(min((int64_t)C::kChunkBytes, nbytes - (int64_t)c * C::kChunkBytes) >> 4);
+            const uint32_t base = smem_u32(ring + (c % S) * C::kChunkBytes);
+            for (int i = threadIdx.x; i < nv; i += kStreamThreads)
+                m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(lds128(base + 16 * i)));
+            if (c + S < nch) {
+                __syncthreads(); // every thread is done with the slot
+                issue(c + S);
+            }
+        }
+        float f = Src<SRC>::mag_to_f32(m);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
+        if (lane == 0)
+            s_red[warp] = f;
+        __syncthreads();
+        if (warp == 0) {
+            g = s_red[lane];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
+            if (gridDim.x > 1) {
+                float unused;
+                if (!grid_exchange_max(a.slots, a.barrier, (int)gridDim.x, (int)blockIdx.x, g,
+                                       0.0f, kExchangeLimit, g, unused) &&
+                    lane == 0)
+                    atomicExch(a.status, (int)NVFP4_ERR_TIMEOUT);
+            }
+            if (SRC == kSrcE4M3)
+                g = __fmul_rn(g, s8); // max |e| * s8 == max |e * s8| (rounding is monotone)
+        }
+    } else {
+        // static amax: the last chunks first (pass 2's order)
+        for (int c = nch - 1; c >= max(0, nch - S); --c)
+            issue(c);
+        if (warp == 0)
+            g = *a.static_amax;
+    }
+    if (threadIdx.x == 0) {
+        const float sg = __fdiv_rn(g, 2688.0f); // 6 * 448
+        s_sg = sg;
+        if (blockIdx.x == 0)
+            *a.global_scale = sg;
+    }
+    __syncthreads();
+    const float sg = s_sg;
+    const float t = __fmul_rn(sg, 6.0f);
+    const float rt = __frcp_rn(t);
+    if (threadIdx.x < 128)
+        s_rcp[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_to_f32(threadIdx.x), sg));
+    __syncthreads();
+    pdl_launch_dependents(); // a dependent GEMM may set up while this grid encodes
+
+    // pass 2: encode, back to front
+    const uint32_t nb = (uint32_t)(a.cols >> 4);
+    const int apb = (int)((nb + 3) >> 2);
+    for (int c = nch - 1; c >= 0; --c) {
+        if (!dyn || c < nch - S)
+            wait_chunk(c);
+        const int64_t item = c0 + (int64_t)c * C::kChunkItems + warp;
+        const int64_t f0 = item * E::kItemBlocks + lane * E::kBpl;
+        if (item < c1 && f0 < nblocks) {
+            const uint32_t src = smem_u32(ring + (c % S) * C::kChunkBytes) + warp * E::kItem +
+                                 lane * (E::kBpl * E::kBlk);
+            uint4 r[NVL];
+#pragma unroll
+            for (int v = 0; v < NVL; ++v)
+                r[v] = lds128(src + 16 * (v ^ k));
+            float m0, m1;
+            lane_maxima_rot<SRC>(r, k, m0, m1);
+            uint32_t cw[2 * E::kBpl], sb0, sb1;
+            lane_encode_rot<SRC>(r, k, m0, m1, s8, sg, t, rt, s_rcp, cw, sb0, sb1);
+            store_lane<SRC>(a, f0, nb, apb, cw, sb0, sb1);
+        }
+        if (c - S >= 0) {
+            __syncthreads(); // every warp is done with the slot
+            issue(c - S);
+        }
+    }
+    zero_pad_rows(a, apb, blockIdx.x, gridDim.x);
 }
 
 template <int SRC>
@@ -1047,7 +1095,7 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
     const uint64_t runs = (nb + 63) / 64;
     qa.runs_magic = runs > 1 ? (uint32_t)((((uint64_t)1 << 32) + runs - 1) / runs) : 0u;
     qa.status = device_status_ptr();
-    qa.partials_out = reinterpret_cast<float *>(ws);
+    qa.slots = reinterpret_cast<float *>(ws);
     // fused single pass when every CTA's share fits in its shared memory
     {
         using E = Enc<SRC>;
@@ -1057,8 +1105,10 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
             g = sms;
         if (g < 1)
             g = 1;
-        if ((nitems + g - 1) / g * E::kItem <= kFusedCap && g <= 160 &&
+        if ((nitems + g - 1) / g * E::kItem <= kFusedCap && g <= kExchangeMaxCtas &&
             qa.nbytes >= kFusedMinBytes) {
+            if (!static_amax && !(qa.barrier = grid_barrier_for(s)))
+                return cudaErrorInvalidValue;
             static std::once_flag fattr[64];
             int dev = 0;
             cudaGetDevice(&dev);
@@ -1082,6 +1132,35 @@ cudaError_t launch_typed(const void *x, const float *fp8_scale, int64_t rows, in
             fc.attrs = fa;
             fc.numAttrs = 2;
             return cudaLaunchKernelEx(&fc, fused_quantize_kernel<SRC>, qa);
+        }
+        // larger tensors: one streamed launch (two passes through a shared-memory ring)
+        if (qa.nbytes >= kFusedMinBytes && sms <= kExchangeMaxCtas) {
+            if (!static_amax && !(qa.barrier = grid_barrier_for(s)))
+                return cudaErrorInvalidValue;
+            static std::once_flag sattr[64];
+            int dev = 0;
+            cudaGetDevice(&dev);
+            cudaError_t se = cudaSuccess;
+            std::call_once(sattr[dev & 63], [&]() {
+                se = cudaFuncSetAttribute(stream_quantize_kernel<SRC>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          StreamCfg<SRC>::kSmem);
+            });
+            if (se != cudaSuccess)
+                return se;
+            cudaLaunchConfig_t sc{};
+            sc.gridDim = dim3((unsigned)sms);
+            sc.blockDim = dim3(kStreamThreads);
+            sc.dynamicSmemBytes = StreamCfg<SRC>::kSmem;
+            sc.stream = s;
+            cudaLaunchAttribute sa[2];
+            sa[0].id = cudaLaunchAttributeCooperative;
+            sa[0].val.cooperative = static_amax ? 0 : 1;
+            sa[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            sa[1].val.programmaticStreamSerializationAllowed = 1;
+            sc.attrs = sa;
+            sc.numAttrs = 2;
+            return cudaLaunchKernelEx(&sc, stream_quantize_kernel<SRC>, qa);
         }
     }
     cudaError_t e;
@@ -1366,8 +1445,9 @@ constexpr int kE8FusedThreads = 1024;
 
 template <int SRC>
 __global__ void __launch_bounds__(kE8FusedThreads, 1)
-    e4m3_fused_kernel(const uint8_t *__restrict__ x, int64_t n, float *__restrict__ partials,
-                      uint8_t *__restrict__ codes, float *__restrict__ scale_out, int *status)
+    e4m3_fused_kernel(const uint8_t *__restrict__ x, int64_t n, float *__restrict__ slots,
+                      GridBarrier *barrier, uint8_t *__restrict__ codes,
+                      float *__restrict__ scale_out, int *status)
 {
     extern __shared__ __align__(128) uint8_t buf[];
     pdl_wait(); // programmatic dependent launch: the previous kernel's writes are visible
@@ -1410,27 +1490,19 @@ __global__ void __launch_bounds__(kE8FusedThreads, 1)
     if ((threadIdx.x & 31) == 0)
         s_red[threadIdx.x >> 5] = f;
     __syncthreads();
-    float g = 0.0f;
     if (threadIdx.x < 32) {
-        g = s_red[threadIdx.x];
+        float g = s_red[threadIdx.x];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
-        if (threadIdx.x == 0)
-            partials[blockIdx.x] = g;
-    }
-    cooperative_groups::this_grid().sync(); // every CTA's partial is visible
-    if (threadIdx.x < 32) {
-        float pv[5]; // gridDim <= 160: one L2 round trip
-#pragma unroll
-        for (int u = 0; u < 5; ++u) {
-            const int i = threadIdx.x + 32 * u;
-            pv[u] = i < (int)gridDim.x ? __ldcg(partials + i) : 0.0f;
+        // every CTA's maximum, through the workspace's exchange slots (bounded)
+        if (gridDim.x > 1) {
+            float unused;
+            if (!grid_exchange_max(slots, barrier, (int)gridDim.x, (int)blockIdx.x, g, 0.0f,
+                                   kExchangeLimit, g, unused) &&
+                threadIdx.x == 0)
+                atomicExch(status, (int)NVFP4_ERR_TIMEOUT);
         }
-        g = fmaxf(fmaxf(fmaxf(pv[0], pv[1]), fmaxf(pv[2], pv[3])), pv[4]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
         if (threadIdx.x == 0) {
             const float sc = __fdiv_rn(g, 448.0f);
             s_s = sc;
@@ -1487,7 +1559,7 @@ cudaError_t launch_e4m3_typed(const void *x, int64_t n, const float *static_amax
         const int64_t nbytes = n * Src<SRC>::kBytes;
         const int64_t per = ((n >> 3) + sms - 1) / sms * 8 * Src<SRC>::kBytes;
         if (!static_amax && (n & 7) == 0 && nbytes >= kFusedMinBytes && per <= kFusedCap &&
-            sms <= 160) {
+            sms <= kExchangeMaxCtas) {
             static std::once_flag fattr[64];
             static cudaError_t fe[64];
             int dev = 0;
@@ -1498,6 +1570,9 @@ cudaError_t launch_e4m3_typed(const void *x, int64_t n, const float *static_amax
             });
             if (fe[dev & 63] != cudaSuccess)
                 return fe[dev & 63];
+            GridBarrier *bar = grid_barrier_for(s);
+            if (!bar)
+                return cudaErrorInvalidValue;
             cudaLaunchConfig_t fc{};
             fc.gridDim = dim3((unsigned)sms);
             fc.blockDim = dim3(kE8FusedThreads);
@@ -1512,7 +1587,7 @@ cudaError_t launch_e4m3_typed(const void *x, int64_t n, const float *static_amax
             fc.numAttrs = 2;
             return cudaLaunchKernelEx(&fc, e4m3_fused_kernel<SRC>,
                                       reinterpret_cast<const uint8_t *>(x), n,
-                                      reinterpret_cast<float *>(ws), codes, scale_out,
+                                      reinterpret_cast<float *>(ws), bar, codes, scale_out,
                                       device_status_ptr());
         }
     }
@@ -1643,7 +1718,7 @@ bool try_fused_pair(const QuantGroup &g, void *ws, cudaStream_t s, cudaError_t *
     // b must fit in registers: kPairRegVecs 16-byte vectors a thread (whole blocks of it)
     const int64_t b_blocks = (int64_t)b.rows * (b.cols / 16);
     const int64_t b_bpt = kPairRegVecs / (g.src[ib] == kSrcF32 ? 4 : g.src[ib] == kSrcBF16 ? 2 : 1);
-    if (grid > 160 || 2 * grid > kAmaxPartials || a.nbytes + b.nbytes < kFusedMinBytes ||
+    if (grid > kExchangeMaxCtas || a.nbytes + b.nbytes < kFusedMinBytes ||
         b.nbytes <= 0 || b_blocks > (int64_t)grid * kPairThreads * b_bpt)
         return false;
     // warp items of a (Enc<>: 32 blocks of fp32, 64 of bf16 / fp8; 2 KB / 2 KB / 1 KB)
@@ -1653,10 +1728,13 @@ bool try_fused_pair(const QuantGroup &g, void *ws, cudaStream_t s, cudaError_t *
     const int64_t items_per_warp_max = kFusedCap / item / (kPairThreads / 32);
     if ((nitems + grid - 1) / grid > items_per_warp_max * (kPairThreads / 32))
         return false;
-    float *part = reinterpret_cast<float *>(ws);
-    a.partials_out = part;
-    b.partials_out = part + grid;
     const bool coop = !a.static_amax || !b.static_amax;
+    a.slots = b.slots = reinterpret_cast<float *>(ws); // one slot per CTA for both tensors
+    a.barrier = b.barrier = coop ? grid_barrier_for(s) : nullptr;
+    if (coop && !a.barrier) {
+        *err = cudaErrorInvalidValue;
+        return true;
+    }
     switch (g.src[ia]) {
     case kSrcF32: *err = launch_fused_pair_b<kSrcF32>(g.src[ib], a, b, grid, coop, s); break;
     case kSrcBF16: *err = launch_fused_pair_b<kSrcBF16>(g.src[ib], a, b, grid, coop, s); break;

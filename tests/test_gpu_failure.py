@@ -45,3 +45,92 @@ def test_timeout_reported_on_the_callers_stream():
         assert lib.nvfp4_selftest_wait_timeout(s.cuda_stream) == L.NVFP4_OK
     assert lib.nvfp4_sync_status(s.cuda_stream) == L.NVFP4_ERR_TIMEOUT
     assert np.int32(lib.nvfp4_sync_status(s.cuda_stream)) == 0
+
+
+# ---- the single-pass quantizers' bounded grid-wide exchange ----------------------------------
+
+def _ws():
+    lib = L.load()
+    n = lib.nvfp4_workspace_bytes(L.NVFP4_OP_QUANTIZE, 1, 0, 32)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    # arbitrary contents: the exchange needs no clearing
+    return torch.randint(0, 256, (n,), dtype=torch.uint8, device="cuda", generator=g)
+
+
+def _exchange(vals, ws, skip=-1, late=-1, late_ns=0, limit=1 << 21, out=None):
+    lib = L.load()
+    v = vals if isinstance(vals, torch.Tensor) else torch.tensor(vals, dtype=torch.float32,
+                                                                 device="cuda")
+    if out is None:
+        out = torch.full((2,), -1.0, dtype=torch.float32, device="cuda")
+    st = lib.nvfp4_selftest_grid_exchange(v.numel(), v.data_ptr(), skip, late, late_ns, limit,
+                                          out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                          torch.cuda.current_stream().cuda_stream or None)
+    return st, out
+
+
+def test_grid_exchange_all_arrive():
+    ws = _ws()
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    for vals in (np.arange(1, n + 1, dtype=np.float32), np.full(n, 3.5, np.float32)):
+        st, out = _exchange(vals.tolist(), ws)
+        assert st == L.NVFP4_OK
+        assert nv.sync_status() == 0
+        assert out.cpu().tolist() == [float(vals.max()), float(vals.max()) / 2]
+
+
+def test_grid_exchange_missing_cta_times_out():
+    # CTA 5 never arrives; its slot still holds the previous launch's token, which must not
+    # count: the others give up after 64 poll rounds, report a timeout and return
+    ws = _ws()
+    n = 148
+    st, out = _exchange([1.0] * n, ws)
+    assert st == L.NVFP4_OK and nv.sync_status() == 0
+    st, out = _exchange([2.0] * n, ws, skip=5, limit=64)
+    assert st == L.NVFP4_OK
+    assert nv.sync_status() == L.NVFP4_ERR_TIMEOUT
+    assert out.cpu().tolist() == [-1.0, -1.0]
+    assert nv.sync_status() == 0
+    x = W.to_bf16_bits(W.normal((64, 256), 1.0, 34, 1))  # the context keeps working
+    assert_quant_equal(gpu_quantize(x), O.quantize(x))
+
+
+def test_grid_exchange_waits_for_a_late_cta():
+    # the largest value sits in a CTA that arrives 0.2 ms late; consecutive launches in the
+    # same workspace, with different values, each get their own maxima
+    ws = _ws()
+    n = 148
+    for big in (1000.0, 500.0, 750.0):
+        vals = [1.0] * n
+        vals[n - 1] = big
+        st, out = _exchange(vals, ws, late=n - 1, late_ns=200_000)
+        assert st == L.NVFP4_OK
+        assert nv.sync_status() == 0
+        assert out.cpu().tolist() == [big, big / 2]
+
+
+def test_grid_exchange_in_graph_replays():
+    # a captured exchange replayed with new values each time: every replay is a new launch
+    # with its own token, so the slots of the previous replay never satisfy the next one
+    ws = _ws()
+    n = 148
+    vals = torch.ones(n, dtype=torch.float32, device="cuda")
+    out = torch.full((2,), -1.0, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        _exchange(vals, ws, late=n - 1, late_ns=200_000, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        _exchange(vals, ws, late=n - 1, late_ns=200_000, out=out)
+    for big in (900.0, 300.0, 600.0):
+        vals.fill_(1.0)
+        vals[n - 1] = big
+        g.replay()
+        torch.cuda.synchronize()
+        assert out.cpu().tolist() == [big, big / 2]
+    assert nv.sync_status() == 0
+    del g

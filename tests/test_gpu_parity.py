@@ -75,6 +75,30 @@ def test_quantize_single_pass_sizes(kind, rows, cols, static):
     assert_quant_equal(gpu_quantize(x, amax=amax), O.quantize(x, amax=amax))
 
 
+# Tensors beyond what the CTAs' shared memory holds (148 x 192 KB) take the streamed
+# single-launch kernel: two passes through a shared-memory ring, the second back to front
+# (the last chunks of each CTA's range still in the ring). Ragged rows and block counts that are
+# not a multiple of 4 again.
+@pytest.mark.parametrize("kind,rows,cols", [("f32", 2100, 4064), ("bf16", 4100, 4064),
+                                            ("e4m3", 8200, 4096), ("bf16", 4096, 12288)])
+@pytest.mark.parametrize("static", [False, True])
+def test_quantize_streamed_sizes(kind, rows, cols, static):
+    x = W.normal((rows, cols), 1.0, 25, rows + cols)
+    x[rows - 1, cols - 1] = 21.0
+    x[0, 17] = -13.0
+    amax = 9.5 if static else None
+    if kind == "e4m3":
+        w8, s8 = W.to_fp8_tensorwise(x)
+        assert w8.nbytes > 148 * 192 * 1024
+        assert_quant_equal(gpu_quantize(w8, amax=amax, fp8_scale=s8),
+                           O.quantize(w8, amax=amax, fp8_scale=s8))
+        return
+    if kind == "bf16":
+        x = W.to_bf16_bits(x)
+    assert x.nbytes > 148 * 192 * 1024
+    assert_quant_equal(gpu_quantize(x, amax=amax), O.quantize(x, amax=amax))
+
+
 def test_quantize_batch_matches_single_calls():
     # a weight re-quantized from FP8, bf16 activations, an fp32 tensor with a static amax, a
     # tiny ragged one: one batched call gives each exactly its own quantization

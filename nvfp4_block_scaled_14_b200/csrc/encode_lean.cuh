@@ -93,6 +93,19 @@ __device__ __forceinline__ uint32_t scale_pair(float m0, float m1, float t, floa
     return e4m3_of_quotient(m0, t, rt) | (e4m3_of_quotient(m1, t, rt) << 8);
 }
 
+// The upper bf16 of a pair as fp32, exactly (sign of zero kept), by the mixed-precision FMA
+// x * 1 + (-0): the widening then runs on the FMA pipe instead of a logic operation on the
+// integer pipe, which the encode keeps busy (the lower one is a shift the compiler already
+// places on the FMA pipe).
+__device__ __forceinline__ float bf16_hi_to_f32(uint32_t w)
+{
+    float d;
+    asm("fma.rn.f32.bf16 %0, %1, %2, %3;"
+        : "=f"(d)
+        : "h"((uint16_t)(w >> 16)), "h"((uint16_t)0x3F80), "f"(-0.0f));
+    return d;
+}
+
 // E2M1 codes (low nibble first) of 8 bf16 values (one 16-byte vector) times r.
 __device__ __forceinline__ uint32_t codes8_bf16(const uint4 &v, float r)
 {
@@ -101,8 +114,8 @@ __device__ __forceinline__ uint32_t codes8_bf16(const uint4 &v, float r)
     float y[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const float2 p = __fmul2_rn(
-            make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u)), rr);
+        const float2 p =
+            __fmul2_rn(make_float2(__uint_as_float(w[j] << 16), bf16_hi_to_f32(w[j])), rr);
         y[2 * j] = p.x;
         y[2 * j + 1] = p.y;
     }

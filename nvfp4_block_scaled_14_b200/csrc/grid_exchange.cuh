@@ -7,11 +7,11 @@
 // before it arrives (the workspace's earlier contents do not matter: every slot read after
 // the barrier was written by this launch).
 //
-// Barrier: a sense-reversing counter (GridBarrier) in device memory that the library owns,
-// zero when the library loads, and left with count 0 by every barrier that completes. A CTA
-// reads the generation, arrives on the counter (release), and the last of the nblk CTAs to
-// arrive resets the counter and advances the generation (release); the others poll the
-// generation (acquire) for at most `limit` rounds. The host gives each stream its own
+// Barrier: a counter word (GridBarrier) in device memory that the library owns, zero when the
+// library loads. Each CTA adds to it once (release): CTA 0 adds 2^31 - (nblk - 1), the others
+// 1, so bit 31 flips exactly when the last CTA arrives and the low bits return to zero (the
+// state the next barrier needs); every CTA polls (acquire) for the flip against the value its
+// own addition returned, for at most `limit` rounds. The host gives each stream its own
 // GridBarrier and every launch captured into a CUDA graph a fresh one, so launches that may
 // run at the same time never share one; launches on one stream are serialized, and each
 // waits for its predecessor (programmatic dependent launch) before it touches the barrier.
@@ -26,16 +26,9 @@ namespace nvfp4 {
 constexpr int kExchangeMaxCtas = 160; // slots read per lane: 5
 
 struct GridBarrier {
-    uint32_t count; // arrivals of the barrier in progress
-    uint32_t gen;   // completed barriers (wraps)
+    uint32_t count; // bit 31: flips once per completed barrier; bits 0-30: arrivals so far
+    uint32_t unused;
 };
-
-__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
 {
@@ -44,26 +37,21 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
     return v;
 }
 
-// Arrive on the barrier and wait (one thread per CTA). The relaxed read of gen comes before
-// the arrival, whose release orders it (and this CTA's slot write) before any later arrival;
-// gen cannot advance before this CTA has arrived. Returns false after `limit` poll rounds.
-__device__ __forceinline__ bool grid_barrier_sync(GridBarrier *bar, int nblk, uint32_t limit)
+// Arrive on the barrier and wait (one thread per CTA; bid: this CTA's index among the nblk).
+// The arrival's release orders this CTA's slot write before it; the additions form one release
+// sequence, so the poll that sees the flip (acquire) sees every CTA's slot. Returns false after
+// `limit` poll rounds.
+__device__ __forceinline__ bool grid_barrier_sync(GridBarrier *bar, int nblk, int bid,
+                                                  uint32_t limit)
 {
-    const uint32_t g0 = ld_relaxed_u32(&bar->gen);
+    const uint32_t add = bid == 0 ? 0x80000000u - (uint32_t)(nblk - 1) : 1u;
     uint32_t old;
-    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
+    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;"
                  : "=r"(old)
-                 : "l"(&bar->count)
+                 : "l"(&bar->count), "r"(add)
                  : "memory");
-    if (old == (uint32_t)nblk - 1u) {
-        // the last arrival: every other CTA's arrival (and what it released) is visible here
-        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(&bar->count) : "memory");
-        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&bar->gen), "r"(g0 + 1u)
-                     : "memory");
-        return true;
-    }
     for (uint32_t round = 0; round < limit; ++round)
-        if (ld_acquire_u32(&bar->gen) != g0)
+        if (((ld_acquire_u32(&bar->count) ^ old) & 0x80000000u) != 0u)
             return true;
     return false;
 }
@@ -82,7 +70,7 @@ __device__ __forceinline__ bool grid_exchange_max(float *slots, GridBarrier *bar
         asm volatile("st.relaxed.gpu.global.v2.f32 [%0], {%1, %2};" ::"l"(slots + 2 * bid),
                      "f"(va), "f"(vb)
                      : "memory");
-        ok = grid_barrier_sync(bar, nblk, limit) ? 1 : 0;
+        ok = grid_barrier_sync(bar, nblk, bid, limit) ? 1 : 0;
     }
     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     __syncwarp();

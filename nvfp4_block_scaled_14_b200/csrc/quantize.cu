@@ -906,22 +906,63 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 }
 
 // Single-launch quantizer for tensors larger than the CTAs' shared memory. One CTA per SM owns
-// a contiguous range of warp items and streams it through a ring of kStreamSlots chunks (one
-// warp item per warp per chunk) with 1-D bulk copies. Dynamic amax: pass 1 folds max |x| over
-// the range front to back; the grid-wide exchange gives sg; pass 2 walks the range back to
-// front, so it starts on the chunks pass 1 left in the ring (no second read) and continues on
-// the ones read last, which L2 still holds; each warp encodes its item of the chunk (block
-// maxima, E4M3 scales, E2M1 codes) and the chunk's slot is refilled with the chunk kStreamSlots
-// further down. Static amax: pass 2 alone. The tensor leaves HBM once and one kernel runs.
-constexpr int kStreamThreads = 1024;
+// a contiguous range of warp items and streams it through a ring of kStreamSlots chunks with
+// 1-D bulk copies; a chunk holds kStreamIpw items per warp. Dynamic amax: pass 1 folds max |x|
+// over the range front to back; the grid-wide exchange gives sg; pass 2 walks the range back
+// to front, so it starts on the chunks pass 1 left in the ring (no second read) and continues
+// on the ones read last, which L2 still holds; each warp encodes its items of the chunk (block
+// maxima, E4M3 scales, E2M1 codes; the two items are independent, so their instructions
+// interleave) and the chunk's slot is refilled with the chunk kStreamSlots further down. Static
+// amax: pass 2 alone. The tensor leaves HBM once and one kernel runs. The encode is bound by
+// the integer pipe, so the per-chunk bookkeeping is kept small: every wait's mbarrier parity
+// is a closed form of the chunk index.
+constexpr int kStreamThreads = 512;
 constexpr int kStreamSlots = 3;
+constexpr int kStreamIpw = 2; // warp items per warp per chunk
 
 template <int SRC> struct StreamCfg {
     static constexpr int kWarps = kStreamThreads / 32;
-    static constexpr int kChunkItems = kWarps; // one warp item per warp per chunk
+    static constexpr int kChunkItems = kWarps * kStreamIpw;
     static constexpr int kChunkBytes = kChunkItems * Enc<SRC>::kItem; // 64 KB (fp8: 32 KB)
     static constexpr int kSmem = kStreamSlots * kChunkBytes;
 };
+
+// max |x| of one 16-byte vector folded into acc (bf16: packed magnitudes, sign bits not
+// meaningful; fp32: the float; fp8: packed f16 magnitudes of |e|)
+template <int SRC> __device__ __forceinline__ uint32_t fold_vec(uint32_t acc, const uint4 &v)
+{
+    if constexpr (SRC == kSrcBF16) {
+        return absmax_bf16x2(acc, absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
+    } else if constexpr (SRC == kSrcF32) {
+        return __float_as_uint(fmaxf(__uint_as_float(acc),
+                                     fmaxf(fmaxf(fabsf(__uint_as_float(v.x)),
+                                                 fabsf(__uint_as_float(v.y))),
+                                           fmaxf(fabsf(__uint_as_float(v.z)),
+                                                 fabsf(__uint_as_float(v.w))))));
+    } else {
+        const uint32_t a0 = absmax_f16x2(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16));
+        const uint32_t a1 = absmax_f16x2(e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
+        const uint32_t a2 = absmax_f16x2(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16));
+        const uint32_t a3 = absmax_f16x2(e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+        return absmax_f16x2(acc, absmax_f16x2(absmax_f16x2(a0, a1), absmax_f16x2(a2, a3)));
+    }
+}
+
+// the folded value as an fp32 maximum (fp8: of |e|)
+template <int SRC> __device__ __forceinline__ float fold_to_f32(uint32_t acc)
+{
+    if constexpr (SRC == kSrcBF16) {
+        return fmaxf(__uint_as_float((acc << 16) & 0x7FFFFFFFu),
+                     __uint_as_float(acc & 0x7FFF0000u));
+    } else if constexpr (SRC == kSrcF32) {
+        return __uint_as_float(acc);
+    } else {
+        __half_raw lo, hi;
+        lo.x = (unsigned short)(acc & 0x7FFFu);
+        hi.x = (unsigned short)((acc >> 16) & 0x7FFFu);
+        return fmaxf(__half2float(__half(lo)), __half2float(__half(hi)));
+    }
+}
 
 template <int SRC>
 __global__ void __launch_bounds__(kStreamThreads, 1) stream_quantize_kernel(const QuantArgs a)
@@ -953,52 +994,37 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_quantize_kernel(cons
         fence_barrier_init();
     }
     __syncthreads();
-    // fills issued per slot (the same count in every thread); a wait for the latest fill of
-    // slot s uses the parity of its number
-    int nfill[S];
-#pragma unroll
-    for (int s = 0; s < S; ++s)
-        nfill[s] = 0;
-    auto issue = [&](int c) {
-        const int s = c % S;
-        if (threadIdx.x == 0) {
-            const int64_t off = (int64_t)c * C::kChunkBytes;
-            const uint32_t n = (uint32_t)min((int64_t)C::kChunkBytes, nbytes - off);
-            mbar_arrive_expect_tx(&full[s], n);
-            bulk_load_1d(ring + s * C::kChunkBytes, a.x + byte0 + off, n, &full[s]);
-        }
-#pragma unroll
-        for (int t = 0; t < S; ++t)
-            nfill[t] += t == s ? 1 : 0;
+    auto issue = [&](int c) { // thread 0 only
+        const int64_t off = (int64_t)c * C::kChunkBytes;
+        const uint32_t n = (uint32_t)min((int64_t)C::kChunkBytes, nbytes - off);
+        mbar_arrive_expect_tx(&full[c % S], n);
+        bulk_load_1d(ring + (c % S) * C::kChunkBytes, a.x + byte0 + off, n, &full[c % S]);
     };
-    auto wait_chunk = [&](int c) {
-        const int s = c % S;
-        int parity = 0;
-#pragma unroll
-        for (int t = 0; t < S; ++t)
-            parity = t == s ? (nfill[t] - 1) & 1 : parity;
-        if (!mbar_wait(&full[s], (uint32_t)parity, kSpinLimit) && lane == 0)
+    auto wait_chunk = [&](int c, uint32_t parity) {
+        if (!mbar_wait(&full[c % S], parity, kSpinLimit) && lane == 0)
             atomicExch(a.status, (int)NVFP4_ERR_TIMEOUT);
     };
 
     float g = 0.0f;
     if (dyn) {
-        // pass 1: max |x| over the range, front to back
-        for (int c = 0; c < min(nch, S); ++c)
-            issue(c);
+        // pass 1: max |x| over the range, front to back; chunk c is fill c / S of its slot
+        if (threadIdx.x == 0)
+            for (int c = 0; c < min(nch, S); ++c)
+                issue(c);
         uint32_t m = 0;
         for (int c = 0; c < nch; ++c) {
-            wait_chunk(c);
+            wait_chunk(c, (uint32_t)(c / S) & 1u);
             const int nv = (int)(min((int64_t)C::kChunkBytes, nbytes - (int64_t)c * C::kChunkBytes) >> 4);
             const uint32_t base = smem_u32(ring + (c % S) * C::kChunkBytes);
             for (int i = threadIdx.x; i < nv; i += kStreamThreads)
-                m = mag_fold<SRC>(m, Src<SRC>::vec_magmax(lds128(base + 16 * i)));
+                m = fold_vec<SRC>(m, lds128(base + 16 * i));
             if (c + S < nch) {
                 __syncthreads(); // every thread is done with the slot
-                issue(c + S);
+                if (threadIdx.x == 0)
+                    issue(c + S);
             }
         }
-        float f = Src<SRC>::mag_to_f32(m);
+        float f = fold_to_f32<SRC>(m);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
@@ -1006,7 +1032,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_quantize_kernel(cons
             s_red[warp] = f;
         __syncthreads();
         if (warp == 0) {
-            g = s_red[lane];
+            g = lane < C::kWarps ? s_red[lane] : 0.0f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 g = fmaxf(g, __shfl_xor_sync(0xFFFFFFFFu, g, o));
@@ -1022,8 +1048,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_quantize_kernel(cons
         }
     } else {
         // static amax: the last chunks first (pass 2's order)
-        for (int c = nch - 1; c >= max(0, nch - S); --c)
-            issue(c);
+        if (threadIdx.x == 0)
+            for (int c = nch - 1; c >= max(0, nch - S); --c)
+                issue(c);
         if (warp == 0)
             g = *a.static_amax;
     }
@@ -1042,30 +1069,43 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_quantize_kernel(cons
     __syncthreads();
     pdl_launch_dependents(); // a dependent GEMM may set up while this grid encodes
 
-    // pass 2: encode, back to front
+    // pass 2: encode, back to front. A chunk below nch - S is a refill: with dynamic amax its
+    // fill number is n1(s) + (nch - S - 1 - c) / S, n1(s) = (nch - 1 - s) / S + 1 fills of
+    // slot s = c % S in pass 1; with a static amax it is 1 + (nch - S - 1 - c) / S (each slot's
+    // first fill holds one of the last S chunks, waited with parity 0).
     const uint32_t nb = (uint32_t)(a.cols >> 4);
     const int apb = (int)((nb + 3) >> 2);
     for (int c = nch - 1; c >= 0; --c) {
-        if (!dyn || c < nch - S)
-            wait_chunk(c);
-        const int64_t item = c0 + (int64_t)c * C::kChunkItems + warp;
-        const int64_t f0 = item * E::kItemBlocks + lane * E::kBpl;
-        if (item < c1 && f0 < nblocks) {
-            const uint32_t src = smem_u32(ring + (c % S) * C::kChunkBytes) + warp * E::kItem +
-                                 lane * (E::kBpl * E::kBlk);
-            uint4 r[NVL];
+        if (c < nch - S) {
+            const int fill = dyn ? (nch - 1 - c % S) / S + 1 + (nch - S - 1 - c) / S
+                                 : 1 + (nch - S - 1 - c) / S;
+            wait_chunk(c, (uint32_t)fill & 1u);
+        } else if (!dyn) {
+            wait_chunk(c, 0u);
+        }
+        const uint32_t slot = smem_u32(ring + (c % S) * C::kChunkBytes);
 #pragma unroll
-            for (int v = 0; v < NVL; ++v)
-                r[v] = lds128(src + 16 * (v ^ k));
-            float m0, m1;
-            lane_maxima_rot<SRC>(r, k, m0, m1);
-            uint32_t cw[2 * E::kBpl], sb0, sb1;
-            lane_encode_rot<SRC>(r, k, m0, m1, s8, sg, t, rt, s_rcp, cw, sb0, sb1);
-            store_lane<SRC>(a, f0, nb, apb, cw, sb0, sb1);
+        for (int h = 0; h < kStreamIpw; ++h) {
+            const int w = warp + C::kWarps * h; // item of the chunk
+            const int64_t item = c0 + (int64_t)c * C::kChunkItems + w;
+            const int64_t f0 = item * E::kItemBlocks + lane * E::kBpl;
+            if (item < c1 && f0 < nblocks) {
+                const uint32_t src = slot + w * E::kItem + lane * (E::kBpl * E::kBlk);
+                uint4 r[NVL];
+#pragma unroll
+                for (int v = 0; v < NVL; ++v)
+                    r[v] = lds128(src + 16 * (v ^ k));
+                float m0, m1;
+                lane_maxima_rot<SRC>(r, k, m0, m1);
+                uint32_t cw[2 * E::kBpl], sb0, sb1;
+                lane_encode_rot<SRC>(r, k, m0, m1, s8, sg, t, rt, s_rcp, cw, sb0, sb1);
+                store_lane<SRC>(a, f0, nb, apb, cw, sb0, sb1);
+            }
         }
         if (c - S >= 0) {
             __syncthreads(); // every warp is done with the slot
-            issue(c - S);
+            if (threadIdx.x == 0)
+                issue(c - S);
         }
     }
     zero_pad_rows(a, apb, blockIdx.x, gridDim.x);

@@ -779,8 +779,59 @@ __device__ __forceinline__ void quantize_out_row(const GemmParams &p, uint32_t t
 // un-split case uses it (TMA-store epilogue).
 // ---------------------------------------------------------------------------------------
 
-struct Pair {
-    static constexpr int kStages = 4;
+// One CTA's 128 x 256 bf16 output tile through a 32 KB staging tile (two 64-column boxes), in
+// two halves: accumulator columns 0-127 are converted and their TMA store issued while columns
+// 128-255 are read from TMEM; `release` follows the last TMEM read; the second half is staged
+// once the first store has left the staging tile. Run by the four epilogue warps (r: this
+// thread's row, TMEM lane; `issuer`: the thread that issues and tracks the stores).
+// Half of the tile's writes thus leave while the MMA warp still waits for the accumulator: the
+// writes that follow the release compete with the next tile's operand loads.
+template <typename Release>
+__device__ __forceinline__ void stage_store_tile_halves(const GemmParams &p, const CUtensorMap *tmY,
+                                                        uint8_t *stg, uint32_t trow, int r,
+                                                        float alpha, bool issuer, int64_t yrow,
+                                                        int64_t ycol, Release release)
+{
+    const uint32_t s = smem_u32(stg);
+    auto store = [&](int half) {
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (issuer) {
+            // boxes that start past the last row or column of Y hold nothing to store
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int64_t col = ycol + (2 * half + b) * 64;
+                if (yrow < p.rows_a && col < p.rows_b)
+                    tma_store_2d(tmY, stg + b * (128 * 128), (int)col, (int)yrow);
+            }
+            bulk_commit_group();
+        }
+    };
+    uint32_t va[64], vb[64];
+    tmem_ld_64cols(trow, va);
+    tmem_ld_wait();
+    tmem_ld_64cols(trow + 64, vb);
+    stage_box_bf16(va, s, 0, r, alpha);
+    tmem_ld_wait();
+    stage_box_bf16(vb, s, 1, r, alpha);
+    tmem_ld_64cols(trow + 128, va);
+    tmem_ld_64cols(trow + 192, vb);
+    store(0);
+    tmem_ld_wait();
+    release();
+    if (issuer)
+        bulk_wait_group_read0(); // the first half has left the staging tile
+    named_bar_sync(1, 128);
+    stage_box_bf16(va, s, 0, r, alpha);
+    stage_box_bf16(vb, s, 1, r, alpha);
+    store(1);
+}
+
+// Shared-memory layout of the pair kernel. bf16 output: five operand stages and a 32 KB bf16
+// staging tile (the output leaves in two halves); quantizing epilogue: four stages and 64 KB
+// of staging (fp32 columns 128-255 of each row while columns 0-127 are quantized).
+template <bool QOUT> struct Pair {
+    static constexpr int kStages = QOUT ? 4 : 5;
     static constexpr int kABytes = 128 * 128;     // this CTA's 128 rows of A
     static constexpr int kBBytes = 128 * 128;     // this CTA's 128 rows of B
     static constexpr int kSfaBytes = 4 * 512;     // SFA atoms of this CTA's rows
@@ -789,7 +840,7 @@ struct Pair {
     static constexpr int kOffSfa = kOffB + kStages * kBBytes;
     static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
     static constexpr int kOffStaging = kOffSfb + kStages * kSfbBytes;
-    static constexpr int kStagingBytes = 128 * 256 * 2;
+    static constexpr int kStagingBytes = QOUT ? 128 * 128 * 4 : 128 * 128 * 2;
     static constexpr int kOffBar = kOffStaging + kStagingBytes;
     static constexpr int kOffRcp = kOffBar + 512; // quantizing epilogue: 128 reciprocals
     static constexpr int kSmemBytes = kOffRcp + 512;
@@ -808,6 +859,7 @@ struct Pair {
                                          ((uint32_t)(256 >> 3) << 17) |
                                          ((uint32_t)(256 >> 4) << 24);
     static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kOffStaging % 1024 == 0, "swizzled staging alignment");
     static_assert(kSfCol + kSfSlots * kSlotCols <= kTmemCols, "TMEM budget");
 };
 
@@ -832,7 +884,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                            const __grid_constant__ CUtensorMap tmT,
                            const __grid_constant__ CUtensorMap tmU, const GemmParams p)
 {
-    using C = Pair;
+    using C = Pair<QOUT>;
     extern __shared__ __align__(1024) uint8_t smem[];
     if ((smem_u32(smem) & 1023u) != 0) {
         if (threadIdx.x == 0)
@@ -1156,26 +1208,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 continue;
             }
             if (threadIdx.x == 64)
-                bulk_wait_group_read0();
+                bulk_wait_group_read0(); // the previous tile's second half has left the staging
             named_bar_sync(1, 128);
-            stage_tile_bf16(trow, smem_u32(smem + C::kOffStaging), q * 32 + lane, alpha, [&]() {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive_remote(leader_acc_empty); // this CTA's accumulator is read
-            });
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (threadIdx.x == 64) {
-                // boxes that start past the last row or column of Y hold nothing to store
-                const int64_t yrow = ta * 256 + rank * 128;
-#pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    if (yrow < p.rows_a && tb * 256 + b * 64 < p.rows_b)
-                        tma_store_2d(&tmY, smem + C::kOffStaging + b * (128 * 128),
-                                     (int)(tb * 256 + b * 64), (int)yrow);
-                bulk_commit_group();
-            }
+            stage_store_tile_halves(p, &tmY, smem + C::kOffStaging, trow, q * 32 + lane, alpha,
+                                    threadIdx.x == 64, ta * 256 + rank * 128, tb * 256, [&]() {
+                                        tc_fence_before();
+                                        __syncwarp();
+                                        if (lane == 0)
+                                            mbar_arrive_remote(leader_acc_empty); // read
+                                    });
             acc_phase ^= 1;
         }
     }
@@ -1983,7 +2024,7 @@ cudaError_t launch_pair(const uint8_t *a_codes, const uint8_t *a_sf, const uint8
     std::call_once(flags[dev & 63], [&]() {
         attr_err = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QOUT, LR>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        Pair::kSmemBytes);
+                                        Pair<QOUT>::kSmemBytes);
     });
     if (attr_err != cudaSuccess)
         return attr_err;
@@ -2001,7 +2042,7 @@ cudaError_t launch_pair(const uint8_t *a_codes, const uint8_t *a_sf, const uint8
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = Pair::kSmemBytes;
+    cfg.dynamicSmemBytes = Pair<QOUT>::kSmemBytes;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

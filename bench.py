@@ -220,7 +220,43 @@ def quantize_launches(nv, nbytes):
     return 1 if nbytes >= (16 << 20) else 2
 
 
-def launches_per_step(nv):
+def graph_kernel_nodes(fns):
+    """Kernel launches of one pass of fns, counted as the kernel nodes of a CUDA graph that
+    captures it; None if the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for f in fns:
+                f()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g):
+            for f in fns:
+                f()
+        h = rt.cudaGraph_t(init_value=int(g.raw_cuda_graph()))
+        err, _, n = rt.cudaGraphGetNodes(h, 0)
+        err2, nodes, n = rt.cudaGraphGetNodes(h, n)
+        if err != rt.cudaError_t.cudaSuccess or err2 != rt.cudaError_t.cudaSuccess:
+            return None
+        kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        count = sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
+        del g
+        return count
+    except Exception:  # an older torch or cuda-python: the caller falls back to its rule
+        return None
+
+
+def launches_per_step(nv, st=None):
+    """Kernel launches of one MLP step: counted in a captured graph of the step when possible,
+    else by rule (quantize: quantize_launches; linear: one launch, two when it needs workspace,
+    i.e. runs a split-K reduction)."""
+    if st is not None:
+        n = graph_kernel_nodes([lambda: st.run(0)])
+        if n is not None:
+            return n
     L = nv.load()
     gemm = lambda m, n, k: 2 if L.nvfp4_workspace_bytes(nv.NVFP4_OP_LINEAR, m, n, k) > 0 else 1
     return (quantize_launches(nv, T * H * 2) + gemm(T, F, H) +
@@ -754,7 +790,7 @@ def run_ours(args):
                 "serial_value": job_tflops(world, e2e_serial_ms, FLOPS),
                 "h2d_bytes_per_step": int(mp.X1.nbytes + mp.X2.nbytes),
                 "d2h_bytes_per_step": int(T * H * 2)},
-        "gpu_launches": launches_per_step(nv) * args.steps,
+        "gpu_launches": launches_per_step(nv, st) * args.steps,
         "clocks": clk,
     }
     if rows is not None:

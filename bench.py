@@ -10,9 +10,9 @@ are quantized to NVFP4 once, before timing, as a deployed layer keeps them.
 
 The headline `value` is the step's throughput in TFLOP/s (2*M*N*K of both GEMMs per step
 over the whole step, activation quantization included), summed over ranks. Each rank runs its
-own independent batch (weak scaling, no collective on the data path). Inputs rotate over
-enough buffer sets that every step reads them cold from HBM (more than 3x the L2 size in
-flight). Steps are replayed from CUDA graphs (one graph per rotation of the input sets).
+own independent batch (weak scaling, no collective on the data path). Inputs and outputs rotate
+over enough buffer sets that every step reads its inputs cold from HBM and writes to buffers
+the previous steps did not leave in L2 (more than 3x the L2 size in flight). Steps are replayed from CUDA graphs (one graph per rotation of the input sets).
 Per-op durations come from CUDA events around graph loops of each op alone over the same
 rotating inputs, on the launching stream (event nodes inside the step graph would break the
 kernels' programmatic dependent launch and add ~15 us per step).
@@ -174,8 +174,9 @@ def clone_q(nv, q):
 
 class MlpStep:
     """The MLP pair over several input sets: quantize X1, GEMM1, quantize X2, GEMM2. Each set
-    holds its own X1, X2 and its own copy of the quantized weights, so every step reads all of
-    its operands from HBM."""
+    holds its own X1, X2, its own copy of the quantized weights and its own outputs (quantized
+    activations, Y1, Y2), so every step reads all of its operands from HBM and writes to
+    buffers that the previous steps did not leave in L2."""
 
     def __init__(self, nv, mp, n_sets, dev):
         self.nv = nv
@@ -186,25 +187,26 @@ class MlpStep:
         self.Q1 = [clone_q(nv, q1) for _ in range(n_sets)]
         self.Q2 = [clone_q(nv, q2) for _ in range(n_sets)]
         del x1, x2, q1, q2
-        self.qx1 = nv.quantize(self.X1[0])
-        self.qx2 = nv.quantize(self.X2[0])
-        self.Y1 = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
-        self.Y2 = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.QX1 = [nv.quantize(x) for x in self.X1]
+        self.QX2 = [nv.quantize(x) for x in self.X2]
+        self.Y1 = [torch.empty((T, F), dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
+        self.Y2 = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
         wq = lambda q: q.codes.numel() + q.scales_swz.numel()
         self.set_bytes = ((self.X1[0].numel() + self.X2[0].numel()) * 2 + wq(self.Q1[0]) +
-                          wq(self.Q2[0]))
+                          wq(self.Q2[0]) + wq(self.QX1[0]) + wq(self.QX2[0]) +
+                          (self.Y1[0].numel() + self.Y2[0].numel()) * 2)
 
     def quantize1(self, i, x=None):
-        self.nv.quantize(self.X1[i] if x is None else x, out=self.qx1)
+        self.nv.quantize(self.X1[i] if x is None else x, out=self.QX1[i])
 
     def gemm1(self, i):
-        self.nv.linear(self.qx1, self.Q1[i], out=self.Y1)
+        self.nv.linear(self.QX1[i], self.Q1[i], out=self.Y1[i])
 
     def quantize2(self, i, x=None):
-        self.nv.quantize(self.X2[i] if x is None else x, out=self.qx2)
+        self.nv.quantize(self.X2[i] if x is None else x, out=self.QX2[i])
 
     def gemm2(self, i, y=None):
-        self.nv.linear(self.qx2, self.Q2[i], out=self.Y2 if y is None else y)
+        self.nv.linear(self.QX2[i], self.Q2[i], out=self.Y2[i] if y is None else y)
 
     def run(self, i):
         self.quantize1(i)
@@ -387,7 +389,7 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
     #     activation), against GEMM1 in bf16 followed by the static-scale quantize
     amax = torch.tensor([float(mlp.X2[0].float().abs().max())], device=dev)
     n_m = len(mlp.X1)
-    sets = list(zip([mlp.qx1] * n_m, mlp.Q1))
+    sets = list(zip(mlp.QX1, mlp.Q1))
     for i in range(n_m):
         mlp.quantize1(i)
     outs = [nv.linear_nvfp4_out(p[0], p[1], amax) for p in sets]
@@ -396,7 +398,7 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
         avg_f, _ = op_timer([lambda p=p, o=o: nv.linear_nvfp4_out(p[0], p[1], amax, act, out=o)
                              for p, o in zip(sets, outs)])
         row[f"nvfp4_out_{act}_us"] = avg_f * 1e3
-    avg_q, _ = op_timer([lambda i=i: nv.quantize(mlp.X2[i], static_amax=amax, out=mlp.qx2)
+    avg_q, _ = op_timer([lambda i=i: nv.quantize(mlp.X2[i], static_amax=amax, out=mlp.QX2[i])
                          for i in range(n_m)])
     row["quantize_x2_static_us"] = avg_q * 1e3
     rows["gemm1_m4096_n12288_k3072_nvfp4_out"] = row
@@ -559,7 +561,7 @@ def e2e_pipelined_ms(st, x1_host, x2_host, steps):
     them)."""
     nslot = 2
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    yd = [torch.empty_like(st.Y2) for _ in range(nslot)]
+    yd = [torch.empty_like(st.Y2[0]) for _ in range(nslot)]
     yh = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(nslot)]
     ev_in = [torch.cuda.Event() for _ in range(nslot)]
     ev_comp = [torch.cuda.Event() for _ in range(nslot)]
@@ -692,7 +694,7 @@ def run_ours(args):
         st.X1[0].view(torch.int16).copy_(x1_host, non_blocking=True)
         st.X2[0].view(torch.int16).copy_(x2_host, non_blocking=True)
         st.run(0)
-        y_host.copy_(st.Y2.view(torch.int16), non_blocking=True)
+        y_host.copy_(st.Y2[0].view(torch.int16), non_blocking=True)
 
     for _ in range(2):
         e2e_serial_step()
@@ -753,7 +755,7 @@ def run_ours(args):
                    "weights": "bf16 -> nvfp4 once, before timing",
                    "activations": "bf16, dynamic per-tensor amax, quantized every step",
                    "out": "bf16",
-                   "l2": f"inputs rotate over {n_sets} buffer sets "
+                   "l2": f"inputs and outputs rotate over {n_sets} buffer sets "
                          f"({n_sets * st.set_bytes / 1e6:.0f} MB > 3x L2)",
                    "parallelism": f"{world} independent ranks"},
         "gemm_tflops": {"gemm1": g1_tf, "gemm2": g2_tf},
@@ -841,7 +843,7 @@ def profile_case(name, reps):
         # each replay pass of a captured launch, so the case keeps it small
         st = MlpStep(nv, W.mlp_pair(), 1, dev)
         amax = torch.tensor([float(st.X2[0].float().abs().max())], device=dev)
-        outs = [nv.linear_nvfp4_out(st.qx1, st.Q1[0], amax)] \
+        outs = [nv.linear_nvfp4_out(st.QX1[0], st.Q1[0], amax)] \
             if name.startswith("nvfp4_out") else None
         st.quantize1(0)
         st.quantize2(0)
@@ -849,9 +851,9 @@ def profile_case(name, reps):
         # the GEMM cases launch only their own GEMM (after the operands' quantize above)
         op3 = {"mlp_step": st.run, "quantize_x1": st.quantize1, "gemm1": st.gemm1,
               "quantize_x2": st.quantize2, "gemm2": st.gemm2,
-              "nvfp4_out_gelu": lambda i: nv.linear_nvfp4_out(st.qx1, st.Q1[i], amax,
+              "nvfp4_out_gelu": lambda i: nv.linear_nvfp4_out(st.QX1[0], st.Q1[i], amax,
                                                               "gelu_tanh", out=outs[i]),
-              "nvfp4_out_identity": lambda i: nv.linear_nvfp4_out(st.qx1, st.Q1[i], amax,
+              "nvfp4_out_identity": lambda i: nv.linear_nvfp4_out(st.QX1[0], st.Q1[i], amax,
                                                                   "identity", out=outs[i])}[name]
         op = lambda i: op3(0)
     elif name in ("smallm_m8", "smallm_m8_resident", "linear_dynamic_m8"):

@@ -14,8 +14,9 @@
 // its K range of x and D through a 4-stage TMA ring into one M128 x N=r MMA accumulator in
 // TMEM. The partial accumulators meet in shared memory: every CTA stages its partial, and
 // after a cluster barrier each CTA sums its share of the band's rows over the cluster's
-// partials in rank order (distributed shared memory, deterministic), multiplies by 1 / alpha,
-// rounds to bf16 and stores.
+// partials in rank order (deterministic), multiplies by 1 / alpha, rounds to bf16 and stores.
+// The other CTAs' rows of that share arrive by bulk copies that their senders push into this
+// CTA's shared memory (remote loads of the same 48 KB a CTA took 3.4 us more, measured).
 #include <cuda.h>
 #include <cstring>
 #include <mutex>
@@ -27,8 +28,7 @@ namespace nvfp4 {
 namespace {
 
 // warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 epilogue; all 8 warps reduce the
-// cluster's partials (globaltimer stamps put that reduce at ~4.3 us of ~13 us with 6 warps, one
-// item in flight a thread and an IEEE division per value)
+// cluster's partials
 constexpr int kDnThreads = 256;
 // K split (CTAs per cluster, a power of two <= 8) and the most TMA ring stages (as many as the
 // shared memory holds, up to this). Measured on M4096 K3072 r128: a split of 4 with one CTA per
@@ -51,6 +51,8 @@ struct DownParams {
     int r;        // rank: multiple of 16, 16..256
     int stages;   // TMA ring depth (3 .. kDnMaxStages; the fp32 partial fits in 3 or more)
     int kt_total; // 64-wide k-tiles of K
+    int push;     // 1: the partials' rows reach their summing CTA by pushed bulk copies into an
+                  // inbox after the partial (dn_push_fits); 0: by remote loads
     const float *a_gs, *w_gs;
     __nv_bfloat16 *t; // [M x r], row stride r
     int *status;
@@ -68,6 +70,14 @@ constexpr int dn_stages(int r)
                : kDnMaxStages;
 }
 constexpr int dn_smem_bytes(int r) { return dn_stages(r) * dn_stage_bytes(r) + 256; }
+// fp32 partial rows of r + 4 floats (the pad spreads a warp's row-strided stores over the banks)
+__host__ __device__ constexpr uint32_t dn_row_bytes(int r) { return (uint32_t)(r + 4) * 4u; }
+// the partial (128 rows) and an inbox of another 128 rows fit in the drained stage buffers
+constexpr bool dn_push_fits(int r)
+{
+    return 256u * dn_row_bytes(r) <= (uint32_t)(dn_stages(r) * dn_stage_bytes(r));
+}
+static_assert(dn_push_fits(128) && dn_push_fits(192), "push reduce for the usual ranks");
 static_assert(dn_stages(256) >= 3 && dn_stages(16) >= 3, "ring depth");
 constexpr int dn_smem_max()
 {
@@ -104,6 +114,18 @@ __device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t cluster_addr)
     return v;
 }
 
+// Bulk copy of `bytes` from this CTA's shared memory to a cluster shared-memory address
+// (dst, mbar: mapa addresses in the receiving CTA); completes as bytes on the receiver's
+// mbarrier. Not a multicast: one destination CTA.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes,
+                                                     uint32_t mbar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes "
+                 "[%0], [%1], %2, [%3];" ::"r"(dst),
+                 "r"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -117,7 +139,8 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                         const __grid_constant__ CUtensorMap tmD, const DownParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
-    pdl_wait(); // programmatic dependent launch: x and the global scales come from earlier kernels
+    // programmatic dependent launch: the set-up below overlaps the previous kernel's tail; the
+    // producer (x) and the reduce (the global scales, T's earlier readers) wait for it
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = p.r;
     const int stage_bytes = dn_stage_bytes(r);
@@ -129,6 +152,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
     uint64_t *empty = full + kDnMaxStages;
     uint64_t *acc_full = empty + kDnMaxStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    uint64_t *inbox_full = acc_full + 2; // push reduce: the other CTAs' rows have arrived
     const bool aligned = (smem_u32(smem) & 1023u) == 0; // uniform over the cluster
     const int kt0 = (int)((int64_t)p.kt_total * rank / S);
     const int nk = (int)((int64_t)p.kt_total * (rank + 1) / S) - kt0; // >= 1 unless K == 0
@@ -140,6 +164,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
+        mbar_init(inbox_full, 1);
         fence_barrier_init();
         if (!aligned)
             atomicExch(p.status, (int)NVFP4_ERR_CUDA);
@@ -159,6 +184,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tmX);
             tma_prefetch_desc(&tmD);
+            pdl_wait();
             for (int i = 0; i < nk; ++i) {
                 const int s = i % nst;
                 const uint32_t ph = (uint32_t)(i / nst) & 1u;
@@ -237,21 +263,76 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                     sts128(prow + (uint32_t)((c + j) * 4), v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
         }
+        fence_proxy_async_smem(); // the partial's rows, before bulk copies read them
     }
+    const int rows_per = 128 / (int)S;
+    const uint32_t chunk = (uint32_t)rows_per * dn_row_bytes(r); // one CTA's share of a partial
+    if (threadIdx.x == 0 && aligned && p.push && S > 1)
+        mbar_arrive_expect_tx(inbox_full, (S - 1) * chunk); // armed before any copy can land
     tc_fence_before();
     __syncwarp();
     cluster_sync(); // every partial of the cluster is in shared memory
     pdl_launch_dependents(); // the GEMM may set up while the partials are reduced
 
     if (aligned) {
+        pdl_wait();
         float alpha = __fmul_rn(*p.a_gs, *p.w_gs);
         if (alpha == 0.0f)
             alpha = 1.0f; // the FP4 product is zero then; the GEMM scales by 1 as well
         const float ralpha = __frcp_rn(alpha);
-        const int rows_per = 128 / (int)S;
         const int v8 = r / 8;
         const int nitems = rows_per * v8;
         const uint32_t base = smem_u32(smem);
+        const uint32_t rb = dn_row_bytes(r);
+        if (p.push) {
+            // rows [rows_per d, rows_per (d + 1)) of this CTA's partial go to CTA d's inbox,
+            // slot `rank`; this CTA's own share stays where it is
+            const uint32_t inbox = base + 128u * rb;
+            if (threadIdx.x == 0)
+                for (uint32_t d = 0; d < S; ++d)
+                    if (d != rank)
+                        bulk_copy_to_cluster(mapa_shared(inbox + rank * chunk, d),
+                                             base + d * chunk, chunk,
+                                             mapa_shared(smem_u32(inbox_full), d));
+            if (S > 1 && !mbar_wait_cluster(inbox_full, 0, kDnWaitLimit)) {
+                if (threadIdx.x == 0)
+                    dn_timeout(p.status);
+            } else {
+                for (int idx = threadIdx.x; idx < nitems; idx += kDnThreads) {
+                    const int lr = idx / v8;
+                    const int c = (idx % v8) * 8;
+                    const int64_t m = band * 128 + (int64_t)rank * rows_per + lr;
+                    if (m >= p.M)
+                        continue;
+                    float acc[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        acc[j] = 0.0f;
+#pragma unroll
+                    for (int s = 0; s < kDnMaxSplit; ++s) // rank order: the same sum every run
+                        if (s < (int)S) {
+                            const uint32_t a =
+                                ((uint32_t)s == rank ? base + rank * chunk : inbox + s * chunk) +
+                                (uint32_t)lr * rb + (uint32_t)c * 4u;
+                            const uint4 u0 = lds128(a), u1 = lds128(a + 16);
+                            acc[0] += __uint_as_float(u0.x);
+                            acc[1] += __uint_as_float(u0.y);
+                            acc[2] += __uint_as_float(u0.z);
+                            acc[3] += __uint_as_float(u0.w);
+                            acc[4] += __uint_as_float(u1.x);
+                            acc[5] += __uint_as_float(u1.y);
+                            acc[6] += __uint_as_float(u1.z);
+                            acc[7] += __uint_as_float(u1.w);
+                        }
+                    uint4 o;
+                    o.x = bf16x2_bits(__fmul_rn(acc[0], ralpha), __fmul_rn(acc[1], ralpha));
+                    o.y = bf16x2_bits(__fmul_rn(acc[2], ralpha), __fmul_rn(acc[3], ralpha));
+                    o.z = bf16x2_bits(__fmul_rn(acc[4], ralpha), __fmul_rn(acc[5], ralpha));
+                    o.w = bf16x2_bits(__fmul_rn(acc[6], ralpha), __fmul_rn(acc[7], ralpha));
+                    *reinterpret_cast<uint4 *>(p.t + m * r + c) = o;
+                }
+            }
+        } else {
         // two items a thread per pass, every rank's loads of both in flight before the sums
         for (int i0 = threadIdx.x; i0 < nitems; i0 += 2 * kDnThreads) {
             float4 lo[2][kDnMaxSplit], hi[2][kDnMaxSplit];
@@ -303,6 +384,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                 o.w = bf16x2_bits(__fmul_rn(acc[6], ralpha), __fmul_rn(acc[7], ralpha));
                 *reinterpret_cast<uint4 *>(p.t + m * r + c) = o;
             }
+        }
         }
     }
     __syncwarp();
@@ -379,6 +461,7 @@ cudaError_t launch_lowrank_down(const void *x, const void *d, int64_t M, int64_t
     p.r = r;
     p.stages = dn_stages(r);
     p.kt_total = (int)((K + 63) / 64);
+    p.push = dn_push_fits(r) ? 1 : 0;
     p.a_gs = a_gs;
     p.w_gs = w_gs;
     p.t = reinterpret_cast<__nv_bfloat16 *>(t);

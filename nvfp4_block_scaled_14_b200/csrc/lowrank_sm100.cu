@@ -116,7 +116,7 @@ __device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t cluster_addr)
 
 // Bulk copy of `bytes` from this CTA's shared memory to a cluster shared-memory address
 // (dst, mbar: mapa addresses in the receiving CTA); completes as bytes on the receiver's
-// mbarrier. Not a multicast: one destination CTA.
+// mbarrier; exactly one destination CTA.
 __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes,
                                                      uint32_t mbar)
 {

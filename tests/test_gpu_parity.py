@@ -470,6 +470,9 @@ def test_linear_large_tile_path(out):
     (1280, 3072, 1024),
     (2000, 2296, 2048),   # ragged M and N, 8 k-tiles
     (4200, 2560, 768),    # two or three tiles per CTA pair (accumulator reuse), ragged M
+    # the 5-stage operand ring with one k-tile per tile (every tile starts at a new ring
+    # position), 85 tiles on 74 pairs
+    (4200, 1280, 256),
 ])
 def test_linear_pair_kernel(M, N, K):
     # every element of the output against the oracle's full product
@@ -485,6 +488,37 @@ def test_linear_pair_kernel(M, N, K):
     assert_quant_equal(qa, ra)
     assert_quant_equal(qw, rw)
     assert_gemm_close(y, O.gemm(ra, rw), True, what=f"pair kernel {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (4200, 1280, 1280),   # exactly as many k-tiles as ring stages, 85 tiles on 74 pairs
+    (2560, 3072, 1792),   # 7 k-tiles: the ring wraps inside a tile, 120 tiles on 74 pairs
+])
+def test_linear_pair_kernel_ring_phases(M, N, K):
+    # every 256 x 256 tile checked at its four corners and 12 seeded interior points against the
+    # oracle's products computed one by one (a wrong ring phase corrupts whole tiles)
+    xa = W.to_bf16_bits(W.normal((M, K), 1.0, 43, M))
+    xw = W.to_bf16_bits(W.normal((N, K), 0.02, 44, N))
+    qa, qw = gpu_quantize(xa), gpu_quantize(xw)
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nv.linear(qa, qw, out=out)
+    torch.cuda.synchronize()
+    y = to_numpy_f64(out)
+    assert np.isfinite(y).all()  # every element written
+    ra, rw = O.quantize(xa), O.quantize(xw)
+    assert_quant_equal(qa, ra)
+    assert_quant_equal(qw, rw)
+    rng = np.random.default_rng(45)
+    ms, ns = [], []
+    for r0 in range(0, M, 256):
+        for c0 in range(0, N, 256):
+            r1, c1 = min(r0 + 256, M) - 1, min(c0 + 256, N) - 1
+            ms += [r0, r0, r1, r1] + list(rng.integers(r0, r1 + 1, 12))
+            ns += [c0, c1, c0, c1] + list(rng.integers(c0, c1 + 1, 12))
+    ms, ns = np.array(ms, np.int64), np.array(ns, np.int64)
+    ref = O.gemm_sampled(ra, rw, ms, ns)
+    # the tolerance's max|Y_ref|: over the sample, the oracle's values only
+    assert_gemm_close(y[ms, ns], ref, True, tol=gemm_tol(ref), what=f"pair kernel {M}x{N}x{K}")
 
 
 # ---------------------------------------------------------------------------------------

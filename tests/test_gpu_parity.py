@@ -389,6 +389,31 @@ def test_linear_resident_weights_back_to_back(M, N, K):
     assert nv.sync_status() == 0
 
 
+def test_linear_degenerate_shapes():
+    # through the C ABI: K == 0 is an empty sum, Y = 0 in both output types (for a small-M and
+    # a large-M shape); M == 0 or N == 0 leaves nothing to compute and nothing is written
+    import ctypes
+    from nvfp4_block_scaled_14_b200 import _lib
+    L = nv.load()
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    for M, N in [(8, 64), (300, 512)]:
+        for dt, tdt in [(_lib.NVFP4_BF16, torch.bfloat16), (_lib.NVFP4_F32, torch.float32)]:
+            y = torch.full((M, N), float("nan"), dtype=tdt, device="cuda")
+            st = L.nvfp4_linear(None, None, None, None, None, None, M, N, 0, dt, ptr(y), None, 0,
+                                s)
+            torch.cuda.synchronize()
+            assert st == _lib.NVFP4_OK
+            assert bool((y == 0).all())
+    y = torch.full((4, 4), 7.0, dtype=torch.float32, device="cuda")
+    for M, N in [(0, 4), (4, 0)]:
+        st = L.nvfp4_linear(None, None, None, None, None, None, M, N, 64, _lib.NVFP4_F32, ptr(y),
+                            None, 0, s)
+        torch.cuda.synchronize()
+        assert st == _lib.NVFP4_OK
+        assert bool((y == 7.0).all())
+
+
 def test_linear_rejects_unknown_flag():
     from nvfp4_block_scaled_14_b200 import _lib as L
     qa = gpu_quantize(W.to_bf16_bits(W.normal((4, 64), 1.0, 32, 0)))

@@ -48,18 +48,6 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b)
     return __half2float(__half(hr));
 }
 
-// Two E4M3 bytes (low half of `b`) -> two fp32, exact.
-__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t b)
-{
-    uint32_t h2;
-    uint16_t in = (uint16_t)(b & 0xFFFFu);
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-    __half2_raw r;
-    r.x = (unsigned short)(h2 & 0xFFFFu);
-    r.y = (unsigned short)(h2 >> 16);
-    return __half22float2(__half2(r));
-}
-
 // One byte of two E2M1 codes -> two fp32 (low nibble first), exact.
 __device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte)
 {
@@ -221,14 +209,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 
 constexpr uint32_t kLayoutSwizzleNone = 0;
 constexpr uint32_t kLayoutSwizzle128B = 2;
-
-// Copy one 512-byte scale-factor atom (32 rows x 16 bytes in smem) to TMEM columns
-// [taddr, taddr + 4), replicated into the four 32-lane sub-partitions.
-__device__ __forceinline__ void tc_cp_sf_atom(uint32_t taddr, uint64_t sdesc)
-{
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
 
 // D(tmem) (+)= A(smem) x B(smem) with per-16 E4M3 block scales from TMEM.
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -511,17 +491,6 @@ __device__ __forceinline__ void pdl_launch_dependents()
 __device__ __forceinline__ void pdl_wait()
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t elect_one()
-{
-    uint32_t pred = 0;
-    asm volatile("{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\t"
-                 "elect.sync rx|px, %1;\n\t"
-                 "@px mov.s32 %0, 1;\n\t}"
-                 : "+r"(pred)
-                 : "r"(0xFFFFFFFFu));
-    return pred;
 }
 
 } // namespace nvfp4

@@ -142,7 +142,8 @@ class ClockSampler:
 
 class AttnStep:
     """The double-quant attention projection step over several input sets: W (FP8 source)
-    and X (bf16, dynamic amax) quantized in one launch, then the GEMM."""
+    and X (bf16, dynamic amax) quantized in one launch, then the GEMM. Each set has its own
+    inputs and its own outputs (quantized W and X, Y)."""
 
     def __init__(self, nv, wl, n_sets, dev):
         self.nv = nv
@@ -152,15 +153,15 @@ class AttnStep:
         self.W = [w8.clone() for _ in range(n_sets)]
         self.X = [xb.clone() for _ in range(n_sets)]
         self.s8 = s8
-        self.qw = nv.quantize_fp8(self.W[0], s8)
-        self.qx = nv.quantize(self.X[0])
-        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.QW = [nv.quantize_fp8(w, s8) for w in self.W]
+        self.QX = [nv.quantize(x) for x in self.X]
+        self.Y = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
 
     def run(self, i):
         nv = self.nv
-        nv.quantize_batch([{"x": self.W[i], "fp8_scale": self.s8, "out": self.qw},
-                           {"x": self.X[i], "out": self.qx}])
-        nv.linear(self.qx, self.qw, out=self.Y)
+        nv.quantize_batch([{"x": self.W[i], "fp8_scale": self.s8, "out": self.QW[i]},
+                           {"x": self.X[i], "out": self.QX[i]}])
+        nv.linear(self.QX[i], self.QW[i], out=self.Y[i])
 
 
 def bf16_dev(a, dev):
@@ -360,16 +361,15 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
     n_a = max(3, math.ceil(3 * L2 / (wl.W_e4m3.nbytes + wl.X_bf16.nbytes)))
     st = AttnStep(nv, wl, n_a, dev)
     step_ms, _ = op_timer([lambda i=i: st.run(i) for i in range(n_a)])
-    qw_ms, _ = op_timer([lambda i=i: nv.quantize_fp8(st.W[i], st.s8, out=st.qw)
+    qw_ms, _ = op_timer([lambda i=i: nv.quantize_fp8(st.W[i], st.s8, out=st.QW[i])
                          for i in range(n_a)])
-    qx_ms, _ = op_timer([lambda i=i: nv.quantize(st.X[i], out=st.qx) for i in range(n_a)])
+    qx_ms, _ = op_timer([lambda i=i: nv.quantize(st.X[i], out=st.QX[i]) for i in range(n_a)])
     qb_ms, _ = op_timer([lambda i=i: nv.quantize_batch([{"x": st.W[i], "fp8_scale": st.s8,
-                                                         "out": st.qw},
-                                                        {"x": st.X[i], "out": st.qx}])
+                                                         "out": st.QW[i]},
+                                                        {"x": st.X[i], "out": st.QX[i]}])
                          for i in range(n_a)])
-    qws = [nv.quantize_fp8(st.W[i], st.s8) for i in range(n_a)]
-    qxs = [nv.quantize(st.X[i]) for i in range(n_a)]
-    g_ms, _ = op_timer([lambda i=i: nv.linear(qxs[i], qws[i], out=st.Y) for i in range(n_a)])
+    g_ms, _ = op_timer([lambda i=i: nv.linear(st.QX[i], st.QW[i], out=st.Y[i])
+                        for i in range(n_a)])
     qx_bytes = M * K * QBYTES_BF16 + 4
     qw_bytes = N * K * (1 + 0.5 + 1 / 16) + 4
     g_tf = A_FLOPS / (g_ms * 1e-3) / 1e12
@@ -382,7 +382,7 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
         "quantize_x_frac_hbm": qx_bytes / (qx_ms * 1e-3) / 1e9 / hbm,
         "quantize_batch_GB/s": (qx_bytes + qw_bytes) / (qb_ms * 1e-3) / 1e9,
         "quantize_batch_frac_hbm": (qx_bytes + qw_bytes) / (qb_ms * 1e-3) / 1e9 / hbm}
-    del st, qws, qxs
+    del st
     torch.cuda.empty_cache()
 
     # --- the MLP's GEMM1 writing GEMM2's NVFP4 operand from its epilogue (static amax of the
@@ -467,12 +467,13 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
         nsw = sets_for(mm * kk + nn * kk)
         a8s = [nv.quantize_e4m3(xs[i % nset]) for i in range(nsw)]
         w8s = [nv.E4M3Tensor(w8.codes.clone(), w8.scale.clone()) for _ in range(nsw)]
-        y = torch.empty((mm, nn), dtype=torch.bfloat16, device=dev)
-        avg_q, _ = op_timer([lambda x=x, a=a8s[0]: nv.quantize_e4m3(x, out=a) for x in xs])
-        avg_g, _ = op_timer([lambda a=a, w=w: nv.linear_e4m3(a, w, out=y)
-                             for a, w in zip(a8s, w8s)])
-        avg_l, _ = op_timer([lambda x=x, a=a8s[i], w=w8s[i]: (nv.quantize_e4m3(x, out=a),
-                                                              nv.linear_e4m3(a, w, out=y))
+        ys = [torch.empty((mm, nn), dtype=torch.bfloat16, device=dev) for _ in range(nsw)]
+        avg_q, _ = op_timer([lambda x=x, a=a8s[i % nsw]: nv.quantize_e4m3(x, out=a)
+                             for i, x in enumerate(xs)])
+        avg_g, _ = op_timer([lambda a=a, w=w, y=y: nv.linear_e4m3(a, w, out=y)
+                             for a, w, y in zip(a8s, w8s, ys)])
+        avg_l, _ = op_timer([lambda x=x, a=a8s[i], w=w8s[i], y=ys[i]:
+                             (nv.quantize_e4m3(x, out=a), nv.linear_e4m3(a, w, out=y))
                              for i, x in enumerate(xs[:nsw] if nsw <= nset else xs)])
         qgbs = mm * kk * 3 / (avg_q * 1e-3) / 1e9
         tf = 2.0 * mm * nn * kk / (avg_g * 1e-3) / 1e12
@@ -480,7 +481,7 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
                      "quantize_x_frac_hbm": qgbs / hbm, "gemm_us": avg_g * 1e3,
                      "gemm_TFLOP/s": tf, "gemm_frac_fp8": tf / fp8_peak,
                      "quantize_x_then_gemm_us": avg_l * 1e3}
-        del xs, a8s, w8s, w8, y
+        del xs, a8s, w8s, w8, ys
         torch.cuda.empty_cache()
     rows["fp8_e4m3_w8a8"] = fp8
 
@@ -497,16 +498,17 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
     xs = [xb.clone() for _ in range(nset)]
     qxs = [nv.quantize(x) for x in xs]
     qws = [clone_q(nv, qw0) for _ in range(nset)]
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    avg_p, _ = op_timer([lambda a=a, w=w: nv.linear(a, w, out=y) for a, w in zip(qxs, qws)])
-    avg_l, _ = op_timer([lambda a=a, w=w, x=x: nv.linear_lowrank(a, w, x, dd, uu, out=y)
-                         for a, w, x in zip(qxs, qws, xs)])
+    ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(nset)]
+    avg_p, _ = op_timer([lambda a=a, w=w, y=y: nv.linear(a, w, out=y)
+                         for a, w, y in zip(qxs, qws, ys)])
+    avg_l, _ = op_timer([lambda a=a, w=w, x=x, y=y: nv.linear_lowrank(a, w, x, dd, uu, out=y)
+                         for a, w, x, y in zip(qxs, qws, xs, ys)])
     flops = 2.0 * M * N * K + 2.0 * M * K * LOWRANK_R + 2.0 * M * N * LOWRANK_R
     rows[f"lowrank_r{LOWRANK_R}_m{M}_n{N}_k{K}"] = {
         "linear_us": avg_p * 1e3, "linear_lowrank_us": avg_l * 1e3,
         "branch_extra_us": (avg_l - avg_p) * 1e3,
         "TFLOP/s": flops / (avg_l * 1e-3) / 1e12}
-    del xs, qxs, qws, y, xb, dd, uu, qw0
+    del xs, qxs, qws, ys, xb, dd, uu, qw0
     torch.cuda.empty_cache()
     return rows
 

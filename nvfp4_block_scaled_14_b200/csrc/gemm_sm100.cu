@@ -724,11 +724,14 @@ __device__ __forceinline__ void quantize_out_chunk(const GemmParams &p, const ui
 // the accumulator is handed back (release()) and the saved half is quantized while the next
 // tile's MMAs run.
 template <int ACT, typename Release>
-__device__ __forceinline__ void quantize_out_row(const GemmParams &p, uint32_t trow, uint32_t stg,
-                                                 int r, int64_t row, int64_t col0, float alpha,
-                                                 float t, float rt, const float *s_rcp,
-                                                 Release release)
+__device__ __forceinline__ void quantize_out_row(const GemmParams &p, uint32_t trow, uint32_t tpark,
+                                                 uint32_t stg, int r, int64_t row, int64_t col0,
+                                                 float alpha, float t, float rt,
+                                                 const float *s_rcp, Release release)
 {
+    // the accumulator is handed back as soon as it is copied: columns 128-255 to the staging
+    // tile (fp32), columns 0-127 to TMEM columns the MMAs do not use (tpark); the activation and
+    // the quantization of the whole tile then overlap the next tile's MMAs
 #pragma unroll 1
     for (int c0 = 128; c0 < 256; c0 += 64) {
         uint32_t v[64];
@@ -748,9 +751,21 @@ __device__ __forceinline__ void quantize_out_row(const GemmParams &p, uint32_t t
         for (int i = 0; i < 4; ++i)
             tmem_ld_32x32b_x16(trow + c0 + 16 * i, v + 16 * i);
         tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            tmem_st_32x32b_x16(tpark + c0 + 16 * i, v + 16 * i);
+    }
+    tmem_st_wait();
+    release();
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 64) {
+        uint32_t v[64];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            tmem_ld_32x32b_x16(tpark + c0 + 16 * i, v + 16 * i);
+        tmem_ld_wait();
         quantize_out_chunk<ACT>(p, v, row, col0 + c0, alpha, t, rt, s_rcp);
     }
-    release();
 #pragma unroll 1
     for (int c0 = 128; c0 < 256; c0 += 64) {
         uint32_t v[64];
@@ -846,9 +861,12 @@ template <bool QOUT> struct Pair {
     static constexpr int kSmemBytes = kOffRcp + 512;
     static constexpr uint32_t kTxAB = 2 * (kABytes + kBBytes); // both CTAs, on the leader
     static constexpr uint32_t kTxSf = kSfaBytes + kSfbBytes;   // own CTA
-    static constexpr int kSfSlots = 4;
+    // quantizing epilogue: two scale slots, so that 128 TMEM columns after them can hold half of
+    // the accumulator while its tile is quantized (quantize_out_row)
+    static constexpr int kSfSlots = QOUT ? 2 : 4;
     static constexpr int kSlotCols = 16 + 32; // SFA 4 x 4, SFB 4 x 8
     static constexpr int kSfCol = 256;
+    static constexpr int kParkCol = kSfCol + kSfSlots * kSlotCols; // QOUT: columns 0-127 kept
     static constexpr int kTmemCols = 512;
     static constexpr uint32_t kIdesc =
         (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
@@ -861,6 +879,7 @@ template <bool QOUT> struct Pair {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kOffStaging % 1024 == 0, "swizzled staging alignment");
     static_assert(kSfCol + kSfSlots * kSlotCols <= kTmemCols, "TMEM budget");
+    static_assert(!QOUT || kParkCol + 128 <= kTmemCols, "TMEM budget of the parked columns");
 };
 
 // 2-SM bf16 MMA issued by the leader CTA (the low-rank k-tiles): D (+)= A x B^T, fp32.
@@ -1198,12 +1217,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 };
                 const uint32_t stg = smem_u32(smem + C::kOffStaging);
                 const int64_t row = ta * 256 + rank * 128 + q * 32 + lane;
+                const uint32_t tpark = trow + C::kParkCol;
                 if (p.act == 1)
-                    quantize_out_row<1>(p, trow, stg, q * 32 + lane, row, tb * 256, alpha, q_t,
-                                        q_rt, s_rcp, release);
+                    quantize_out_row<1>(p, trow, tpark, stg, q * 32 + lane, row, tb * 256, alpha,
+                                        q_t, q_rt, s_rcp, release);
                 else
-                    quantize_out_row<0>(p, trow, stg, q * 32 + lane, row, tb * 256, alpha, q_t,
-                                        q_rt, s_rcp, release);
+                    quantize_out_row<0>(p, trow, tpark, stg, q * 32 + lane, row, tb * 256, alpha,
+                                        q_t, q_rt, s_rcp, release);
                 acc_phase ^= 1;
                 continue;
             }

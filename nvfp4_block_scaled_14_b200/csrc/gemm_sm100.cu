@@ -842,9 +842,10 @@ __device__ __forceinline__ void stage_store_tile_halves(const GemmParams &p, con
     store(1);
 }
 
-// Shared-memory layout of the pair kernel. bf16 output: five operand stages and a 32 KB bf16
-// staging tile (the output leaves in two halves); quantizing epilogue: four stages and 64 KB
-// of staging (fp32 columns 128-255 of each row while columns 0-127 are quantized).
+// Shared-memory and TMEM layout of the pair kernel. bf16 output: five operand stages and a 32 KB
+// bf16 staging tile (the output leaves in two halves), four scale slots; quantizing epilogue:
+// four stages and 64 KB of staging (fp32 columns 128-255 of each row), two scale slots and 128
+// TMEM columns for columns 0-127 (both kept while the tile is quantized after the hand-back).
 template <bool QOUT> struct Pair {
     static constexpr int kStages = QOUT ? 4 : 5;
     static constexpr int kABytes = 128 * 128;     // this CTA's 128 rows of A

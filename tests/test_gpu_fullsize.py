@@ -183,6 +183,97 @@ def test_step_in_cuda_graph_matches_eager():
     del g
 
 
+def test_mlp_step_in_cuda_graph_matches_eager():
+    # the bench's headline step (quantize X1 4096x3072, GEMM1 N12288 K3072, quantize X2
+    # 4096x12288, GEMM2 N3072 K12288) for two input sets, captured in one CUDA graph and replayed
+    # twice: the single-pass and streamed quantizers take a fresh grid barrier per captured
+    # launch, the pair GEMMs run their five-stage ring; every output must match the eager run bit
+    # for bit
+    mp = W.mlp_pair()
+    w1, w2 = nv.quantize(dev_tensor(mp.W1)), nv.quantize(dev_tensor(mp.W2))
+    x1s = [dev_tensor(mp.X1), dev_tensor(W.to_bf16_bits(W.normal((4096, 3072), 1.0, 81, 1)))]
+    x2s = [dev_tensor(mp.X2), dev_tensor(W.to_bf16_bits(np.abs(W.normal((4096, 12288), 1.0, 82,
+                                                                         2))))]
+    ref = []
+    for x1, x2 in zip(x1s, x2s):
+        y1 = nv.linear(nv.quantize(x1), w1)
+        y2 = nv.linear(nv.quantize(x2), w2)
+        ref.append((y1.clone(), y2.clone()))
+    q1, q2 = nv.quantize(x1s[0]), nv.quantize(x2s[0])
+    y1 = torch.empty_like(ref[0][0])
+    y2 = torch.empty_like(ref[0][1])
+    outs = [(torch.empty_like(y1), torch.empty_like(y2)) for _ in range(2)]
+
+    def step(i):
+        nv.quantize(x1s[i], out=q1)
+        nv.linear(q1, w1, out=y1)
+        nv.quantize(x2s[i], out=q2)
+        nv.linear(q2, w2, out=y2)
+        outs[i][0].copy_(y1)
+        outs[i][1].copy_(y2)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(0)
+        step(1)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(0)
+        step(1)
+    for _ in range(2):
+        for o in outs:
+            o[0].zero_()
+            o[1].zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert nv.sync_status() == 0
+        for i in range(2):
+            for k in range(2):
+                assert torch.equal(outs[i][k].view(torch.int16), ref[i][k].view(torch.int16)), (i, k)
+    del g
+
+
+def test_decode_chain_in_cuda_graph_matches_eager():
+    # back-to-back decode GEMVs (M 8 and M 1, N12288 K4096) with the resident-weights flag, as the
+    # bench chains them: each call requests its first weight tiles before waiting for the
+    # previous kernel; captured in a CUDA graph and replayed, they match the eager calls bit for
+    # bit
+    dc = W.decode(Ms=(1, 8))
+    wd = dev_tensor(dc.W)
+    qws = [nv.quantize(wd), nv.quantize((wd.float() * 0.5).to(torch.bfloat16)),
+           nv.quantize((wd.float() * -1.5).to(torch.bfloat16))]
+    qas = [nv.quantize(dev_tensor(dc.X[m])) for m in (8, 1)]
+    calls = [(qas[i % 2], qws[i % 3]) for i in range(6)]
+    ref = [nv.linear(a, w, resident_weights=True).clone() for a, w in calls]
+    ys = [torch.empty_like(r) for r in ref]
+
+    def chain():
+        for (a, w), y in zip(calls, ys):
+            nv.linear(a, w, out=y, resident_weights=True)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        chain()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        chain()
+    for _ in range(3):
+        for y in ys:
+            y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert nv.sync_status() == 0
+        for i, (y, r) in enumerate(zip(ys, ref)):
+            assert torch.equal(y.view(torch.int16), r.view(torch.int16)), i
+    del g
+
+
 @pytest.mark.parametrize("offset", [0, 16])
 def test_dequantize_full_weight(offset):
     # the MLP's 12288 x 3072 weight, as the bench times it: every warp of the grid takes several

@@ -73,7 +73,10 @@ size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
  * whole 128 x 4 atoms (swizzled = 1). */
 size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int swizzled);
 
-/* Device workspace the call needs (0 if none). Returns 0 for an unknown op. */
+/* Device workspace the call needs (0 if none). Returns 0 for an unknown op. A workspace holds
+ * the call's state (partial maxima, split-K partials) from the launch until its kernels have
+ * finished: calls that may run at the same time (on different streams or host threads) need
+ * different workspaces; calls on one stream may reuse one. */
 size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k);
 
 /*

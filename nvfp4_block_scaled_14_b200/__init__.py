@@ -63,9 +63,14 @@ _ws_cache = {}
 
 
 def _workspace(device, nbytes):
+    """The calling stream's workspace on `device` (grown as needed). A workspace holds a call's
+    state until its kernels finish, so calls on different streams, which may run at the same
+    time, never share one; a buffer is only ever used (and freed) on the stream that
+    allocated it."""
     if nbytes == 0:
         return None
-    key = (device.index if device.index is not None else torch.cuda.current_device())
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    key = (idx, torch.cuda.current_stream(idx).cuda_stream)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)

@@ -134,3 +134,33 @@ def test_grid_exchange_in_graph_replays():
         assert out.cpu().tolist() == [big, big / 2]
     assert nv.sync_status() == 0
     del g
+
+
+def test_quantizers_on_two_streams_at_once():
+    # single-pass quantizers (X1-sized, fused) and streamed ones (X2-sized) launched on two
+    # streams without ordering between them: each stream has its own grid barrier and its own
+    # workspace, so every result equals the one-at-a-time result
+    xs = [W.to_bf16_bits(W.normal((4096, 3072), 1.0, 90, 1)),
+          W.to_bf16_bits(W.normal((4096, 3072), 3.0, 90, 2)),
+          W.to_bf16_bits(W.normal((4096, 12288), 1.0, 90, 3)),
+          W.to_bf16_bits(W.normal((4096, 12288), 0.5, 90, 4))]
+    dx = [torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) for x in xs]
+    ref = [nv.quantize(x) for x in dx]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [nv.quantize(x) for x in dx]
+    for _ in range(3):
+        torch.cuda.synchronize()
+        for o in outs:
+            o.codes.zero_()
+            o.scales_swz.zero_()
+        torch.cuda.synchronize()
+        for i, x in enumerate(dx):
+            with torch.cuda.stream(streams[i % 2]):
+                nv.quantize(x, out=outs[i])
+        torch.cuda.synchronize()
+        assert nv.sync_status() == 0
+        for o, r in zip(outs, ref):
+            assert torch.equal(o.codes, r.codes)
+            assert torch.equal(o.scales_swz, r.scales_swz)
+            assert torch.equal(o.global_scale, r.global_scale)

@@ -361,9 +361,11 @@ nvfp4_status nvfp4_selftest_wait_timeout(cudaStream_t stream);
  * Test of the single-pass quantizers' grid-wide exchange. No counterpart in the paper. Those
  * kernels (nvfp4_quantize of 16 MB and more with a dynamic amax, the two-tensor
  * nvfp4_quantize_batch, nvfp4_quantize_e4m3) meet once all their CTAs have folded their
- * share of the tensor: each CTA writes its partial maximum and a token naming the launch into
- * a 16-byte slot of the workspace, then polls every slot until all carry that token, at most
- * a bounded number of rounds. This call runs the exchange alone, on a cooperative grid of nblk
+ * share of the tensor: each CTA writes its partial maxima into an 8-byte slot of the
+ * workspace and adds once to a barrier counter in library memory (one per stream, a fresh one
+ * per launch captured into a CUDA graph) whose top bit flips at the last arrival; every CTA
+ * polls for the flip for a bounded number of rounds, then reads all the slots. This call runs
+ * the exchange alone, on a cooperative grid of nblk
  * (1..160) CTAs of one warp: CTA i contributes vals[i] (device fp32; and vals[i] / 2 as the
  * second value); CTA skip_cta (-1: none) never arrives; CTA late_cta (-1: none) arrives after
  * spinning late_ns nanoseconds; poll_limit bounds the rounds. If every CTA arrived, out[0..1]
@@ -379,8 +381,9 @@ nvfp4_status nvfp4_selftest_grid_exchange(int nblk, const float *vals, int skip_
 
 /*
  * Synchronize the stream, then report and clear the library's device-side status word
- * (set by a kernel whose bounded wait gave up: NVFP4_ERR_TIMEOUT). Returns NVFP4_ERR_CUDA if
- * the synchronization itself failed.
+ * (set by a kernel whose bounded wait gave up: NVFP4_ERR_TIMEOUT). After a timeout it also
+ * resets the library's grid-barrier counters, which an exchange that gave up leaves
+ * unbalanced. Returns NVFP4_ERR_CUDA if the synchronization itself failed.
  */
 nvfp4_status nvfp4_sync_status(cudaStream_t stream);
 

@@ -607,8 +607,9 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
 // Fused single-pass quantizer for tensors that fit in the CTAs' shared memory (one CTA per
 // SM, up to kFusedCap bytes each): each CTA bulk-loads its contiguous share of warp items in
 // 32 KB copies. Dynamic amax: it folds max |x| over its share as the copies land, publishes
-// one partial, meets the other CTAs at a grid-wide barrier (cooperative launch: all CTAs are
-// co-resident), reduces the partials to the global scale and encodes from shared memory, so
+// one partial, meets the other CTAs at the library's bounded grid-wide barrier (cooperative
+// launch: all CTAs are co-resident; grid_exchange.cuh), reduces the partials to the global
+// scale and encodes from shared memory, so
 // the tensor is read from HBM once and no second kernel is launched. Static amax: no
 // barrier, each item is encoded as soon as its copy lands. Each lane reads its 64 (fp8: 32)
 // contiguous bytes as 16-byte vectors in a rotated order (lane_rotation): conflict-free.
@@ -621,8 +622,10 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const QuantArgs 
 // before a's shared-memory encode. Two tensors then cost one launch, one barrier and one HBM
 // read each, with all of both in flight at once (nvfp4_quantize_batch of, e.g., a layer's FP8
 // weight and its activations). Measured on W 3072x3072 FP8 + X 4096x3072 bf16 (globaltimer
-// stamps in an instrumented copy): loads and maxima ~7-8 us, grid barrier ~2 us, partials +
-// W's encode ~6 us, X's encode ~3.5 us; 1024 threads x 4 vectors beat 768 x 6 by ~0.5 us.
+// stamps in an instrumented copy, with the earlier cooperative-groups barrier): loads and
+// maxima ~7-8 us, grid barrier ~2 us (the library's own one-atomic barrier takes ~1 us),
+// partials + W's encode ~6 us, X's encode ~3.5 us; 1024 threads x 4 vectors beat 768 x 6 by
+// ~0.5 us.
 constexpr int kPairThreads = 1024; // 64 registers a thread: b's 16 plus the encode's
 constexpr int kPairRegVecs = 4;
 

@@ -26,7 +26,7 @@ from ._lib import (NVFP4_BF16, NVFP4_F32, NVFP4_LINEAR_DEFAULT, NVFP4_LINEAR_RES
 
 __all__ = ["NVFP4Tensor", "quantize", "quantize_fp8", "quantize_batch", "dequantize", "linear",
            "linear_dynamic", "linear_nvfp4_out", "linear_lowrank", "E4M3Tensor", "quantize_e4m3", "linear_e4m3",
-           "calib_percentile_amax", "sync_status", "load", "NVFP4Error"]
+           "calib_percentile_amax", "sync_status", "free_workspaces", "load", "NVFP4Error"]
 
 
 def __getattr__(name):
@@ -66,7 +66,8 @@ def _workspace(device, nbytes):
     """The calling stream's workspace on `device` (grown as needed). A workspace holds a call's
     state until its kernels finish, so calls on different streams, which may run at the same
     time, never share one; a buffer is only ever used (and freed) on the stream that
-    allocated it."""
+    allocated it. Each stream that has called the library keeps its workspace (at least
+    1 MiB) for the life of the process; free_workspaces() drops them all."""
     if nbytes == 0:
         return None
     idx = device.index if device.index is not None else torch.cuda.current_device()
@@ -76,6 +77,12 @@ def _workspace(device, nbytes):
         buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
         _ws_cache[key] = buf
     return buf
+
+
+def free_workspaces():
+    """Drop every cached workspace (after the device work that used them has finished, e.g.
+    after torch.cuda.synchronize()); later calls allocate afresh."""
+    _ws_cache.clear()
 
 
 def _alloc_outputs(rows, cols, device, swizzled, linear):

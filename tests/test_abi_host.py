@@ -143,3 +143,12 @@ def test_linear_lowrank_checks(lib):
     assert lr(*ops, 256, 256, 64, 128, FAKE, None, 0, None) == L.NVFP4_ERR_WORKSPACE
     assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_LINEAR_LOWRANK, 4096, 128, 0) == 4096 * 128 * 2
     assert lib.nvfp4_workspace_bytes(L.NVFP4_OP_LINEAR_LOWRANK, 4096, 512, 0) == 0
+
+
+def test_free_workspaces_empties_the_cache():
+    # host logic only: the binding's per-(device, stream) workspace cache and its reset
+    import nvfp4_block_scaled_14_b200 as nv
+    nv._ws_cache[(0, 12345)] = object()
+    assert "free_workspaces" in nv.__all__
+    nv.free_workspaces()
+    assert nv._ws_cache == {}

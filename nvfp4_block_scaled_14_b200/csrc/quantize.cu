@@ -8,10 +8,13 @@
 // quantization): "Qwen-Rapid-AIO FP8 -> NVFP4", "1. Double Quantization".
 //
 // Tensors of 16 MB up to what the CTAs' shared memory holds (148 x 192 KB) take one fused
-// single-pass kernel (fused_quantize_kernel, below); two tensors of a batch, the larger of that
-// size and the smaller up to what the threads' registers hold, take one fused launch together
-// (fused_pair_quantize_kernel). Every other size takes two kernels, both HBM-bound, chained by
-// programmatic dependent launch:
+// single-pass kernel (fused_quantize_kernel, below); larger ones take one streamed launch that
+// reads the tensor twice through a shared-memory ring, amax then encode
+// (stream_quantize_kernel); two tensors of a batch, the larger of the fused size and the
+// smaller up to what the threads' registers hold, take one fused launch together
+// (fused_pair_quantize_kernel). Tensors below 16 MB, and batches the pair launch does not fit
+// (amax_group_kernel / encode_group_kernel, one launch of each for all the batch's tensors),
+// take two kernels, both HBM-bound, chained by programmatic dependent launch:
 //   amax_kernel   (dynamic amax only) -- one CTA per SM streams a contiguous byte range of
 //                 the tensor (whole 16-byte vectors) through a 4 x 32 KB shared-memory ring of
 //                 1-D bulk copies and reduces max |x| with native packed max (exact,

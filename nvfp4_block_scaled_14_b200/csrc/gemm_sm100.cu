@@ -25,6 +25,14 @@
 //               the next tile's mainloop. (fp32 outputs / split-K partials store chunk-wise.)
 // Large M with few tiles splits K over CTAs of this kernel and a second kernel adds the fp32
 // partials in split order (deterministic).
+// Large M with bf16 output (and the NVFP4-output epilogue and the low-rank branch) runs
+// nvfp4_gemm_pair_kernel instead: the two CTAs of a cluster share 256 x 256 tiles
+// (tcgen05 cta_group::2, M256 x N256 x K64 MMAs issued by the leader; each CTA loads 128 rows
+// of A and 128 rows of B and holds its 128 rows of the accumulator), with the same warp roles.
+// Its bf16 epilogue stores the first half of a tile before it hands the accumulator back and
+// the second half after; the NVFP4-output form parks half of the accumulator in spare TMEM
+// columns and the other half in shared memory, so the whole tile is activated and quantized
+// while the next tile's MMAs run.
 // Small M (<= 128) runs swap-AB in its own kernel (nvfp4_gemm_smallm_kernel): the weights take
 // the MMA's M side (128 rows of W per tile) and the activation rows the N side (8..128), so
 // the tensor cores stream the weight matrix at full width; K is split over a thread-block

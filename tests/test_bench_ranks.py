@@ -52,3 +52,28 @@ def test_job_throughput_is_weak_scaling():
     assert bench.job_tflops(2, 0.044, flops) == pytest.approx(2 * one)
     assert one == pytest.approx(flops / 0.044e-3 / 1e12)
     assert bench.max_over_ranks(0.044, None, torch.device("cpu")) == 0.044
+
+
+def test_reference_arm_prints_one_contract_line():
+    # the reference arm (the CPU oracle on a bounded sample) runs without a GPU: one JSON line
+    # with the arm's own metric, unit and config, a cpu_baseline describing the run and an e2e
+    # entry that moves no bytes
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] == 3
+    assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True and d["value"] > 0
+    assert d["config"]["workload"] == "dit_mlp_pair_m4096_h3072_f12288"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    e = d["e2e"]
+    assert e["value"] == d["value"] and e["unit"] == d["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0

@@ -513,6 +513,18 @@ def extras(nv, W, dev, hbm, fp4_peak, mlp):
     return rows
 
 
+def oracle_threads():
+    """Threads the OpenMP oracle runs on: OMP_NUM_THREADS when set, else the CPUs this
+    process may run on (libgomp's default), not the machine's total."""
+    n = os.environ.get("OMP_NUM_THREADS", "").split(",")[0].strip()
+    if n.isdigit() and int(n) > 0:
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
 def oracle_sample(O, W):
     """A bounded sample of the MLP step for the CPU oracle: the weights quantized once (as the
     GPU step keeps them); per call, quantize X1 rows 0..63 and X2 rows 0..15 with their
@@ -550,7 +562,7 @@ def cpu_baseline(seconds=10.0):
         if time.time() - t0 >= seconds:
             break
     dt = (time.time() - t0) / reps
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = oracle_threads()
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{desc}; {reps} repetitions, {dt:.3f} s each"}
 
@@ -818,7 +830,7 @@ def run_reference(args):
         call()
     dt = (time.time() - t0) / args.steps
     value = flops / dt / 1e12
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = oracle_threads()
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,

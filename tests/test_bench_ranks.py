@@ -77,3 +77,13 @@ def test_reference_arm_prints_one_contract_line():
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_oracle_thread_count(monkeypatch):
+    # the cores a CPU-baseline line states are the oracle's OpenMP threads
+    import os
+    import bench
+    monkeypatch.setenv("OMP_NUM_THREADS", "3")
+    assert bench.oracle_threads() == 3
+    monkeypatch.delenv("OMP_NUM_THREADS")
+    assert bench.oracle_threads() == len(os.sched_getaffinity(0))

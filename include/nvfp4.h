@@ -22,7 +22,9 @@
  *       global_scale: one fp32 in device memory.
  *   - Blocks run along cols (the GEMM's K dimension). cols must be a multiple of 32.
  *   - The caller owns every buffer; the library never allocates or frees memory. Every
- *     pointer is a device pointer unless stated otherwise, 16-byte aligned.
+ *     pointer is a device pointer unless stated otherwise: arrays 16-byte aligned, pointers
+ *     to a single fp32 (global scales, static amax, fp8 scales, percentile outputs) 4-byte
+ *     aligned (NVFP4_ERR_ALIGNMENT otherwise).
  *   - Every call is asynchronous on the given stream. Argument checks run on the host before
  *     any launch and return an error without touching memory.
  *   - Numbers of rows, cols, M, N, K are >= 0 and < 2^31. Empty inputs are allowed.

@@ -166,7 +166,8 @@ nvfp4_status check_quantize(const void *x, int64_t rows, int64_t cols, const flo
     if (!empty && (!x || !codes || (!scales_swz && !scales_lin)))
         return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(codes) || !aligned16(scales_swz) || !aligned16(scales_lin) ||
-        (reinterpret_cast<uintptr_t>(global_scale) & 3u) || !aligned16(ws))
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(static_amax) & 3u) || !aligned16(ws))
         return NVFP4_ERR_ALIGNMENT;
     if (!static_amax && (!ws || ws_bytes < quantize_ws_bytes()))
         return NVFP4_ERR_WORKSPACE;
@@ -178,19 +179,10 @@ nvfp4_status quantize_common(const void *x, int src_type, const float *fp8_scale
                              uint8_t *scales_swz, uint8_t *scales_lin, float *global_scale,
                              void *ws, size_t ws_bytes, cudaStream_t s)
 {
-    nvfp4_status st = check_matrix(rows, cols);
+    nvfp4_status st = check_quantize(x, rows, cols, static_amax, codes, scales_swz, scales_lin,
+                                     global_scale, ws, ws_bytes);
     if (st != NVFP4_OK)
         return st;
-    const bool empty = rows == 0 || cols == 0;
-    if (!global_scale)
-        return NVFP4_ERR_INVALID_ARG;
-    if (!empty && (!x || !codes || (!scales_swz && !scales_lin)))
-        return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales_swz) || !aligned16(scales_lin) ||
-        (reinterpret_cast<uintptr_t>(global_scale) & 3u) || !aligned16(ws))
-        return NVFP4_ERR_ALIGNMENT;
-    if (!static_amax && (!ws || ws_bytes < quantize_ws_bytes()))
-        return NVFP4_ERR_WORKSPACE;
     if ((st = check_device()) != NVFP4_OK)
         return st;
     return map_cuda(launch_quantize(x, src_type, fp8_scale, rows, cols, static_amax, codes,
@@ -250,6 +242,8 @@ nvfp4_status nvfp4_quantize_batch(const nvfp4_quant_job *jobs, int njobs, void *
         const nvfp4_quant_job &q = jobs[j];
         if (q.src != NVFP4_SRC_F32 && q.src != NVFP4_SRC_BF16 && q.src != NVFP4_SRC_E4M3)
             return NVFP4_ERR_INVALID_ARG;
+        if (q.src == NVFP4_SRC_E4M3 && (reinterpret_cast<uintptr_t>(q.fp8_scale) & 3u))
+            return NVFP4_ERR_ALIGNMENT;
         const nvfp4_status st =
             check_quantize(q.x, q.rows, q.cols, q.static_amax, q.codes, q.scales_swz,
                            q.scales_lin, q.global_scale, ws, ws_bytes);

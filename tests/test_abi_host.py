@@ -152,3 +152,23 @@ def test_free_workspaces_empties_the_cache():
     assert "free_workspaces" in nv.__all__
     nv.free_workspaces()
     assert nv._ws_cache == {}
+
+
+def test_scalar_pointers_must_be_4_byte_aligned(lib):
+    # a static amax or an fp8 scale is one fp32 the kernels load as such
+    q = lib.nvfp4_quantize
+    assert q(FAKE, 1, 8, 64, FAKE + 2, FAKE, FAKE, None, FAKE, None, 0, None) == \
+        L.NVFP4_ERR_ALIGNMENT
+    f = lib.nvfp4_quantize_fp8_src
+    assert f(FAKE, FAKE, 8, 64, FAKE + 1, FAKE, FAKE, None, FAKE, None, 0, None) == \
+        L.NVFP4_ERR_ALIGNMENT
+    jobs = (L.QuantJob * 2)()
+    for j in jobs:
+        j.x, j.rows, j.cols, j.codes, j.scales_swz, j.global_scale = FAKE, 8, 64, FAKE, FAKE, FAKE
+        j.static_amax = FAKE
+    jobs[0].src, jobs[1].src = L.NVFP4_SRC_BF16, L.NVFP4_SRC_E4M3
+    jobs[1].fp8_scale = FAKE + 2
+    assert lib.nvfp4_quantize_batch(jobs, 2, None, 0, None) == L.NVFP4_ERR_ALIGNMENT
+    jobs[1].fp8_scale = FAKE
+    jobs[0].static_amax = FAKE + 2
+    assert lib.nvfp4_quantize_batch(jobs, 2, None, 0, None) == L.NVFP4_ERR_ALIGNMENT
